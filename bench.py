@@ -1,0 +1,352 @@
+#!/usr/bin/env python
+"""Optimizer-step benchmark of the B200 Gram Newton-Schulz Muon update.
+
+One step = dmu_momentum_normalize + dmu_gram_ns_batched (K = 5, quintic) +
+dmu_apply_update over the whole workload (default: 28 Qwen2.5-7B-shaped
+decoder layers, 196 bf16 matrices), inputs resident in HBM.  The inputs
+(~100 GB touched per step) are far larger than the 126 MB L2, so no L2
+flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the fp64 oracle on host cores
+
+Multi-GPU (torchrun, one process per GPU): every rank owns a full layer set
+of its own (owner-sharded by matrix, no collective on the data path), so
+per-GPU work is fixed (weak scaling); the step time is the max over ranks.
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "Gram-NS optimizer-step ms on 7B-shape layer set; TFLOP/s vs B200 bf16 peak"
+DEFAULT_WORKLOAD = "qwen2.5-7b-layer-set-x28"
+K_STEPS = 5
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def alg_flops(shapes, k=K_STEPS):
+    """Algorithmic flops of one step: SYRK m^2 n + (4K-3) symmetric m^3
+    products + final 2 m^2 n, per matrix (m = min, n = max)."""
+    tot = 0.0
+    for r, c in shapes:
+        m, n = min(r, c), max(r, c)
+        tot += 3.0 * m * m * n + (4 * k - 3) * float(m) ** 3
+    return tot
+
+
+def momentum_bytes(shapes, grad_bytes=2):
+    """HBM bytes of the momentum pass: read G and M, write M and Mb."""
+    e = sum(r * c for r, c in shapes)
+    return e * (grad_bytes + 4 + 4 + 2)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            out_dir = os.path.join(ROOT, "gpurun_out")
+            os.makedirs(out_dir, exist_ok=True)
+            self.path = os.path.join(out_dir, f"clocks_rank{self.index}.csv")
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def oracle_sample_seconds(shapes, budget_s=20.0):
+    """Time the fp64 oracle (as it stands) on a bounded sample and scale to
+    the full workload by each bucket's fp64 flop count."""
+    import numpy as np
+    import torch
+    from threadpoolctl import threadpool_info
+    import oracle
+    from gram_newton_schulz_b200 import synth
+
+    def rect_flops(r, c):
+        m, n = min(r, c), max(r, c)
+        return K_STEPS * (4.0 * m * m * n + 2.0 * m ** 3)
+
+    buckets = {}
+    for s in shapes:
+        buckets[s] = buckets.get(s, 0) + 1
+    # sample: one matrix of each bucket whose fp64 cost fits the budget,
+    # smallest first; the other buckets are scaled by flop count
+    order = sorted(buckets, key=lambda s: rect_flops(*s))
+    w = synth.custom("sample", order, seed=99)
+    timed, spent = {}, 0.0
+    for i, s in enumerate(order):
+        est = rect_flops(*s) / 2e11  # a conservative fp64 rate guess
+        if timed and spent + est > budget_s:
+            break
+        g = synth.gradient(w, i).to(torch.float64).numpy()
+        wt = synth.weight(w, i).to(torch.float64).numpy()
+        t0 = time.perf_counter()
+        oracle.muon_step(wt, np.zeros_like(g), g, beta=0.95, lr=0.02)
+        dt = time.perf_counter() - t0
+        timed[s] = dt
+        spent += dt
+    rate = sum(rect_flops(*s) for s in timed) / sum(timed.values())
+    total = 0.0
+    for s, n in buckets.items():
+        total += n * (timed[s] if s in timed else rect_flops(*s) / rate)
+    threads = max((d.get("num_threads", 1) for d in threadpool_info()), default=os.cpu_count())
+    sample = ("fp64 oracle muon_step timed on one matrix each of " +
+              ", ".join(f"{r}x{c}" for r, c in timed) +
+              ("; other buckets scaled by fp64 flop count" if len(timed) < len(buckets) else "") +
+              f"; scaled to {len(shapes)} matrices")
+    return total, threads, sample, spent
+
+
+def run_reference(args):
+    """--impl reference: the oracle on the host cores (bounded samples)."""
+    from gram_newton_schulz_b200 import synth
+    w = synth.workload(args.workload)
+    vals = []
+    for k in range(args.warmup + args.steps):
+        total, threads, sample, _ = oracle_sample_seconds(w.shapes, budget_s=args.ref_budget)
+        if k >= args.warmup:
+            vals.append(total * 1e3)
+    v = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "ms", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(v, 3), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "matrices": w.count, "K": K_STEPS, "coeffs": [3.4445, -4.7750, 2.0315]},
+        "cpu_baseline": {"value": round(v, 3), "unit": "ms", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(v, 3), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="dmu", choices=["dmu", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--prec", default="auto")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-budget", type=float, default=10.0)
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from gram_newton_schulz_b200 import dmu, synth
+
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    w = synth.workload(args.workload)
+    grads = synth.gradients(w, dev)
+    weights = synth.weights(w, dev)
+    moms = [torch.zeros(s, dtype=torch.float32, device=dev) for s in w.shapes]
+    plan = dmu.Plan(w.shapes, dtype=w.dtype, prec=args.prec, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        plan.momentum_normalize(grads, moms, beta=w.beta, eps=1e-7)
+        n0 = plan.last_launch_count()
+        plan.gram_ns_batched(None, dmu.QUINTIC, K_STEPS)
+        n1 = plan.last_launch_count()
+        plan.apply_update(weights, lr=w.lr)
+        n2 = plan.last_launch_count()
+        return n0 + n1 + n2
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if plan.read_status() != 0:
+        raise SystemExit("device status word set during warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(dev)
+    launches = 0
+    for k in range(K):
+        ev[k][0].record(stream)
+        plan.momentum_normalize(grads, moms, beta=w.beta, eps=1e-7)
+        launches += plan.last_launch_count()
+        ev[k][1].record(stream)
+        plan.gram_ns_batched(None, dmu.QUINTIC, K_STEPS)
+        launches += plan.last_launch_count()
+        ev[k][2].record(stream)
+        plan.apply_update(weights, lr=w.lr)
+        launches += plan.last_launch_count()
+        ev[k][3].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    total_ms = ev[0][0].elapsed_time(ev[K - 1][3])
+    t_mom = sum(e[0].elapsed_time(e[1]) for e in ev)
+    t_gram = sum(e[1].elapsed_time(e[2]) for e in ev)
+    t_upd = sum(e[2].elapsed_time(e[3]) for e in ev)
+    step_ms = total_ms / K
+    if world > 1:
+        t = torch.tensor([step_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_ms = float(t.item())
+    status = plan.read_status()
+
+    peaks, peak_kind = load_peaks()
+    flops = alg_flops(w.shapes)
+    tc_s = (t_gram + t_upd) / K / 1e3
+    achieved_tf = flops / tc_s / 1e12
+    peak_tf = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    mom_s = t_mom / K / 1e3
+    mom_gbs = momentum_bytes(w.shapes) / mom_s / 1e9
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+
+    # end to end through the public API with host buffers: pinned gradients
+    # in, updated weights out, every step
+    e2e = None
+    if not args.no_e2e:
+        h_grads = [g.to("cpu").pin_memory() for g in grads]
+        h_w = [x.to("cpu").pin_memory() for x in weights]
+        h2d = sum(t.numel() * t.element_size() for t in h_grads)
+        d2h = sum(t.numel() * t.element_size() for t in h_w)
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            for hg, g in zip(h_grads, grads):
+                g.copy_(hg, non_blocking=True)
+            step()
+            for hw, x in zip(h_w, weights):
+                hw.copy_(x, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": round(e2e_ms, 3), "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        total_s, threads, sample, _ = oracle_sample_seconds(w.shapes)
+        cpu = {"value": round(total_s * 1e3, 1), "unit": "ms", "cores": threads, "kind": "oracle",
+               "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(step_ms, 3), "unit": "ms", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": round(step_ms, 3), "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+            "data": "synthetic",
+            "config": {"workload": w.name, "matrices": w.count, "matrices_total": w.count * world,
+                       "K": K_STEPS, "coeffs": [3.4445, -4.7750, 2.0315], "precision": args.prec,
+                       "parallelism": f"owner-sharded x{world} (independent layer sets)",
+                       "l2": "inputs larger than L2 (no flush needed)"},
+            "throughput": {"matrices_per_s": round(w.count * world / (step_ms / 1e3), 1),
+                           "alg_tflops": round(flops * world / (step_ms / 1e3) / 1e12, 1),
+                           "alg_tflops_frac": round(flops / (step_ms / 1e3) / 1e12 / peak_tf, 4)},
+            "split_ms": {"momentum": round(t_mom / K, 3), "gram": round(t_gram / K, 3),
+                         "update": round(t_upd / K, 3)},
+            "roofline": {"bound": "tensor", "achieved": round(achieved_tf, 1), "peak": peak_tf,
+                         "unit": "TFLOP/s", "frac": round(achieved_tf / peak_tf, 4), "traffic": None,
+                         "kernel": "k_gemm_tc (all Gram-space and final launches)",
+                         "peak_kind": f"{peak_kind} bf16 sustained"},
+            "hbm_kernel": {"kernel": "k_momentum", "achieved": round(mom_gbs, 1), "peak": hbm,
+                           "unit": "GB/s", "frac": round(mom_gbs / hbm, 4), "peak_kind": peak_kind},
+            "gpu_launches": launches,
+            "status_word": status,
+            "clocks": clk,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    plan.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,142 @@
+// Internal types shared by the planner (plan.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "dmu.h"
+
+namespace dmu {
+
+// ---------------------------------------------------------------- tiles
+// One CTA computes a BM x BN fp32 tile in TMEM with tcgen05.mma
+// (M = 128, N = 256, K = 16 per instruction), K-blocks of BK = 64 bf16
+// (one 128-byte swizzle atom per row).
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;
+constexpr int UMMA_K = 16;
+constexpr int A_PART_BYTES = BM * BK * 2;  // 16 KB
+constexpr int B_PART_BYTES = BN * BK * 2;  // 32 KB
+constexpr int GEMM_THREADS = 192;          // TMA warp, MMA warp, 4 epilogue warps
+constexpr int TMEM_COLS = 512;             // two BN-column accumulators
+
+constexpr int MAX_MAPS = 16;
+constexpr int MAX_PROBS = 8;
+
+// Gram-space storage slots (each a bf16 matrix); hi/lo pairs.
+enum GramSlot : int {
+  SLOT_G_HI = 0, SLOT_G_LO, SLOT_R_HI, SLOT_R_LO, SLOT_T_HI, SLOT_T_LO,
+  SLOT_PA_HI, SLOT_PA_LO, SLOT_PB_HI, SLOT_PB_LO, NUM_SLOTS
+};
+// fp32 path: one fp32 matrix per quantity.
+enum GramSlotF32 : int { FSLOT_G = 0, FSLOT_R, FSLOT_T, FSLOT_PA, FSLOT_PB, NUM_FSLOTS };
+
+enum Epi : int { EPI_GRAM = 0, EPI_UPDATE = 1 };
+enum AlphaMode : int { ALPHA_CONST = 0, ALPHA_INV2 = 1, ALPHA_INV = 2 };
+
+// Term bits: which bf16 products the MMA warp issues per K slice.
+enum Terms : int { TERM_HH = 1, TERM_HL = 2, TERM_LH = 4 };
+
+// One grouped-GEMM problem: `count` independent matrices of the same
+// geometry.  Output tile (bi, bj) of matrix `mat` is
+//   D[i][j] = sum_k A(i, k) * B(j, k),   i in [0, M), j in [0, N)
+// where A and B are read by TMA from 3-D tensor maps; z = base + mat.
+struct GemmProblem {
+  int count, M, N, K;
+  int tiles_m, tiles_n, tiles_per_mat;
+  int tile_begin;       // first global tile index of this problem
+  int sym;              // upper-triangle tiles only, mirrored write (M == N)
+  int a_map, b_map;     // indices into GemmParams::maps
+  int a_mn, b_mn;       // 1: operand is MN-major (M/N contiguous)
+  int a_z[2], b_z[2];   // z base of the hi and lo parts
+  int terms;            // Terms bits
+  // epilogue
+  int epi;
+  int alpha_mode;
+  float alpha, beta, gamma, gamma2;
+  const float* inv;     // per-matrix 1/(||M||+eps), indexed by inv_base + mat
+  int inv_base;
+  // EPI_GRAM: out = alpha' * acc + beta * Cin + gamma * I  (bf16 hi/lo pair)
+  const __nv_bfloat16* cin_hi;
+  const __nv_bfloat16* cin_lo;
+  __nv_bfloat16* out_hi;
+  __nv_bfloat16* out_lo;   // may be null
+  __nv_bfloat16* out2_hi;  // optional second output out + gamma2 * I
+  __nv_bfloat16* out2_lo;
+  long long ld;            // row stride (elements) of Cin/out
+  long long mat_stride;    // matrix stride (elements) of Cin/out
+  // EPI_UPDATE: W += alpha * inv * acc in W's layout; O = inv * acc
+  void* const* w_ptrs;     // device table, indexed by ptr_base + mat
+  float* const* o_ptrs;    // device table (may be null)
+  int ptr_base;
+  int w_f32;               // W is fp32 (else bf16)
+  int w_transposed;        // output tile is W^T (tall matrix)
+  long long w_cols;        // W's row length
+};
+
+struct __align__(64) GemmParams {
+  CUtensorMap maps[MAX_MAPS];
+  GemmProblem prob[MAX_PROBS];
+  int nprob;
+  int total_tiles;
+  unsigned int* status;    // device status word
+  long long timeout_ns;    // bounded-wait limit
+};
+
+// ---------------------------------------------------------------- momentum
+struct MomChunk {
+  long long start;  // first element (flat, row-major) within the matrix
+  int slot;         // matrix slot (bucket order)
+  int len;          // elements in this chunk
+};
+
+struct MomMat {     // per-slot geometry for the momentum/normalise pass
+  long long rows, cols, ldc;
+  long long mb_off;     // element offset of this matrix's image in the Mb area
+  int chunk_begin, chunk_end;
+};
+
+constexpr int MOM_CHUNK = 16384;
+
+// ---------------------------------------------------------------- fp32 path
+struct SimtProblem {
+  int count, M, N, K;
+  int sym;
+  // A(i,k) = a + mat*a_ms + i*a_si + k*a_sk ; same for B(j,k)
+  const float* a; long long a_ms, a_si, a_sk;
+  const float* b; long long b_ms, b_si, b_sk;
+  int epi, alpha_mode;
+  float alpha, beta, gamma, gamma2;
+  const float* inv; int inv_base;
+  const float* cin; float* out; float* out2;
+  long long ld, mat_stride;
+  void* const* w_ptrs; float* const* o_ptrs; int ptr_base;
+  int w_f32, w_transposed; long long w_cols;
+};
+
+// ---------------------------------------------------------------- launchers
+cudaError_t launch_gemm_tc(const GemmParams& p, int na, int nb, int num_sms, cudaStream_t s);
+cudaError_t gemm_tc_configure();
+cudaError_t launch_wait_selftest(unsigned int* status, long long timeout_ns, cudaStream_t s);
+int gemm_tc_stages(int na, int nb);
+
+cudaError_t launch_momentum(const MomChunk* chunks, int nchunks, const MomMat* mats,
+                            const void* const* grads, float* const* momenta, int grad_f32,
+                            void* mb, int mb_f32, float beta, float* partial,
+                            int vec_ok, int num_sms, cudaStream_t s);
+cudaError_t launch_norm_finalize(const MomMat* mats, int nmats, const float* partial,
+                                 float eps, float* inv, unsigned int* status, cudaStream_t s);
+cudaError_t launch_simt_gemm(const SimtProblem& p, cudaStream_t s);
+cudaError_t launch_identity_bf16(__nv_bfloat16* hi, __nv_bfloat16* lo, int count, int m,
+                                 long long ld, long long mat_stride, cudaStream_t s);
+cudaError_t launch_identity_f32(float* p, int count, int m, long long ld, long long mat_stride,
+                                cudaStream_t s);
+cudaError_t launch_pair_to_f32(const __nv_bfloat16* hi, const __nv_bfloat16* lo, long long rows,
+                               long long cols, long long ld, float* out, cudaStream_t s);
+cudaError_t launch_f32_copy2d(const float* src, long long rows, long long cols, long long ld,
+                              float* out, cudaStream_t s);
+
+}  // namespace dmu

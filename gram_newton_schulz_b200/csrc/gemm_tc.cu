@@ -1,0 +1,612 @@
+// Grouped bf16 GEMM on the 5th-generation tensor cores (tcgen05), sm_100a.
+//
+// Every product of the Muon update is one "problem" here:
+//   * the Gram matrix G0 = s^2 X X^T (SYRK: only upper-triangle tiles,
+//     mirrored on write) -- DMuon page, section 2.2 (Gram-space recursion,
+//     SYRK-style symmetric path); Dion3 review, section 3 (symmetric GEMM);
+//   * the Gram-space products G G, R G, R P, T R of the recursion
+//     Q = aI + bG + cG^2, G <- QGQ, P <- QP, written as R = Q - aI so the
+//     identity terms are applied exactly in the fp32 epilogue:
+//       R = bG + c(GG),  T = aG + RG,  G' = aT + TR,  P' = aP + RP
+//     (all operands are polynomials in G0, hence symmetric and commuting;
+//     only upper tiles are computed);
+//   * the final O = P X0 with the weight update fused in the epilogue.
+//
+// Structure (one CTA per SM, persistent, static round-robin over tiles):
+//   warp 0     TMA producer: 3-D tensor maps, 128-byte swizzle, a ring of
+//              shared-memory stages guarded by full/empty mbarriers;
+//   warp 1     MMA issuer: one thread issues tcgen05.mma (M=128, N=256,
+//              K=16) into one of two TMEM accumulators (2 x 256 columns);
+//   warps 2-5  epilogue: tcgen05.ld of their 32-lane quarter, fp32 affine
+//              epilogue, bf16 hi/lo split, direct + mirrored stores; the
+//              epilogue of tile t overlaps the main loop of tile t+1.
+// Operand precision: each stage holds up to two bf16 parts of A (hi, lo)
+// and of B; the problem's term bits choose hi*hi, hi*lo, lo*hi.
+// Every mbarrier wait is bounded by a wall-clock limit; on expiry the CTA
+// sets DMU_FLAG_TIMEOUT in the status word and winds down.
+#include "dmu_internal.h"
+#include "ptx.cuh"
+
+namespace dmu {
+
+template <int NA, int NB>
+struct TcCfg {
+  static constexpr int STAGE_BYTES = NA * A_PART_BYTES + NB * B_PART_BYTES;
+  static constexpr int STAGES = (200 * 1024) / STAGE_BYTES;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static_assert(STAGES >= 2, "at least two stages");
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+};
+
+struct TileCoord {
+  int pi, mat, bi, bj;
+};
+
+__device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int t) {
+  TileCoord c;
+  int pi = 0;
+  while (pi + 1 < p.nprob && t >= p.prob[pi + 1].tile_begin) ++pi;
+  const GemmProblem& pr = p.prob[pi];
+  int local = t - pr.tile_begin;
+  int mat = local / pr.tiles_per_mat;
+  int tl = local - mat * pr.tiles_per_mat;
+  int bi, bj;
+  if (!pr.sym) {
+    bi = tl % pr.tiles_m;
+    bj = tl / pr.tiles_m;
+  } else {
+    // column block bj holds row blocks 0 .. min(tiles_m, ((bj+1)*BN-1)/BM + 1) - 1
+    bj = 0;
+    for (;;) {
+      int cnt = min(pr.tiles_m, ((bj + 1) * BN - 1) / BM + 1);
+      if (tl < cnt) break;
+      tl -= cnt;
+      ++bj;
+    }
+    bi = tl;
+  }
+  c.pi = pi;
+  c.mat = mat;
+  c.bi = bi;
+  c.bj = bj;
+  return c;
+}
+
+// Bounded wait on an mbarrier phase.  Returns false when the CTA is
+// winding down (this or another role timed out).
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         const GemmParams& p) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  uint32_t n = 0;
+  for (;;) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if ((++n & 63u) == 0) {
+      if (*abort_flag) return false;
+      if ((long long)(ptx::globaltimer() - t0) > p.timeout_ns) {
+        *abort_flag = 1;
+        atomicOr(p.status, DMU_FLAG_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------- epilogue
+__device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+__device__ __forceinline__ void unpack8(const uint4& u, float* f) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    float2 t = __bfloat1622float2(h[q]);
+    f[2 * q] = t.x;
+    f[2 * q + 1] = t.y;
+  }
+}
+
+__device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&hi);
+  __nv_bfloat162* l = reinterpret_cast<__nv_bfloat162*>(&lo);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    __nv_bfloat16 h0 = __float2bfloat16_rn(v[2 * q]);
+    __nv_bfloat16 h1 = __float2bfloat16_rn(v[2 * q + 1]);
+    h[q] = __halves2bfloat162(h0, h1);
+    l[q] = __halves2bfloat162(__float2bfloat16_rn(v[2 * q] - bf2f(h0)),
+                              __float2bfloat16_rn(v[2 * q + 1] - bf2f(h1)));
+  }
+}
+
+// Store value v at (i, j) of a hi/lo pair.
+__device__ __forceinline__ void store_pair(__nv_bfloat16* hi, __nv_bfloat16* lo, long long off,
+                                           float v) {
+  __nv_bfloat16 h = __float2bfloat16_rn(v);
+  hi[off] = h;
+  if (lo) lo[off] = __float2bfloat16_rn(v - bf2f(h));
+}
+
+// One 32-column chunk of a Gram-space output tile for the thread's row i.
+__device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, int i, int col0,
+                                               const uint32_t (&r)[32]) {
+  const int M = pr.M, N = pr.N;
+  if (i >= M) return;
+  float coef = pr.alpha;
+  if (pr.alpha_mode == ALPHA_INV2) {
+    float s = pr.inv[pr.inv_base + mat];
+    coef *= s * s;
+  } else if (pr.alpha_mode == ALPHA_INV) {
+    coef *= pr.inv[pr.inv_base + mat];
+  }
+  float v[32];
+#pragma unroll
+  for (int c = 0; c < 32; ++c) v[c] = coef * __uint_as_float(r[c]);
+
+  const long long mbase = (long long)mat * pr.mat_stride;
+  const long long rowoff = mbase + (long long)i * pr.ld;
+  const bool full = (col0 + 32 <= N);
+  const bool all_upper = !pr.sym || (i <= col0);
+
+  if (pr.cin_hi) {
+    if (full) {
+      const uint4* ph = reinterpret_cast<const uint4*>(pr.cin_hi + rowoff + col0);
+      const uint4* pl = pr.cin_lo ? reinterpret_cast<const uint4*>(pr.cin_lo + rowoff + col0) : nullptr;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float fh[8], fl[8];
+        unpack8(ph[q], fh);
+        if (pl) {
+          unpack8(pl[q], fl);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) fl[e] = 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[8 * q + e] += pr.beta * (fh[e] + fl[e]);
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        if (col0 + c < N) {
+          float x = bf2f(pr.cin_hi[rowoff + col0 + c]);
+          if (pr.cin_lo) x += bf2f(pr.cin_lo[rowoff + col0 + c]);
+          v[c] += pr.beta * x;
+        }
+      }
+    }
+  }
+  const int dc = i - col0;  // diagonal column within the chunk
+  if (dc >= 0 && dc < 32) {
+#pragma unroll
+    for (int c = 0; c < 32; ++c)
+      if (c == dc) v[c] += pr.gamma;
+  }
+
+  for (int pass = 0; pass < 2; ++pass) {
+    __nv_bfloat16* oh = pass == 0 ? pr.out_hi : pr.out2_hi;
+    __nv_bfloat16* ol = pass == 0 ? pr.out_lo : pr.out2_lo;
+    if (!oh) continue;
+    if (pass == 1 && dc >= 0 && dc < 32) {
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (c == dc) v[c] += pr.gamma2;
+    }
+    // direct stores (i, j), j >= i when symmetric
+    if (full && all_upper) {
+      uint4* dh = reinterpret_cast<uint4*>(oh + rowoff + col0);
+      uint4* dl = ol ? reinterpret_cast<uint4*>(ol + rowoff + col0) : nullptr;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 h, l;
+        split8(v + 8 * q, h, l);
+        dh[q] = h;
+        if (dl) dl[q] = l;
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const int j = col0 + c;
+        if (j < N && (!pr.sym || i <= j)) store_pair(oh, ol, rowoff + j, v[c]);
+      }
+    }
+    // mirrored stores (j, i) for j > i: consecutive lanes write consecutive
+    // columns of row j, so each store instruction is coalesced.
+    if (pr.sym) {
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const int j = col0 + c;
+        if (j < N && i < j) store_pair(oh, ol, mbase + (long long)j * pr.ld + i, v[c]);
+      }
+    }
+  }
+}
+
+// One 32-column chunk of the final O = P X0 tile, fused with the update.
+// Row i of the tile is row i of O (m x n); element (i, j) lives at W[i][j]
+// for a wide matrix and at W[j][i] for a tall one (w_transposed).
+__device__ __forceinline__ void epi_update_chunk(const GemmProblem& pr, int mat, int i, int col0,
+                                                 const uint32_t (&r)[32]) {
+  const int M = pr.M, N = pr.N;
+  if (i >= M) return;
+  const float s = pr.inv[pr.inv_base + mat];
+  const float cw = pr.alpha * s;  // -lr * scale / (||M|| + eps)
+  float o[32];
+#pragma unroll
+  for (int c = 0; c < 32; ++c) o[c] = __uint_as_float(r[c]);
+  void* wp = pr.w_ptrs ? pr.w_ptrs[pr.ptr_base + mat] : nullptr;
+  float* op = pr.o_ptrs ? pr.o_ptrs[pr.ptr_base + mat] : nullptr;
+  const long long wc = pr.w_cols;
+  if (!pr.w_transposed) {
+    const long long rowoff = (long long)i * wc;
+    const bool full = (col0 + 32 <= N);
+    if (wp) {
+      if (!pr.w_f32) {
+        __nv_bfloat16* w = reinterpret_cast<__nv_bfloat16*>(wp);
+        const bool vec = full && ((wc & 7) == 0) && ((reinterpret_cast<uintptr_t>(w) & 15) == 0);
+        if (vec) {
+          uint4* pw = reinterpret_cast<uint4*>(w + rowoff + col0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float f[8];
+            unpack8(pw[q], f);
+            uint4 h;
+            __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&h);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              hh[e] = __floats2bfloat162_rn(f[2 * e] + cw * o[8 * q + 2 * e],
+                                            f[2 * e + 1] + cw * o[8 * q + 2 * e + 1]);
+            pw[q] = h;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (col0 + c < N) {
+              long long off = rowoff + col0 + c;
+              w[off] = __float2bfloat16_rn(bf2f(w[off]) + cw * o[c]);
+            }
+        }
+      } else {
+        float* w = reinterpret_cast<float*>(wp);
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if (col0 + c < N) w[rowoff + col0 + c] += cw * o[c];
+      }
+    }
+    if (op) {
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (col0 + c < N) op[rowoff + col0 + c] = s * o[c];
+    }
+  } else {
+    // W is n x m (rows = N here, cols = M); element (i, j) -> W[j][i].
+    if (wp) {
+      if (!pr.w_f32) {
+        __nv_bfloat16* w = reinterpret_cast<__nv_bfloat16*>(wp);
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if (col0 + c < N) {
+            long long off = (long long)(col0 + c) * wc + i;
+            w[off] = __float2bfloat16_rn(bf2f(w[off]) + cw * o[c]);
+          }
+      } else {
+        float* w = reinterpret_cast<float*>(wp);
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if (col0 + c < N) w[(long long)(col0 + c) * wc + i] += cw * o[c];
+      }
+    }
+    if (op) {
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (col0 + c < N) op[(long long)(col0 + c) * wc + i] = s * o[c];
+    }
+  }
+}
+
+// ------------------------------------------------------------- kernel
+template <int NA, int NB>
+__global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_constant__ GemmParams p) {
+  using Cfg = TcCfg<NA, NB>;
+  constexpr int S = Cfg::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = ptx::smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  const uint32_t ring = base;
+  const uint32_t bars = base + S * Cfg::STAGE_BYTES;
+  auto full_bar = [&](int s) { return bars + 8u * s; };
+  auto empty_bar = [&](int s) { return bars + 8u * (S + s); };
+  auto tfull_bar = [&](int b) { return bars + 8u * (2 * S + b); };
+  auto tempty_bar = [&](int b) { return bars + 8u * (2 * S + 2 + b); };
+  const uint32_t drain_bar = bars + 8u * (2 * S + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S * Cfg::STAGE_BYTES + 8 * (2 * S + 5));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      ptx::mbar_init(full_bar(s), 1);
+      ptx::mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(tfull_bar(b), 1);
+      ptx::mbar_init(tempty_bar(b), 4);
+    }
+    ptx::mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+    ptx::fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int pi = 0; pi < p.nprob; ++pi) {
+      ptx::prefetch_tmap(&p.maps[p.prob[pi].a_map]);
+      ptx::prefetch_tmap(&p.maps[p.prob[pi].b_map]);
+    }
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      uint32_t issued_mask = 0, issued_par = 0;  // per stage: a load was issued, its phase parity
+      for (int t = blockIdx.x; ok && t < p.total_tiles; t += gridDim.x) {
+        const TileCoord tc = decode_tile(p, t);
+        const GemmProblem& pr = p.prob[tc.pi];
+        const CUtensorMap* am = &p.maps[pr.a_map];
+        const CUtensorMap* bm = &p.maps[pr.b_map];
+        const int na = (NA > 1 && (pr.terms & TERM_LH)) ? 2 : 1;
+        const int nb = (NB > 1 && (pr.terms & TERM_HL)) ? 2 : 1;
+        const uint32_t bytes = na * A_PART_BYTES + nb * B_PART_BYTES;
+        const int nk = (pr.K + BK - 1) / BK;
+        const int arow = tc.bi * BM, brow = tc.bj * BN;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!wait_bar(empty_bar(stage), phase ^ 1u, abort_flag, p)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = full_bar(stage);
+          ptx::mbar_arrive_expect_tx(fb, bytes);
+          issued_mask |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          const int k0 = kb * BK;
+          const uint32_t sa = ring + stage * Cfg::STAGE_BYTES;
+          const uint32_t sb = sa + NA * A_PART_BYTES;
+          for (int part = 0; part < na; ++part) {
+            const uint32_t dst = sa + part * A_PART_BYTES;
+            const int z = pr.a_z[part] + tc.mat;
+            if (!pr.a_mn) {
+              ptx::tma_load_3d(dst, am, fb, k0, arow, z);
+            } else {
+              ptx::tma_load_3d(dst, am, fb, arow, k0, z);
+              ptx::tma_load_3d(dst + 8192, am, fb, arow + 64, k0, z);
+            }
+          }
+          for (int part = 0; part < nb; ++part) {
+            const uint32_t dst = sb + part * B_PART_BYTES;
+            const int z = pr.b_z[part] + tc.mat;
+            if (!pr.b_mn) {
+              ptx::tma_load_3d(dst, bm, fb, k0, brow, z);
+              ptx::tma_load_3d(dst + 16384, bm, fb, k0, brow + 128, z);
+            } else {
+#pragma unroll
+              for (int c = 0; c < 4; ++c) ptx::tma_load_3d(dst + 8192 * c, bm, fb, brow + 64 * c, k0, z);
+            }
+          }
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Before the CTA may exit, every bulk copy it issued must have landed
+      // (normally already true: the MMA warp consumed them).
+      for (int s2 = 0; s2 < S; ++s2) {
+        if (!(issued_mask & (1u << s2))) continue;
+        const uint32_t par = (issued_par >> s2) & 1u;
+        const uint64_t t0 = ptx::globaltimer();
+        while (!ptx::mbar_try_wait(full_bar(s2), par)) {
+          if ((long long)(ptx::globaltimer() - t0) > p.timeout_ns) {
+            atomicOr(p.status, DMU_FLAG_TIMEOUT);
+            break;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      bool issued = false;
+      for (int t = blockIdx.x; ok && t < p.total_tiles; t += gridDim.x) {
+        const TileCoord tc = decode_tile(p, t);
+        const GemmProblem& pr = p.prob[tc.pi];
+        const int nk = (pr.K + BK - 1) / BK;
+        const uint32_t idesc = ptx::make_idesc_bf16(BM, BN, pr.a_mn, pr.b_mn);
+        if (!wait_bar(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        const uint32_t a_lbo = pr.a_mn ? 8192u : 16u, a_sbo = 1024u;
+        const uint32_t b_lbo = pr.b_mn ? 8192u : 16u, b_sbo = 1024u;
+        const uint32_t a_kstep = pr.a_mn ? 2048u : 32u;
+        const uint32_t b_kstep = pr.b_mn ? 2048u : 32u;
+        uint32_t accumulate = 0;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!wait_bar(full_bar(stage), phase, abort_flag, p)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t sa = ring + stage * Cfg::STAGE_BYTES;
+          const uint32_t sb = sa + NA * A_PART_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+#pragma unroll
+            for (int term = 0; term < 3; ++term) {
+              const int bit = 1 << term;
+              if (!(pr.terms & bit)) continue;
+              if (term == 1 && NB < 2) continue;
+              if (term == 2 && NA < 2) continue;
+              const uint32_t pa = sa + (term == 2 ? A_PART_BYTES : 0);
+              const uint32_t pb = sb + (term == 1 ? B_PART_BYTES : 0);
+              const uint64_t ad = ptx::make_sw128_desc(pa + kk * a_kstep, a_lbo, a_sbo);
+              const uint64_t bd = ptx::make_sw128_desc(pb + kk * b_kstep, b_lbo, b_sbo);
+              ptx::mma_bf16(d_tmem, ad, bd, idesc, accumulate);
+              accumulate = 1;
+              issued = true;
+            }
+          }
+          ptx::mma_commit(empty_bar(stage));
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        ptx::mma_commit(tfull_bar(acc));
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      if (!ok && issued) {
+        // wind down: wait (bounded) for the MMAs already issued
+        ptx::mma_commit(drain_bar);
+        const uint64_t t0 = ptx::globaltimer();
+        while (!ptx::mbar_try_wait(drain_bar, 0)) {
+          if ((long long)(ptx::globaltimer() - t0) > p.timeout_ns) break;
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
+      const TileCoord tc = decode_tile(p, t);
+      const GemmProblem& pr = p.prob[tc.pi];
+      int ok = 1;
+      if (lane == 0) ok = wait_bar(tfull_bar(acc), acc_phase, abort_flag, p) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      ptx::tc_fence_after();
+      const int row_lo = tc.bi * BM + q * 32;
+      const int i = row_lo + lane;
+      for (int ch = 0; ch < BN / 32; ++ch) {
+        const int col0 = tc.bj * BN + ch * 32;
+        if (col0 >= pr.N) break;
+        if (pr.sym && col0 + 31 < row_lo) continue;  // chunk strictly below the diagonal
+        if (row_lo >= pr.M) break;
+        uint32_t r[32];
+        ptx::tmem_ld32(tmem_base + (uint32_t)(acc * BN + ch * 32) + ((uint32_t)(q * 32) << 16), r);
+        ptx::tmem_wait_ld();
+        if (pr.epi == EPI_GRAM)
+          epi_gram_chunk(pr, tc.mat, i, col0, r);
+        else
+          epi_update_chunk(pr, tc.mat, i, col0, r);
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(tempty_bar(acc));
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// Bounded-wait self-test: one thread waits on an mbarrier that nothing
+// arrives on; the wait gives up after timeout_ns and sets DMU_FLAG_TIMEOUT.
+__global__ void k_wait_selftest(unsigned int* status, long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(ptx::smem_u32(&bar), 1);
+    abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint64_t t0 = ptx::globaltimer();
+    uint32_t n = 0;
+    for (;;) {
+      if (ptx::mbar_try_wait(ptx::smem_u32(&bar), 0)) break;
+      if ((++n & 63u) == 0 && (long long)(ptx::globaltimer() - t0) > timeout_ns) {
+        atomicOr(status, DMU_FLAG_TIMEOUT);
+        break;
+      }
+    }
+  }
+}
+
+cudaError_t launch_wait_selftest(unsigned int* status, long long timeout_ns, cudaStream_t s) {
+  k_wait_selftest<<<1, 32, 0, s>>>(status, timeout_ns);
+  return cudaGetLastError();
+}
+
+template <int NA, int NB>
+static cudaError_t configure_one() {
+  return cudaFuncSetAttribute(k_gemm_tc<NA, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              TcCfg<NA, NB>::SMEM_BYTES);
+}
+
+cudaError_t gemm_tc_configure() {
+  cudaError_t e;
+  if ((e = configure_one<1, 1>()) != cudaSuccess) return e;
+  if ((e = configure_one<2, 1>()) != cudaSuccess) return e;
+  if ((e = configure_one<2, 2>()) != cudaSuccess) return e;
+  return cudaSuccess;
+}
+
+int gemm_tc_stages(int na, int nb) {
+  if (na == 1 && nb == 1) return TcCfg<1, 1>::STAGES;
+  if (na == 2 && nb == 1) return TcCfg<2, 1>::STAGES;
+  if (na == 2 && nb == 2) return TcCfg<2, 2>::STAGES;
+  return 0;
+}
+
+template <int NA, int NB>
+static cudaError_t launch_one(const GemmParams& p, int num_sms, cudaStream_t s) {
+  const int grid = p.total_tiles < num_sms ? p.total_tiles : num_sms;
+  if (grid <= 0) return cudaSuccess;
+  k_gemm_tc<NA, NB><<<grid, GEMM_THREADS, TcCfg<NA, NB>::SMEM_BYTES, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_tc(const GemmParams& p, int na, int nb, int num_sms, cudaStream_t s) {
+  if (na == 1 && nb == 1) return launch_one<1, 1>(p, num_sms, s);
+  if (na == 2 && nb == 1) return launch_one<2, 1>(p, num_sms, s);
+  if (na == 2 && nb == 2) return launch_one<2, 2>(p, num_sms, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace dmu

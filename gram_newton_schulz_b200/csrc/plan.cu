@@ -1,0 +1,940 @@
+// Planner and C ABI of libdmu (see include/dmu.h for the contract).
+//
+// The planner groups matrices into shape buckets (equal rows, cols) and
+// Gram classes (equal m = min(rows, cols)); the batched recursion then runs
+// one grouped launch per product over all matrices of all classes that
+// share a precision (DMuon page, section 2.2: batching of similar-shape
+// matrices so the Gram recursion runs jointly and dispatch is amortised).
+// Tall matrices are transposed logically: their Gram matrix is Mb^T Mb
+// read through an MN-major tensor map, and their update is written into W
+// transposed; nothing is copied.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstring>
+#include <map>
+#include <string>
+#include <utility>
+#include <vector>
+
+#include "dmu_internal.h"
+
+using namespace dmu;
+
+namespace {
+
+thread_local std::string g_err;
+
+dmu_status fail(dmu_status s, const std::string& msg) {
+  g_err = msg;
+  return s;
+}
+
+#define CUDA_TRY(x)                                                                   \
+  do {                                                                                \
+    cudaError_t e_ = (x);                                                             \
+    if (e_ != cudaSuccess) return fail(DMU_ERR_CUDA, std::string(#x) + ": " + cudaGetErrorString(e_)); \
+  } while (0)
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+int64_t round_up64(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+struct Bucket {
+  int64_t rows = 0, cols = 0, m = 0, n = 0;
+  bool tall = false;
+  int count = 0;
+  std::vector<int> mats;  // plan indices, in slot order
+  int first_slot = 0;
+  int cls = 0, cls_off = 0;
+  int64_t ldc = 0;
+  int64_t mb_off = 0;  // element offset of the bucket's first image
+  int map_k = -1, map_mn = -1;
+};
+
+struct GClass {
+  int64_t m = 0, ldg = 0;
+  int count = 0;
+  size_t off = 0;  // byte offset in the workspace
+  int prec = DMU_PREC_FAST;
+  int map = -1;
+};
+
+enum { TBL_GRADS = 0, TBL_MOMS, TBL_W, TBL_O, TBL_IN, NUM_TBL };
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+struct DevGuard {
+  int prev = -1;
+  explicit DevGuard(int d) {
+    if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+    if (prev != d) cudaSetDevice(d);
+  }
+  ~DevGuard() {
+    int cur = -1;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+}  // namespace
+
+struct dmu_plan_s {
+  int device = 0, num_sms = 0;
+  bool has_device = false;
+  dmu_dtype dtype = DMU_BF16;
+  dmu_prec prec = DMU_PREC_AUTO;
+  int count = 0;
+  std::vector<dmu_shape> shapes;
+  std::vector<Bucket> buckets;
+  std::vector<GClass> classes;
+  std::vector<int> slot_of;
+  std::vector<MomChunk> chunks;
+  std::vector<MomMat> mats;
+  bool vec_shapes = true;
+  size_t esize = 2;
+  // workspace layout (bytes)
+  size_t off_status = 0, off_inv = 0, off_partial = 0, off_chunks = 0, off_mats = 0, off_tbl = 0,
+         off_mb = 0, off_gram = 0, total = 0;
+  char* ws = nullptr;
+  size_t ws_bytes = 0;
+  std::vector<CUtensorMap> maps;
+  std::vector<const void*> tbl_cache[NUM_TBL];
+  bool tbl_valid[NUM_TBL] = {};
+  void* pinned[NUM_TBL] = {};
+  cudaEvent_t tbl_ev[NUM_TBL] = {};
+  bool have_mb = false, have_p = false;
+  int p_final = 0;  // 0: P buffer A, 1: P buffer B
+  float eps = 1e-7f;
+  int launches = 0;
+  long long timeout_ns = 2000000000LL;
+
+  unsigned int* status_dev() const { return reinterpret_cast<unsigned int*>(ws + off_status); }
+  float* inv_dev() const { return reinterpret_cast<float*>(ws + off_inv); }
+  float* partial_dev() const { return reinterpret_cast<float*>(ws + off_partial); }
+  const MomChunk* chunks_dev() const { return reinterpret_cast<const MomChunk*>(ws + off_chunks); }
+  const MomMat* mats_dev() const { return reinterpret_cast<const MomMat*>(ws + off_mats); }
+  void** tbl_dev(int t) const { return reinterpret_cast<void**>(ws + off_tbl) + (size_t)t * count; }
+  char* mb_dev() const { return ws + off_mb; }
+  // bf16 Gram slot of class c (first matrix of the class)
+  __nv_bfloat16* slot_bf16(int c, int slot) const {
+    const GClass& g = classes[c];
+    return reinterpret_cast<__nv_bfloat16*>(ws + g.off) + (size_t)slot * g.count * g.m * g.ldg;
+  }
+  float* slot_f32(int c, int slot) const {
+    const GClass& g = classes[c];
+    return reinterpret_cast<float*>(ws + g.off) + (size_t)slot * g.count * g.m * g.ldg;
+  }
+};
+
+namespace {
+
+dmu_status check_plan(dmu_plan p, bool need_ws) {
+  if (!p) return fail(DMU_ERR_INVALID_ARG, "plan is NULL");
+  if (need_ws && !p->ws) return fail(DMU_ERR_WORKSPACE, "no workspace set (dmu_set_workspace)");
+  if (need_ws && !p->has_device) return fail(DMU_ERR_CUDA, "no CUDA device");
+  return DMU_OK;
+}
+
+dmu_status upload_table(dmu_plan p, int t, const void* const* ptrs, cudaStream_t s, bool allow_null = false) {
+  std::vector<const void*> v(p->count);
+  for (int i = 0; i < p->count; ++i) {
+    if (!ptrs[i] && !allow_null)
+      return fail(DMU_ERR_INVALID_ARG, "null device pointer in table, matrix " + std::to_string(i));
+    v[p->slot_of[i]] = ptrs[i];
+  }
+  if (p->tbl_valid[t] && v == p->tbl_cache[t]) return DMU_OK;
+  const size_t bytes = sizeof(void*) * (size_t)p->count;
+  if (!p->pinned[t]) {
+    CUDA_TRY(cudaMallocHost(&p->pinned[t], bytes));
+    CUDA_TRY(cudaEventCreateWithFlags(&p->tbl_ev[t], cudaEventDisableTiming));
+  } else {
+    CUDA_TRY(cudaEventSynchronize(p->tbl_ev[t]));  // previous upload has left the staging buffer
+  }
+  std::memcpy(p->pinned[t], v.data(), bytes);
+  CUDA_TRY(cudaMemcpyAsync(p->tbl_dev(t), p->pinned[t], bytes, cudaMemcpyHostToDevice, s));
+  CUDA_TRY(cudaEventRecord(p->tbl_ev[t], s));
+  p->tbl_cache[t] = std::move(v);
+  p->tbl_valid[t] = true;
+  return DMU_OK;
+}
+
+bool aligned16(const void* const* ptrs, int n) {
+  for (int i = 0; i < n; ++i)
+    if (reinterpret_cast<uintptr_t>(ptrs[i]) & 15) return false;
+  return true;
+}
+
+int tiles_for(int M, int N, bool sym, int* tm, int* tn) {
+  *tm = (M + BM - 1) / BM;
+  *tn = (N + BN - 1) / BN;
+  if (!sym) return (*tm) * (*tn);
+  int t = 0;
+  for (int bj = 0; bj < *tn; ++bj) {
+    int c = ((bj + 1) * BN - 1) / BM + 1;
+    t += c < *tm ? c : *tm;
+  }
+  return t;
+}
+
+// ---------------------------------------------------------------- tc launches
+struct Prob {
+  GemmProblem g;
+  int amap, bmap;  // plan map indices
+};
+
+dmu_status run_tc(dmu_plan p, std::vector<Prob>& probs, int na, int nb, cudaStream_t s) {
+  size_t i = 0;
+  while (i < probs.size()) {
+    GemmParams gp;
+    std::memset(&gp, 0, sizeof(gp));
+    std::vector<int> used;
+    int nprob = 0, tiles = 0;
+    while (i < probs.size() && nprob < MAX_PROBS) {
+      int need = 0;
+      bool fa = false, fb = false;
+      for (int u : used) {
+        fa |= (u == probs[i].amap);
+        fb |= (u == probs[i].bmap);
+      }
+      need = (fa ? 0 : 1) + (fb || probs[i].bmap == probs[i].amap ? 0 : 1);
+      if ((int)used.size() + need > MAX_MAPS) break;
+      auto slot = [&](int pm) {
+        for (size_t k = 0; k < used.size(); ++k)
+          if (used[k] == pm) return (int)k;
+        used.push_back(pm);
+        return (int)used.size() - 1;
+      };
+      GemmProblem g = probs[i].g;
+      g.a_map = slot(probs[i].amap);
+      g.b_map = slot(probs[i].bmap);
+      g.tile_begin = tiles;
+      tiles += g.count * g.tiles_per_mat;
+      gp.prob[nprob++] = g;
+      ++i;
+    }
+    for (size_t k = 0; k < used.size(); ++k) gp.maps[k] = p->maps[used[k]];
+    gp.nprob = nprob;
+    gp.total_tiles = tiles;
+    gp.status = p->status_dev();
+    gp.timeout_ns = p->timeout_ns;
+    CUDA_TRY(launch_gemm_tc(gp, na, nb, p->num_sms, s));
+    p->launches++;
+  }
+  return DMU_OK;
+}
+
+void prec_shape(int prec, int* na, int* nb, int* terms) {
+  switch (prec) {
+    case DMU_PREC_SPLIT2: *na = 2; *nb = 1; *terms = TERM_HH | TERM_LH; break;
+    case DMU_PREC_SPLIT3: *na = 2; *nb = 2; *terms = TERM_HH | TERM_HL | TERM_LH; break;
+    default: *na = 1; *nb = 1; *terms = TERM_HH; break;
+  }
+}
+
+// A Gram-space product over all matrices of class c:
+//   out = alpha * (A B) + beta * Cin + gamma * I   [, out2 = out + gamma2 * I]
+Prob gram_prob(dmu_plan p, int c, int a_slot, int b_slot, int terms, float alpha, float beta,
+               int cin_slot, int out_slot, bool out_lo, int out2_slot, float gamma2) {
+  const GClass& gc = p->classes[c];
+  Prob pr;
+  std::memset(&pr, 0, sizeof(pr));
+  GemmProblem& g = pr.g;
+  g.count = gc.count;
+  g.M = g.N = g.K = (int)gc.m;
+  g.sym = 1;
+  g.tiles_per_mat = tiles_for(g.M, g.N, true, &g.tiles_m, &g.tiles_n);
+  g.a_mn = g.b_mn = 0;
+  g.a_z[0] = a_slot * gc.count;
+  g.a_z[1] = (a_slot + 1) * gc.count;
+  g.b_z[0] = b_slot * gc.count;
+  g.b_z[1] = (b_slot + 1) * gc.count;
+  g.terms = terms;
+  g.epi = EPI_GRAM;
+  g.alpha_mode = ALPHA_CONST;
+  g.alpha = alpha;
+  g.beta = beta;
+  g.gamma = 0.f;
+  g.gamma2 = gamma2;
+  if (cin_slot >= 0) {
+    g.cin_hi = p->slot_bf16(c, cin_slot);
+    g.cin_lo = p->slot_bf16(c, cin_slot + 1);
+  }
+  g.out_hi = p->slot_bf16(c, out_slot);
+  g.out_lo = out_lo ? p->slot_bf16(c, out_slot + 1) : nullptr;
+  if (out2_slot >= 0) {
+    g.out2_hi = p->slot_bf16(c, out2_slot);
+    g.out2_lo = p->slot_bf16(c, out2_slot + 1);
+  }
+  g.ld = gc.ldg;
+  g.mat_stride = gc.m * gc.ldg;
+  pr.amap = pr.bmap = gc.map;
+  return pr;
+}
+
+enum Product { PROD_R, PROD_T, PROD_P, PROD_G };
+
+// Operands and epilogue of one product of step k for class c (R-form):
+//   R = bG + c(GG),  T = aG + RG,  P' = aP + RP (P0 = aI + R),  G' = aT + TR
+Prob product(dmu_plan p, int c, Product what, int k, const float co[3], int p_in, int p_out) {
+  const GClass& gc = p->classes[c];
+  int na, nb, terms;
+  prec_shape(gc.prec, &na, &nb, &terms);
+  const bool r_lo = gc.prec != DMU_PREC_FAST;
+  const int PA = SLOT_PA_HI, PB = SLOT_PB_HI;
+  const int pin = p_in == 0 ? PA : PB, pout = p_out == 0 ? PA : PB;
+  switch (what) {
+    case PROD_R:
+      return gram_prob(p, c, SLOT_G_HI, SLOT_G_HI, terms, co[2], co[1], SLOT_G_HI, SLOT_R_HI, r_lo,
+                       k == 0 ? PA : -1, co[0]);
+    case PROD_T:
+      return gram_prob(p, c, SLOT_R_HI, SLOT_G_HI, terms, 1.f, co[0], SLOT_G_HI, SLOT_T_HI, true, -1, 0.f);
+    case PROD_P:
+      if (gc.prec == DMU_PREC_SPLIT2)
+        return gram_prob(p, c, pin, SLOT_R_HI, terms, 1.f, co[0], pin, pout, true, -1, 0.f);
+      return gram_prob(p, c, SLOT_R_HI, pin, terms, 1.f, co[0], pin, pout, true, -1, 0.f);
+    case PROD_G:
+    default:
+      return gram_prob(p, c, SLOT_T_HI, SLOT_R_HI, terms, 1.f, co[0], SLOT_T_HI, SLOT_G_HI, true, -1, 0.f);
+  }
+}
+
+// Run one or two kinds of product for every class, one grouped launch per
+// precision group.
+dmu_status run_products(dmu_plan p, const std::vector<std::pair<Product, bool>>& kinds, int k,
+                        const float co[3], int p_in, int p_out, cudaStream_t s) {
+  const int precs[3] = {DMU_PREC_FAST, DMU_PREC_SPLIT2, DMU_PREC_SPLIT3};
+  for (int pr : precs) {
+    std::vector<Prob> probs;
+    for (size_t c = 0; c < p->classes.size(); ++c) {
+      if (p->classes[c].prec != pr) continue;
+      for (auto& kd : kinds)
+        if (kd.second) probs.push_back(product(p, (int)c, kd.first, k, co, p_in, p_out));
+    }
+    if (probs.empty()) continue;
+    int na, nb, terms;
+    prec_shape(pr, &na, &nb, &terms);
+    dmu_status st = run_tc(p, probs, na, nb, s);
+    if (st != DMU_OK) return st;
+  }
+  return DMU_OK;
+}
+
+dmu_status gram_bf16(dmu_plan p, const float co[3], int steps, cudaStream_t s) {
+  // G0 = s^2 X X^T, one problem per shape bucket (SYRK, upper tiles only)
+  std::vector<Prob> syrk;
+  for (const Bucket& b : p->buckets) {
+    const GClass& gc = p->classes[b.cls];
+    Prob pr;
+    std::memset(&pr, 0, sizeof(pr));
+    GemmProblem& g = pr.g;
+    g.count = b.count;
+    g.M = g.N = (int)b.m;
+    g.K = (int)b.n;
+    g.sym = 1;
+    g.tiles_per_mat = tiles_for(g.M, g.N, true, &g.tiles_m, &g.tiles_n);
+    g.a_mn = g.b_mn = b.tall ? 1 : 0;
+    g.terms = TERM_HH;
+    g.epi = EPI_GRAM;
+    g.alpha_mode = ALPHA_INV2;
+    g.alpha = 1.f;
+    g.inv = p->inv_dev();
+    g.inv_base = b.first_slot;
+    const size_t moff = (size_t)b.cls_off * gc.m * gc.ldg;
+    g.out_hi = p->slot_bf16(b.cls, SLOT_G_HI) + moff;
+    g.out_lo = p->slot_bf16(b.cls, SLOT_G_LO) + moff;
+    g.ld = gc.ldg;
+    g.mat_stride = gc.m * gc.ldg;
+    pr.amap = pr.bmap = b.tall ? b.map_mn : b.map_k;
+    syrk.push_back(pr);
+  }
+  dmu_status st = run_tc(p, syrk, 1, 1, s);
+  if (st != DMU_OK) return st;
+
+  if (steps == 0) {
+    for (size_t c = 0; c < p->classes.size(); ++c) {
+      const GClass& gc = p->classes[c];
+      CUDA_TRY(launch_identity_bf16(p->slot_bf16((int)c, SLOT_PA_HI), p->slot_bf16((int)c, SLOT_PA_LO),
+                                    gc.count, (int)gc.m, gc.ldg, gc.m * gc.ldg, s));
+      p->launches++;
+    }
+    p->p_final = 0;
+    return DMU_OK;
+  }
+  int p_cur = 0;  // P_k lives in buffer p_cur (after step 0: buffer A)
+  for (int k = 0; k < steps; ++k) {
+    const bool last = (k == steps - 1);
+    st = run_products(p, {{PROD_R, true}}, k, co, 0, 0, s);
+    if (st != DMU_OK) return st;
+    const int p_next = (k == 0) ? 0 : 1 - p_cur;
+    st = run_products(p, {{PROD_T, !last}, {PROD_P, k >= 1}}, k, co, p_cur, p_next, s);
+    if (st != DMU_OK) return st;
+    p_cur = p_next;
+    if (!last) {
+      st = run_products(p, {{PROD_G, true}}, k, co, 0, 0, s);
+      if (st != DMU_OK) return st;
+    }
+  }
+  p->p_final = p_cur;
+  return DMU_OK;
+}
+
+// ---------------------------------------------------------------- fp32 path
+SimtProblem simt_gram(dmu_plan p, int c, int a_slot, int b_slot, float alpha, float beta, int cin_slot,
+                      int out_slot, int out2_slot, float gamma2) {
+  const GClass& gc = p->classes[c];
+  SimtProblem q;
+  std::memset(&q, 0, sizeof(q));
+  q.count = gc.count;
+  q.M = q.N = q.K = (int)gc.m;
+  q.sym = 1;
+  q.a = p->slot_f32(c, a_slot);
+  q.a_ms = gc.m * gc.ldg;
+  q.a_si = gc.ldg;
+  q.a_sk = 1;
+  q.b = p->slot_f32(c, b_slot);
+  q.b_ms = gc.m * gc.ldg;
+  q.b_si = gc.ldg;
+  q.b_sk = 1;
+  q.epi = EPI_GRAM;
+  q.alpha_mode = ALPHA_CONST;
+  q.alpha = alpha;
+  q.beta = beta;
+  q.gamma2 = gamma2;
+  q.cin = cin_slot >= 0 ? p->slot_f32(c, cin_slot) : nullptr;
+  q.out = p->slot_f32(c, out_slot);
+  q.out2 = out2_slot >= 0 ? p->slot_f32(c, out2_slot) : nullptr;
+  q.ld = gc.ldg;
+  q.mat_stride = gc.m * gc.ldg;
+  return q;
+}
+
+dmu_status gram_f32(dmu_plan p, const float co[3], int steps, cudaStream_t s) {
+  for (const Bucket& b : p->buckets) {
+    const GClass& gc = p->classes[b.cls];
+    SimtProblem q;
+    std::memset(&q, 0, sizeof(q));
+    q.count = b.count;
+    q.M = q.N = (int)b.m;
+    q.K = (int)b.n;
+    q.sym = 1;
+    q.a = reinterpret_cast<const float*>(p->mb_dev()) + b.mb_off;
+    q.a_ms = b.rows * b.ldc;
+    q.a_si = b.tall ? 1 : b.ldc;
+    q.a_sk = b.tall ? b.ldc : 1;
+    q.b = q.a;
+    q.b_ms = q.a_ms;
+    q.b_si = q.a_si;
+    q.b_sk = q.a_sk;
+    q.epi = EPI_GRAM;
+    q.alpha_mode = ALPHA_INV2;
+    q.alpha = 1.f;
+    q.inv = p->inv_dev();
+    q.inv_base = b.first_slot;
+    q.out = p->slot_f32(b.cls, FSLOT_G) + (size_t)b.cls_off * gc.m * gc.ldg;
+    q.ld = gc.ldg;
+    q.mat_stride = gc.m * gc.ldg;
+    CUDA_TRY(launch_simt_gemm(q, s));
+    p->launches++;
+  }
+  if (steps == 0) {
+    for (size_t c = 0; c < p->classes.size(); ++c) {
+      const GClass& gc = p->classes[c];
+      CUDA_TRY(launch_identity_f32(p->slot_f32((int)c, FSLOT_PA), gc.count, (int)gc.m, gc.ldg,
+                                   gc.m * gc.ldg, s));
+      p->launches++;
+    }
+    p->p_final = 0;
+    return DMU_OK;
+  }
+  int p_cur = 0;
+  for (int k = 0; k < steps; ++k) {
+    const bool last = (k == steps - 1);
+    const int p_next = (k == 0) ? 0 : 1 - p_cur;
+    const int pin = p_cur == 0 ? FSLOT_PA : FSLOT_PB, pout = p_next == 0 ? FSLOT_PA : FSLOT_PB;
+    for (size_t c = 0; c < p->classes.size(); ++c) {
+      const int ci = (int)c;
+      std::vector<SimtProblem> qs;
+      qs.push_back(simt_gram(p, ci, FSLOT_G, FSLOT_G, co[2], co[1], FSLOT_G, FSLOT_R, k == 0 ? FSLOT_PA : -1, co[0]));
+      if (!last) qs.push_back(simt_gram(p, ci, FSLOT_R, FSLOT_G, 1.f, co[0], FSLOT_G, FSLOT_T, -1, 0.f));
+      if (k >= 1) qs.push_back(simt_gram(p, ci, FSLOT_R, pin, 1.f, co[0], pin, pout, -1, 0.f));
+      if (!last) qs.push_back(simt_gram(p, ci, FSLOT_T, FSLOT_R, 1.f, co[0], FSLOT_T, FSLOT_G, -1, 0.f));
+      for (auto& q : qs) {
+        CUDA_TRY(launch_simt_gemm(q, s));
+        p->launches++;
+      }
+    }
+    p_cur = p_next;
+  }
+  p->p_final = p_cur;
+  return DMU_OK;
+}
+
+dmu_status run_normalize(dmu_plan p, int tbl, bool with_mom, float beta, float eps, bool vec, cudaStream_t s) {
+  const bool f32 = p->dtype == DMU_F32;
+  CUDA_TRY(launch_momentum(p->chunks_dev(), (int)p->chunks.size(), p->mats_dev(),
+                           const_cast<const void* const*>(p->tbl_dev(tbl)),
+                           with_mom ? reinterpret_cast<float* const*>(p->tbl_dev(TBL_MOMS)) : nullptr,
+                           f32 ? 1 : 0, p->mb_dev(), f32 ? 1 : 0, beta, p->partial_dev(), vec ? 1 : 0,
+                           p->num_sms, s));
+  CUDA_TRY(launch_norm_finalize(p->mats_dev(), p->count, p->partial_dev(), eps, p->inv_dev(),
+                                p->status_dev(), s));
+  p->launches += 2;
+  p->eps = eps;
+  p->have_mb = true;
+  p->have_p = false;
+  return DMU_OK;
+}
+
+dmu_status encode_map(CUtensorMap* map, void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+                      uint64_t s2, uint32_t box0, uint32_t box1) {
+  auto enc = get_encode();
+  if (!enc) return fail(DMU_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1, s2};
+  cuuint32_t box[3] = {box0, box1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DMU_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
+  return DMU_OK;
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+extern "C" {
+
+int dmu_version(void) { return DMU_VERSION; }
+
+const char* dmu_last_error(void) { return g_err.c_str(); }
+
+dmu_status dmu_plan_create(const dmu_shape* shapes, int count, dmu_dtype dtype, dmu_prec prec, int device,
+                           dmu_plan* out) {
+  g_err.clear();
+  if (!out) return fail(DMU_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (!shapes) return fail(DMU_ERR_INVALID_ARG, "shapes is NULL");
+  if (count <= 0) return fail(DMU_ERR_INVALID_ARG, "count must be positive");
+  if (dtype != DMU_BF16 && dtype != DMU_F32) return fail(DMU_ERR_INVALID_ARG, "unknown dtype");
+  if (prec < DMU_PREC_AUTO || prec > DMU_PREC_SPLIT3) return fail(DMU_ERR_INVALID_ARG, "unknown precision");
+  for (int i = 0; i < count; ++i) {
+    if (shapes[i].rows <= 0 || shapes[i].cols <= 0)
+      return fail(DMU_ERR_INVALID_ARG, "non-positive extent at matrix " + std::to_string(i));
+    if (shapes[i].rows > (1 << 20) || shapes[i].cols > (1 << 20) ||
+        std::min(shapes[i].rows, shapes[i].cols) > 65536)
+      return fail(DMU_ERR_UNSUPPORTED, "extent too large at matrix " + std::to_string(i));
+  }
+  dmu_plan p = new dmu_plan_s();
+  p->device = device;
+  p->dtype = dtype;
+  p->prec = prec;
+  p->count = count;
+  p->shapes.assign(shapes, shapes + count);
+  p->esize = dtype == DMU_BF16 ? 2 : 4;
+
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) == cudaSuccess && ndev > 0) {
+    if (device < 0 || device >= ndev) {
+      delete p;
+      return fail(DMU_ERR_INVALID_ARG, "device index out of range");
+    }
+    int major = 0, minor = 0, sms = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, device);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
+    if (dtype == DMU_BF16 && !(major == 10 && minor == 0)) {
+      delete p;
+      return fail(DMU_ERR_UNSUPPORTED, "the bf16 path is built for sm_100a (compute capability 10.0)");
+    }
+    p->has_device = true;
+    p->num_sms = sms;
+  } else {
+    cudaGetLastError();  // clear "no device"
+  }
+
+  // buckets (equal rows, cols) in order of first appearance; classes (equal m)
+  std::map<std::pair<int64_t, int64_t>, int> bidx;
+  std::map<int64_t, int> cidx;
+  for (int i = 0; i < count; ++i) {
+    auto key = std::make_pair(shapes[i].rows, shapes[i].cols);
+    auto it = bidx.find(key);
+    if (it == bidx.end()) {
+      Bucket b;
+      b.rows = shapes[i].rows;
+      b.cols = shapes[i].cols;
+      b.tall = b.rows > b.cols;
+      b.m = std::min(b.rows, b.cols);
+      b.n = std::max(b.rows, b.cols);
+      auto ci = cidx.find(b.m);
+      if (ci == cidx.end()) {
+        GClass g;
+        g.m = b.m;
+        g.ldg = dtype == DMU_BF16 ? round_up64(b.m, 8) : b.m;
+        if (dtype == DMU_BF16) {
+          if (prec == DMU_PREC_AUTO)
+            g.prec = b.m >= 1024 ? DMU_PREC_FAST : DMU_PREC_SPLIT3;
+          else
+            g.prec = prec;
+        }
+        cidx[b.m] = (int)p->classes.size();
+        p->classes.push_back(g);
+      }
+      b.cls = cidx[b.m];
+      bidx[key] = (int)p->buckets.size();
+      p->buckets.push_back(b);
+      it = bidx.find(key);
+    }
+    p->buckets[it->second].mats.push_back(i);
+  }
+  p->slot_of.assign(count, 0);
+  int slot = 0;
+  int64_t mb_elems = 0;
+  for (Bucket& b : p->buckets) {
+    b.count = (int)b.mats.size();
+    b.first_slot = slot;
+    for (int k = 0; k < b.count; ++k) p->slot_of[b.mats[k]] = slot + k;
+    slot += b.count;
+    GClass& g = p->classes[b.cls];
+    b.cls_off = g.count;
+    g.count += b.count;
+    b.ldc = dtype == DMU_BF16 ? round_up64(b.cols, 8) : b.cols;
+    if (b.cols % 8) p->vec_shapes = false;
+    b.mb_off = mb_elems;
+    mb_elems += round_up64((int64_t)b.count * b.rows * b.ldc, 128);
+  }
+  // momentum chunks and per-slot geometry
+  p->mats.resize(count);
+  for (const Bucket& b : p->buckets) {
+    for (int k = 0; k < b.count; ++k) {
+      MomMat mm;
+      mm.rows = b.rows;
+      mm.cols = b.cols;
+      mm.ldc = b.ldc;
+      mm.mb_off = b.mb_off + (int64_t)k * b.rows * b.ldc;
+      mm.chunk_begin = (int)p->chunks.size();
+      const int64_t total = b.rows * b.cols;
+      for (int64_t st = 0; st < total; st += MOM_CHUNK) {
+        MomChunk ch;
+        ch.start = st;
+        ch.slot = b.first_slot + k;
+        ch.len = (int)std::min<int64_t>(MOM_CHUNK, total - st);
+        p->chunks.push_back(ch);
+      }
+      mm.chunk_end = (int)p->chunks.size();
+      p->mats[b.first_slot + k] = mm;
+    }
+  }
+  // workspace layout
+  size_t off = 0;
+  p->off_status = off;
+  off = align_up(off + 16, 256);
+  p->off_inv = off;
+  off = align_up(off + sizeof(float) * count, 256);
+  p->off_partial = off;
+  off = align_up(off + sizeof(float) * p->chunks.size(), 256);
+  p->off_chunks = off;
+  off = align_up(off + sizeof(MomChunk) * p->chunks.size(), 256);
+  p->off_mats = off;
+  off = align_up(off + sizeof(MomMat) * count, 256);
+  p->off_tbl = off;
+  off = align_up(off + sizeof(void*) * NUM_TBL * (size_t)count, 256);
+  p->off_mb = off;
+  off = align_up(off + p->esize * (size_t)mb_elems, 1024);
+  p->off_gram = off;
+  const int nslots = dtype == DMU_BF16 ? NUM_SLOTS : NUM_FSLOTS;
+  for (GClass& g : p->classes) {
+    g.off = off;
+    off = align_up(off + p->esize * (size_t)nslots * g.count * g.m * g.ldg, 1024);
+  }
+  p->total = off;
+  *out = p;
+  return DMU_OK;
+}
+
+size_t dmu_workspace_bytes(dmu_plan plan) { return plan ? plan->total : 0; }
+
+dmu_status dmu_set_workspace(dmu_plan p, void* dev_ptr, size_t bytes) {
+  g_err.clear();
+  dmu_status st = check_plan(p, false);
+  if (st != DMU_OK) return st;
+  if (!p->has_device) return fail(DMU_ERR_CUDA, "no CUDA device");
+  if (!dev_ptr) return fail(DMU_ERR_WORKSPACE, "workspace pointer is NULL");
+  if (reinterpret_cast<uintptr_t>(dev_ptr) & 255) return fail(DMU_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (bytes < p->total)
+    return fail(DMU_ERR_WORKSPACE, "workspace too small: " + std::to_string(bytes) + " < " + std::to_string(p->total));
+  DevGuard dg(p->device);
+  p->ws = reinterpret_cast<char*>(dev_ptr);
+  p->ws_bytes = bytes;
+  for (int t = 0; t < NUM_TBL; ++t) p->tbl_valid[t] = false;
+  p->have_mb = p->have_p = false;
+  CUDA_TRY(cudaMemset(p->ws + p->off_status, 0, 16));
+  CUDA_TRY(cudaMemcpy(p->ws + p->off_chunks, p->chunks.data(), sizeof(MomChunk) * p->chunks.size(),
+                      cudaMemcpyHostToDevice));
+  CUDA_TRY(cudaMemcpy(p->ws + p->off_mats, p->mats.data(), sizeof(MomMat) * p->mats.size(),
+                      cudaMemcpyHostToDevice));
+  p->maps.clear();
+  if (p->dtype == DMU_BF16) {
+    CUDA_TRY(gemm_tc_configure());
+    for (Bucket& b : p->buckets) {
+      CUtensorMap mk, mn;
+      void* base = p->mb_dev() + 2 * (size_t)b.mb_off;
+      const uint64_t s1 = (uint64_t)b.ldc * 2, s2 = (uint64_t)b.rows * b.ldc * 2;
+      st = encode_map(&mk, base, (uint64_t)b.cols, (uint64_t)b.rows, (uint64_t)b.count, s1, s2, 64, 128);
+      if (st != DMU_OK) return st;
+      st = encode_map(&mn, base, (uint64_t)b.cols, (uint64_t)b.rows, (uint64_t)b.count, s1, s2, 64, 64);
+      if (st != DMU_OK) return st;
+      b.map_k = (int)p->maps.size();
+      p->maps.push_back(mk);
+      b.map_mn = (int)p->maps.size();
+      p->maps.push_back(mn);
+    }
+    for (GClass& g : p->classes) {
+      CUtensorMap mg;
+      const uint64_t s1 = (uint64_t)g.ldg * 2, s2 = (uint64_t)g.m * g.ldg * 2;
+      st = encode_map(&mg, p->ws + g.off, (uint64_t)g.m, (uint64_t)g.m, (uint64_t)NUM_SLOTS * g.count, s1, s2,
+                      64, 128);
+      if (st != DMU_OK) return st;
+      g.map = (int)p->maps.size();
+      p->maps.push_back(mg);
+    }
+  }
+  return DMU_OK;
+}
+
+dmu_status dmu_momentum_normalize(dmu_plan p, const void* const* grads, float* const* momenta, float beta,
+                                  float eps, void* stream) {
+  g_err.clear();
+  dmu_status st = check_plan(p, true);
+  if (st != DMU_OK) return st;
+  if (!grads) return fail(DMU_ERR_INVALID_ARG, "grads is NULL");
+  if (!(eps >= 0.f) || !std::isfinite(beta)) return fail(DMU_ERR_INVALID_ARG, "eps must be >= 0 and beta finite");
+  DevGuard dg(p->device);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  p->launches = 0;
+  st = upload_table(p, TBL_GRADS, grads, s);
+  if (st != DMU_OK) return st;
+  bool vec = p->vec_shapes && aligned16(grads, p->count);
+  if (momenta) {
+    st = upload_table(p, TBL_MOMS, reinterpret_cast<const void* const*>(momenta), s);
+    if (st != DMU_OK) return st;
+    vec = vec && aligned16(reinterpret_cast<const void* const*>(momenta), p->count);
+  }
+  return run_normalize(p, TBL_GRADS, momenta != nullptr, beta, eps, vec, s);
+}
+
+dmu_status dmu_gram_ns_batched(dmu_plan p, const void* const* ptrs, const dmu_shape* shapes, int count,
+                               const float coeffs[3], int steps, void* stream) {
+  g_err.clear();
+  dmu_status st = check_plan(p, true);
+  if (st != DMU_OK) return st;
+  if (!shapes || !coeffs) return fail(DMU_ERR_INVALID_ARG, "shapes or coeffs is NULL");
+  if (count != p->count) return fail(DMU_ERR_NOT_PLANNED, "count differs from the plan");
+  for (int i = 0; i < count; ++i)
+    if (shapes[i].rows != p->shapes[i].rows || shapes[i].cols != p->shapes[i].cols)
+      return fail(DMU_ERR_NOT_PLANNED, "shape of matrix " + std::to_string(i) + " differs from the plan");
+  if (steps < 0 || steps > 64) return fail(DMU_ERR_INVALID_ARG, "steps must be in [0, 64]");
+  for (int k = 0; k < 3; ++k)
+    if (!std::isfinite(coeffs[k])) return fail(DMU_ERR_INVALID_ARG, "coefficients must be finite");
+  DevGuard dg(p->device);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  p->launches = 0;
+  if (ptrs) {
+    st = upload_table(p, TBL_IN, ptrs, s);
+    if (st != DMU_OK) return st;
+    st = run_normalize(p, TBL_IN, false, 0.f, p->eps, p->vec_shapes && aligned16(ptrs, p->count), s);
+    if (st != DMU_OK) return st;
+  } else if (!p->have_mb) {
+    return fail(DMU_ERR_NOT_PLANNED, "no input: call dmu_momentum_normalize first or pass ptrs");
+  }
+  st = p->dtype == DMU_BF16 ? gram_bf16(p, coeffs, steps, s) : gram_f32(p, coeffs, steps, s);
+  if (st != DMU_OK) return st;
+  p->have_p = true;
+  return DMU_OK;
+}
+
+dmu_status dmu_apply_update(dmu_plan p, void* const* weights, float lr, float* const* out_o, void* stream) {
+  g_err.clear();
+  dmu_status st = check_plan(p, true);
+  if (st != DMU_OK) return st;
+  if (!p->have_p) return fail(DMU_ERR_NOT_PLANNED, "call dmu_gram_ns_batched first");
+  if (!std::isfinite(lr)) return fail(DMU_ERR_INVALID_ARG, "lr must be finite");
+  DevGuard dg(p->device);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  p->launches = 0;
+  if (weights) {
+    st = upload_table(p, TBL_W, reinterpret_cast<const void* const*>(weights), s);
+    if (st != DMU_OK) return st;
+  }
+  if (out_o) {
+    st = upload_table(p, TBL_O, reinterpret_cast<const void* const*>(out_o), s, true);
+    if (st != DMU_OK) return st;
+  }
+  if (!weights && !out_o) return DMU_OK;
+  if (p->dtype == DMU_BF16) {
+    std::vector<Prob> probs;
+    const int pf_hi = p->p_final == 0 ? SLOT_PA_HI : SLOT_PB_HI;
+    for (const Bucket& b : p->buckets) {
+      const GClass& gc = p->classes[b.cls];
+      Prob pr;
+      std::memset(&pr, 0, sizeof(pr));
+      GemmProblem& g = pr.g;
+      g.count = b.count;
+      g.M = (int)b.m;
+      g.N = (int)b.n;
+      g.K = (int)b.m;
+      g.sym = 0;
+      g.tiles_per_mat = tiles_for(g.M, g.N, false, &g.tiles_m, &g.tiles_n);
+      g.a_mn = 0;
+      g.a_z[0] = pf_hi * gc.count + b.cls_off;
+      g.a_z[1] = (pf_hi + 1) * gc.count + b.cls_off;
+      g.b_mn = b.tall ? 0 : 1;
+      g.terms = TERM_HH | TERM_LH;
+      g.epi = EPI_UPDATE;
+      g.alpha = -lr * (float)std::sqrt(std::max(1.0, (double)b.rows / (double)b.cols));
+      g.inv = p->inv_dev();
+      g.inv_base = b.first_slot;
+      g.w_ptrs = weights ? reinterpret_cast<void* const*>(p->tbl_dev(TBL_W)) : nullptr;
+      g.o_ptrs = out_o ? reinterpret_cast<float* const*>(p->tbl_dev(TBL_O)) : nullptr;
+      g.ptr_base = b.first_slot;
+      g.w_f32 = 0;
+      g.w_transposed = b.tall ? 1 : 0;
+      g.w_cols = b.cols;
+      pr.amap = gc.map;
+      pr.bmap = b.tall ? b.map_k : b.map_mn;
+      probs.push_back(pr);
+    }
+    return run_tc(p, probs, 2, 1, s);
+  }
+  const int pf = p->p_final == 0 ? FSLOT_PA : FSLOT_PB;
+  for (const Bucket& b : p->buckets) {
+    const GClass& gc = p->classes[b.cls];
+    SimtProblem q;
+    std::memset(&q, 0, sizeof(q));
+    q.count = b.count;
+    q.M = (int)b.m;
+    q.N = (int)b.n;
+    q.K = (int)b.m;
+    q.a = p->slot_f32(b.cls, pf) + (size_t)b.cls_off * gc.m * gc.ldg;
+    q.a_ms = gc.m * gc.ldg;
+    q.a_si = gc.ldg;
+    q.a_sk = 1;
+    q.b = reinterpret_cast<const float*>(p->mb_dev()) + b.mb_off;
+    q.b_ms = b.rows * b.ldc;
+    q.b_si = b.tall ? b.ldc : 1;
+    q.b_sk = b.tall ? 1 : b.ldc;
+    q.epi = EPI_UPDATE;
+    q.alpha = -lr * (float)std::sqrt(std::max(1.0, (double)b.rows / (double)b.cols));
+    q.alpha_mode = ALPHA_INV;
+    q.inv = p->inv_dev();
+    q.inv_base = b.first_slot;
+    q.w_ptrs = weights ? reinterpret_cast<void* const*>(p->tbl_dev(TBL_W)) : nullptr;
+    q.o_ptrs = out_o ? reinterpret_cast<float* const*>(p->tbl_dev(TBL_O)) : nullptr;
+    q.ptr_base = b.first_slot;
+    q.w_f32 = 1;
+    q.w_transposed = b.tall ? 1 : 0;
+    q.w_cols = b.cols;
+    CUDA_TRY(launch_simt_gemm(q, s));
+    p->launches++;
+  }
+  return DMU_OK;
+}
+
+dmu_status dmu_read_status(dmu_plan p, uint32_t* flags) {
+  g_err.clear();
+  dmu_status st = check_plan(p, true);
+  if (st != DMU_OK) return st;
+  DevGuard dg(p->device);
+  unsigned int v = 0;
+  CUDA_TRY(cudaDeviceSynchronize());
+  CUDA_TRY(cudaMemcpy(&v, p->status_dev(), sizeof(v), cudaMemcpyDeviceToHost));
+  CUDA_TRY(cudaMemset(p->status_dev(), 0, sizeof(v)));
+  if (flags) *flags = v;
+  if (v & DMU_FLAG_TIMEOUT) return fail(DMU_ERR_TIMEOUT, "a device wait timed out");
+  if (v & DMU_FLAG_NONFINITE) return fail(DMU_ERR_NONFINITE, "a momentum norm is not finite");
+  return DMU_OK;
+}
+
+dmu_status dmu_debug_gram(dmu_plan p, int which, int index, float* out, void* stream) {
+  g_err.clear();
+  dmu_status st = check_plan(p, true);
+  if (st != DMU_OK) return st;
+  if (!out) return fail(DMU_ERR_INVALID_ARG, "out is NULL");
+  if (which < 0 || which > 8) return fail(DMU_ERR_INVALID_ARG, "which must be in [0, 8]");
+  if (which < 6 && (index < 0 || index >= p->count)) return fail(DMU_ERR_INVALID_ARG, "index out of range");
+  if (which == 7 && (index < 0 || index >= p->count)) return fail(DMU_ERR_INVALID_ARG, "index out of range");
+  DevGuard dg(p->device);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (which == 8) {
+    // bounded-wait self-test: wait `index` microseconds on a barrier nothing completes
+    if (index < 1 || index > 1000000) return fail(DMU_ERR_INVALID_ARG, "self-test wait must be 1..1e6 us");
+    CUDA_TRY(launch_wait_selftest(p->status_dev(), 1000LL * index, s));
+    CUDA_TRY(cudaStreamSynchronize(s));
+    return DMU_OK;
+  }
+  if (which == 6) {
+    CUDA_TRY(cudaMemcpyAsync(out, p->inv_dev(), sizeof(float) * p->count, cudaMemcpyDeviceToDevice, s));
+    CUDA_TRY(cudaStreamSynchronize(s));
+    return DMU_OK;
+  }
+  const int slot = p->slot_of[index];
+  const Bucket* bk = nullptr;
+  for (const Bucket& b : p->buckets)
+    if (slot >= b.first_slot && slot < b.first_slot + b.count) bk = &b;
+  const int local = slot - bk->first_slot;
+  if (which == 5) {
+    const MomMat& mm = p->mats[slot];
+    if (p->dtype == DMU_BF16) {
+      CUDA_TRY(launch_pair_to_f32(reinterpret_cast<const __nv_bfloat16*>(p->mb_dev()) + mm.mb_off, nullptr,
+                                  mm.rows, mm.cols, mm.ldc, out, s));
+    } else {
+      CUDA_TRY(launch_f32_copy2d(reinterpret_cast<const float*>(p->mb_dev()) + mm.mb_off, mm.rows, mm.cols,
+                                 mm.ldc, out, s));
+    }
+    CUDA_TRY(cudaStreamSynchronize(s));
+    return DMU_OK;
+  }
+  const GClass& gc = p->classes[bk->cls];
+  const size_t moff = (size_t)(bk->cls_off + local) * gc.m * gc.ldg;
+  int q = which;
+  if (which == 7) q = p->p_final == 0 ? 3 : 4;
+  if (p->dtype == DMU_BF16) {
+    const int slots[5] = {SLOT_G_HI, SLOT_R_HI, SLOT_T_HI, SLOT_PA_HI, SLOT_PB_HI};
+    const int sh = slots[q];
+    const bool has_lo = !(sh == SLOT_R_HI && gc.prec == DMU_PREC_FAST);
+    CUDA_TRY(launch_pair_to_f32(p->slot_bf16(bk->cls, sh) + moff,
+                                has_lo ? p->slot_bf16(bk->cls, sh + 1) + moff : nullptr, gc.m, gc.m, gc.ldg,
+                                out, s));
+  } else {
+    CUDA_TRY(launch_f32_copy2d(p->slot_f32(bk->cls, q) + moff, gc.m, gc.m, gc.ldg, out, s));
+  }
+  CUDA_TRY(cudaStreamSynchronize(s));
+  return DMU_OK;
+}
+
+int dmu_last_launch_count(dmu_plan p) { return p ? p->launches : 0; }
+
+void dmu_plan_destroy(dmu_plan p) {
+  if (!p) return;
+  for (int t = 0; t < NUM_TBL; ++t) {
+    if (p->tbl_ev[t]) {
+      cudaEventSynchronize(p->tbl_ev[t]);
+      cudaEventDestroy(p->tbl_ev[t]);
+    }
+    if (p->pinned[t]) cudaFreeHost(p->pinned[t]);
+  }
+  delete p;
+}
+
+}  // extern "C"

@@ -16,6 +16,7 @@ Recipes (one entry per workload):
   projection shapes (q, o 3584 x 3584; k, v 512 x 3584; gate, up
   18944 x 3584; down 3584 x 18944), each drawn like the uniform workload.
   Only the shapes come from that model; no weights are used.
+  ``qwen2.5-7b-layer-set-x<L>`` is the same with L layers (profiling).
 * ``small-swarm-4096``: 2048 gradients 128 x 512 and 2048 gradients
   256 x 1024, N(0, 1) times a per-matrix scale 10**U(-4, -1), bf16.
 * ``large-dense-24``: 16 gradients 8192 x 8192 and 8 of 8192 x 28672,
@@ -83,6 +84,10 @@ def workload(name: str) -> Workload:
         return Workload(name, 2, "bf16", ((512, 2048),) * 64, "spiked", 1e-3, 8)
     if name == "qwen2.5-7b-layer-set-x28":
         s, l = _qwen_shapes(28)
+        return Workload(name, 3, "bf16", s, "spiked", 1e-3, 8, labels=l)
+    if name.startswith("qwen2.5-7b-layer-set-x") and name != "qwen2.5-7b-layer-set-x28":
+        layers = int(name.rsplit("x", 1)[1])
+        s, l = _qwen_shapes(layers)
         return Workload(name, 3, "bf16", s, "spiked", 1e-3, 8, labels=l)
     if name == "small-swarm-4096":
         return Workload(name, 4, "bf16", ((128, 512),) * 2048 + ((256, 1024),) * 2048,

@@ -1,0 +1,198 @@
+/*
+ * dmu.h -- C ABI of libdmu: the owner-side Muon update on one B200 GPU.
+ *
+ * The update, per weight matrix W (rows x cols, row-major, contiguous):
+ *
+ *   1. momentum        M <- beta * M + G
+ *   2. orientation     X = M if rows <= cols, else X = M^T   (m = min, n = max)
+ *   3. normalisation   X0 = X / (||M||_F + eps)
+ *   4. Gram recursion  G0 = X0 X0^T, P0 = I;  K times:
+ *                        Q = a I + b G + c G^2,  G <- Q G Q,  P <- Q P
+ *   5. update          O = P X0 (in W's orientation);
+ *                      W <- W - lr * sqrt(max(1, rows / cols)) * O
+ *
+ * Sources (page title and section):
+ *   - "DMuon: Efficient Distributed Muon Training with Near-Adam Overhead",
+ *     technical summary, section 1: Muon applies Newton-Schulz to the
+ *     momentum-accumulated gradient of each weight matrix (steps 1, 4, 5).
+ *   - same page, section 2.2: the recursion runs in the m x m Gram space
+ *     G = X X^T, the symmetric products take a SYRK-style path, and
+ *     similar-shape matrices are batched (steps 2, 4; the batching below).
+ *   - same page, section 2.4: per-shape kernel schedules are tuned and
+ *     cached (the per-plan schedule choice).
+ *   - "DeMuon" technical summary, Method 1: the target of the iteration is
+ *     the matrix sign msgn(X) = U V^T.
+ *   - "Dion3: Full-Stack Orthogonal Updates" review, sections 1 and 3:
+ *     Gram Newton-Schulz and a symmetric GEMM kernel.
+ * The pages give no coefficients, step count, eps, momentum form or scale
+ * rule; the defaults here are (a,b,c) = (3.4445, -4.7750, 2.0315), K = 5,
+ * eps = 1e-7, the plain accumulation above and sqrt(max(1, rows/cols)).
+ *
+ * Conventions for every call:
+ *   - Ownership: the caller owns all device memory -- gradients, momenta,
+ *     weights and the workspace (dmu_set_workspace).  The library owns only
+ *     its host-side plan and a small pinned staging buffer for pointer
+ *     tables.  Pointer arrays are HOST arrays of DEVICE pointers; the
+ *     library copies them to the workspace when they differ from the last
+ *     call's (stream-ordered), so steady-state steps upload nothing.
+ *   - Asynchrony: compute calls enqueue work on `stream` (a cudaStream_t,
+ *     passed as void*; NULL = legacy default stream) and return without
+ *     synchronising.  Only dmu_read_status and dmu_debug_gram synchronise.
+ *   - Errors: every call returns a dmu_status.  Argument errors are
+ *     detected before any launch.  CUDA errors map to DMU_ERR_CUDA.
+ *     dmu_last_error() returns the message of the calling thread's last
+ *     error.  There are no device traps: device-side faults of the data
+ *     (non-finite norms) and bounded-wait timeouts set bits of a device
+ *     status word that dmu_read_status returns.
+ *   - Layout: every matrix i is contiguous row-major with the shape given
+ *     to dmu_plan_create.  Device pointers must be 16-byte aligned for the
+ *     vectorised paths (misaligned pointers take a scalar path).
+ *   - Threads: a plan must not be used by two host threads at once.
+ */
+#ifndef DMU_H
+#define DMU_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DMU_VERSION 100
+
+#if defined(__GNUC__)
+#define DMU_API __attribute__((visibility("default")))
+#else
+#define DMU_API
+#endif
+
+typedef enum {
+  DMU_OK = 0,
+  DMU_ERR_INVALID_ARG = 1,  /* null pointer, bad shape, count mismatch   */
+  DMU_ERR_UNSUPPORTED = 2,  /* device is not sm_100, or a mode not built */
+  DMU_ERR_WORKSPACE = 3,    /* workspace missing, too small, misaligned  */
+  DMU_ERR_CUDA = 4,         /* a CUDA runtime or driver call failed       */
+  DMU_ERR_NONFINITE = 5,    /* a momentum norm was NaN or Inf             */
+  DMU_ERR_NOT_PLANNED = 6,  /* shapes differ from the plan, or call order */
+  DMU_ERR_TIMEOUT = 7       /* a bounded device-side wait gave up         */
+} dmu_status;
+
+typedef enum {
+  DMU_BF16 = 0, /* gradients and weights bf16; tensor-core (tcgen05) path */
+  DMU_F32 = 1   /* gradients and weights fp32; exact fp32 FFMA path        */
+} dmu_dtype;
+
+/* Precision of the Gram-space products on the bf16 path.  Gram-space
+ * matrices are always stored as a bf16 pair (hi, lo = bf16(x - hi)) and
+ * the final P X0 product always uses both halves of P.
+ *   FAST   : one bf16 MMA per product (hi x hi).
+ *   SPLIT2 : two MMAs per product (hi x hi + lo x hi).
+ *   SPLIT3 : three MMAs per product (hi x hi + hi x lo + lo x hi).
+ *   AUTO   : FAST for m >= 1024, SPLIT3 below (per shape bucket). */
+typedef enum {
+  DMU_PREC_AUTO = 0,
+  DMU_PREC_FAST = 1,
+  DMU_PREC_SPLIT2 = 2,
+  DMU_PREC_SPLIT3 = 3
+} dmu_prec;
+
+/* Bits of the device status word (dmu_read_status). */
+#define DMU_FLAG_NONFINITE 0x1u /* a Frobenius norm was not finite  */
+#define DMU_FLAG_TIMEOUT 0x2u   /* a device wait hit its time limit */
+
+typedef struct {
+  int64_t rows; /* W.shape[0] (out_features) */
+  int64_t cols; /* W.shape[1] (in_features)  */
+} dmu_shape;
+
+typedef struct dmu_plan_s* dmu_plan;
+
+/* Build a plan for `count` matrices with these shapes on CUDA `device`.
+ * Matrices are grouped into buckets of equal (rows, cols) and, for the
+ * Gram-space recursion, into classes of equal m = min(rows, cols); tall
+ * matrices are handled by logical transposition (no copy).  No device
+ * memory is allocated.  Errors: INVALID_ARG (count <= 0, a non-positive
+ * extent, out == NULL), UNSUPPORTED (device not compute capability 10.x
+ * for DMU_BF16), CUDA. */
+DMU_API dmu_status dmu_plan_create(const dmu_shape* shapes, int count, dmu_dtype dtype,
+                           dmu_prec prec, int device, dmu_plan* out);
+
+/* Bytes of device workspace the plan needs (0 for an invalid plan). */
+DMU_API size_t dmu_workspace_bytes(dmu_plan plan);
+
+/* Give the plan its workspace: `bytes` >= dmu_workspace_bytes, 256-byte
+ * aligned, on the plan's device, owned by the caller and kept alive while
+ * the plan is used.  Uploads the plan's tables (synchronous) and encodes
+ * the TMA tensor maps.  Errors: WORKSPACE, INVALID_ARG, CUDA. */
+DMU_API dmu_status dmu_set_workspace(dmu_plan plan, void* dev_ptr, size_t bytes);
+
+/* Step 1 + the norm of step 3, for all matrices of the plan.
+ *   grads[i]   : device pointer, rows*cols elements of the plan dtype.
+ *   momenta[i] : device pointer, rows*cols fp32, updated in place
+ *                (M <- beta*M + G).  momenta == NULL means "no state":
+ *                M = G and nothing is written back.
+ * Writes the bf16 (or fp32) image of M and 1/(||M||_F + eps) for every
+ * matrix into the workspace.  Source: DMuon page, section 1. */
+DMU_API dmu_status dmu_momentum_normalize(dmu_plan plan, const void* const* grads,
+                                  float* const* momenta, float beta, float eps,
+                                  void* stream);
+
+/* Steps 2-4: the Gram Newton-Schulz recursion, batched over all matrices.
+ *   ptrs   : NULL to use the matrices left by dmu_momentum_normalize; or
+ *            device pointers to `count` matrices (plan dtype) to
+ *            orthogonalise directly (they are normalised first, with the
+ *            eps of the last dmu_momentum_normalize call, 1e-7 if none).
+ *   shapes, count : must equal the plan's (else NOT_PLANNED).
+ *   coeffs : (a, b, c);  steps : K >= 0 (K = 0 gives P = I).
+ * Result: P_K per matrix, kept in the workspace for dmu_apply_update.
+ * Sources: DMuon page, section 2.2; Dion3 review, sections 1 and 3. */
+DMU_API dmu_status dmu_gram_ns_batched(dmu_plan plan, const void* const* ptrs,
+                               const dmu_shape* shapes, int count,
+                               const float coeffs[3], int steps, void* stream);
+
+/* Step 5: O = P X0 fused with W <- W - lr * sqrt(max(1, rows/cols)) * O.
+ *   weights[i] : device pointer, rows*cols of the plan dtype, updated in
+ *                place; weights == NULL skips the update.
+ *   out_o[i]   : optional fp32 device buffers (rows*cols) that receive O
+ *                in W's orientation; out_o == NULL skips them all, a NULL
+ *                entry skips that matrix.
+ * Requires a completed dmu_gram_ns_batched (else NOT_PLANNED). */
+DMU_API dmu_status dmu_apply_update(dmu_plan plan, void* const* weights, float lr,
+                            float* const* out_o, void* stream);
+
+/* Synchronise the plan's device, read and clear the status word.
+ * Returns NONFINITE or TIMEOUT when the matching bit was set. */
+DMU_API dmu_status dmu_read_status(dmu_plan plan, uint32_t* flags);
+
+/* Test hook: write one workspace quantity as fp32 into `out` (device).
+ *   which 0..4 : Gram-space matrix G, R, T, P(buffer A), P(buffer B) of
+ *                matrix `index` (m*m floats, hi + lo combined);
+ *   which 5    : the normalised input image Mb of matrix `index`
+ *                (rows*cols floats, unscaled);
+ *   which 6    : 1/(||M||_F + eps) of every matrix (count floats);
+ *   which 7    : the final P of matrix `index` (m*m floats);
+ *   which 8    : bounded-wait self-test, writes nothing to `out`: a kernel
+ *                waits `index` microseconds (1..1e6) on a barrier that
+ *                nothing completes, gives up, and sets DMU_FLAG_TIMEOUT
+ *                (read it with dmu_read_status).
+ * Synchronises `stream`. */
+DMU_API dmu_status dmu_debug_gram(dmu_plan plan, int which, int index, float* out, void* stream);
+
+/* Number of kernel launches the last compute call enqueued. */
+DMU_API int dmu_last_launch_count(dmu_plan plan);
+
+/* Message for the calling thread's last error ("" if none). */
+DMU_API const char* dmu_last_error(void);
+
+/* Library version (DMU_VERSION). */
+DMU_API int dmu_version(void);
+
+/* Free the host-side plan.  Does not touch the caller's device memory. */
+DMU_API void dmu_plan_destroy(dmu_plan plan);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DMU_H */

@@ -1,0 +1,145 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+* libdmu.so loads and exports every function include/dmu.h declares;
+* argument errors come back as status codes before any CUDA call;
+* planning (bucketing, Gram classes, workspace layout) works without a
+  device, and compute calls then fail cleanly.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from gram_newton_schulz_b200 import dmu, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dmu.h")
+NO_GPU = not torch.cuda.is_available()
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"DMU_API\s+[\w\s\*]+?\b(dmu_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("dmu_momentum_normalize", "dmu_gram_ns_batched", "dmu_apply_update", "dmu_plan_create",
+              "dmu_set_workspace", "dmu_workspace_bytes", "dmu_read_status", "dmu_plan_destroy"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = dmu.load()
+    for n in _declared():
+        assert hasattr(lib, n), n
+    assert set(_declared()) <= set(dmu.SIGNATURES)
+    assert lib.dmu_version() == 100
+
+
+def _shapes(pairs):
+    arr = (dmu.Shape * max(len(pairs), 1))(*[dmu.Shape(r, c) for r, c in pairs])
+    return ctypes.cast(arr, ctypes.c_void_p), arr
+
+
+def _create(pairs, dtype=0, prec=0, count=None):
+    lib = dmu.load()
+    p, keep = _shapes(pairs)
+    h = ctypes.c_void_p()
+    st = lib.dmu_plan_create(p, len(pairs) if count is None else count, dtype, prec, 0, ctypes.byref(h))
+    return st, h, keep
+
+
+def test_argument_errors():
+    lib = dmu.load()
+    h = ctypes.c_void_p()
+    assert lib.dmu_plan_create(None, 1, 0, 0, 0, ctypes.byref(h)) == dmu.ERR_INVALID_ARG
+    assert b"NULL" in lib.dmu_last_error()
+    assert _create([(4, 4)], count=0)[0] == dmu.ERR_INVALID_ARG
+    assert _create([(0, 4)])[0] == dmu.ERR_INVALID_ARG
+    assert _create([(4, -1)])[0] == dmu.ERR_INVALID_ARG
+    assert _create([(4, 4)], dtype=7)[0] == dmu.ERR_INVALID_ARG
+    assert _create([(4, 4)], prec=9)[0] == dmu.ERR_INVALID_ARG
+    assert _create([(4, 1 << 21)])[0] == dmu.ERR_UNSUPPORTED
+    p, keep = _shapes([(4, 4)])
+    assert lib.dmu_plan_create(p, 1, 0, 0, 0, None) == dmu.ERR_INVALID_ARG
+    # calls on a NULL plan
+    assert lib.dmu_set_workspace(None, None, 0) == dmu.ERR_INVALID_ARG
+    assert lib.dmu_momentum_normalize(None, None, None, 0.9, 1e-7, None) == dmu.ERR_INVALID_ARG
+    co = (ctypes.c_float * 3)(*dmu.QUINTIC)
+    assert lib.dmu_gram_ns_batched(None, None, p, 1, ctypes.cast(co, ctypes.c_void_p), 5, None) == dmu.ERR_INVALID_ARG
+    assert lib.dmu_apply_update(None, None, 0.02, None, None) == dmu.ERR_INVALID_ARG
+    assert lib.dmu_workspace_bytes(None) == 0
+    lib.dmu_plan_destroy(None)
+
+
+def _ws_expected(shapes, nslots, esize=2):
+    mb = 0
+    buckets = {}
+    for r, c in shapes:
+        buckets.setdefault((r, c), 0)
+        buckets[(r, c)] += 1
+    for (r, c), n in buckets.items():
+        ldc = -(-c // 8) * 8
+        mb += n * r * ldc
+    gram = 0
+    classes = {}
+    for r, c in shapes:
+        m = min(r, c)
+        classes[m] = classes.get(m, 0) + 1
+    for m, n in classes.items():
+        ldg = -(-m // 8) * 8
+        gram += nslots * n * m * ldg
+    return esize * (mb + gram)
+
+
+@pytest.mark.skipif(not NO_GPU, reason="host-only planning is checked where no device exists")
+def test_host_only_plan_layout_qwen7b():
+    w = synth.workload("qwen2.5-7b-layer-set-x28")
+    st, h, keep = _create(w.shapes)
+    assert st == dmu.OK
+    lib = dmu.load()
+    total = lib.dmu_workspace_bytes(h)
+    expect = _ws_expected(w.shapes, 10)
+    # tables, per-chunk partial sums and alignment add a little on top
+    assert expect <= total <= expect * 1.002
+    assert 45e9 < total < 55e9
+    # no device: setting a workspace or computing fails cleanly
+    assert lib.dmu_set_workspace(h, ctypes.c_void_p(256), total) == dmu.ERR_CUDA
+    assert lib.dmu_momentum_normalize(h, None, None, 0.9, 1e-7, None) == dmu.ERR_WORKSPACE
+    lib.dmu_plan_destroy(h)
+
+
+@pytest.mark.skipif(not NO_GPU, reason="host-only planning is checked where no device exists")
+@pytest.mark.parametrize("name", ["single-64x256-fp32", "uniform-64x512x2048", "small-swarm-4096",
+                                  "large-dense-24"])
+def test_host_only_plan_sizes(name):
+    w = synth.workload(name)
+    st, h, keep = _create(w.shapes, dtype=0 if w.dtype == "bf16" else 1)
+    assert st == dmu.OK
+    total = dmu.load().dmu_workspace_bytes(h)
+    expect = _ws_expected(w.shapes, 10 if w.dtype == "bf16" else 5, 2 if w.dtype == "bf16" else 4)
+    assert expect <= total <= expect * 1.01 + (1 << 20)
+    dmu.load().dmu_plan_destroy(h)
+
+
+def test_binding_rejects_mismatched_tensors():
+    # shape/dtype validation happens in the binding before the C call
+    class Fake:
+        shape = (3, 3)
+        dtype = torch.bfloat16
+        device = torch.device("cpu")
+
+        def is_contiguous(self):
+            return True
+
+    p = dmu.Plan.__new__(dmu.Plan)
+    p.count = 1
+    p.shapes = [(4, 4)]
+    p.device = torch.device("cuda", 0)
+    with pytest.raises(ValueError):
+        p._check_tensors([Fake()], "grads", torch.bfloat16)
+    with pytest.raises(ValueError):
+        p._check_tensors([], "grads", torch.bfloat16)
