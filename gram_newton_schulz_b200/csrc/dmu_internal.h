@@ -40,6 +40,14 @@ enum AlphaMode : int { ALPHA_CONST = 0, ALPHA_INV2 = 1, ALPHA_INV = 2 };
 // Term bits: which bf16 products the MMA warp issues per K slice.
 enum Terms : int { TERM_HH = 1, TERM_HL = 2, TERM_LH = 4 };
 
+// Operand kind of a tensor-core launch: bf16 (kind::f16, K = 16 per MMA)
+// or tf32 (kind::tf32 on fp32 storage, K = 8 per MMA).  Either way a
+// K-block is one 128-byte swizzle row: 64 bf16 or 32 fp32 elements.
+enum MmaKind : int { KIND_BF16 = 0, KIND_TF32 = 1 };
+
+// Storage format of an epilogue input/output matrix.
+enum Fmt : int { FMT_PAIR = 0, FMT_F32 = 1 };
+
 // One grouped-GEMM problem: `count` independent matrices of the same
 // geometry.  Output tile (bi, bj) of matrix `mat` is
 //   D[i][j] = sum_k A(i, k) * B(j, k),   i in [0, M), j in [0, N)
@@ -68,6 +76,10 @@ struct GemmProblem {
   __nv_bfloat16* out2_lo;
   long long ld;            // row stride (elements) of Cin/out
   long long mat_stride;    // matrix stride (elements) of Cin/out
+  int cin_fmt, out_fmt, out2_fmt;  // Fmt of Cin, out, out2
+  const float* cin_f;      // FMT_F32 variants of Cin / out / out2
+  float* out_f;
+  float* out2_f;
   // EPI_UPDATE: W += alpha * inv * acc in W's layout; O = inv * acc
   void* const* w_ptrs;     // device table, indexed by ptr_base + mat
   float* const* o_ptrs;    // device table (may be null)
@@ -118,7 +130,7 @@ struct SimtProblem {
 };
 
 // ---------------------------------------------------------------- launchers
-cudaError_t launch_gemm_tc(const GemmParams& p, int na, int nb, int num_sms, cudaStream_t s);
+cudaError_t launch_gemm_tc(const GemmParams& p, int na, int nb, int kind, int num_sms, cudaStream_t s);
 cudaError_t gemm_tc_configure();
 cudaError_t launch_wait_selftest(unsigned int* status, long long timeout_ns, cudaStream_t s);
 int gemm_tc_stages(int na, int nb);

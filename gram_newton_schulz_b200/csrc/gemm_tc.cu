@@ -30,7 +30,7 @@
 namespace dmu {
 
 template <int NA, int NB>
-struct TcCfg {
+struct TcCfg {  // stage geometry is the same for both operand kinds
   static constexpr int STAGE_BYTES = NA * A_PART_BYTES + NB * B_PART_BYTES;
   static constexpr int STAGES = (200 * 1024) / STAGE_BYTES;
   static constexpr int BAR_BYTES = 256;
@@ -128,6 +128,7 @@ __device__ __forceinline__ void store_pair(__nv_bfloat16* hi, __nv_bfloat16* lo,
 }
 
 // One 32-column chunk of a Gram-space output tile for the thread's row i.
+// Input and outputs are bf16 hi/lo pairs (FMT_PAIR) or fp32 (FMT_F32).
 __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, int i, int col0,
                                                const uint32_t (&r)[32]) {
   const int M = pr.M, N = pr.N;
@@ -148,7 +149,23 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
   const bool full = (col0 + 32 <= N);
   const bool all_upper = !pr.sym || (i <= col0);
 
-  if (pr.cin_hi) {
+  if (pr.cin_fmt == FMT_F32 && pr.cin_f) {
+    if (full) {
+      const float4* pc = reinterpret_cast<const float4*>(pr.cin_f + rowoff + col0);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 t = pc[q];
+        v[4 * q] += pr.beta * t.x;
+        v[4 * q + 1] += pr.beta * t.y;
+        v[4 * q + 2] += pr.beta * t.z;
+        v[4 * q + 3] += pr.beta * t.w;
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (col0 + c < N) v[c] += pr.beta * pr.cin_f[rowoff + col0 + c];
+    }
+  } else if (pr.cin_fmt == FMT_PAIR && pr.cin_hi) {
     if (full) {
       const uint4* ph = reinterpret_cast<const uint4*>(pr.cin_hi + rowoff + col0);
       const uint4* pl = pr.cin_lo ? reinterpret_cast<const uint4*>(pr.cin_lo + rowoff + col0) : nullptr;
@@ -184,14 +201,38 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
   }
 
   for (int pass = 0; pass < 2; ++pass) {
-    __nv_bfloat16* oh = pass == 0 ? pr.out_hi : pr.out2_hi;
-    __nv_bfloat16* ol = pass == 0 ? pr.out_lo : pr.out2_lo;
-    if (!oh) continue;
+    const int fmt = pass == 0 ? pr.out_fmt : pr.out2_fmt;
     if (pass == 1 && dc >= 0 && dc < 32) {
 #pragma unroll
       for (int c = 0; c < 32; ++c)
         if (c == dc) v[c] += pr.gamma2;
     }
+    if (fmt == FMT_F32) {
+      float* of = pass == 0 ? pr.out_f : pr.out2_f;
+      if (!of) continue;
+      if (full && all_upper) {
+        float4* d4 = reinterpret_cast<float4*>(of + rowoff + col0);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) d4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int j = col0 + c;
+          if (j < N && (!pr.sym || i <= j)) of[rowoff + j] = v[c];
+        }
+      }
+      if (pr.sym) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int j = col0 + c;
+          if (j < N && i < j) of[mbase + (long long)j * pr.ld + i] = v[c];
+        }
+      }
+      continue;
+    }
+    __nv_bfloat16* oh = pass == 0 ? pr.out_hi : pr.out2_hi;
+    __nv_bfloat16* ol = pass == 0 ? pr.out_lo : pr.out2_lo;
+    if (!oh) continue;
     // direct stores (i, j), j >= i when symmetric
     if (full && all_upper) {
       uint4* dh = reinterpret_cast<uint4*>(oh + rowoff + col0);
@@ -305,9 +346,10 @@ __device__ __forceinline__ void epi_update_chunk(const GemmProblem& pr, int mat,
 }
 
 // ------------------------------------------------------------- kernel
-template <int NA, int NB>
+template <int NA, int NB, int KIND>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_constant__ GemmParams p) {
   using Cfg = TcCfg<NA, NB>;
+  constexpr int BKE = KIND == KIND_TF32 ? 32 : 64;  // elements per 128-byte K-block row
   constexpr int S = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = ptx::smem_u32(smem_raw);
@@ -370,7 +412,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
         const int na = (NA > 1 && (pr.terms & TERM_LH)) ? 2 : 1;
         const int nb = (NB > 1 && (pr.terms & TERM_HL)) ? 2 : 1;
         const uint32_t bytes = na * A_PART_BYTES + nb * B_PART_BYTES;
-        const int nk = (pr.K + BK - 1) / BK;
+        const int nk = (pr.K + BKE - 1) / BKE;
         const int arow = tc.bi * BM, brow = tc.bj * BN;
         for (int kb = 0; kb < nk; ++kb) {
           if (!wait_bar(empty_bar(stage), phase ^ 1u, abort_flag, p)) {
@@ -381,7 +423,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
           ptx::mbar_arrive_expect_tx(fb, bytes);
           issued_mask |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-          const int k0 = kb * BK;
+          const int k0 = kb * BKE;
           const uint32_t sa = ring + stage * Cfg::STAGE_BYTES;
           const uint32_t sb = sa + NA * A_PART_BYTES;
           for (int part = 0; part < na; ++part) {
@@ -438,8 +480,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
       for (int t = blockIdx.x; ok && t < p.total_tiles; t += gridDim.x) {
         const TileCoord tc = decode_tile(p, t);
         const GemmProblem& pr = p.prob[tc.pi];
-        const int nk = (pr.K + BK - 1) / BK;
-        const uint32_t idesc = ptx::make_idesc_bf16(BM, BN, pr.a_mn, pr.b_mn);
+        const int nk = (pr.K + BKE - 1) / BKE;
+        const uint32_t idesc = ptx::make_idesc(BM, BN, pr.a_mn, pr.b_mn, KIND == KIND_TF32 ? 2 : 1);
         if (!wait_bar(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p)) {
           ok = false;
           break;
@@ -460,7 +502,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
           const uint32_t sa = ring + stage * Cfg::STAGE_BYTES;
           const uint32_t sb = sa + NA * A_PART_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+          for (int kk = 0; kk < 4; ++kk) {  // 4 MMAs x 32 bytes of K per 128-byte row
 #pragma unroll
             for (int term = 0; term < 3; ++term) {
               const int bit = 1 << term;
@@ -471,7 +513,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
               const uint32_t pb = sb + (term == 1 ? B_PART_BYTES : 0);
               const uint64_t ad = ptx::make_sw128_desc(pa + kk * a_kstep, a_lbo, a_sbo);
               const uint64_t bd = ptx::make_sw128_desc(pb + kk * b_kstep, b_lbo, b_sbo);
-              ptx::mma_bf16(d_tmem, ad, bd, idesc, accumulate);
+              if (KIND == KIND_TF32)
+                ptx::mma_tf32(d_tmem, ad, bd, idesc, accumulate);
+              else
+                ptx::mma_bf16(d_tmem, ad, bd, idesc, accumulate);
               accumulate = 1;
               issued = true;
             }
@@ -573,17 +618,18 @@ cudaError_t launch_wait_selftest(unsigned int* status, long long timeout_ns, cud
   return cudaGetLastError();
 }
 
-template <int NA, int NB>
+template <int NA, int NB, int KIND>
 static cudaError_t configure_one() {
-  return cudaFuncSetAttribute(k_gemm_tc<NA, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  return cudaFuncSetAttribute(k_gemm_tc<NA, NB, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               TcCfg<NA, NB>::SMEM_BYTES);
 }
 
 cudaError_t gemm_tc_configure() {
   cudaError_t e;
-  if ((e = configure_one<1, 1>()) != cudaSuccess) return e;
-  if ((e = configure_one<2, 1>()) != cudaSuccess) return e;
-  if ((e = configure_one<2, 2>()) != cudaSuccess) return e;
+  if ((e = configure_one<1, 1, KIND_BF16>()) != cudaSuccess) return e;
+  if ((e = configure_one<2, 1, KIND_BF16>()) != cudaSuccess) return e;
+  if ((e = configure_one<2, 2, KIND_BF16>()) != cudaSuccess) return e;
+  if ((e = configure_one<1, 1, KIND_TF32>()) != cudaSuccess) return e;
   return cudaSuccess;
 }
 
@@ -594,18 +640,22 @@ int gemm_tc_stages(int na, int nb) {
   return 0;
 }
 
-template <int NA, int NB>
+template <int NA, int NB, int KIND>
 static cudaError_t launch_one(const GemmParams& p, int num_sms, cudaStream_t s) {
   const int grid = p.total_tiles < num_sms ? p.total_tiles : num_sms;
   if (grid <= 0) return cudaSuccess;
-  k_gemm_tc<NA, NB><<<grid, GEMM_THREADS, TcCfg<NA, NB>::SMEM_BYTES, s>>>(p);
+  k_gemm_tc<NA, NB, KIND><<<grid, GEMM_THREADS, TcCfg<NA, NB>::SMEM_BYTES, s>>>(p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm_tc(const GemmParams& p, int na, int nb, int num_sms, cudaStream_t s) {
-  if (na == 1 && nb == 1) return launch_one<1, 1>(p, num_sms, s);
-  if (na == 2 && nb == 1) return launch_one<2, 1>(p, num_sms, s);
-  if (na == 2 && nb == 2) return launch_one<2, 2>(p, num_sms, s);
+cudaError_t launch_gemm_tc(const GemmParams& p, int na, int nb, int kind, int num_sms, cudaStream_t s) {
+  if (kind == KIND_TF32) {
+    if (na == 1 && nb == 1) return launch_one<1, 1, KIND_TF32>(p, num_sms, s);
+    return cudaErrorInvalidValue;
+  }
+  if (na == 1 && nb == 1) return launch_one<1, 1, KIND_BF16>(p, num_sms, s);
+  if (na == 2 && nb == 1) return launch_one<2, 1, KIND_BF16>(p, num_sms, s);
+  if (na == 2 && nb == 2) return launch_one<2, 2, KIND_BF16>(p, num_sms, s);
   return cudaErrorInvalidValue;
 }
 

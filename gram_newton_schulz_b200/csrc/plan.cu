@@ -54,9 +54,12 @@ struct Bucket {
 struct GClass {
   int64_t m = 0, ldg = 0;
   int count = 0;
-  size_t off = 0;  // byte offset in the workspace
+  size_t off = 0;     // byte offset in the workspace
+  size_t off_pf = 0;  // TF32 classes: bf16 hi/lo pair of the final P
   int prec = DMU_PREC_FAST;
-  int map = -1;
+  int kind = KIND_BF16;
+  int map = -1;       // TMA map over the Gram slots (bf16 pairs or fp32)
+  int map_pf = -1;    // TF32 classes: bf16 map over the final-P pair
 };
 
 enum { TBL_GRADS = 0, TBL_MOMS, TBL_W, TBL_O, TBL_IN, NUM_TBL };
@@ -135,6 +138,11 @@ struct dmu_plan_s {
     const GClass& g = classes[c];
     return reinterpret_cast<float*>(ws + g.off) + (size_t)slot * g.count * g.m * g.ldg;
   }
+  // TF32 classes: half 0 = hi, 1 = lo of the final P
+  __nv_bfloat16* pf_bf16(int c, int half) const {
+    const GClass& g = classes[c];
+    return reinterpret_cast<__nv_bfloat16*>(ws + g.off_pf) + (size_t)half * g.count * g.m * g.ldg;
+  }
 };
 
 namespace {
@@ -193,7 +201,7 @@ struct Prob {
   int amap, bmap;  // plan map indices
 };
 
-dmu_status run_tc(dmu_plan p, std::vector<Prob>& probs, int na, int nb, cudaStream_t s) {
+dmu_status run_tc(dmu_plan p, std::vector<Prob>& probs, int na, int nb, int kind, cudaStream_t s) {
   size_t i = 0;
   while (i < probs.size()) {
     GemmParams gp;
@@ -228,16 +236,18 @@ dmu_status run_tc(dmu_plan p, std::vector<Prob>& probs, int na, int nb, cudaStre
     gp.total_tiles = tiles;
     gp.status = p->status_dev();
     gp.timeout_ns = p->timeout_ns;
-    CUDA_TRY(launch_gemm_tc(gp, na, nb, p->num_sms, s));
+    CUDA_TRY(launch_gemm_tc(gp, na, nb, kind, p->num_sms, s));
     p->launches++;
   }
   return DMU_OK;
 }
 
-void prec_shape(int prec, int* na, int* nb, int* terms) {
+void prec_shape(int prec, int* na, int* nb, int* terms, int* kind) {
+  *kind = KIND_BF16;
   switch (prec) {
     case DMU_PREC_SPLIT2: *na = 2; *nb = 1; *terms = TERM_HH | TERM_LH; break;
     case DMU_PREC_SPLIT3: *na = 2; *nb = 2; *terms = TERM_HH | TERM_HL | TERM_LH; break;
+    case DMU_PREC_TF32: *na = 1; *nb = 1; *terms = TERM_HH; *kind = KIND_TF32; break;
     default: *na = 1; *nb = 1; *terms = TERM_HH; break;
   }
 }
@@ -282,14 +292,72 @@ Prob gram_prob(dmu_plan p, int c, int a_slot, int b_slot, int terms, float alpha
   return pr;
 }
 
+// TF32 classes: fp32 slots; out_slot == OUT_PF writes the final P as a
+// bf16 hi/lo pair (the operand of the final bf16 GEMM).
+constexpr int OUT_PF = -2;
+
+void set_f32_out(dmu_plan p, int c, int slot, int* fmt, float** f, __nv_bfloat16** hi, __nv_bfloat16** lo) {
+  if (slot == OUT_PF) {
+    *fmt = FMT_PAIR;
+    *hi = p->pf_bf16(c, 0);
+    *lo = p->pf_bf16(c, 1);
+  } else if (slot >= 0) {
+    *fmt = FMT_F32;
+    *f = p->slot_f32(c, slot);
+  }
+}
+
+Prob gram_prob_f32(dmu_plan p, int c, int a_slot, int b_slot, float alpha, float beta, int cin_slot,
+                   int out_slot, int out2_slot, float gamma2) {
+  const GClass& gc = p->classes[c];
+  Prob pr;
+  std::memset(&pr, 0, sizeof(pr));
+  GemmProblem& g = pr.g;
+  g.count = gc.count;
+  g.M = g.N = g.K = (int)gc.m;
+  g.sym = 1;
+  g.tiles_per_mat = tiles_for(g.M, g.N, true, &g.tiles_m, &g.tiles_n);
+  g.a_z[0] = g.a_z[1] = a_slot * gc.count;
+  g.b_z[0] = g.b_z[1] = b_slot * gc.count;
+  g.terms = TERM_HH;
+  g.epi = EPI_GRAM;
+  g.alpha_mode = ALPHA_CONST;
+  g.alpha = alpha;
+  g.beta = beta;
+  g.gamma2 = gamma2;
+  g.cin_fmt = FMT_F32;
+  if (cin_slot >= 0) g.cin_f = p->slot_f32(c, cin_slot);
+  set_f32_out(p, c, out_slot, &g.out_fmt, &g.out_f, &g.out_hi, &g.out_lo);
+  set_f32_out(p, c, out2_slot, &g.out2_fmt, &g.out2_f, &g.out2_hi, &g.out2_lo);
+  g.ld = gc.ldg;
+  g.mat_stride = gc.m * gc.ldg;
+  pr.amap = pr.bmap = gc.map;
+  return pr;
+}
+
 enum Product { PROD_R, PROD_T, PROD_P, PROD_G };
 
 // Operands and epilogue of one product of step k for class c (R-form):
 //   R = bG + c(GG),  T = aG + RG,  P' = aP + RP (P0 = aI + R),  G' = aT + TR
-Prob product(dmu_plan p, int c, Product what, int k, const float co[3], int p_in, int p_out) {
+Prob product(dmu_plan p, int c, Product what, int k, bool last, const float co[3], int p_in, int p_out) {
   const GClass& gc = p->classes[c];
-  int na, nb, terms;
-  prec_shape(gc.prec, &na, &nb, &terms);
+  int na, nb, terms, kind;
+  prec_shape(gc.prec, &na, &nb, &terms, &kind);
+  if (kind == KIND_TF32) {
+    const int fin = p_in == 0 ? FSLOT_PA : FSLOT_PB, fout = p_out == 0 ? FSLOT_PA : FSLOT_PB;
+    switch (what) {
+      case PROD_R:
+        return gram_prob_f32(p, c, FSLOT_G, FSLOT_G, co[2], co[1], FSLOT_G, FSLOT_R,
+                             k == 0 ? (last ? OUT_PF : FSLOT_PA) : -1, co[0]);
+      case PROD_T:
+        return gram_prob_f32(p, c, FSLOT_R, FSLOT_G, 1.f, co[0], FSLOT_G, FSLOT_T, -1, 0.f);
+      case PROD_P:
+        return gram_prob_f32(p, c, FSLOT_R, fin, 1.f, co[0], fin, last ? OUT_PF : fout, -1, 0.f);
+      case PROD_G:
+      default:
+        return gram_prob_f32(p, c, FSLOT_T, FSLOT_R, 1.f, co[0], FSLOT_T, FSLOT_G, -1, 0.f);
+    }
+  }
   const bool r_lo = gc.prec != DMU_PREC_FAST;
   const int PA = SLOT_PA_HI, PB = SLOT_PB_HI;
   const int pin = p_in == 0 ? PA : PB, pout = p_out == 0 ? PA : PB;
@@ -311,20 +379,20 @@ Prob product(dmu_plan p, int c, Product what, int k, const float co[3], int p_in
 
 // Run one or two kinds of product for every class, one grouped launch per
 // precision group.
-dmu_status run_products(dmu_plan p, const std::vector<std::pair<Product, bool>>& kinds, int k,
+dmu_status run_products(dmu_plan p, const std::vector<std::pair<Product, bool>>& kinds, int k, bool last,
                         const float co[3], int p_in, int p_out, cudaStream_t s) {
-  const int precs[3] = {DMU_PREC_FAST, DMU_PREC_SPLIT2, DMU_PREC_SPLIT3};
+  const int precs[4] = {DMU_PREC_TF32, DMU_PREC_FAST, DMU_PREC_SPLIT2, DMU_PREC_SPLIT3};
   for (int pr : precs) {
     std::vector<Prob> probs;
     for (size_t c = 0; c < p->classes.size(); ++c) {
       if (p->classes[c].prec != pr) continue;
       for (auto& kd : kinds)
-        if (kd.second) probs.push_back(product(p, (int)c, kd.first, k, co, p_in, p_out));
+        if (kd.second) probs.push_back(product(p, (int)c, kd.first, k, last, co, p_in, p_out));
     }
     if (probs.empty()) continue;
-    int na, nb, terms;
-    prec_shape(pr, &na, &nb, &terms);
-    dmu_status st = run_tc(p, probs, na, nb, s);
+    int na, nb, terms, kind;
+    prec_shape(pr, &na, &nb, &terms, &kind);
+    dmu_status st = run_tc(p, probs, na, nb, kind, s);
     if (st != DMU_OK) return st;
   }
   return DMU_OK;
@@ -351,20 +419,27 @@ dmu_status gram_bf16(dmu_plan p, const float co[3], int steps, cudaStream_t s) {
     g.inv = p->inv_dev();
     g.inv_base = b.first_slot;
     const size_t moff = (size_t)b.cls_off * gc.m * gc.ldg;
-    g.out_hi = p->slot_bf16(b.cls, SLOT_G_HI) + moff;
-    g.out_lo = p->slot_bf16(b.cls, SLOT_G_LO) + moff;
+    if (gc.kind == KIND_TF32) {
+      g.out_fmt = FMT_F32;
+      g.out_f = p->slot_f32(b.cls, FSLOT_G) + moff;
+    } else {
+      g.out_hi = p->slot_bf16(b.cls, SLOT_G_HI) + moff;
+      g.out_lo = p->slot_bf16(b.cls, SLOT_G_LO) + moff;
+    }
     g.ld = gc.ldg;
     g.mat_stride = gc.m * gc.ldg;
     pr.amap = pr.bmap = b.tall ? b.map_mn : b.map_k;
     syrk.push_back(pr);
   }
-  dmu_status st = run_tc(p, syrk, 1, 1, s);
+  dmu_status st = run_tc(p, syrk, 1, 1, KIND_BF16, s);
   if (st != DMU_OK) return st;
 
   if (steps == 0) {
     for (size_t c = 0; c < p->classes.size(); ++c) {
       const GClass& gc = p->classes[c];
-      CUDA_TRY(launch_identity_bf16(p->slot_bf16((int)c, SLOT_PA_HI), p->slot_bf16((int)c, SLOT_PA_LO),
+      const bool tf = gc.kind == KIND_TF32;
+      CUDA_TRY(launch_identity_bf16(tf ? p->pf_bf16((int)c, 0) : p->slot_bf16((int)c, SLOT_PA_HI),
+                                    tf ? p->pf_bf16((int)c, 1) : p->slot_bf16((int)c, SLOT_PA_LO),
                                     gc.count, (int)gc.m, gc.ldg, gc.m * gc.ldg, s));
       p->launches++;
     }
@@ -374,14 +449,14 @@ dmu_status gram_bf16(dmu_plan p, const float co[3], int steps, cudaStream_t s) {
   int p_cur = 0;  // P_k lives in buffer p_cur (after step 0: buffer A)
   for (int k = 0; k < steps; ++k) {
     const bool last = (k == steps - 1);
-    st = run_products(p, {{PROD_R, true}}, k, co, 0, 0, s);
+    st = run_products(p, {{PROD_R, true}}, k, last, co, 0, 0, s);
     if (st != DMU_OK) return st;
     const int p_next = (k == 0) ? 0 : 1 - p_cur;
-    st = run_products(p, {{PROD_T, !last}, {PROD_P, k >= 1}}, k, co, p_cur, p_next, s);
+    st = run_products(p, {{PROD_T, !last}, {PROD_P, k >= 1}}, k, last, co, p_cur, p_next, s);
     if (st != DMU_OK) return st;
     p_cur = p_next;
     if (!last) {
-      st = run_products(p, {{PROD_G, true}}, k, co, 0, 0, s);
+      st = run_products(p, {{PROD_G, true}}, k, last, co, 0, 0, s);
       if (st != DMU_OK) return st;
     }
   }
@@ -497,14 +572,15 @@ dmu_status run_normalize(dmu_plan p, int tbl, bool with_mom, float beta, float e
 }
 
 dmu_status encode_map(CUtensorMap* map, void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
-                      uint64_t s2, uint32_t box0, uint32_t box1) {
+                      uint64_t s2, uint32_t box0, uint32_t box1,
+                      CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   auto enc = get_encode();
   if (!enc) return fail(DMU_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
   cuuint64_t dims[3] = {d0, d1, d2};
   cuuint64_t strides[2] = {s1, s2};
   cuuint32_t box[3] = {box0, box1, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+  CUresult r = enc(map, dt, 3, base, dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(DMU_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
@@ -528,7 +604,7 @@ dmu_status dmu_plan_create(const dmu_shape* shapes, int count, dmu_dtype dtype, 
   if (!shapes) return fail(DMU_ERR_INVALID_ARG, "shapes is NULL");
   if (count <= 0) return fail(DMU_ERR_INVALID_ARG, "count must be positive");
   if (dtype != DMU_BF16 && dtype != DMU_F32) return fail(DMU_ERR_INVALID_ARG, "unknown dtype");
-  if (prec < DMU_PREC_AUTO || prec > DMU_PREC_SPLIT3) return fail(DMU_ERR_INVALID_ARG, "unknown precision");
+  if (prec < DMU_PREC_AUTO || prec > DMU_PREC_TF32) return fail(DMU_ERR_INVALID_ARG, "unknown precision");
   for (int i = 0; i < count; ++i) {
     if (shapes[i].rows <= 0 || shapes[i].cols <= 0)
       return fail(DMU_ERR_INVALID_ARG, "non-positive extent at matrix " + std::to_string(i));
@@ -584,9 +660,10 @@ dmu_status dmu_plan_create(const dmu_shape* shapes, int count, dmu_dtype dtype, 
         g.ldg = dtype == DMU_BF16 ? round_up64(b.m, 8) : b.m;
         if (dtype == DMU_BF16) {
           if (prec == DMU_PREC_AUTO)
-            g.prec = b.m >= 1024 ? DMU_PREC_FAST : DMU_PREC_SPLIT3;
+            g.prec = b.m >= 1024 ? DMU_PREC_TF32 : DMU_PREC_SPLIT3;
           else
             g.prec = prec;
+          g.kind = g.prec == DMU_PREC_TF32 ? KIND_TF32 : KIND_BF16;
         }
         cidx[b.m] = (int)p->classes.size();
         p->classes.push_back(g);
@@ -653,10 +730,18 @@ dmu_status dmu_plan_create(const dmu_shape* shapes, int count, dmu_dtype dtype, 
   p->off_mb = off;
   off = align_up(off + p->esize * (size_t)mb_elems, 1024);
   p->off_gram = off;
-  const int nslots = dtype == DMU_BF16 ? NUM_SLOTS : NUM_FSLOTS;
   for (GClass& g : p->classes) {
     g.off = off;
-    off = align_up(off + p->esize * (size_t)nslots * g.count * g.m * g.ldg, 1024);
+    const size_t elems = (size_t)g.count * g.m * g.ldg;
+    if (dtype == DMU_F32) {
+      off = align_up(off + 4 * (size_t)NUM_FSLOTS * elems, 1024);
+    } else if (g.kind == KIND_TF32) {
+      off = align_up(off + 4 * (size_t)NUM_FSLOTS * elems, 1024);
+      g.off_pf = off;
+      off = align_up(off + 2 * 2 * elems, 1024);
+    } else {
+      off = align_up(off + 2 * (size_t)NUM_SLOTS * elems, 1024);
+    }
   }
   p->total = off;
   *out = p;
@@ -702,12 +787,28 @@ dmu_status dmu_set_workspace(dmu_plan p, void* dev_ptr, size_t bytes) {
     }
     for (GClass& g : p->classes) {
       CUtensorMap mg;
-      const uint64_t s1 = (uint64_t)g.ldg * 2, s2 = (uint64_t)g.m * g.ldg * 2;
-      st = encode_map(&mg, p->ws + g.off, (uint64_t)g.m, (uint64_t)g.m, (uint64_t)NUM_SLOTS * g.count, s1, s2,
-                      64, 128);
-      if (st != DMU_OK) return st;
-      g.map = (int)p->maps.size();
-      p->maps.push_back(mg);
+      if (g.kind == KIND_TF32) {
+        const uint64_t s1 = (uint64_t)g.ldg * 4, s2 = (uint64_t)g.m * g.ldg * 4;
+        st = encode_map(&mg, p->ws + g.off, (uint64_t)g.m, (uint64_t)g.m, (uint64_t)NUM_FSLOTS * g.count, s1,
+                        s2, 32, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
+        if (st != DMU_OK) return st;
+        g.map = (int)p->maps.size();
+        p->maps.push_back(mg);
+        CUtensorMap mp;
+        const uint64_t t1 = (uint64_t)g.ldg * 2, t2 = (uint64_t)g.m * g.ldg * 2;
+        st = encode_map(&mp, p->ws + g.off_pf, (uint64_t)g.m, (uint64_t)g.m, (uint64_t)2 * g.count, t1, t2, 64,
+                        128);
+        if (st != DMU_OK) return st;
+        g.map_pf = (int)p->maps.size();
+        p->maps.push_back(mp);
+      } else {
+        const uint64_t s1 = (uint64_t)g.ldg * 2, s2 = (uint64_t)g.m * g.ldg * 2;
+        st = encode_map(&mg, p->ws + g.off, (uint64_t)g.m, (uint64_t)g.m, (uint64_t)NUM_SLOTS * g.count, s1,
+                        s2, 64, 128);
+        if (st != DMU_OK) return st;
+        g.map = (int)p->maps.size();
+        p->maps.push_back(mg);
+      }
     }
   }
   return DMU_OK;
@@ -797,8 +898,13 @@ dmu_status dmu_apply_update(dmu_plan p, void* const* weights, float lr, float* c
       g.sym = 0;
       g.tiles_per_mat = tiles_for(g.M, g.N, false, &g.tiles_m, &g.tiles_n);
       g.a_mn = 0;
-      g.a_z[0] = pf_hi * gc.count + b.cls_off;
-      g.a_z[1] = (pf_hi + 1) * gc.count + b.cls_off;
+      if (gc.kind == KIND_TF32) {
+        g.a_z[0] = b.cls_off;
+        g.a_z[1] = gc.count + b.cls_off;
+      } else {
+        g.a_z[0] = pf_hi * gc.count + b.cls_off;
+        g.a_z[1] = (pf_hi + 1) * gc.count + b.cls_off;
+      }
       g.b_mn = b.tall ? 0 : 1;
       g.terms = TERM_HH | TERM_LH;
       g.epi = EPI_UPDATE;
@@ -811,11 +917,11 @@ dmu_status dmu_apply_update(dmu_plan p, void* const* weights, float lr, float* c
       g.w_f32 = 0;
       g.w_transposed = b.tall ? 1 : 0;
       g.w_cols = b.cols;
-      pr.amap = gc.map;
+      pr.amap = gc.kind == KIND_TF32 ? gc.map_pf : gc.map;
       pr.bmap = b.tall ? b.map_k : b.map_mn;
       probs.push_back(pr);
     }
-    return run_tc(p, probs, 2, 1, s);
+    return run_tc(p, probs, 2, 1, KIND_BF16, s);
   }
   const int pf = p->p_final == 0 ? FSLOT_PA : FSLOT_PB;
   for (const Bucket& b : p->buckets) {
@@ -909,7 +1015,14 @@ dmu_status dmu_debug_gram(dmu_plan p, int which, int index, float* out, void* st
   const size_t moff = (size_t)(bk->cls_off + local) * gc.m * gc.ldg;
   int q = which;
   if (which == 7) q = p->p_final == 0 ? 3 : 4;
-  if (p->dtype == DMU_BF16) {
+  if (p->dtype == DMU_BF16 && gc.kind == KIND_TF32) {
+    if (which == 7) {
+      CUDA_TRY(launch_pair_to_f32(p->pf_bf16(bk->cls, 0) + moff, p->pf_bf16(bk->cls, 1) + moff, gc.m, gc.m,
+                                  gc.ldg, out, s));
+    } else {
+      CUDA_TRY(launch_f32_copy2d(p->slot_f32(bk->cls, q) + moff, gc.m, gc.m, gc.ldg, out, s));
+    }
+  } else if (p->dtype == DMU_BF16) {
     const int slots[5] = {SLOT_G_HI, SLOT_R_HI, SLOT_T_HI, SLOT_PA_HI, SLOT_PB_HI};
     const int sh = slots[q];
     const bool has_lo = !(sh == SLOT_R_HI && gc.prec == DMU_PREC_FAST);

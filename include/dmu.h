@@ -85,16 +85,23 @@ typedef enum {
 
 /* Precision of the Gram-space products on the bf16 path.  Gram-space
  * matrices are always stored as a bf16 pair (hi, lo = bf16(x - hi)) and
- * the final P X0 product always uses both halves of P.
- *   FAST   : one bf16 MMA per product (hi x hi).
- *   SPLIT2 : two MMAs per product (hi x hi + lo x hi).
- *   SPLIT3 : three MMAs per product (hi x hi + hi x lo + lo x hi).
- *   AUTO   : FAST for m >= 1024, SPLIT3 below (per shape bucket). */
+ * the final P X0 product always uses both halves of P.  Each symmetric
+ * product is computed on its upper-triangle tiles and mirrored, which
+ * turns the antisymmetric part of the operand rounding error into a
+ * symmetric one; with one bf16 MMA per product that error shifts the small
+ * eigenvalues of G enough to miss 2e-2 on spiked inputs, so:
+ *   FAST   : one bf16 MMA per product (hi x hi)        -- low precision;
+ *   SPLIT2 : two MMAs per product (hi x hi + lo x hi)  -- low precision;
+ *   SPLIT3 : three MMAs per product (hi x hi + hi x lo + lo x hi);
+ *   TF32   : Gram-space state in fp32, one kind::tf32 MMA per product
+ *            (half the bf16 rate; 10-bit operand mantissa);
+ *   AUTO   : TF32 for m >= 1024, SPLIT3 below (per Gram class). */
 typedef enum {
   DMU_PREC_AUTO = 0,
   DMU_PREC_FAST = 1,
   DMU_PREC_SPLIT2 = 2,
-  DMU_PREC_SPLIT3 = 3
+  DMU_PREC_SPLIT3 = 3,
+  DMU_PREC_TF32 = 4
 } dmu_prec;
 
 /* Bits of the device status word (dmu_read_status). */
