@@ -43,10 +43,12 @@ enum Terms : int { TERM_HH = 1, TERM_HL = 2, TERM_LH = 4 };
 // Operand kind of a tensor-core launch: bf16 (kind::f16, K = 16 per MMA)
 // or tf32 (kind::tf32 on fp32 storage, K = 8 per MMA).  Either way a
 // K-block is one 128-byte swizzle row: 64 bf16 or 32 fp32 elements.
-enum MmaKind : int { KIND_BF16 = 0, KIND_TF32 = 1 };
+enum MmaKind : int { KIND_BF16 = 0, KIND_TF32 = 1, KIND_F16 = 2 };
 
-// Storage format of an epilogue input/output matrix.
-enum Fmt : int { FMT_PAIR = 0, FMT_F32 = 1 };
+// Storage format of an epilogue input/output matrix: bf16 hi/lo pair,
+// fp32, or fp16 hi/lo pair (values pre-scaled by a power of two chosen by
+// the planner so fp16's exponent range holds them).
+enum Fmt : int { FMT_PAIR = 0, FMT_F32 = 1, FMT_PAIR_H = 2 };
 
 // One grouped-GEMM problem: `count` independent matrices of the same
 // geometry.  Output tile (bi, bj) of matrix `mat` is
@@ -77,6 +79,7 @@ struct GemmProblem {
   long long ld;            // row stride (elements) of Cin/out
   long long mat_stride;    // matrix stride (elements) of Cin/out
   int cin_fmt, out_fmt, out2_fmt;  // Fmt of Cin, out, out2
+  float scale2;            // out2 = scale2 * out + gamma2 * I
   const float* cin_f;      // FMT_F32 variants of Cin / out / out2
   float* out_f;
   float* out2_f;
@@ -148,6 +151,8 @@ cudaError_t launch_identity_f32(float* p, int count, int m, long long ld, long l
                                 cudaStream_t s);
 cudaError_t launch_pair_to_f32(const __nv_bfloat16* hi, const __nv_bfloat16* lo, long long rows,
                                long long cols, long long ld, float* out, cudaStream_t s);
+cudaError_t launch_pair_h_to_f32(const void* hi, const void* lo, long long rows, long long cols, long long ld,
+                                 float scale, float* out, cudaStream_t s);
 cudaError_t launch_f32_copy2d(const float* src, long long rows, long long cols, long long ld,
                               float* out, cudaStream_t s);
 

@@ -24,6 +24,8 @@
 // and of B; the problem's term bits choose hi*hi, hi*lo, lo*hi.
 // Every mbarrier wait is bounded by a wall-clock limit; on expiry the CTA
 // sets DMU_FLAG_TIMEOUT in the status word and winds down.
+#include <cuda_fp16.h>
+
 #include "dmu_internal.h"
 #include "ptx.cuh"
 
@@ -119,6 +121,35 @@ __device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
   }
 }
 
+__device__ __forceinline__ void unpack8_h(const uint4& u, float* f) {
+  const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    float2 t = __half22float2(h[q]);
+    f[2 * q] = t.x;
+    f[2 * q + 1] = t.y;
+  }
+}
+
+__device__ __forceinline__ void split8_h(const float* v, uint4& hi, uint4& lo) {
+  __half2* h = reinterpret_cast<__half2*>(&hi);
+  __half2* l = reinterpret_cast<__half2*>(&lo);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    __half h0 = __float2half_rn(v[2 * q]);
+    __half h1 = __float2half_rn(v[2 * q + 1]);
+    h[q] = __halves2half2(h0, h1);
+    l[q] = __halves2half2(__float2half_rn(v[2 * q] - __half2float(h0)),
+                          __float2half_rn(v[2 * q + 1] - __half2float(h1)));
+  }
+}
+
+__device__ __forceinline__ void store_pair_h(__half* hi, __half* lo, long long off, float v) {
+  __half h = __float2half_rn(v);
+  hi[off] = h;
+  if (lo) lo[off] = __float2half_rn(v - __half2float(h));
+}
+
 // Store value v at (i, j) of a hi/lo pair.
 __device__ __forceinline__ void store_pair(__nv_bfloat16* hi, __nv_bfloat16* lo, long long off,
                                            float v) {
@@ -165,6 +196,32 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
       for (int c = 0; c < 32; ++c)
         if (col0 + c < N) v[c] += pr.beta * pr.cin_f[rowoff + col0 + c];
     }
+  } else if (pr.cin_fmt == FMT_PAIR_H && pr.cin_hi) {
+    const __half* ch = reinterpret_cast<const __half*>(pr.cin_hi);
+    const __half* cl = reinterpret_cast<const __half*>(pr.cin_lo);
+    if (full) {
+      const uint4* ph = reinterpret_cast<const uint4*>(ch + rowoff + col0);
+      const uint4* pl = reinterpret_cast<const uint4*>(cl + rowoff + col0);
+      uint4 uh[4], ul[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uh[q] = ph[q];
+        ul[q] = pl[q];
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float fh[8], fl[8];
+        unpack8_h(uh[q], fh);
+        unpack8_h(ul[q], fl);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[8 * q + e] += pr.beta * (fh[e] + fl[e]);
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (col0 + c < N)
+          v[c] += pr.beta * (__half2float(ch[rowoff + col0 + c]) + __half2float(cl[rowoff + col0 + c]));
+    }
   } else if (pr.cin_fmt == FMT_PAIR && pr.cin_hi) {
     if (full) {
       const uint4* ph = reinterpret_cast<const uint4*>(pr.cin_hi + rowoff + col0);
@@ -202,10 +259,40 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
 
   for (int pass = 0; pass < 2; ++pass) {
     const int fmt = pass == 0 ? pr.out_fmt : pr.out2_fmt;
-    if (pass == 1 && dc >= 0 && dc < 32) {
+    if (pass == 1) {
+      if (!pr.out2_hi && !pr.out2_f) break;
 #pragma unroll
-      for (int c = 0; c < 32; ++c)
-        if (c == dc) v[c] += pr.gamma2;
+      for (int c = 0; c < 32; ++c) v[c] = v[c] * pr.scale2 + (c == dc ? pr.gamma2 : 0.f);
+    }
+    if (fmt == FMT_PAIR_H) {
+      __half* oh = reinterpret_cast<__half*>(pass == 0 ? pr.out_hi : pr.out2_hi);
+      __half* ol = reinterpret_cast<__half*>(pass == 0 ? pr.out_lo : pr.out2_lo);
+      if (!oh) continue;
+      if (full && all_upper) {
+        uint4* dh = reinterpret_cast<uint4*>(oh + rowoff + col0);
+        uint4* dl = ol ? reinterpret_cast<uint4*>(ol + rowoff + col0) : nullptr;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 h, l;
+          split8_h(v + 8 * q, h, l);
+          dh[q] = h;
+          if (dl) dl[q] = l;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int j = col0 + c;
+          if (j < N && (!pr.sym || i <= j)) store_pair_h(oh, ol, rowoff + j, v[c]);
+        }
+      }
+      if (pr.sym) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int j = col0 + c;
+          if (j < N && i < j) store_pair_h(oh, ol, mbase + (long long)j * pr.ld + i, v[c]);
+        }
+      }
+      continue;
     }
     if (fmt == FMT_F32) {
       float* of = pass == 0 ? pr.out_f : pr.out2_f;
@@ -265,7 +352,9 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
 
 // One 32-column chunk of the final O = P X0 tile, fused with the update.
 // Row i of the tile is row i of O (m x n); element (i, j) lives at W[i][j]
-// for a wide matrix and at W[j][i] for a tall one (w_transposed).
+// for a wide matrix and at W[j][i] for a tall one (w_transposed).  All W
+// loads of the chunk are issued before any store, so they overlap instead
+// of serialising behind stores the compiler cannot prove independent.
 __device__ __forceinline__ void epi_update_chunk(const GemmProblem& pr, int mat, int i, int col0,
                                                  const uint32_t (&r)[32]) {
   const int M = pr.M, N = pr.N;
@@ -278,19 +367,22 @@ __device__ __forceinline__ void epi_update_chunk(const GemmProblem& pr, int mat,
   void* wp = pr.w_ptrs ? pr.w_ptrs[pr.ptr_base + mat] : nullptr;
   float* op = pr.o_ptrs ? pr.o_ptrs[pr.ptr_base + mat] : nullptr;
   const long long wc = pr.w_cols;
+  const bool full = (col0 + 32 <= N);
   if (!pr.w_transposed) {
     const long long rowoff = (long long)i * wc;
-    const bool full = (col0 + 32 <= N);
     if (wp) {
       if (!pr.w_f32) {
         __nv_bfloat16* w = reinterpret_cast<__nv_bfloat16*>(wp);
         const bool vec = full && ((wc & 7) == 0) && ((reinterpret_cast<uintptr_t>(w) & 15) == 0);
         if (vec) {
           uint4* pw = reinterpret_cast<uint4*>(w + rowoff + col0);
+          uint4 wv[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) wv[q] = pw[q];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             float f[8];
-            unpack8(pw[q], f);
+            unpack8(wv[q], f);
             uint4 h;
             __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&h);
 #pragma unroll
@@ -300,18 +392,21 @@ __device__ __forceinline__ void epi_update_chunk(const GemmProblem& pr, int mat,
             pw[q] = h;
           }
         } else {
+          float wv[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) wv[c] = (col0 + c < N) ? bf2f(w[rowoff + col0 + c]) : 0.f;
 #pragma unroll
           for (int c = 0; c < 32; ++c)
-            if (col0 + c < N) {
-              long long off = rowoff + col0 + c;
-              w[off] = __float2bfloat16_rn(bf2f(w[off]) + cw * o[c]);
-            }
+            if (col0 + c < N) w[rowoff + col0 + c] = __float2bfloat16_rn(wv[c] + cw * o[c]);
         }
       } else {
         float* w = reinterpret_cast<float*>(wp);
+        float wv[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) wv[c] = (col0 + c < N) ? w[rowoff + col0 + c] : 0.f;
 #pragma unroll
         for (int c = 0; c < 32; ++c)
-          if (col0 + c < N) w[rowoff + col0 + c] += cw * o[c];
+          if (col0 + c < N) w[rowoff + col0 + c] = wv[c] + cw * o[c];
       }
     }
     if (op) {
@@ -320,21 +415,25 @@ __device__ __forceinline__ void epi_update_chunk(const GemmProblem& pr, int mat,
         if (col0 + c < N) op[rowoff + col0 + c] = s * o[c];
     }
   } else {
-    // W is n x m (rows = N here, cols = M); element (i, j) -> W[j][i].
+    // W is n x m (rows = N here, cols = M); element (i, j) -> W[j][i]; each
+    // store instruction of the warp covers 32 consecutive columns of a row.
     if (wp) {
       if (!pr.w_f32) {
         __nv_bfloat16* w = reinterpret_cast<__nv_bfloat16*>(wp);
+        float wv[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) wv[c] = (col0 + c < N) ? bf2f(w[(long long)(col0 + c) * wc + i]) : 0.f;
 #pragma unroll
         for (int c = 0; c < 32; ++c)
-          if (col0 + c < N) {
-            long long off = (long long)(col0 + c) * wc + i;
-            w[off] = __float2bfloat16_rn(bf2f(w[off]) + cw * o[c]);
-          }
+          if (col0 + c < N) w[(long long)(col0 + c) * wc + i] = __float2bfloat16_rn(wv[c] + cw * o[c]);
       } else {
         float* w = reinterpret_cast<float*>(wp);
+        float wv[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) wv[c] = (col0 + c < N) ? w[(long long)(col0 + c) * wc + i] : 0.f;
 #pragma unroll
         for (int c = 0; c < 32; ++c)
-          if (col0 + c < N) w[(long long)(col0 + c) * wc + i] += cw * o[c];
+          if (col0 + c < N) w[(long long)(col0 + c) * wc + i] = wv[c] + cw * o[c];
       }
     }
     if (op) {
@@ -350,6 +449,7 @@ template <int NA, int NB, int KIND>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_constant__ GemmParams p) {
   using Cfg = TcCfg<NA, NB>;
   constexpr int BKE = KIND == KIND_TF32 ? 32 : 64;  // elements per 128-byte K-block row
+  constexpr int OPFMT = KIND == KIND_TF32 ? 2 : (KIND == KIND_F16 ? 0 : 1);  // idesc A/B format code
   constexpr int S = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = ptx::smem_u32(smem_raw);
@@ -481,7 +581,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
         const TileCoord tc = decode_tile(p, t);
         const GemmProblem& pr = p.prob[tc.pi];
         const int nk = (pr.K + BKE - 1) / BKE;
-        const uint32_t idesc = ptx::make_idesc(BM, BN, pr.a_mn, pr.b_mn, KIND == KIND_TF32 ? 2 : 1);
+        const uint32_t idesc = ptx::make_idesc(BM, BN, pr.a_mn, pr.b_mn, OPFMT);
         if (!wait_bar(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p)) {
           ok = false;
           break;
@@ -630,6 +730,7 @@ cudaError_t gemm_tc_configure() {
   if ((e = configure_one<2, 1, KIND_BF16>()) != cudaSuccess) return e;
   if ((e = configure_one<2, 2, KIND_BF16>()) != cudaSuccess) return e;
   if ((e = configure_one<1, 1, KIND_TF32>()) != cudaSuccess) return e;
+  if ((e = configure_one<1, 1, KIND_F16>()) != cudaSuccess) return e;
   return cudaSuccess;
 }
 
@@ -651,6 +752,10 @@ static cudaError_t launch_one(const GemmParams& p, int num_sms, cudaStream_t s) 
 cudaError_t launch_gemm_tc(const GemmParams& p, int na, int nb, int kind, int num_sms, cudaStream_t s) {
   if (kind == KIND_TF32) {
     if (na == 1 && nb == 1) return launch_one<1, 1, KIND_TF32>(p, num_sms, s);
+    return cudaErrorInvalidValue;
+  }
+  if (kind == KIND_F16) {
+    if (na == 1 && nb == 1) return launch_one<1, 1, KIND_F16>(p, num_sms, s);
     return cudaErrorInvalidValue;
   }
   if (na == 1 && nb == 1) return launch_one<1, 1, KIND_BF16>(p, num_sms, s);

@@ -8,6 +8,8 @@
 //   * k_simt_gemm: the fp32 FFMA path (exact fp32 products) with the same
 //     epilogues as the tensor-core kernel, used for fp32 plans;
 //   * small helpers: identity P, hi/lo -> fp32 conversion for test hooks.
+#include <cuda_fp16.h>
+
 #include "dmu_internal.h"
 
 namespace dmu {
@@ -179,6 +181,16 @@ __global__ void k_pair_to_f32(const __nv_bfloat16* hi, const __nv_bfloat16* lo, 
   }
 }
 
+__global__ void k_pair_h_to_f32(const __half* hi, const __half* lo, long long rows, long long cols,
+                                long long ld, float scale, float* out) {
+  const long long total = rows * cols;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+       e += (long long)gridDim.x * blockDim.x) {
+    const long long r = e / cols, c = e % cols;
+    out[e] = (__half2float(hi[r * ld + c]) + __half2float(lo[r * ld + c])) * scale;
+  }
+}
+
 __global__ void k_f32_copy2d(const float* src, long long rows, long long cols, long long ld, float* out) {
   const long long total = rows * cols;
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
@@ -208,6 +220,13 @@ cudaError_t launch_identity_f32(float* p, int count, int m, long long ld, long l
 cudaError_t launch_pair_to_f32(const __nv_bfloat16* hi, const __nv_bfloat16* lo, long long rows,
                                long long cols, long long ld, float* out, cudaStream_t s) {
   k_pair_to_f32<<<grid_for(rows * cols), 256, 0, s>>>(hi, lo, rows, cols, ld, out);
+  return cudaGetLastError();
+}
+cudaError_t launch_pair_h_to_f32(const void* hi, const void* lo, long long rows, long long cols, long long ld,
+                                 float scale, float* out, cudaStream_t s) {
+  k_pair_h_to_f32<<<grid_for(rows * cols), 256, 0, s>>>(reinterpret_cast<const __half*>(hi),
+                                                        reinterpret_cast<const __half*>(lo), rows, cols, ld, scale,
+                                                        out);
   return cudaGetLastError();
 }
 cudaError_t launch_f32_copy2d(const float* src, long long rows, long long cols, long long ld, float* out,

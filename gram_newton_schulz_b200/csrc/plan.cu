@@ -248,6 +248,7 @@ void prec_shape(int prec, int* na, int* nb, int* terms, int* kind) {
     case DMU_PREC_SPLIT2: *na = 2; *nb = 1; *terms = TERM_HH | TERM_LH; break;
     case DMU_PREC_SPLIT3: *na = 2; *nb = 2; *terms = TERM_HH | TERM_HL | TERM_LH; break;
     case DMU_PREC_TF32: *na = 1; *nb = 1; *terms = TERM_HH; *kind = KIND_TF32; break;
+    case DMU_PREC_F16: *na = 1; *nb = 1; *terms = TERM_HH; *kind = KIND_F16; break;
     default: *na = 1; *nb = 1; *terms = TERM_HH; break;
   }
 }
@@ -276,6 +277,7 @@ Prob gram_prob(dmu_plan p, int c, int a_slot, int b_slot, int terms, float alpha
   g.beta = beta;
   g.gamma = 0.f;
   g.gamma2 = gamma2;
+  g.scale2 = 1.f;
   if (cin_slot >= 0) {
     g.cin_hi = p->slot_bf16(c, cin_slot);
     g.cin_lo = p->slot_bf16(c, cin_slot + 1);
@@ -325,10 +327,71 @@ Prob gram_prob_f32(dmu_plan p, int c, int a_slot, int b_slot, float alpha, float
   g.alpha = alpha;
   g.beta = beta;
   g.gamma2 = gamma2;
+  g.scale2 = 1.f;
   g.cin_fmt = FMT_F32;
   if (cin_slot >= 0) g.cin_f = p->slot_f32(c, cin_slot);
   set_f32_out(p, c, out_slot, &g.out_fmt, &g.out_f, &g.out_hi, &g.out_lo);
   set_f32_out(p, c, out2_slot, &g.out2_fmt, &g.out2_f, &g.out2_hi, &g.out2_lo);
+  g.ld = gc.ldg;
+  g.mat_stride = gc.m * gc.ldg;
+  pr.amap = pr.bmap = gc.map;
+  return pr;
+}
+
+// F16 classes: every Gram-space quantity is stored as an fp16 hi/lo pair
+// pre-scaled by a power of two so its entries sit well inside fp16's
+// normal range: G, R, T by 2^8 (their entries are O(1/m)), P by 1 (its
+// eigenvalues reach ~500).  The scales are folded exactly into the
+// epilogue coefficients.  The final P is written as a bf16 pair (unscaled)
+// because the final GEMM multiplies it with the bf16 image of M.
+float half_slot_scale(int slot) { return slot >= SLOT_PA_HI ? 1.f : 256.f; }
+
+void set_h_out(dmu_plan p, int c, int slot, int* fmt, __nv_bfloat16** hi, __nv_bfloat16** lo, float* scale) {
+  if (slot == OUT_PF) {
+    *fmt = FMT_PAIR;
+    *hi = p->pf_bf16(c, 0);
+    *lo = p->pf_bf16(c, 1);
+    *scale = 1.f;
+  } else if (slot >= 0) {
+    *fmt = FMT_PAIR_H;
+    *hi = p->slot_bf16(c, slot);  // fp16 bits; same element size as bf16
+    *lo = p->slot_bf16(c, slot + 1);
+    *scale = half_slot_scale(slot);
+  } else {
+    *scale = 1.f;
+  }
+}
+
+Prob gram_prob_h(dmu_plan p, int c, int a_slot, int b_slot, float alpha, float beta, int cin_slot, int out_slot,
+                 int out2_slot, float gamma2) {
+  const GClass& gc = p->classes[c];
+  Prob pr;
+  std::memset(&pr, 0, sizeof(pr));
+  GemmProblem& g = pr.g;
+  g.count = gc.count;
+  g.M = g.N = g.K = (int)gc.m;
+  g.sym = 1;
+  g.tiles_per_mat = tiles_for(g.M, g.N, true, &g.tiles_m, &g.tiles_n);
+  g.a_z[0] = a_slot * gc.count;
+  g.a_z[1] = (a_slot + 1) * gc.count;
+  g.b_z[0] = b_slot * gc.count;
+  g.b_z[1] = (b_slot + 1) * gc.count;
+  g.terms = TERM_HH;
+  g.epi = EPI_GRAM;
+  g.alpha_mode = ALPHA_CONST;
+  float s_out = 1.f, s_out2 = 1.f;
+  set_h_out(p, c, out_slot, &g.out_fmt, &g.out_hi, &g.out_lo, &s_out);
+  set_h_out(p, c, out2_slot, &g.out2_fmt, &g.out2_hi, &g.out2_lo, &s_out2);
+  g.alpha = alpha * s_out / (half_slot_scale(a_slot) * half_slot_scale(b_slot));
+  g.gamma = 0.f;
+  if (cin_slot >= 0) {
+    g.cin_fmt = FMT_PAIR_H;
+    g.cin_hi = p->slot_bf16(c, cin_slot);
+    g.cin_lo = p->slot_bf16(c, cin_slot + 1);
+    g.beta = beta * s_out / half_slot_scale(cin_slot);
+  }
+  g.scale2 = s_out2 / s_out;
+  g.gamma2 = gamma2 * s_out2;
   g.ld = gc.ldg;
   g.mat_stride = gc.m * gc.ldg;
   pr.amap = pr.bmap = gc.map;
@@ -343,6 +406,21 @@ Prob product(dmu_plan p, int c, Product what, int k, bool last, const float co[3
   const GClass& gc = p->classes[c];
   int na, nb, terms, kind;
   prec_shape(gc.prec, &na, &nb, &terms, &kind);
+  if (kind == KIND_F16) {
+    const int hin = p_in == 0 ? SLOT_PA_HI : SLOT_PB_HI, hout = p_out == 0 ? SLOT_PA_HI : SLOT_PB_HI;
+    switch (what) {
+      case PROD_R:
+        return gram_prob_h(p, c, SLOT_G_HI, SLOT_G_HI, co[2], co[1], SLOT_G_HI, SLOT_R_HI,
+                           k == 0 ? (last ? OUT_PF : SLOT_PA_HI) : -1, co[0]);
+      case PROD_T:
+        return gram_prob_h(p, c, SLOT_R_HI, SLOT_G_HI, 1.f, co[0], SLOT_G_HI, SLOT_T_HI, -1, 0.f);
+      case PROD_P:
+        return gram_prob_h(p, c, SLOT_R_HI, hin, 1.f, co[0], hin, last ? OUT_PF : hout, -1, 0.f);
+      case PROD_G:
+      default:
+        return gram_prob_h(p, c, SLOT_T_HI, SLOT_R_HI, 1.f, co[0], SLOT_T_HI, SLOT_G_HI, -1, 0.f);
+    }
+  }
   if (kind == KIND_TF32) {
     const int fin = p_in == 0 ? FSLOT_PA : FSLOT_PB, fout = p_out == 0 ? FSLOT_PA : FSLOT_PB;
     switch (what) {
@@ -381,7 +459,7 @@ Prob product(dmu_plan p, int c, Product what, int k, bool last, const float co[3
 // precision group.
 dmu_status run_products(dmu_plan p, const std::vector<std::pair<Product, bool>>& kinds, int k, bool last,
                         const float co[3], int p_in, int p_out, cudaStream_t s) {
-  const int precs[4] = {DMU_PREC_TF32, DMU_PREC_FAST, DMU_PREC_SPLIT2, DMU_PREC_SPLIT3};
+  const int precs[5] = {DMU_PREC_F16, DMU_PREC_TF32, DMU_PREC_FAST, DMU_PREC_SPLIT2, DMU_PREC_SPLIT3};
   for (int pr : precs) {
     std::vector<Prob> probs;
     for (size_t c = 0; c < p->classes.size(); ++c) {
@@ -422,6 +500,11 @@ dmu_status gram_bf16(dmu_plan p, const float co[3], int steps, cudaStream_t s) {
     if (gc.kind == KIND_TF32) {
       g.out_fmt = FMT_F32;
       g.out_f = p->slot_f32(b.cls, FSLOT_G) + moff;
+    } else if (gc.kind == KIND_F16) {
+      g.out_fmt = FMT_PAIR_H;
+      g.alpha = half_slot_scale(SLOT_G_HI);
+      g.out_hi = p->slot_bf16(b.cls, SLOT_G_HI) + moff;
+      g.out_lo = p->slot_bf16(b.cls, SLOT_G_LO) + moff;
     } else {
       g.out_hi = p->slot_bf16(b.cls, SLOT_G_HI) + moff;
       g.out_lo = p->slot_bf16(b.cls, SLOT_G_LO) + moff;
@@ -437,7 +520,7 @@ dmu_status gram_bf16(dmu_plan p, const float co[3], int steps, cudaStream_t s) {
   if (steps == 0) {
     for (size_t c = 0; c < p->classes.size(); ++c) {
       const GClass& gc = p->classes[c];
-      const bool tf = gc.kind == KIND_TF32;
+      const bool tf = gc.kind != KIND_BF16;  // TF32 / F16 classes keep the final P in the bf16 pair area
       CUDA_TRY(launch_identity_bf16(tf ? p->pf_bf16((int)c, 0) : p->slot_bf16((int)c, SLOT_PA_HI),
                                     tf ? p->pf_bf16((int)c, 1) : p->slot_bf16((int)c, SLOT_PA_LO),
                                     gc.count, (int)gc.m, gc.ldg, gc.m * gc.ldg, s));
@@ -604,7 +687,7 @@ dmu_status dmu_plan_create(const dmu_shape* shapes, int count, dmu_dtype dtype, 
   if (!shapes) return fail(DMU_ERR_INVALID_ARG, "shapes is NULL");
   if (count <= 0) return fail(DMU_ERR_INVALID_ARG, "count must be positive");
   if (dtype != DMU_BF16 && dtype != DMU_F32) return fail(DMU_ERR_INVALID_ARG, "unknown dtype");
-  if (prec < DMU_PREC_AUTO || prec > DMU_PREC_TF32) return fail(DMU_ERR_INVALID_ARG, "unknown precision");
+  if (prec < DMU_PREC_AUTO || prec > DMU_PREC_F16) return fail(DMU_ERR_INVALID_ARG, "unknown precision");
   for (int i = 0; i < count; ++i) {
     if (shapes[i].rows <= 0 || shapes[i].cols <= 0)
       return fail(DMU_ERR_INVALID_ARG, "non-positive extent at matrix " + std::to_string(i));
@@ -660,10 +743,10 @@ dmu_status dmu_plan_create(const dmu_shape* shapes, int count, dmu_dtype dtype, 
         g.ldg = dtype == DMU_BF16 ? round_up64(b.m, 8) : b.m;
         if (dtype == DMU_BF16) {
           if (prec == DMU_PREC_AUTO)
-            g.prec = b.m >= 1024 ? DMU_PREC_TF32 : DMU_PREC_SPLIT3;
+            g.prec = b.m >= 1024 ? DMU_PREC_F16 : DMU_PREC_SPLIT3;
           else
             g.prec = prec;
-          g.kind = g.prec == DMU_PREC_TF32 ? KIND_TF32 : KIND_BF16;
+          g.kind = g.prec == DMU_PREC_TF32 ? KIND_TF32 : (g.prec == DMU_PREC_F16 ? KIND_F16 : KIND_BF16);
         }
         cidx[b.m] = (int)p->classes.size();
         p->classes.push_back(g);
@@ -739,6 +822,10 @@ dmu_status dmu_plan_create(const dmu_shape* shapes, int count, dmu_dtype dtype, 
       off = align_up(off + 4 * (size_t)NUM_FSLOTS * elems, 1024);
       g.off_pf = off;
       off = align_up(off + 2 * 2 * elems, 1024);
+    } else if (g.kind == KIND_F16) {
+      off = align_up(off + 2 * (size_t)NUM_SLOTS * elems, 1024);
+      g.off_pf = off;
+      off = align_up(off + 2 * 2 * elems, 1024);
     } else {
       off = align_up(off + 2 * (size_t)NUM_SLOTS * elems, 1024);
     }
@@ -804,10 +891,19 @@ dmu_status dmu_set_workspace(dmu_plan p, void* dev_ptr, size_t bytes) {
       } else {
         const uint64_t s1 = (uint64_t)g.ldg * 2, s2 = (uint64_t)g.m * g.ldg * 2;
         st = encode_map(&mg, p->ws + g.off, (uint64_t)g.m, (uint64_t)g.m, (uint64_t)NUM_SLOTS * g.count, s1,
-                        s2, 64, 128);
+                        s2, 64, 128,
+                        g.kind == KIND_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
         if (st != DMU_OK) return st;
         g.map = (int)p->maps.size();
         p->maps.push_back(mg);
+        if (g.kind == KIND_F16) {
+          CUtensorMap mp;
+          st = encode_map(&mp, p->ws + g.off_pf, (uint64_t)g.m, (uint64_t)g.m, (uint64_t)2 * g.count, s1, s2, 64,
+                          128);
+          if (st != DMU_OK) return st;
+          g.map_pf = (int)p->maps.size();
+          p->maps.push_back(mp);
+        }
       }
     }
   }
@@ -898,7 +994,7 @@ dmu_status dmu_apply_update(dmu_plan p, void* const* weights, float lr, float* c
       g.sym = 0;
       g.tiles_per_mat = tiles_for(g.M, g.N, false, &g.tiles_m, &g.tiles_n);
       g.a_mn = 0;
-      if (gc.kind == KIND_TF32) {
+      if (gc.kind != KIND_BF16) {
         g.a_z[0] = b.cls_off;
         g.a_z[1] = gc.count + b.cls_off;
       } else {
@@ -917,7 +1013,7 @@ dmu_status dmu_apply_update(dmu_plan p, void* const* weights, float lr, float* c
       g.w_f32 = 0;
       g.w_transposed = b.tall ? 1 : 0;
       g.w_cols = b.cols;
-      pr.amap = gc.kind == KIND_TF32 ? gc.map_pf : gc.map;
+      pr.amap = gc.kind != KIND_BF16 ? gc.map_pf : gc.map;
       pr.bmap = b.tall ? b.map_k : b.map_mn;
       probs.push_back(pr);
     }
@@ -1015,7 +1111,17 @@ dmu_status dmu_debug_gram(dmu_plan p, int which, int index, float* out, void* st
   const size_t moff = (size_t)(bk->cls_off + local) * gc.m * gc.ldg;
   int q = which;
   if (which == 7) q = p->p_final == 0 ? 3 : 4;
-  if (p->dtype == DMU_BF16 && gc.kind == KIND_TF32) {
+  if (p->dtype == DMU_BF16 && gc.kind == KIND_F16) {
+    if (which == 7) {
+      CUDA_TRY(launch_pair_to_f32(p->pf_bf16(bk->cls, 0) + moff, p->pf_bf16(bk->cls, 1) + moff, gc.m, gc.m,
+                                  gc.ldg, out, s));
+    } else {
+      const int slots[5] = {SLOT_G_HI, SLOT_R_HI, SLOT_T_HI, SLOT_PA_HI, SLOT_PB_HI};
+      const int sh = slots[q];
+      CUDA_TRY(launch_pair_h_to_f32(p->slot_bf16(bk->cls, sh) + moff, p->slot_bf16(bk->cls, sh + 1) + moff, gc.m,
+                                    gc.m, gc.ldg, 1.f / half_slot_scale(sh), out, s));
+    }
+  } else if (p->dtype == DMU_BF16 && gc.kind == KIND_TF32) {
     if (which == 7) {
       CUDA_TRY(launch_pair_to_f32(p->pf_bf16(bk->cls, 0) + moff, p->pf_bf16(bk->cls, 1) + moff, gc.m, gc.m,
                                   gc.ldg, out, s));

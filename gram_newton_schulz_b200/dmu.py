@@ -26,7 +26,7 @@ LIB_PATH = os.path.join(_HERE, "_lib", "libdmu.so")
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_NONFINITE, ERR_NOT_PLANNED, ERR_TIMEOUT = range(8)
 STATUS_NAMES = ["OK", "INVALID_ARG", "UNSUPPORTED", "WORKSPACE", "CUDA", "NONFINITE", "NOT_PLANNED", "TIMEOUT"]
 DTYPES = {"bf16": 0, "f32": 1}
-PRECS = {"auto": 0, "fast": 1, "split2": 2, "split3": 3, "tf32": 4}
+PRECS = {"auto": 0, "fast": 1, "split2": 2, "split3": 3, "tf32": 4, "f16": 5}
 FLAG_NONFINITE, FLAG_TIMEOUT = 1, 2
 
 # name -> (restype, argtypes); every symbol of include/dmu.h

@@ -95,13 +95,17 @@ typedef enum {
  *   SPLIT3 : three MMAs per product (hi x hi + hi x lo + lo x hi);
  *   TF32   : Gram-space state in fp32, one kind::tf32 MMA per product
  *            (half the bf16 rate; 10-bit operand mantissa);
- *   AUTO   : TF32 for m >= 1024, SPLIT3 below (per Gram class). */
+ *   F16    : Gram-space state as fp16 hi/lo pairs pre-scaled by powers of
+ *            two, one fp16 MMA per product at the full rate, with the same
+ *            10-bit operand mantissa as TF32;
+ *   AUTO   : F16 for m >= 1024, SPLIT3 below (per Gram class). */
 typedef enum {
   DMU_PREC_AUTO = 0,
   DMU_PREC_FAST = 1,
   DMU_PREC_SPLIT2 = 2,
   DMU_PREC_SPLIT3 = 3,
-  DMU_PREC_TF32 = 4
+  DMU_PREC_TF32 = 4,
+  DMU_PREC_F16 = 5
 } dmu_prec;
 
 /* Bits of the device status word (dmu_read_status). */
@@ -197,6 +201,7 @@ DMU_API int dmu_version(void);
 
 /* Free the host-side plan.  Does not touch the caller's device memory. */
 DMU_API void dmu_plan_destroy(dmu_plan plan);
+
 
 #ifdef __cplusplus
 }
