@@ -672,6 +672,11 @@ dmu_status encode_map(CUtensorMap* map, void* base, uint64_t d0, uint64_t d1, ui
 
 }  // namespace
 
+namespace dmu {
+// Lets entry points defined in other files report through dmu_last_error.
+void set_last_error(const char* msg) { g_err = msg ? msg : ""; }
+}  // namespace dmu
+
 // =================================================================== C ABI
 extern "C" {
 

@@ -44,6 +44,8 @@ SIGNATURES = {
     "dmu_last_error": (ctypes.c_char_p, []),
     "dmu_version": (ctypes.c_int, []),
     "dmu_plan_destroy": (None, [_VP]),
+    "dmu_momentum_norm_static": (ctypes.c_int, [_VP, _VP, _VP, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                                                ctypes.c_float, ctypes.c_float, _VP, _VP]),
 }
 
 

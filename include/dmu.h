@@ -202,6 +202,30 @@ DMU_API int dmu_version(void);
 /* Free the host-side plan.  Does not touch the caller's device memory. */
 DMU_API void dmu_plan_destroy(dmu_plan plan);
 
+/* Momentum + Frobenius norm of ONE matrix without allocating anything.
+ * The pages describe no such call; it exists for callers that cannot
+ * allocate device memory themselves -- a process whose device memory
+ * belongs to another framework's pool, a plugin that may not call the CUDA
+ * allocator, or a hot loop where cudaMalloc/cudaFree would synchronise.
+ * It computes what dmu_momentum_normalize computes for one matrix, with
+ * its scratch (one partial sum per 16384 elements) in a fixed 64 KB
+ * __device__ array inside the library instead of a workspace:
+ *   grad         : device, rows*cols elements of `dtype`;
+ *   momentum     : device fp32 rows*cols, updated in place (M <- beta*M + G);
+ *                  NULL means M = G and nothing is written back;
+ *   image_out    : device, rows*cols of `dtype` receiving M rounded to the
+ *                  dtype (bf16 image for DMU_BF16); may be NULL;
+ *   inv_norm_out : device, one float, receives 1/(||M||_F + eps).
+ * Limit: rows*cols <= 2^28 (268435456); larger returns DMU_ERR_UNSUPPORTED
+ * before any launch.  The first call on a device (with that device
+ * current) looks up the array's device address; make that first call
+ * before any stream capture.  Every call on a device shares the array:
+ * calls that overlap on the GPU race and must be ordered by the caller.
+ * The array needs no clearing (each call writes every slot it reads).
+ * Allocates nothing (no cudaMalloc, cudaFree or allocating library call). */
+DMU_API dmu_status dmu_momentum_norm_static(const void* grad, float* momentum, void* image_out,
+                                            int64_t rows, int64_t cols, dmu_dtype dtype, float beta,
+                                            float eps, float* inv_norm_out, void* stream);
 
 #ifdef __cplusplus
 }

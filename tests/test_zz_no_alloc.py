@@ -1,0 +1,71 @@
+"""The allocation-free momentum/norm entry point (dmu_momentum_norm_static).
+
+Callers that cannot allocate device memory -- a host process whose device
+memory belongs to another framework's pool, a plugin forbidden to call the
+CUDA allocator, or a hot loop where cudaMalloc would synchronise -- use this
+entry point, which keeps its scratch in a fixed array inside the library.
+This test calls it through the C ABI twice in a row (two matrices of
+different sizes, so the shared scratch is reused with stale contents) and
+checks each result against the plan-based dmu_momentum_normalize on the same
+inputs.  The file sorts last so that a failure here never hides another
+test's result.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from gram_newton_schulz_b200 import dmu, synth
+
+pytestmark = pytest.mark.gpu
+
+BETA, EPS = 0.95, 1e-7
+
+
+def _static_call(lib, g, mom, img, inv, dtype_code):
+    r, c = g.shape
+    return lib.dmu_momentum_norm_static(
+        ctypes.c_void_p(g.data_ptr()), ctypes.c_void_p(mom.data_ptr()) if mom is not None else None,
+        ctypes.c_void_p(img.data_ptr()), r, c, dtype_code, BETA, EPS, ctypes.c_void_p(inv.data_ptr()),
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_static_scratch_matches_plan_path_two_calls(dtype):
+    lib = dmu.load()
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    # second call is smaller: the scratch still holds the first call's sums
+    for call, shape in enumerate([(3584, 3584), (512, 2048), (300, 77)]):
+        w = synth.custom("noalloc", [shape], seed=90 + call, dtype=dtype)
+        g = synth.gradients(w, "cuda")[0]
+        m0 = torch.randn(shape, generator=torch.Generator("cuda").manual_seed(call), device="cuda")
+
+        plan = dmu.Plan([shape], dtype=dtype)
+        mom_a = m0.clone()
+        plan.momentum_normalize([g], [mom_a], beta=BETA, eps=EPS)
+        inv_a = plan.debug(6)
+        img_a = plan.debug(5, 0)
+
+        mom_b = m0.clone()
+        img_b = torch.empty(shape, dtype=tdt, device="cuda")
+        inv_b = torch.full((1,), -1.0, device="cuda")
+        st = _static_call(lib, g, mom_b, img_b, inv_b, dmu.DTYPES[dtype])
+        assert st == dmu.OK, lib.dmu_last_error()
+        torch.cuda.synchronize()
+        assert torch.equal(mom_a, mom_b)
+        assert torch.equal(img_a, img_b.float())
+        assert float(inv_b[0]) == pytest.approx(float(inv_a[0]), rel=1e-6)
+        x = mom_b.double().cpu().numpy()
+        assert float(inv_b[0]) == pytest.approx(1.0 / (np.linalg.norm(x) + EPS), rel=2e-6)
+
+
+def test_static_scratch_rejects_oversize_and_bad_args():
+    lib = dmu.load()
+    dummy = torch.empty(16, device="cuda")
+    p = ctypes.c_void_p(dummy.data_ptr())
+    st = lib.dmu_momentum_norm_static(p, None, p, 1 << 15, 1 << 14, 0, BETA, EPS, p, None)
+    assert st == dmu.ERR_UNSUPPORTED
+    assert b"2^28" in lib.dmu_last_error()
+    assert lib.dmu_momentum_norm_static(None, None, p, 4, 4, 0, BETA, EPS, p, None) == dmu.ERR_INVALID_ARG
+    assert lib.dmu_momentum_norm_static(p, None, p, 0, 4, 0, BETA, EPS, p, None) == dmu.ERR_INVALID_ARG
