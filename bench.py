@@ -157,10 +157,21 @@ def oracle_sample_seconds(shapes, budget_s=20.0):
     return total, threads, sample, spent
 
 
+def custom_workload(spec: str):
+    """'RxC*N,...' -> a spiked bf16 workload drawn like the layer-set recipe."""
+    from gram_newton_schulz_b200 import synth
+    shapes = []
+    for part in spec.split(","):
+        dims, _, n = part.partition("*")
+        r, c = dims.lower().split("x")
+        shapes += [(int(r), int(c))] * int(n or 1)
+    return synth.custom("custom-" + spec, shapes, seed=3)
+
+
 def run_reference(args):
     """--impl reference: the oracle on the host cores (bounded samples)."""
     from gram_newton_schulz_b200 import synth
-    w = synth.workload(args.workload)
+    w = custom_workload(args.shapes) if args.shapes else synth.workload(args.workload)
     vals = []
     for k in range(args.warmup + args.steps):
         total, threads, sample, _ = oracle_sample_seconds(w.shapes, budget_s=args.ref_budget)
@@ -185,6 +196,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="dmu", choices=["dmu", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--shard", default="replica", choices=["replica", "owner"],
+                    help="replica: every rank owns a full layer set (weak scaling); owner: the ranks "
+                         "split one layer set by LPT owner assignment (strong scaling)")
+    ap.add_argument("--shapes", default=None,
+                    help="custom spiked bf16 workload for profiling, e.g. 3584x3584*8,512x3584*4")
     ap.add_argument("--prec", default="auto")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
@@ -217,9 +233,16 @@ def main():
         if world > 1:
             dist.barrier()
 
-    w = synth.workload(args.workload)
-    grads = synth.gradients(w, dev)
-    weights = synth.weights(w, dev)
+    from gram_newton_schulz_b200 import owners
+    w_full = custom_workload(args.shapes) if args.shapes else synth.workload(args.workload)
+    if args.shard == "owner" and world > 1:
+        mine = owners.owned_indices(owners.assign_shapes(w_full.shapes, world), rank)
+    else:
+        mine = list(range(w_full.count))
+    w = synth.Workload(w_full.name, w_full.seed, w_full.dtype, tuple(w_full.shapes[i] for i in mine),
+                       w_full.dist, w_full.var, w_full.rank, w_full.beta, w_full.lr)
+    grads = synth.gradients(w_full, dev, indices=mine)
+    weights = synth.weights(w_full, dev, indices=mine)
     moms = [torch.zeros(s, dtype=torch.float32, device=dev) for s in w.shapes]
     plan = dmu.Plan(w.shapes, dtype=w.dtype, prec=args.prec, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -265,15 +288,13 @@ def main():
     t_mom = sum(e[0].elapsed_time(e[1]) for e in ev)
     t_gram = sum(e[1].elapsed_time(e[2]) for e in ev)
     t_upd = sum(e[2].elapsed_time(e[3]) for e in ev)
-    step_ms = total_ms / K
-    if world > 1:
-        t = torch.tensor([step_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms = float(t.item())
+    step_ms = owners.max_over_ranks(total_ms / K, device=dev)
     status = plan.read_status()
 
     peaks, peak_kind = load_peaks()
     flops = alg_flops(w.shapes)
+    job_shapes = w_full.shapes if args.shard == "owner" else w_full.shapes * world
+    job_flops = alg_flops(job_shapes)
     tc_s = (t_gram + t_upd) / K / 1e3
     achieved_tf = flops / tc_s / 1e12
     peak_tf = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
@@ -302,11 +323,7 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = owners.max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, device=dev)
         e2e = {"value": round(e2e_ms, 3), "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     cpu = None
@@ -319,15 +336,16 @@ def main():
         line = {
             "metric": METRIC, "value": round(step_ms, 3), "unit": "ms", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": round(step_ms, 3), "higher_is_better": False,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
-            "data": "synthetic",
-            "config": {"workload": w.name, "matrices": w.count, "matrices_total": w.count * world,
+            "scaling": "strong" if args.shard == "owner" else "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": {"workload": w_full.name, "matrices": w_full.count, "matrices_total": len(job_shapes),
                        "K": K_STEPS, "coeffs": [3.4445, -4.7750, 2.0315], "precision": args.prec,
-                       "parallelism": f"owner-sharded x{world} (independent layer sets)",
+                       "parallelism": (f"owner x{world} (LPT owners of one layer set)" if args.shard == "owner"
+                                       else f"replica x{world} (one owned layer set per rank)"),
                        "l2": "inputs larger than L2 (no flush needed)"},
-            "throughput": {"matrices_per_s": round(w.count * world / (step_ms / 1e3), 1),
-                           "alg_tflops": round(flops * world / (step_ms / 1e3) / 1e12, 1),
-                           "alg_tflops_frac": round(flops / (step_ms / 1e3) / 1e12 / peak_tf, 4)},
+            "throughput": {"matrices_per_s": round(len(job_shapes) / (step_ms / 1e3), 1),
+                           "alg_tflops": round(job_flops / (step_ms / 1e3) / 1e12, 1),
+                           "alg_tflops_frac_per_gpu": round(job_flops / world / (step_ms / 1e3) / 1e12 / peak_tf, 4)},
             "split_ms": {"momentum": round(t_mom / K, 3), "gram": round(t_gram / K, 3),
                          "update": round(t_upd / K, 3)},
             "roofline": {"bound": "tensor", "achieved": round(achieved_tf, 1), "peak": peak_tf,

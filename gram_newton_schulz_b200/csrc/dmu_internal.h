@@ -20,7 +20,8 @@ constexpr int BK = 64;
 constexpr int UMMA_K = 16;
 constexpr int A_PART_BYTES = BM * BK * 2;  // 16 KB
 constexpr int B_PART_BYTES = BN * BK * 2;  // 32 KB
-constexpr int GEMM_THREADS = 192;          // TMA warp, MMA warp, 4 epilogue warps
+constexpr int GEMM_THREADS = 320;          // TMA warp, MMA warp, 8 epilogue warps
+constexpr int EPI_WARPS = 8;               // two per TMEM lane quarter, each on half the columns
 constexpr int TMEM_COLS = 512;             // two BN-column accumulators
 
 constexpr int MAX_MAPS = 16;

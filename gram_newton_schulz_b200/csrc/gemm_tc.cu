@@ -17,8 +17,9 @@
 //              shared-memory stages guarded by full/empty mbarriers;
 //   warp 1     MMA issuer: one thread issues tcgen05.mma (M=128, N=256,
 //              K=16) into one of two TMEM accumulators (2 x 256 columns);
-//   warps 2-5  epilogue: tcgen05.ld of their 32-lane quarter, fp32 affine
-//              epilogue, bf16 hi/lo split, direct + mirrored stores; the
+//   warps 2-9  epilogue: tcgen05.ld of their 32-lane quarter (two warps per
+//              quarter, each on half of the tile's columns), fp32 affine
+//              epilogue, hi/lo split, direct + mirrored stores; the
 //              epilogue of tile t overlaps the main loop of tile t+1.
 // Operand precision: each stage holds up to two bf16 parts of A (hi, lo)
 // and of B; the problem's term bits choose hi*hi, hi*lo, lo*hi.
@@ -158,10 +159,13 @@ __device__ __forceinline__ void store_pair(__nv_bfloat16* hi, __nv_bfloat16* lo,
   if (lo) lo[off] = __float2bfloat16_rn(v - bf2f(h));
 }
 
-// One 32-column chunk of a Gram-space output tile for the thread's row i.
+// Columns per epilogue chunk (one tcgen05.ld of 32 lanes x CW columns).
+constexpr int CW = 16;
+
+// One CW-column chunk of a Gram-space output tile for the thread's row i.
 // Input and outputs are bf16 hi/lo pairs (FMT_PAIR) or fp32 (FMT_F32).
 __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, int i, int col0,
-                                               const uint32_t (&r)[32]) {
+                                               const uint32_t (&r)[CW]) {
   const int M = pr.M, N = pr.N;
   if (i >= M) return;
   float coef = pr.alpha;
@@ -171,20 +175,20 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
   } else if (pr.alpha_mode == ALPHA_INV) {
     coef *= pr.inv[pr.inv_base + mat];
   }
-  float v[32];
+  float v[CW];
 #pragma unroll
-  for (int c = 0; c < 32; ++c) v[c] = coef * __uint_as_float(r[c]);
+  for (int c = 0; c < CW; ++c) v[c] = coef * __uint_as_float(r[c]);
 
   const long long mbase = (long long)mat * pr.mat_stride;
   const long long rowoff = mbase + (long long)i * pr.ld;
-  const bool full = (col0 + 32 <= N);
+  const bool full = (col0 + CW <= N);
   const bool all_upper = !pr.sym || (i <= col0);
 
   if (pr.cin_fmt == FMT_F32 && pr.cin_f) {
     if (full) {
       const float4* pc = reinterpret_cast<const float4*>(pr.cin_f + rowoff + col0);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
+      for (int q = 0; q < CW / 4; ++q) {
         const float4 t = pc[q];
         v[4 * q] += pr.beta * t.x;
         v[4 * q + 1] += pr.beta * t.y;
@@ -193,7 +197,7 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
       }
     } else {
 #pragma unroll
-      for (int c = 0; c < 32; ++c)
+      for (int c = 0; c < CW; ++c)
         if (col0 + c < N) v[c] += pr.beta * pr.cin_f[rowoff + col0 + c];
     }
   } else if (pr.cin_fmt == FMT_PAIR_H && pr.cin_hi) {
@@ -202,14 +206,14 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
     if (full) {
       const uint4* ph = reinterpret_cast<const uint4*>(ch + rowoff + col0);
       const uint4* pl = reinterpret_cast<const uint4*>(cl + rowoff + col0);
-      uint4 uh[4], ul[4];
+      uint4 uh[CW / 8], ul[CW / 8];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < CW / 8; ++q) {
         uh[q] = ph[q];
         ul[q] = pl[q];
       }
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < CW / 8; ++q) {
         float fh[8], fl[8];
         unpack8_h(uh[q], fh);
         unpack8_h(ul[q], fl);
@@ -218,7 +222,7 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
       }
     } else {
 #pragma unroll
-      for (int c = 0; c < 32; ++c)
+      for (int c = 0; c < CW; ++c)
         if (col0 + c < N)
           v[c] += pr.beta * (__half2float(ch[rowoff + col0 + c]) + __half2float(cl[rowoff + col0 + c]));
     }
@@ -227,7 +231,7 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
       const uint4* ph = reinterpret_cast<const uint4*>(pr.cin_hi + rowoff + col0);
       const uint4* pl = pr.cin_lo ? reinterpret_cast<const uint4*>(pr.cin_lo + rowoff + col0) : nullptr;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < CW / 8; ++q) {
         float fh[8], fl[8];
         unpack8(ph[q], fh);
         if (pl) {
@@ -241,7 +245,7 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
       }
     } else {
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
+      for (int c = 0; c < CW; ++c) {
         if (col0 + c < N) {
           float x = bf2f(pr.cin_hi[rowoff + col0 + c]);
           if (pr.cin_lo) x += bf2f(pr.cin_lo[rowoff + col0 + c]);
@@ -251,9 +255,9 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
     }
   }
   const int dc = i - col0;  // diagonal column within the chunk
-  if (dc >= 0 && dc < 32) {
+  if (dc >= 0 && dc < CW) {
 #pragma unroll
-    for (int c = 0; c < 32; ++c)
+    for (int c = 0; c < CW; ++c)
       if (c == dc) v[c] += pr.gamma;
   }
 
@@ -262,7 +266,7 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
     if (pass == 1) {
       if (!pr.out2_hi && !pr.out2_f) break;
 #pragma unroll
-      for (int c = 0; c < 32; ++c) v[c] = v[c] * pr.scale2 + (c == dc ? pr.gamma2 : 0.f);
+      for (int c = 0; c < CW; ++c) v[c] = v[c] * pr.scale2 + (c == dc ? pr.gamma2 : 0.f);
     }
     if (fmt == FMT_PAIR_H) {
       __half* oh = reinterpret_cast<__half*>(pass == 0 ? pr.out_hi : pr.out2_hi);
@@ -272,7 +276,7 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
         uint4* dh = reinterpret_cast<uint4*>(oh + rowoff + col0);
         uint4* dl = ol ? reinterpret_cast<uint4*>(ol + rowoff + col0) : nullptr;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < CW / 8; ++q) {
           uint4 h, l;
           split8_h(v + 8 * q, h, l);
           dh[q] = h;
@@ -280,14 +284,14 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
         }
       } else {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
+        for (int c = 0; c < CW; ++c) {
           const int j = col0 + c;
           if (j < N && (!pr.sym || i <= j)) store_pair_h(oh, ol, rowoff + j, v[c]);
         }
       }
       if (pr.sym) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
+        for (int c = 0; c < CW; ++c) {
           const int j = col0 + c;
           if (j < N && i < j) store_pair_h(oh, ol, mbase + (long long)j * pr.ld + i, v[c]);
         }
@@ -300,17 +304,17 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
       if (full && all_upper) {
         float4* d4 = reinterpret_cast<float4*>(of + rowoff + col0);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) d4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        for (int q = 0; q < CW / 4; ++q) d4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
       } else {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
+        for (int c = 0; c < CW; ++c) {
           const int j = col0 + c;
           if (j < N && (!pr.sym || i <= j)) of[rowoff + j] = v[c];
         }
       }
       if (pr.sym) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
+        for (int c = 0; c < CW; ++c) {
           const int j = col0 + c;
           if (j < N && i < j) of[mbase + (long long)j * pr.ld + i] = v[c];
         }
@@ -325,7 +329,7 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
       uint4* dh = reinterpret_cast<uint4*>(oh + rowoff + col0);
       uint4* dl = ol ? reinterpret_cast<uint4*>(ol + rowoff + col0) : nullptr;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < CW / 8; ++q) {
         uint4 h, l;
         split8(v + 8 * q, h, l);
         dh[q] = h;
@@ -333,7 +337,7 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
       }
     } else {
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
+      for (int c = 0; c < CW; ++c) {
         const int j = col0 + c;
         if (j < N && (!pr.sym || i <= j)) store_pair(oh, ol, rowoff + j, v[c]);
       }
@@ -342,7 +346,7 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
     // columns of row j, so each store instruction is coalesced.
     if (pr.sym) {
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
+      for (int c = 0; c < CW; ++c) {
         const int j = col0 + c;
         if (j < N && i < j) store_pair(oh, ol, mbase + (long long)j * pr.ld + i, v[c]);
       }
@@ -350,24 +354,24 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
   }
 }
 
-// One 32-column chunk of the final O = P X0 tile, fused with the update.
+// One CW-column chunk of the final O = P X0 tile, fused with the update.
 // Row i of the tile is row i of O (m x n); element (i, j) lives at W[i][j]
 // for a wide matrix and at W[j][i] for a tall one (w_transposed).  All W
 // loads of the chunk are issued before any store, so they overlap instead
 // of serialising behind stores the compiler cannot prove independent.
 __device__ __forceinline__ void epi_update_chunk(const GemmProblem& pr, int mat, int i, int col0,
-                                                 const uint32_t (&r)[32]) {
+                                                 const uint32_t (&r)[CW]) {
   const int M = pr.M, N = pr.N;
   if (i >= M) return;
   const float s = pr.inv[pr.inv_base + mat];
   const float cw = pr.alpha * s;  // -lr * scale / (||M|| + eps)
-  float o[32];
+  float o[CW];
 #pragma unroll
-  for (int c = 0; c < 32; ++c) o[c] = __uint_as_float(r[c]);
+  for (int c = 0; c < CW; ++c) o[c] = __uint_as_float(r[c]);
   void* wp = pr.w_ptrs ? pr.w_ptrs[pr.ptr_base + mat] : nullptr;
   float* op = pr.o_ptrs ? pr.o_ptrs[pr.ptr_base + mat] : nullptr;
   const long long wc = pr.w_cols;
-  const bool full = (col0 + 32 <= N);
+  const bool full = (col0 + CW <= N);
   if (!pr.w_transposed) {
     const long long rowoff = (long long)i * wc;
     if (wp) {
@@ -376,11 +380,11 @@ __device__ __forceinline__ void epi_update_chunk(const GemmProblem& pr, int mat,
         const bool vec = full && ((wc & 7) == 0) && ((reinterpret_cast<uintptr_t>(w) & 15) == 0);
         if (vec) {
           uint4* pw = reinterpret_cast<uint4*>(w + rowoff + col0);
-          uint4 wv[4];
+          uint4 wv[CW / 8];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) wv[q] = pw[q];
+          for (int q = 0; q < CW / 8; ++q) wv[q] = pw[q];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+          for (int q = 0; q < CW / 8; ++q) {
             float f[8];
             unpack8(wv[q], f);
             uint4 h;
@@ -392,26 +396,26 @@ __device__ __forceinline__ void epi_update_chunk(const GemmProblem& pr, int mat,
             pw[q] = h;
           }
         } else {
-          float wv[32];
+          float wv[CW];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) wv[c] = (col0 + c < N) ? bf2f(w[rowoff + col0 + c]) : 0.f;
+          for (int c = 0; c < CW; ++c) wv[c] = (col0 + c < N) ? bf2f(w[rowoff + col0 + c]) : 0.f;
 #pragma unroll
-          for (int c = 0; c < 32; ++c)
+          for (int c = 0; c < CW; ++c)
             if (col0 + c < N) w[rowoff + col0 + c] = __float2bfloat16_rn(wv[c] + cw * o[c]);
         }
       } else {
         float* w = reinterpret_cast<float*>(wp);
-        float wv[32];
+        float wv[CW];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) wv[c] = (col0 + c < N) ? w[rowoff + col0 + c] : 0.f;
+        for (int c = 0; c < CW; ++c) wv[c] = (col0 + c < N) ? w[rowoff + col0 + c] : 0.f;
 #pragma unroll
-        for (int c = 0; c < 32; ++c)
+        for (int c = 0; c < CW; ++c)
           if (col0 + c < N) w[rowoff + col0 + c] = wv[c] + cw * o[c];
       }
     }
     if (op) {
 #pragma unroll
-      for (int c = 0; c < 32; ++c)
+      for (int c = 0; c < CW; ++c)
         if (col0 + c < N) op[rowoff + col0 + c] = s * o[c];
     }
   } else {
@@ -420,25 +424,25 @@ __device__ __forceinline__ void epi_update_chunk(const GemmProblem& pr, int mat,
     if (wp) {
       if (!pr.w_f32) {
         __nv_bfloat16* w = reinterpret_cast<__nv_bfloat16*>(wp);
-        float wv[32];
+        float wv[CW];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) wv[c] = (col0 + c < N) ? bf2f(w[(long long)(col0 + c) * wc + i]) : 0.f;
+        for (int c = 0; c < CW; ++c) wv[c] = (col0 + c < N) ? bf2f(w[(long long)(col0 + c) * wc + i]) : 0.f;
 #pragma unroll
-        for (int c = 0; c < 32; ++c)
+        for (int c = 0; c < CW; ++c)
           if (col0 + c < N) w[(long long)(col0 + c) * wc + i] = __float2bfloat16_rn(wv[c] + cw * o[c]);
       } else {
         float* w = reinterpret_cast<float*>(wp);
-        float wv[32];
+        float wv[CW];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) wv[c] = (col0 + c < N) ? w[(long long)(col0 + c) * wc + i] : 0.f;
+        for (int c = 0; c < CW; ++c) wv[c] = (col0 + c < N) ? w[(long long)(col0 + c) * wc + i] : 0.f;
 #pragma unroll
-        for (int c = 0; c < 32; ++c)
+        for (int c = 0; c < CW; ++c)
           if (col0 + c < N) w[(long long)(col0 + c) * wc + i] = wv[c] + cw * o[c];
       }
     }
     if (op) {
 #pragma unroll
-      for (int c = 0; c < 32; ++c)
+      for (int c = 0; c < CW; ++c)
         if (col0 + c < N) op[(long long)(col0 + c) * wc + i] = s * o[c];
     }
   }
@@ -475,7 +479,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(tfull_bar(b), 1);
-      ptx::mbar_init(tempty_bar(b), 4);
+      ptx::mbar_init(tempty_bar(b), EPI_WARPS);
     }
     ptx::mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -645,8 +649,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------ epilogue (warps 2..5)
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    // ------------------------------------------------ epilogue (warps 2..9)
+    const int q = warp & 3;                        // TMEM lane quarter this warp may access
+    const int ch_begin = ((warp - 2) >> 2) * (BN / 2 / CW);  // column half of the tile
+    const int ch_end = ch_begin + BN / 2 / CW;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
@@ -659,13 +665,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
       ptx::tc_fence_after();
       const int row_lo = tc.bi * BM + q * 32;
       const int i = row_lo + lane;
-      for (int ch = 0; ch < BN / 32; ++ch) {
-        const int col0 = tc.bj * BN + ch * 32;
+      for (int ch = ch_begin; ch < ch_end; ++ch) {
+        const int col0 = tc.bj * BN + ch * CW;
         if (col0 >= pr.N) break;
-        if (pr.sym && col0 + 31 < row_lo) continue;  // chunk strictly below the diagonal
+        if (pr.sym && col0 + CW - 1 < row_lo) continue;  // chunk strictly below the diagonal
         if (row_lo >= pr.M) break;
-        uint32_t r[32];
-        ptx::tmem_ld32(tmem_base + (uint32_t)(acc * BN + ch * 32) + ((uint32_t)(q * 32) << 16), r);
+        uint32_t r[CW];
+        ptx::tmem_ld16(tmem_base + (uint32_t)(acc * BN + ch * CW) + ((uint32_t)(q * 32) << 16), r);
         ptx::tmem_wait_ld();
         if (pr.epi == EPI_GRAM)
           epi_gram_chunk(pr, tc.mat, i, col0, r);

@@ -187,7 +187,7 @@ __global__ void k_pair_h_to_f32(const __half* hi, const __half* lo, long long ro
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
        e += (long long)gridDim.x * blockDim.x) {
     const long long r = e / cols, c = e % cols;
-    out[e] = (__half2float(hi[r * ld + c]) + __half2float(lo[r * ld + c])) * scale;
+    out[e] = (__half2float(hi[r * ld + c]) + (lo ? __half2float(lo[r * ld + c]) : 0.f)) * scale;
   }
 }
 

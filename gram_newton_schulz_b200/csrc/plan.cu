@@ -363,7 +363,7 @@ void set_h_out(dmu_plan p, int c, int slot, int* fmt, __nv_bfloat16** hi, __nv_b
 }
 
 Prob gram_prob_h(dmu_plan p, int c, int a_slot, int b_slot, float alpha, float beta, int cin_slot, int out_slot,
-                 int out2_slot, float gamma2) {
+                 int out2_slot, float gamma2, bool out_lo = true) {
   const GClass& gc = p->classes[c];
   Prob pr;
   std::memset(&pr, 0, sizeof(pr));
@@ -382,6 +382,7 @@ Prob gram_prob_h(dmu_plan p, int c, int a_slot, int b_slot, float alpha, float b
   float s_out = 1.f, s_out2 = 1.f;
   set_h_out(p, c, out_slot, &g.out_fmt, &g.out_hi, &g.out_lo, &s_out);
   set_h_out(p, c, out2_slot, &g.out2_fmt, &g.out2_hi, &g.out2_lo, &s_out2);
+  if (!out_lo) g.out_lo = nullptr;
   g.alpha = alpha * s_out / (half_slot_scale(a_slot) * half_slot_scale(b_slot));
   g.gamma = 0.f;
   if (cin_slot >= 0) {
@@ -410,8 +411,9 @@ Prob product(dmu_plan p, int c, Product what, int k, bool last, const float co[3
     const int hin = p_in == 0 ? SLOT_PA_HI : SLOT_PB_HI, hout = p_out == 0 ? SLOT_PA_HI : SLOT_PB_HI;
     switch (what) {
       case PROD_R:
+        // R is only ever an MMA operand (hi): its lo half is not stored
         return gram_prob_h(p, c, SLOT_G_HI, SLOT_G_HI, co[2], co[1], SLOT_G_HI, SLOT_R_HI,
-                           k == 0 ? (last ? OUT_PF : SLOT_PA_HI) : -1, co[0]);
+                           k == 0 ? (last ? OUT_PF : SLOT_PA_HI) : -1, co[0], false);
       case PROD_T:
         return gram_prob_h(p, c, SLOT_R_HI, SLOT_G_HI, 1.f, co[0], SLOT_G_HI, SLOT_T_HI, -1, 0.f);
       case PROD_P:
@@ -1123,8 +1125,9 @@ dmu_status dmu_debug_gram(dmu_plan p, int which, int index, float* out, void* st
     } else {
       const int slots[5] = {SLOT_G_HI, SLOT_R_HI, SLOT_T_HI, SLOT_PA_HI, SLOT_PB_HI};
       const int sh = slots[q];
-      CUDA_TRY(launch_pair_h_to_f32(p->slot_bf16(bk->cls, sh) + moff, p->slot_bf16(bk->cls, sh + 1) + moff, gc.m,
-                                    gc.m, gc.ldg, 1.f / half_slot_scale(sh), out, s));
+      CUDA_TRY(launch_pair_h_to_f32(p->slot_bf16(bk->cls, sh) + moff,
+                                    sh == SLOT_R_HI ? nullptr : p->slot_bf16(bk->cls, sh + 1) + moff, gc.m, gc.m,
+                                    gc.ldg, 1.f / half_slot_scale(sh), out, s));
     }
   } else if (p->dtype == DMU_BF16 && gc.kind == KIND_TF32) {
     if (which == 7) {
