@@ -46,6 +46,7 @@ struct TileCoord {
   int pi, mat, bi, bj;
 };
 
+template <int TBM>
 __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int t) {
   TileCoord c;
   int pi = 0;
@@ -59,10 +60,10 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int t) {
     bi = tl % pr.tiles_m;
     bj = tl / pr.tiles_m;
   } else {
-    // column block bj holds row blocks 0 .. min(tiles_m, ((bj+1)*BN-1)/BM + 1) - 1
+    // column block bj holds row blocks 0 .. min(tiles_m, ((bj+1)*BN-1)/TBM + 1) - 1
     bj = 0;
     for (;;) {
-      int cnt = min(pr.tiles_m, ((bj + 1) * BN - 1) / BM + 1);
+      int cnt = min(pr.tiles_m, ((bj + 1) * BN - 1) / TBM + 1);
       if (tl < cnt) break;
       tl -= cnt;
       ++bj;
@@ -509,7 +510,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
       bool ok = true;
       uint32_t issued_mask = 0, issued_par = 0;  // per stage: a load was issued, its phase parity
       for (int t = blockIdx.x; ok && t < p.total_tiles; t += gridDim.x) {
-        const TileCoord tc = decode_tile(p, t);
+        const TileCoord tc = decode_tile<BM>(p, t);
         const GemmProblem& pr = p.prob[tc.pi];
         const CUtensorMap* am = &p.maps[pr.a_map];
         const CUtensorMap* bm = &p.maps[pr.b_map];
@@ -582,7 +583,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
       bool ok = true;
       bool issued = false;
       for (int t = blockIdx.x; ok && t < p.total_tiles; t += gridDim.x) {
-        const TileCoord tc = decode_tile(p, t);
+        const TileCoord tc = decode_tile<BM>(p, t);
         const GemmProblem& pr = p.prob[tc.pi];
         const int nk = (pr.K + BKE - 1) / BKE;
         const uint32_t idesc = ptx::make_idesc(BM, BN, pr.a_mn, pr.b_mn, OPFMT);
@@ -656,7 +657,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
-      const TileCoord tc = decode_tile(p, t);
+      const TileCoord tc = decode_tile<BM>(p, t);
       const GemmProblem& pr = p.prob[tc.pi];
       int ok = 1;
       if (lane == 0) ok = wait_bar(tfull_bar(acc), acc_phase, abort_flag, p) ? 1 : 0;
@@ -695,6 +696,298 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
   }
 }
 
+// ------------------------------------------------------------- CTA-pair kernel
+// Same problems and epilogues, computed by CTA pairs (a cluster of 2) on
+// 256 x 256 output tiles with tcgen05.mma.cta_group::2 (M = 256, N = 256):
+// CTA r of the pair TMA-loads rows [128 r, 128 r + 128) of the tile's A
+// block and of its B block into its own shared memory and holds rows
+// [128 r, 128 r + 128) of the accumulator in its own TMEM.  Per SM this
+// halves the B operand bytes of the 128 x 256 single-CTA tile (64 instead
+// of 96 bytes per MMA clock), and one K-block stage is only 32 KB, so six
+// stages fit.  The leader (rank 0) arms the stage barrier with both CTAs'
+// bytes and issues the MMAs; its commits arrive on both CTAs' barriers;
+// both epilogues arrive on the leader's TMEM-empty barrier.  No load uses
+// cluster multicast: every byte a CTA reads comes from its own TMA loads.
+constexpr int BM2 = 256;
+constexpr int HALF_BYTES = 128 * 128;  // 128 rows x 128-byte K row
+
+template <int NA, int NB>
+struct Tc2Cfg {
+  static constexpr int STAGE_BYTES = (NA + NB) * HALF_BYTES;
+  static constexpr int STAGES = (200 * 1024) / STAGE_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+  static_assert(STAGES >= 2 && STAGES <= 8, "stage count");
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+};
+
+__device__ __forceinline__ bool wait_bar_cluster(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                                 const GemmParams& p) {
+  if (ptx::mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  uint32_t n = 0;
+  for (;;) {
+    if (ptx::mbar_try_wait_cluster(bar, parity)) return true;
+    if ((++n & 63u) == 0) {
+      if (*abort_flag) return false;
+      if ((long long)(ptx::globaltimer() - t0) > p.timeout_ns) {
+        *abort_flag = 1;
+        atomicOr(p.status, DMU_FLAG_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+template <int NA, int NB, int KIND>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
+    k_gemm_tc2(const __grid_constant__ GemmParams p) {
+  using Cfg = Tc2Cfg<NA, NB>;
+  constexpr int S = Cfg::STAGES;
+  constexpr int BKE = KIND == KIND_TF32 ? 32 : 64;
+  constexpr int OPFMT = KIND == KIND_TF32 ? 2 : (KIND == KIND_F16 ? 0 : 1);
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = ptx::smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  const uint32_t ring = base;
+  const uint32_t bars = base + S * Cfg::STAGE_BYTES;
+  auto full_bar = [&](int s) { return bars + 8u * s; };
+  auto empty_bar = [&](int s) { return bars + 8u * (S + s); };
+  auto tfull_bar = [&](int b) { return bars + 8u * (2 * S + b); };
+  auto tempty_bar = [&](int b) { return bars + 8u * (2 * S + 2 + b); };
+  const uint32_t drain_bar = bars + 8u * (2 * S + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S * Cfg::STAGE_BYTES + 8 * (2 * S + 5));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      ptx::mbar_init(full_bar(s), 1);
+      ptx::mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(tfull_bar(b), 1);
+      ptx::mbar_init(tempty_bar(b), 2 * EPI_WARPS);
+    }
+    ptx::mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+    ptx::fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int pi = 0; pi < p.nprob; ++pi) {
+      ptx::prefetch_tmap(&p.maps[p.prob[pi].a_map]);
+      ptx::prefetch_tmap(&p.maps[p.prob[pi].b_map]);
+    }
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc2(ptx::smem_u32(tmem_slot), TMEM_COLS);
+    ptx::tmem_relinquish2();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync();  // both CTAs' barriers exist before any remote arrive
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      uint32_t issued_mask = 0, issued_par = 0;
+      for (int t = pair; ok && t < p.total_tiles; t += npairs) {
+        const TileCoord tc = decode_tile<BM2>(p, t);
+        const GemmProblem& pr = p.prob[tc.pi];
+        const CUtensorMap* am = &p.maps[pr.a_map];
+        const CUtensorMap* bm = &p.maps[pr.b_map];
+        const int na = (NA > 1 && (pr.terms & TERM_LH)) ? 2 : 1;
+        const int nb = (NB > 1 && (pr.terms & TERM_HL)) ? 2 : 1;
+        const uint32_t bytes_pair = 2u * (uint32_t)(na + nb) * HALF_BYTES;
+        const int nk = (pr.K + BKE - 1) / BKE;
+        const int arow = tc.bi * BM2 + (int)rank * 128, brow = tc.bj * BN + (int)rank * 128;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!wait_bar_cluster(empty_bar(stage), phase ^ 1u, abort_flag, p)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb_leader = ptx::mapa_shared(full_bar(stage), 0);
+          if (leader) {
+            ptx::mbar_arrive_expect_tx(full_bar(stage), bytes_pair);
+            issued_mask |= 1u << stage;
+            issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          }
+          const int k0 = kb * BKE;
+          const uint32_t sa = ring + stage * Cfg::STAGE_BYTES;
+          const uint32_t sb = sa + NA * HALF_BYTES;
+          for (int part = 0; part < na; ++part) {
+            const uint32_t dst = sa + part * HALF_BYTES;
+            const int z = pr.a_z[part] + tc.mat;
+            if (!pr.a_mn) {
+              ptx::tma_load_3d_pair(dst, am, fb_leader, k0, arow, z);
+            } else {
+              ptx::tma_load_3d_pair(dst, am, fb_leader, arow, k0, z);
+              ptx::tma_load_3d_pair(dst + 8192, am, fb_leader, arow + 64, k0, z);
+            }
+          }
+          for (int part = 0; part < nb; ++part) {
+            const uint32_t dst = sb + part * HALF_BYTES;
+            const int z = pr.b_z[part] + tc.mat;
+            if (!pr.b_mn) {
+              ptx::tma_load_3d_pair(dst, bm, fb_leader, k0, brow, z);
+            } else {
+              ptx::tma_load_3d_pair(dst, bm, fb_leader, brow, k0, z);
+              ptx::tma_load_3d_pair(dst + 8192, bm, fb_leader, brow + 64, k0, z);
+            }
+          }
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // The leader's stage barriers count both CTAs' bytes: wait until every
+      // phase it armed has landed before the pair may exit.
+      for (int s2 = 0; s2 < S; ++s2) {
+        if (!(issued_mask & (1u << s2))) continue;
+        const uint32_t par = (issued_par >> s2) & 1u;
+        const uint64_t t0 = ptx::globaltimer();
+        while (!ptx::mbar_try_wait_cluster(full_bar(s2), par)) {
+          if ((long long)(ptx::globaltimer() - t0) > p.timeout_ns) {
+            atomicOr(p.status, DMU_FLAG_TIMEOUT);
+            break;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer (leader only)
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      bool issued = false;
+      for (int t = pair; ok && t < p.total_tiles; t += npairs) {
+        const TileCoord tc = decode_tile<BM2>(p, t);
+        const GemmProblem& pr = p.prob[tc.pi];
+        const int nk = (pr.K + BKE - 1) / BKE;
+        const uint32_t idesc = ptx::make_idesc(BM2, BN, pr.a_mn, pr.b_mn, OPFMT);
+        if (!wait_bar_cluster(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        const uint32_t a_lbo = pr.a_mn ? 8192u : 16u, b_lbo = pr.b_mn ? 8192u : 16u;
+        const uint32_t a_kstep = pr.a_mn ? 2048u : 32u, b_kstep = pr.b_mn ? 2048u : 32u;
+        uint32_t accumulate = 0;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!wait_bar_cluster(full_bar(stage), phase, abort_flag, p)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t sa = ring + stage * Cfg::STAGE_BYTES;
+          const uint32_t sb = sa + NA * HALF_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+            for (int term = 0; term < 3; ++term) {
+              if (!(pr.terms & (1 << term))) continue;
+              if (term == 1 && NB < 2) continue;
+              if (term == 2 && NA < 2) continue;
+              const uint32_t pa = sa + (term == 2 ? HALF_BYTES : 0);
+              const uint32_t pb = sb + (term == 1 ? HALF_BYTES : 0);
+              const uint64_t ad = ptx::make_sw128_desc(pa + kk * a_kstep, a_lbo, 1024u);
+              const uint64_t bd = ptx::make_sw128_desc(pb + kk * b_kstep, b_lbo, 1024u);
+              if (KIND == KIND_TF32)
+                ptx::mma2_tf32(d_tmem, ad, bd, idesc, accumulate);
+              else
+                ptx::mma2_f16(d_tmem, ad, bd, idesc, accumulate);
+              accumulate = 1;
+              issued = true;
+            }
+          }
+          ptx::mma2_commit_both(empty_bar(stage));
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        ptx::mma2_commit_both(tfull_bar(acc));
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      if (!ok && issued) {
+        ptx::mma2_commit_both(drain_bar);
+        const uint64_t t0 = ptx::globaltimer();
+        while (!ptx::mbar_try_wait_cluster(drain_bar, 0)) {
+          if ((long long)(ptx::globaltimer() - t0) > p.timeout_ns) break;
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ epilogue (both CTAs, warps 2..9)
+    const int q = warp & 3;
+    const int ch_begin = ((warp - 2) >> 2) * (BN / 2 / CW);
+    const int ch_end = ch_begin + BN / 2 / CW;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = pair; t < p.total_tiles; t += npairs) {
+      const TileCoord tc = decode_tile<BM2>(p, t);
+      const GemmProblem& pr = p.prob[tc.pi];
+      int ok = 1;
+      if (lane == 0) ok = wait_bar_cluster(tfull_bar(acc), acc_phase, abort_flag, p) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      ptx::tc_fence_after();
+      const int row_lo = tc.bi * BM2 + (int)rank * 128 + q * 32;
+      const int i = row_lo + lane;
+      for (int ch = ch_begin; ch < ch_end; ++ch) {
+        const int col0 = tc.bj * BN + ch * CW;
+        if (col0 >= pr.N) break;
+        if (pr.sym && col0 + CW - 1 < row_lo) continue;
+        if (row_lo >= pr.M) break;
+        uint32_t r[CW];
+        ptx::tmem_ld16(tmem_base + (uint32_t)(acc * BN + ch * CW) + ((uint32_t)(q * 32) << 16), r);
+        ptx::tmem_wait_ld();
+        if (pr.epi == EPI_GRAM)
+          epi_gram_chunk(pr, tc.mat, i, col0, r);
+        else
+          epi_update_chunk(pr, tc.mat, i, col0, r);
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive_cluster(ptx::mapa_shared(tempty_bar(acc), 0));
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  __syncthreads();
+  ptx::cluster_sync();  // no CTA leaves while its peer may still signal it
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc2(tmem_base, TMEM_COLS);
+  }
+}
+
 // Bounded-wait self-test: one thread waits on an mbarrier that nothing
 // arrives on; the wait gives up after timeout_ns and sets DMU_FLAG_TIMEOUT.
 __global__ void k_wait_selftest(unsigned int* status, long long timeout_ns) {
@@ -730,6 +1023,12 @@ static cudaError_t configure_one() {
                               TcCfg<NA, NB>::SMEM_BYTES);
 }
 
+template <int NA, int NB, int KIND>
+static cudaError_t configure_two() {
+  return cudaFuncSetAttribute(k_gemm_tc2<NA, NB, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              Tc2Cfg<NA, NB>::SMEM_BYTES);
+}
+
 cudaError_t gemm_tc_configure() {
   cudaError_t e;
   if ((e = configure_one<1, 1, KIND_BF16>()) != cudaSuccess) return e;
@@ -737,6 +1036,11 @@ cudaError_t gemm_tc_configure() {
   if ((e = configure_one<2, 2, KIND_BF16>()) != cudaSuccess) return e;
   if ((e = configure_one<1, 1, KIND_TF32>()) != cudaSuccess) return e;
   if ((e = configure_one<1, 1, KIND_F16>()) != cudaSuccess) return e;
+  if ((e = configure_two<1, 1, KIND_BF16>()) != cudaSuccess) return e;
+  if ((e = configure_two<2, 1, KIND_BF16>()) != cudaSuccess) return e;
+  if ((e = configure_two<2, 2, KIND_BF16>()) != cudaSuccess) return e;
+  if ((e = configure_two<1, 1, KIND_TF32>()) != cudaSuccess) return e;
+  if ((e = configure_two<1, 1, KIND_F16>()) != cudaSuccess) return e;
   return cudaSuccess;
 }
 
@@ -753,6 +1057,30 @@ static cudaError_t launch_one(const GemmParams& p, int num_sms, cudaStream_t s) 
   if (grid <= 0) return cudaSuccess;
   k_gemm_tc<NA, NB, KIND><<<grid, GEMM_THREADS, TcCfg<NA, NB>::SMEM_BYTES, s>>>(p);
   return cudaGetLastError();
+}
+
+template <int NA, int NB, int KIND>
+static cudaError_t launch_two(const GemmParams& p, int num_sms, cudaStream_t s) {
+  int pairs = num_sms / 2;
+  if (p.total_tiles < pairs) pairs = p.total_tiles;
+  if (pairs <= 0) return cudaSuccess;
+  k_gemm_tc2<NA, NB, KIND><<<2 * pairs, GEMM_THREADS, Tc2Cfg<NA, NB>::SMEM_BYTES, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_tc2(const GemmParams& p, int na, int nb, int kind, int num_sms, cudaStream_t s) {
+  if (kind == KIND_TF32) {
+    if (na == 1 && nb == 1) return launch_two<1, 1, KIND_TF32>(p, num_sms, s);
+    return cudaErrorInvalidValue;
+  }
+  if (kind == KIND_F16) {
+    if (na == 1 && nb == 1) return launch_two<1, 1, KIND_F16>(p, num_sms, s);
+    return cudaErrorInvalidValue;
+  }
+  if (na == 1 && nb == 1) return launch_two<1, 1, KIND_BF16>(p, num_sms, s);
+  if (na == 2 && nb == 1) return launch_two<2, 1, KIND_BF16>(p, num_sms, s);
+  if (na == 2 && nb == 2) return launch_two<2, 2, KIND_BF16>(p, num_sms, s);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_gemm_tc(const GemmParams& p, int na, int nb, int kind, int num_sms, cudaStream_t s) {

@@ -18,11 +18,11 @@ namespace dmu {
 __device__ __forceinline__ void load8_grad(const void* g, int f32, long long idx, float* out) {
   if (f32) {
     const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(g) + idx);
-    float4 a = p[0], b = p[1];
+    float4 a = __ldg(p), b = __ldg(p + 1);
     out[0] = a.x; out[1] = a.y; out[2] = a.z; out[3] = a.w;
     out[4] = b.x; out[5] = b.y; out[6] = b.z; out[7] = b.w;
   } else {
-    uint4 u = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(g) + idx);
+    uint4 u = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(g) + idx));
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -33,7 +33,24 @@ __device__ __forceinline__ void load8_grad(const void* g, int f32, long long idx
   }
 }
 
-__global__ void __launch_bounds__(256) k_momentum(const MomChunk* __restrict__ chunks, int nchunks,
+__device__ __forceinline__ void store8_image(void* __restrict__ mb, int mb_f32, long long o, const float* v) {
+  if (mb_f32) {
+    float4* d = reinterpret_cast<float4*>(reinterpret_cast<float*>(mb) + o);
+    d[0] = make_float4(v[0], v[1], v[2], v[3]);
+    d[1] = make_float4(v[4], v[5], v[6], v[7]);
+  } else {
+    uint4 u;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) h[q] = __floats2bfloat162_rn(v[2 * q], v[2 * q + 1]);
+    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(mb) + o) = u;
+  }
+}
+
+// Vector path: each thread takes two 8-element vectors per iteration and
+// issues every load (G, M) before any store, so two vectors' loads are in
+// flight per thread; G, M and the image are distinct buffers (restrict).
+__global__ void __launch_bounds__(256, 6) k_momentum(const MomChunk* __restrict__ chunks, int nchunks,
                                                   const MomMat* __restrict__ mats,
                                                   const void* const* __restrict__ grads,
                                                   float* const* __restrict__ momenta, int grad_f32,
@@ -43,35 +60,47 @@ __global__ void __launch_bounds__(256) k_momentum(const MomChunk* __restrict__ c
   for (int c = blockIdx.x; c < nchunks; c += gridDim.x) {
     const MomChunk ch = chunks[c];
     const MomMat mm = mats[ch.slot];
-    const void* g = grads[ch.slot];
-    float* mom = momenta ? momenta[ch.slot] : nullptr;
+    const void* __restrict__ g = grads[ch.slot];
+    float* __restrict__ mom = momenta ? momenta[ch.slot] : nullptr;
     float ss = 0.f;
     if (vec) {
-      for (int e = threadIdx.x * 8; e < ch.len; e += blockDim.x * 8) {
-        const long long idx = ch.start + e;
-        float v[8];
-        load8_grad(g, grad_f32, idx, v);
+      const int stride = blockDim.x * 8;
+      for (int e = threadIdx.x * 8; e < ch.len; e += 2 * stride) {
+        const long long i0 = ch.start + e, i1 = i0 + stride;
+        const bool has1 = e + stride < ch.len;
+        float v0[8], v1[8];
+        float4 m0a, m0b, m1a, m1b;
+        load8_grad(g, grad_f32, i0, v0);
+        if (has1) load8_grad(g, grad_f32, i1, v1);
         if (mom) {
-          float4* pm = reinterpret_cast<float4*>(mom + idx);
-          float4 a = pm[0], b = pm[1];
-          v[0] += beta * a.x; v[1] += beta * a.y; v[2] += beta * a.z; v[3] += beta * a.w;
-          v[4] += beta * b.x; v[5] += beta * b.y; v[6] += beta * b.z; v[7] += beta * b.w;
-          pm[0] = make_float4(v[0], v[1], v[2], v[3]);
-          pm[1] = make_float4(v[4], v[5], v[6], v[7]);
+          const float4* p0 = reinterpret_cast<const float4*>(mom + i0);
+          m0a = p0[0];
+          m0b = p0[1];
+          if (has1) {
+            const float4* p1 = reinterpret_cast<const float4*>(mom + i1);
+            m1a = p1[0];
+            m1b = p1[1];
+          }
+          v0[0] += beta * m0a.x; v0[1] += beta * m0a.y; v0[2] += beta * m0a.z; v0[3] += beta * m0a.w;
+          v0[4] += beta * m0b.x; v0[5] += beta * m0b.y; v0[6] += beta * m0b.z; v0[7] += beta * m0b.w;
+          float4* q0 = reinterpret_cast<float4*>(mom + i0);
+          q0[0] = make_float4(v0[0], v0[1], v0[2], v0[3]);
+          q0[1] = make_float4(v0[4], v0[5], v0[6], v0[7]);
+          if (has1) {
+            v1[0] += beta * m1a.x; v1[1] += beta * m1a.y; v1[2] += beta * m1a.z; v1[3] += beta * m1a.w;
+            v1[4] += beta * m1b.x; v1[5] += beta * m1b.y; v1[6] += beta * m1b.z; v1[7] += beta * m1b.w;
+            float4* q1 = reinterpret_cast<float4*>(mom + i1);
+            q1[0] = make_float4(v1[0], v1[1], v1[2], v1[3]);
+            q1[1] = make_float4(v1[4], v1[5], v1[6], v1[7]);
+          }
         }
 #pragma unroll
-        for (int q = 0; q < 8; ++q) ss += v[q] * v[q];
-        const long long o = mm.mb_off + idx;  // ldc == cols on the vector path
-        if (mb_f32) {
-          float4* d = reinterpret_cast<float4*>(reinterpret_cast<float*>(mb) + o);
-          d[0] = make_float4(v[0], v[1], v[2], v[3]);
-          d[1] = make_float4(v[4], v[5], v[6], v[7]);
-        } else {
-          uint4 u;
-          __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+        for (int q = 0; q < 8; ++q) ss += v0[q] * v0[q];
+        store8_image(mb, mb_f32, mm.mb_off + i0, v0);  // ldc == cols on the vector path
+        if (has1) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) h[q] = __floats2bfloat162_rn(v[2 * q], v[2 * q + 1]);
-          *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(mb) + o) = u;
+          for (int q = 0; q < 8; ++q) ss += v1[q] * v1[q];
+          store8_image(mb, mb_f32, mm.mb_off + i1, v1);
         }
       }
     } else {
@@ -130,7 +159,7 @@ cudaError_t launch_momentum(const MomChunk* chunks, int nchunks, const MomMat* m
                             int mb_f32, float beta, float* partial, int vec_ok, int num_sms,
                             cudaStream_t s) {
   if (nchunks <= 0) return cudaSuccess;
-  int grid = num_sms * 8;
+  int grid = num_sms * 6;
   if (grid > nchunks) grid = nchunks;
   k_momentum<<<grid, 256, 0, s>>>(chunks, nchunks, mats, grads, momenta, grad_f32, mb, mb_f32, beta,
                                   partial, vec_ok);

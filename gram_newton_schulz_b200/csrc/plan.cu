@@ -11,7 +11,11 @@
 #include <cudaTypedefs.h>
 
 #include <cmath>
+#include <cstdio>
+#include <cstdlib>
 #include <cstring>
+#include <fstream>
+#include <sstream>
 #include <map>
 #include <string>
 #include <utility>
@@ -121,6 +125,7 @@ struct dmu_plan_s {
   float eps = 1e-7f;
   int launches = 0;
   long long timeout_ns = 2000000000LL;
+  bool cta_pair = true;  // tensor-core launches on CTA pairs (256 x 256 tiles)
 
   unsigned int* status_dev() const { return reinterpret_cast<unsigned int*>(ws + off_status); }
   float* inv_dev() const { return reinterpret_cast<float*>(ws + off_inv); }
@@ -183,13 +188,16 @@ bool aligned16(const void* const* ptrs, int n) {
   return true;
 }
 
-int tiles_for(int M, int N, bool sym, int* tm, int* tn) {
-  *tm = (M + BM - 1) / BM;
+// Tile grid of one problem for row blocks of `bm` (128: one CTA per tile;
+// 256: a CTA pair per tile) and column blocks of BN; symmetric problems keep
+// only the tiles that touch the upper triangle (same rule as the kernels).
+int tiles_for(int M, int N, bool sym, int* tm, int* tn, int bm = BM) {
+  *tm = (M + bm - 1) / bm;
   *tn = (N + BN - 1) / BN;
   if (!sym) return (*tm) * (*tn);
   int t = 0;
   for (int bj = 0; bj < *tn; ++bj) {
-    int c = ((bj + 1) * BN - 1) / BM + 1;
+    int c = ((bj + 1) * BN - 1) / bm + 1;
     t += c < *tm ? c : *tm;
   }
   return t;
@@ -226,6 +234,7 @@ dmu_status run_tc(dmu_plan p, std::vector<Prob>& probs, int na, int nb, int kind
       GemmProblem g = probs[i].g;
       g.a_map = slot(probs[i].amap);
       g.b_map = slot(probs[i].bmap);
+      g.tiles_per_mat = tiles_for(g.M, g.N, g.sym != 0, &g.tiles_m, &g.tiles_n, p->cta_pair ? 256 : BM);
       g.tile_begin = tiles;
       tiles += g.count * g.tiles_per_mat;
       gp.prob[nprob++] = g;
@@ -236,7 +245,10 @@ dmu_status run_tc(dmu_plan p, std::vector<Prob>& probs, int na, int nb, int kind
     gp.total_tiles = tiles;
     gp.status = p->status_dev();
     gp.timeout_ns = p->timeout_ns;
-    CUDA_TRY(launch_gemm_tc(gp, na, nb, kind, p->num_sms, s));
+    if (p->cta_pair)
+      CUDA_TRY(launch_gemm_tc2(gp, na, nb, kind, p->num_sms, s));
+    else
+      CUDA_TRY(launch_gemm_tc(gp, na, nb, kind, p->num_sms, s));
     p->launches++;
   }
   return DMU_OK;
@@ -709,6 +721,7 @@ dmu_status dmu_plan_create(const dmu_shape* shapes, int count, dmu_dtype dtype, 
   p->count = count;
   p->shapes.assign(shapes, shapes + count);
   p->esize = dtype == DMU_BF16 ? 2 : 4;
+  if (const char* e = std::getenv("DMU_CTA_PAIR")) p->cta_pair = std::atoi(e) != 0;
 
   int ndev = 0;
   if (cudaGetDeviceCount(&ndev) == cudaSuccess && ndev > 0) {
@@ -1151,6 +1164,88 @@ dmu_status dmu_debug_gram(dmu_plan p, int which, int index, float* out, void* st
 }
 
 int dmu_last_launch_count(dmu_plan p) { return p ? p->launches : 0; }
+
+// Schedule cache (DMuon page, section 2.4: tuned configs are cached and
+// reused).  The key names the device and the plan's shapes, dtype and
+// precision; the value is the chosen schedule and the times that chose it.
+static std::string schedule_key(dmu_plan p) {
+  cudaDeviceProp prop;
+  std::memset(&prop, 0, sizeof(prop));
+  cudaGetDeviceProperties(&prop, p->device);
+  std::ostringstream k;
+  std::string name = prop.name;
+  for (char& c : name)
+    if (c == ' ') c = '_';
+  k << name << "/sm" << prop.multiProcessorCount << "/d" << (int)p->dtype << "/p" << (int)p->prec;
+  unsigned long long h = 1469598103934665603ULL;  // FNV-1a over the shape list
+  for (const dmu_shape& sh : p->shapes) {
+    const int64_t v[2] = {sh.rows, sh.cols};
+    const unsigned char* b = reinterpret_cast<const unsigned char*>(v);
+    for (size_t i = 0; i < sizeof(v); ++i) h = (h ^ b[i]) * 1099511628211ULL;
+  }
+  k << "/n" << p->count << "/h" << std::hex << h;
+  return k.str();
+}
+
+int dmu_get_schedule(dmu_plan p) { return p ? (p->cta_pair ? 1 : 0) : -1; }
+
+dmu_status dmu_autotune(dmu_plan p, const char* cache_path, void* stream) {
+  g_err.clear();
+  dmu_status st = check_plan(p, true);
+  if (st != DMU_OK) return st;
+  if (!p->have_mb) return fail(DMU_ERR_NOT_PLANNED, "call dmu_momentum_normalize before dmu_autotune");
+  if (p->dtype != DMU_BF16) return DMU_OK;  // one schedule on the fp32 path
+  DevGuard dg(p->device);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const std::string key = schedule_key(p);
+  if (cache_path) {
+    std::ifstream in(cache_path);
+    std::string line;
+    while (std::getline(in, line)) {
+      std::istringstream ls(line);
+      std::string k;
+      int pair = -1;
+      if ((ls >> k >> pair) && k == key && (pair == 0 || pair == 1)) {
+        p->cta_pair = pair == 1;
+        return DMU_OK;
+      }
+    }
+  }
+  const float co[3] = {3.4445f, -4.7750f, 2.0315f};
+  float ms[2] = {0.f, 0.f};
+  cudaEvent_t e0, e1;
+  CUDA_TRY(cudaEventCreate(&e0));
+  CUDA_TRY(cudaEventCreate(&e1));
+  const bool keep = p->cta_pair;
+  for (int variant = 0; variant < 2; ++variant) {
+    p->cta_pair = variant == 1;
+    st = gram_bf16(p, co, 5, s);  // warm-up
+    for (int rep = 0; st == DMU_OK && rep < 3; ++rep) {
+      CUDA_TRY(cudaEventRecord(e0, s));
+      st = gram_bf16(p, co, 5, s);
+      CUDA_TRY(cudaEventRecord(e1, s));
+      CUDA_TRY(cudaEventSynchronize(e1));
+      float t = 0.f;
+      CUDA_TRY(cudaEventElapsedTime(&t, e0, e1));
+      ms[variant] = rep == 0 ? t : std::min(ms[variant], t);
+    }
+    if (st != DMU_OK) {
+      p->cta_pair = keep;
+      cudaEventDestroy(e0);
+      cudaEventDestroy(e1);
+      return st;
+    }
+  }
+  cudaEventDestroy(e0);
+  cudaEventDestroy(e1);
+  p->cta_pair = ms[1] <= ms[0];
+  p->have_p = true;
+  if (cache_path) {
+    std::ofstream out(cache_path, std::ios::app);
+    if (out) out << key << " " << (p->cta_pair ? 1 : 0) << " pair_ms=" << ms[1] << " single_ms=" << ms[0] << "\n";
+  }
+  return DMU_OK;
+}
 
 void dmu_plan_destroy(dmu_plan p) {
   if (!p) return;

@@ -44,6 +44,8 @@ SIGNATURES = {
     "dmu_last_error": (ctypes.c_char_p, []),
     "dmu_version": (ctypes.c_int, []),
     "dmu_plan_destroy": (None, [_VP]),
+    "dmu_autotune": (ctypes.c_int, [_VP, ctypes.c_char_p, _VP]),
+    "dmu_get_schedule": (ctypes.c_int, [_VP]),
     "dmu_momentum_norm_static": (ctypes.c_int, [_VP, _VP, _VP, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
                                                 ctypes.c_float, ctypes.c_float, _VP, _VP]),
 }
@@ -196,6 +198,13 @@ class Plan:
         self.momentum_normalize(grads, momenta, beta, eps, stream)
         self.gram_ns_batched(None, coeffs, steps, stream)
         self.apply_update(weights, lr, out_o, stream)
+
+    def autotune(self, cache_path: Optional[str] = None, stream=None) -> int:
+        """Choose the faster tensor-core schedule by measurement (needs a prior
+        momentum_normalize); returns 1 for CTA pairs, 0 for single CTAs."""
+        _check(self.lib.dmu_autotune(self.handle, cache_path.encode() if cache_path else None,
+                                     _stream_handle(stream, self.device)))
+        return int(self.lib.dmu_get_schedule(self.handle))
 
     def read_status(self) -> int:
         flags = ctypes.c_uint32(0)

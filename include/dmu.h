@@ -48,6 +48,10 @@
  *     to dmu_plan_create.  Device pointers must be 16-byte aligned for the
  *     vectorised paths (misaligned pointers take a scalar path).
  *   - Threads: a plan must not be used by two host threads at once.
+ *   - Schedule: tensor-core launches run on CTA pairs (256 x 256 tiles,
+ *     tcgen05.mma.cta_group::2) unless the environment variable
+ *     DMU_CTA_PAIR=0 is set when the plan is created (one CTA per
+ *     128 x 256 tile).
  */
 #ifndef DMU_H
 #define DMU_H
@@ -189,6 +193,20 @@ DMU_API dmu_status dmu_read_status(dmu_plan plan, uint32_t* flags);
  *                (read it with dmu_read_status).
  * Synchronises `stream`. */
 DMU_API dmu_status dmu_debug_gram(dmu_plan plan, int which, int index, float* out, void* stream);
+
+/* Pick the faster tensor-core schedule for this plan by measurement (DMuon
+ * page, section 2.4: per-shape kernel configurations are tuned once and
+ * cached).  Times the whole Gram recursion (K = 5) with CTA-pair kernels
+ * (256 x 256 tiles) and with single-CTA kernels (128 x 256 tiles) on the
+ * data left by dmu_momentum_normalize, keeps the faster, and appends the
+ * choice to the text file `cache_path` (may be NULL: no cache).  A cached
+ * entry for the same device, shapes, dtype and precision is reused without
+ * timing.  Synchronises `stream`; overwrites the plan's Gram-space state.
+ * Errors: NOT_PLANNED (no dmu_momentum_normalize yet), CUDA. */
+DMU_API dmu_status dmu_autotune(dmu_plan plan, const char* cache_path, void* stream);
+
+/* Current schedule of the plan: 1 = CTA pairs, 0 = single CTA. */
+DMU_API int dmu_get_schedule(dmu_plan plan);
 
 /* Number of kernel launches the last compute call enqueued. */
 DMU_API int dmu_last_launch_count(dmu_plan plan);

@@ -308,3 +308,42 @@ def test_plan_errors_on_gpu():
     st = lib.dmu_gram_ns_batched(plan.handle, None, ctypes.cast(bad, ctypes.c_void_p), 1,
                                  ctypes.cast(co, ctypes.c_void_p), 5, None)
     assert st == dmu.ERR_NOT_PLANNED
+
+
+@pytest.mark.parametrize("prec", ["auto", "split3", "tf32"])
+def test_cta_pair_and_single_cta_agree(prec, monkeypatch):
+    """The CTA-pair kernels (256 x 256 tiles, cta_group::2) and the single-CTA
+    kernels (128 x 256 tiles) accumulate every element over K in the same
+    order, so they must give bitwise-equal results."""
+    shapes = [(1100, 3000), (3000, 1100), (512, 2048), (520, 200), (384, 384)]
+    w = synth.custom("pair", shapes, seed=29)
+    monkeypatch.setenv("DMU_CTA_PAIR", "1")
+    a = run_step(w, prec=prec)
+    monkeypatch.setenv("DMU_CTA_PAIR", "0")
+    b = run_step(w, prec=prec)
+    for i in range(w.count):
+        assert torch.equal(a["o"][i], b["o"][i]), shapes[i]
+        assert torch.equal(a["w_after"][i], b["w_after"][i]), shapes[i]
+
+
+def test_autotune_picks_and_caches_schedule(tmp_path):
+    shapes = [(1024, 4096), (4096, 1024), (512, 2048)]
+    w = synth.custom("tune", shapes, seed=33)
+    grads = synth.gradients(w, "cuda")
+    cache = str(tmp_path / "dmu_schedule.txt")
+    plan = dmu.Plan(shapes)
+    plan.momentum_normalize(grads, None, beta=0.0)
+    choice = plan.autotune(cache)
+    assert choice in (0, 1)
+    text = open(cache).read()
+    assert "pair_ms=" in text and "single_ms=" in text
+    # a second plan with the same shapes reuses the cached choice
+    plan2 = dmu.Plan(shapes)
+    plan2.momentum_normalize(grads, None, beta=0.0)
+    assert plan2.autotune(cache) == choice
+    assert open(cache).read() == text
+    outs = [torch.empty(s, dtype=torch.float32, device="cuda") for s in shapes]
+    plan2.gram_ns_batched(None)
+    plan2.apply_update(None, out_o=outs)
+    for i in range(len(shapes)):
+        assert rel(f64(outs[i]), oracle_o(grads[i], torch.zeros(shapes[i]), 0.0)) < 2e-2
