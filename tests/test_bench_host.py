@@ -1,0 +1,53 @@
+"""Host-side pieces of bench.py (no GPU): the algorithmic flop and byte
+counts behind the roofline fields, the workload parser, the oracle
+CPU-baseline sampler, and the reference arm's JSON line."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+import bench
+from gram_newton_schulz_b200 import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_alg_flops_closed_form():
+    # 3 m^2 n + 17 m^3 per matrix, orientation-free
+    assert bench.alg_flops([(2, 4)]) == 3 * 4 * 4 + 17 * 8
+    assert bench.alg_flops([(4, 2)]) == bench.alg_flops([(2, 4)])
+    w = synth.workload("qwen2.5-7b-layer-set-x28")
+    assert bench.alg_flops(w.shapes) == pytest.approx(1.789e14, rel=2e-3)
+
+
+def test_momentum_bytes():
+    assert bench.momentum_bytes([(10, 10)]) == 100 * 12
+    assert bench.momentum_bytes([(10, 10)], grad_bytes=4) == 100 * 14
+
+
+def test_custom_workload_parser():
+    w = bench.custom_workload("3584x3584*2,512x3584")
+    assert w.shapes == ((3584, 3584), (3584, 3584), (512, 3584))
+    assert w.dtype == "bf16" and w.dist == "spiked"
+
+
+def test_oracle_sample_is_bounded_and_scaled():
+    shapes = [(64, 256)] * 3 + [(128, 512)] * 2
+    total, threads, sample, spent = bench.oracle_sample_seconds(shapes, budget_s=5.0)
+    assert total > 0 and threads >= 1
+    assert "64x256" in sample and "scaled to 5 matrices" in sample
+    assert spent < 30
+
+
+def test_reference_arm_prints_one_json_line():
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1", "--warmup", "0",
+           "--shapes", "64x256*2", "--ref-budget", "2"]
+    out = subprocess.run(cmd, capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert out.returncode == 0, out.stderr
+    lines = [l for l in out.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "ms" and d["higher_is_better"] is False
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
