@@ -62,6 +62,13 @@ struct GemmProblem {
   int sym;              // upper-triangle tiles only, mirrored write (M == N)
   int a_map, b_map;     // indices into GemmParams::maps
   int a_mn, b_mn;       // 1: operand is MN-major (M/N contiguous)
+  // Half-stored symmetric operands: only 256 x 256 blocks (r, c) with
+  // r <= c hold data.  A K-atom of rows in block r and columns in block c
+  // is read directly (K-major, *_map) when r <= c, else as the transposed
+  // block (MN-major, *_map_t).  half_out: the output is written half-stored
+  // (whole tiles, no mirror).
+  int half_a, half_b, half_out;
+  int a_map_t, b_map_t;
   int a_z[2], b_z[2];   // z base of the hi and lo parts
   int terms;            // Terms bits
   // epilogue
@@ -153,11 +160,14 @@ cudaError_t launch_identity_bf16(__nv_bfloat16* hi, __nv_bfloat16* lo, int count
                                  long long ld, long long mat_stride, cudaStream_t s);
 cudaError_t launch_identity_f32(float* p, int count, int m, long long ld, long long mat_stride,
                                 cudaStream_t s);
+// Test-hook conversions; `half` reads a half-stored symmetric matrix
+// (element (r, c) with block(r) > block(c) comes from (c, r)).
 cudaError_t launch_pair_to_f32(const __nv_bfloat16* hi, const __nv_bfloat16* lo, long long rows,
-                               long long cols, long long ld, float* out, cudaStream_t s);
+                               long long cols, long long ld, float* out, cudaStream_t s, int half = 0);
 cudaError_t launch_pair_h_to_f32(const void* hi, const void* lo, long long rows, long long cols, long long ld,
-                                 float scale, float* out, cudaStream_t s);
+                                 float scale, float* out, cudaStream_t s, int half = 0);
 cudaError_t launch_f32_copy2d(const float* src, long long rows, long long cols, long long ld,
                               float* out, cudaStream_t s);
+constexpr int HALF_BLOCK = 256;  // block size of half-stored symmetric matrices
 
 }  // namespace dmu

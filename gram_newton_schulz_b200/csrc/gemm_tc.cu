@@ -165,8 +165,10 @@ constexpr int CW = 16;
 
 // One CW-column chunk of a Gram-space output tile for the thread's row i.
 // Input and outputs are bf16 hi/lo pairs (FMT_PAIR) or fp32 (FMT_F32).
+// `tri`: store only i <= j and mirror (symmetric outputs, except the
+// off-diagonal tiles of half-stored outputs, which are written whole).
 __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, int i, int col0,
-                                               const uint32_t (&r)[CW]) {
+                                               const uint32_t (&r)[CW], bool tri) {
   const int M = pr.M, N = pr.N;
   if (i >= M) return;
   float coef = pr.alpha;
@@ -183,7 +185,7 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
   const long long mbase = (long long)mat * pr.mat_stride;
   const long long rowoff = mbase + (long long)i * pr.ld;
   const bool full = (col0 + CW <= N);
-  const bool all_upper = !pr.sym || (i <= col0);
+  const bool all_upper = !tri || (i <= col0);
 
   if (pr.cin_fmt == FMT_F32 && pr.cin_f) {
     if (full) {
@@ -287,10 +289,10 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
 #pragma unroll
         for (int c = 0; c < CW; ++c) {
           const int j = col0 + c;
-          if (j < N && (!pr.sym || i <= j)) store_pair_h(oh, ol, rowoff + j, v[c]);
+          if (j < N && (!tri || i <= j)) store_pair_h(oh, ol, rowoff + j, v[c]);
         }
       }
-      if (pr.sym) {
+      if (tri) {
 #pragma unroll
         for (int c = 0; c < CW; ++c) {
           const int j = col0 + c;
@@ -310,10 +312,10 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
 #pragma unroll
         for (int c = 0; c < CW; ++c) {
           const int j = col0 + c;
-          if (j < N && (!pr.sym || i <= j)) of[rowoff + j] = v[c];
+          if (j < N && (!tri || i <= j)) of[rowoff + j] = v[c];
         }
       }
-      if (pr.sym) {
+      if (tri) {
 #pragma unroll
         for (int c = 0; c < CW; ++c) {
           const int j = col0 + c;
@@ -340,12 +342,12 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
 #pragma unroll
       for (int c = 0; c < CW; ++c) {
         const int j = col0 + c;
-        if (j < N && (!pr.sym || i <= j)) store_pair(oh, ol, rowoff + j, v[c]);
+        if (j < N && (!tri || i <= j)) store_pair(oh, ol, rowoff + j, v[c]);
       }
     }
     // mirrored stores (j, i) for j > i: consecutive lanes write consecutive
     // columns of row j, so each store instruction is coalesced.
-    if (pr.sym) {
+    if (tri) {
 #pragma unroll
       for (int c = 0; c < CW; ++c) {
         const int j = col0 + c;
@@ -531,25 +533,30 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
           const int k0 = kb * BKE;
           const uint32_t sa = ring + stage * Cfg::STAGE_BYTES;
           const uint32_t sb = sa + NA * A_PART_BYTES;
+          const int ktile = k0 / HALF_BLOCK;
+          const bool a_t = pr.half_a && (arow / HALF_BLOCK) > ktile;  // read the transposed block
+          const bool b_t = pr.half_b && (brow / HALF_BLOCK) > ktile;
+          const CUtensorMap* am_k = a_t ? &p.maps[pr.a_map_t] : am;
+          const CUtensorMap* bm_k = b_t ? &p.maps[pr.b_map_t] : bm;
           for (int part = 0; part < na; ++part) {
             const uint32_t dst = sa + part * A_PART_BYTES;
             const int z = pr.a_z[part] + tc.mat;
-            if (!pr.a_mn) {
-              ptx::tma_load_3d(dst, am, fb, k0, arow, z);
+            if (!pr.a_mn && !a_t) {
+              ptx::tma_load_3d(dst, am_k, fb, k0, arow, z);
             } else {
-              ptx::tma_load_3d(dst, am, fb, arow, k0, z);
-              ptx::tma_load_3d(dst + 8192, am, fb, arow + 64, k0, z);
+              ptx::tma_load_3d(dst, am_k, fb, arow, k0, z);
+              ptx::tma_load_3d(dst + 8192, am_k, fb, arow + 64, k0, z);
             }
           }
           for (int part = 0; part < nb; ++part) {
             const uint32_t dst = sb + part * B_PART_BYTES;
             const int z = pr.b_z[part] + tc.mat;
-            if (!pr.b_mn) {
-              ptx::tma_load_3d(dst, bm, fb, k0, brow, z);
-              ptx::tma_load_3d(dst + 16384, bm, fb, k0, brow + 128, z);
+            if (!pr.b_mn && !b_t) {
+              ptx::tma_load_3d(dst, bm_k, fb, k0, brow, z);
+              ptx::tma_load_3d(dst + 16384, bm_k, fb, k0, brow + 128, z);
             } else {
 #pragma unroll
-              for (int c = 0; c < 4; ++c) ptx::tma_load_3d(dst + 8192 * c, bm, fb, brow + 64 * c, k0, z);
+              for (int c = 0; c < 4; ++c) ptx::tma_load_3d(dst + 8192 * c, bm_k, fb, brow + 64 * c, k0, z);
             }
           }
           if (++stage == S) {
@@ -586,17 +593,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
         const TileCoord tc = decode_tile<BM>(p, t);
         const GemmProblem& pr = p.prob[tc.pi];
         const int nk = (pr.K + BKE - 1) / BKE;
-        const uint32_t idesc = ptx::make_idesc(BM, BN, pr.a_mn, pr.b_mn, OPFMT);
         if (!wait_bar(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        const uint32_t a_lbo = pr.a_mn ? 8192u : 16u, a_sbo = 1024u;
-        const uint32_t b_lbo = pr.b_mn ? 8192u : 16u, b_sbo = 1024u;
-        const uint32_t a_kstep = pr.a_mn ? 2048u : 32u;
-        const uint32_t b_kstep = pr.b_mn ? 2048u : 32u;
+        const uint32_t a_sbo = 1024u, b_sbo = 1024u;
+        const int arow_blk = (tc.bi * BM) / HALF_BLOCK, brow_blk = (tc.bj * BN) / HALF_BLOCK;
         uint32_t accumulate = 0;
         for (int kb = 0; kb < nk; ++kb) {
           if (!wait_bar(full_bar(stage), phase, abort_flag, p)) {
@@ -604,6 +608,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
             break;
           }
           ptx::tc_fence_after();
+          const int ktile = (kb * BKE) / HALF_BLOCK;
+          const int a_mn = pr.a_mn | ((pr.half_a && arow_blk > ktile) ? 1 : 0);
+          const int b_mn = pr.b_mn | ((pr.half_b && brow_blk > ktile) ? 1 : 0);
+          const uint32_t idesc = ptx::make_idesc(BM, BN, a_mn, b_mn, OPFMT);
+          const uint32_t a_lbo = a_mn ? 8192u : 16u, b_lbo = b_mn ? 8192u : 16u;
+          const uint32_t a_kstep = a_mn ? 2048u : 32u, b_kstep = b_mn ? 2048u : 32u;
           const uint32_t sa = ring + stage * Cfg::STAGE_BYTES;
           const uint32_t sb = sa + NA * A_PART_BYTES;
 #pragma unroll
@@ -665,17 +675,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
       if (!ok) break;
       ptx::tc_fence_after();
       const int row_lo = tc.bi * BM + q * 32;
+      const bool tri = pr.sym && (!pr.half_out || (tc.bi * BM) / HALF_BLOCK == tc.bj);
       const int i = row_lo + lane;
       for (int ch = ch_begin; ch < ch_end; ++ch) {
         const int col0 = tc.bj * BN + ch * CW;
         if (col0 >= pr.N) break;
-        if (pr.sym && col0 + CW - 1 < row_lo) continue;  // chunk strictly below the diagonal
+        if (tri && col0 + CW - 1 < row_lo) continue;  // chunk strictly below the diagonal
         if (row_lo >= pr.M) break;
         uint32_t r[CW];
         ptx::tmem_ld16(tmem_base + (uint32_t)(acc * BN + ch * CW) + ((uint32_t)(q * 32) << 16), r);
         ptx::tmem_wait_ld();
         if (pr.epi == EPI_GRAM)
-          epi_gram_chunk(pr, tc.mat, i, col0, r);
+          epi_gram_chunk(pr, tc.mat, i, col0, r, tri);
         else
           epi_update_chunk(pr, tc.mat, i, col0, r);
       }
@@ -711,9 +722,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
 constexpr int BM2 = 256;
 constexpr int HALF_BYTES = 128 * 128;  // 128 rows x 128-byte K row
 
+// K atoms (128-byte rows) per stage: measured on the GPU, every stage
+// boundary costs ~700 cycles of MMA-pipe time beyond the MMAs themselves,
+// so the one-MMA-per-slice configurations take two atoms (8 MMAs) per
+// stage; the split configurations already issue 8-12 MMAs per atom.
 template <int NA, int NB>
 struct Tc2Cfg {
-  static constexpr int STAGE_BYTES = (NA + NB) * HALF_BYTES;
+  static constexpr int KAT = (NA + NB <= 2) ? 2 : 1;
+  static constexpr int STAGE_BYTES = (NA + NB) * HALF_BYTES * KAT;
   static constexpr int STAGES = (200 * 1024) / STAGE_BYTES;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
   static_assert(STAGES >= 2 && STAGES <= 8, "stage count");
@@ -743,7 +759,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     k_gemm_tc2(const __grid_constant__ GemmParams p) {
   using Cfg = Tc2Cfg<NA, NB>;
   constexpr int S = Cfg::STAGES;
-  constexpr int BKE = KIND == KIND_TF32 ? 32 : 64;
+  constexpr int KATOMS = Cfg::KAT;
+  constexpr int ATOM_E = KIND == KIND_TF32 ? 32 : 64;  // elements per 128-byte K row
+  constexpr int BKE = ATOM_E * KATOMS;                 // K elements per stage
   constexpr int OPFMT = KIND == KIND_TF32 ? 2 : (KIND == KIND_F16 ? 0 : 1);
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = ptx::smem_u32(smem_raw);
@@ -810,7 +828,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         const CUtensorMap* bm = &p.maps[pr.b_map];
         const int na = (NA > 1 && (pr.terms & TERM_LH)) ? 2 : 1;
         const int nb = (NB > 1 && (pr.terms & TERM_HL)) ? 2 : 1;
-        const uint32_t bytes_pair = 2u * (uint32_t)(na + nb) * HALF_BYTES;
+        const uint32_t bytes_pair = 2u * (uint32_t)(na + nb) * HALF_BYTES * KATOMS;
         const int nk = (pr.K + BKE - 1) / BKE;
         const int arow = tc.bi * BM2 + (int)rank * 128, brow = tc.bj * BN + (int)rank * 128;
         for (int kb = 0; kb < nk; ++kb) {
@@ -824,27 +842,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
             issued_mask |= 1u << stage;
             issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
           }
-          const int k0 = kb * BKE;
+          // stage layout: [A parts][B parts], each part KATOMS 16 KB atoms
           const uint32_t sa = ring + stage * Cfg::STAGE_BYTES;
-          const uint32_t sb = sa + NA * HALF_BYTES;
-          for (int part = 0; part < na; ++part) {
-            const uint32_t dst = sa + part * HALF_BYTES;
-            const int z = pr.a_z[part] + tc.mat;
-            if (!pr.a_mn) {
-              ptx::tma_load_3d_pair(dst, am, fb_leader, k0, arow, z);
-            } else {
-              ptx::tma_load_3d_pair(dst, am, fb_leader, arow, k0, z);
-              ptx::tma_load_3d_pair(dst + 8192, am, fb_leader, arow + 64, k0, z);
+          const uint32_t sb = sa + NA * KATOMS * HALF_BYTES;
+          for (int at = 0; at < KATOMS; ++at) {
+            const int k0 = kb * BKE + at * ATOM_E;
+            const int ktile = k0 / HALF_BLOCK;
+            const bool a_t = pr.half_a && tc.bi > ktile;  // rows of block bi, K in an earlier block
+            const bool b_t = pr.half_b && tc.bj > ktile;
+            const CUtensorMap* am_k = a_t ? &p.maps[pr.a_map_t] : am;
+            const CUtensorMap* bm_k = b_t ? &p.maps[pr.b_map_t] : bm;
+            for (int part = 0; part < na; ++part) {
+              const uint32_t dst = sa + (part * KATOMS + at) * HALF_BYTES;
+              const int z = pr.a_z[part] + tc.mat;
+              if (!pr.a_mn && !a_t) {
+                ptx::tma_load_3d_pair(dst, am_k, fb_leader, k0, arow, z);
+              } else {
+                ptx::tma_load_3d_pair(dst, am_k, fb_leader, arow, k0, z);
+                ptx::tma_load_3d_pair(dst + 8192, am_k, fb_leader, arow + 64, k0, z);
+              }
             }
-          }
-          for (int part = 0; part < nb; ++part) {
-            const uint32_t dst = sb + part * HALF_BYTES;
-            const int z = pr.b_z[part] + tc.mat;
-            if (!pr.b_mn) {
-              ptx::tma_load_3d_pair(dst, bm, fb_leader, k0, brow, z);
-            } else {
-              ptx::tma_load_3d_pair(dst, bm, fb_leader, brow, k0, z);
-              ptx::tma_load_3d_pair(dst + 8192, bm, fb_leader, brow + 64, k0, z);
+            for (int part = 0; part < nb; ++part) {
+              const uint32_t dst = sb + (part * KATOMS + at) * HALF_BYTES;
+              const int z = pr.b_z[part] + tc.mat;
+              if (!pr.b_mn && !b_t) {
+                ptx::tma_load_3d_pair(dst, bm_k, fb_leader, k0, brow, z);
+              } else {
+                ptx::tma_load_3d_pair(dst, bm_k, fb_leader, brow, k0, z);
+                ptx::tma_load_3d_pair(dst + 8192, bm_k, fb_leader, brow + 64, k0, z);
+              }
             }
           }
           if (++stage == S) {
@@ -881,15 +907,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         const TileCoord tc = decode_tile<BM2>(p, t);
         const GemmProblem& pr = p.prob[tc.pi];
         const int nk = (pr.K + BKE - 1) / BKE;
-        const uint32_t idesc = ptx::make_idesc(BM2, BN, pr.a_mn, pr.b_mn, OPFMT);
         if (!wait_bar_cluster(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        const uint32_t a_lbo = pr.a_mn ? 8192u : 16u, b_lbo = pr.b_mn ? 8192u : 16u;
-        const uint32_t a_kstep = pr.a_mn ? 2048u : 32u, b_kstep = pr.b_mn ? 2048u : 32u;
         uint32_t accumulate = 0;
         for (int kb = 0; kb < nk; ++kb) {
           if (!wait_bar_cluster(full_bar(stage), phase, abort_flag, p)) {
@@ -898,16 +921,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
           }
           ptx::tc_fence_after();
           const uint32_t sa = ring + stage * Cfg::STAGE_BYTES;
-          const uint32_t sb = sa + NA * HALF_BYTES;
+          const uint32_t sb = sa + NA * KATOMS * HALF_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
+          for (int kq = 0; kq < 4 * KATOMS; ++kq) {
+            const int at = kq >> 2, kk = kq & 3;
+            const int ktile = (kb * BKE + at * ATOM_E) / HALF_BLOCK;
+            const int a_mn = pr.a_mn | ((pr.half_a && tc.bi > ktile) ? 1 : 0);
+            const int b_mn = pr.b_mn | ((pr.half_b && tc.bj > ktile) ? 1 : 0);
+            const uint32_t idesc = ptx::make_idesc(BM2, BN, a_mn, b_mn, OPFMT);
+            const uint32_t a_lbo = a_mn ? 8192u : 16u, b_lbo = b_mn ? 8192u : 16u;
+            const uint32_t a_kstep = a_mn ? 2048u : 32u, b_kstep = b_mn ? 2048u : 32u;
 #pragma unroll
             for (int term = 0; term < 3; ++term) {
               if (!(pr.terms & (1 << term))) continue;
               if (term == 1 && NB < 2) continue;
               if (term == 2 && NA < 2) continue;
-              const uint32_t pa = sa + (term == 2 ? HALF_BYTES : 0);
-              const uint32_t pb = sb + (term == 1 ? HALF_BYTES : 0);
+              const uint32_t pa = sa + ((term == 2 ? KATOMS : 0) + at) * HALF_BYTES;
+              const uint32_t pb = sb + ((term == 1 ? KATOMS : 0) + at) * HALF_BYTES;
               const uint64_t ad = ptx::make_sw128_desc(pa + kk * a_kstep, a_lbo, 1024u);
               const uint64_t bd = ptx::make_sw128_desc(pb + kk * b_kstep, b_lbo, 1024u);
               if (KIND == KIND_TF32)
@@ -956,17 +986,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       if (!ok) break;
       ptx::tc_fence_after();
       const int row_lo = tc.bi * BM2 + (int)rank * 128 + q * 32;
+      const bool tri = pr.sym && (!pr.half_out || tc.bi == tc.bj);
       const int i = row_lo + lane;
       for (int ch = ch_begin; ch < ch_end; ++ch) {
         const int col0 = tc.bj * BN + ch * CW;
         if (col0 >= pr.N) break;
-        if (pr.sym && col0 + CW - 1 < row_lo) continue;
+        if (tri && col0 + CW - 1 < row_lo) continue;
         if (row_lo >= pr.M) break;
         uint32_t r[CW];
         ptx::tmem_ld16(tmem_base + (uint32_t)(acc * BN + ch * CW) + ((uint32_t)(q * 32) << 16), r);
         ptx::tmem_wait_ld();
         if (pr.epi == EPI_GRAM)
-          epi_gram_chunk(pr, tc.mat, i, col0, r);
+          epi_gram_chunk(pr, tc.mat, i, col0, r, tri);
         else
           epi_update_chunk(pr, tc.mat, i, col0, r);
       }

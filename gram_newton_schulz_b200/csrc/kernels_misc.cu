@@ -198,25 +198,32 @@ __global__ void k_identity_f32(float* p, int count, int m, long long ld, long lo
   }
 }
 
+__device__ __forceinline__ long long half_offset(long long r, long long c, long long ld, int half) {
+  if (half && (r / HALF_BLOCK) > (c / HALF_BLOCK)) return c * ld + r;
+  return r * ld + c;
+}
+
 __global__ void k_pair_to_f32(const __nv_bfloat16* hi, const __nv_bfloat16* lo, long long rows,
-                              long long cols, long long ld, float* out) {
+                              long long cols, long long ld, float* out, int half) {
   const long long total = rows * cols;
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
        e += (long long)gridDim.x * blockDim.x) {
     const long long r = e / cols, c = e % cols;
-    float v = __bfloat162float(hi[r * ld + c]);
-    if (lo) v += __bfloat162float(lo[r * ld + c]);
+    const long long o = half_offset(r, c, ld, half);
+    float v = __bfloat162float(hi[o]);
+    if (lo) v += __bfloat162float(lo[o]);
     out[e] = v;
   }
 }
 
 __global__ void k_pair_h_to_f32(const __half* hi, const __half* lo, long long rows, long long cols,
-                                long long ld, float scale, float* out) {
+                                long long ld, float scale, float* out, int half) {
   const long long total = rows * cols;
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
        e += (long long)gridDim.x * blockDim.x) {
     const long long r = e / cols, c = e % cols;
-    out[e] = (__half2float(hi[r * ld + c]) + (lo ? __half2float(lo[r * ld + c]) : 0.f)) * scale;
+    const long long o = half_offset(r, c, ld, half);
+    out[e] = (__half2float(hi[o]) + (lo ? __half2float(lo[o]) : 0.f)) * scale;
   }
 }
 
@@ -247,15 +254,15 @@ cudaError_t launch_identity_f32(float* p, int count, int m, long long ld, long l
   return cudaGetLastError();
 }
 cudaError_t launch_pair_to_f32(const __nv_bfloat16* hi, const __nv_bfloat16* lo, long long rows,
-                               long long cols, long long ld, float* out, cudaStream_t s) {
-  k_pair_to_f32<<<grid_for(rows * cols), 256, 0, s>>>(hi, lo, rows, cols, ld, out);
+                               long long cols, long long ld, float* out, cudaStream_t s, int half) {
+  k_pair_to_f32<<<grid_for(rows * cols), 256, 0, s>>>(hi, lo, rows, cols, ld, out, half);
   return cudaGetLastError();
 }
 cudaError_t launch_pair_h_to_f32(const void* hi, const void* lo, long long rows, long long cols, long long ld,
-                                 float scale, float* out, cudaStream_t s) {
+                                 float scale, float* out, cudaStream_t s, int half) {
   k_pair_h_to_f32<<<grid_for(rows * cols), 256, 0, s>>>(reinterpret_cast<const __half*>(hi),
                                                         reinterpret_cast<const __half*>(lo), rows, cols, ld, scale,
-                                                        out);
+                                                        out, half);
   return cudaGetLastError();
 }
 cudaError_t launch_f32_copy2d(const float* src, long long rows, long long cols, long long ld, float* out,

@@ -64,6 +64,11 @@ struct GClass {
   int kind = KIND_BF16;
   int map = -1;       // TMA map over the Gram slots (bf16 pairs or fp32)
   int map_pf = -1;    // TF32 classes: bf16 map over the final-P pair
+  // Half storage (all but TF32 classes): symmetric Gram-space matrices keep
+  // only their upper 256 x 256 blocks; lower blocks are read transposed
+  // through MN-major maps (64 x 64 boxes).
+  bool half = false;
+  int map_t = -1, map_pf_t = -1;
 };
 
 enum { TBL_GRADS = 0, TBL_MOMS, TBL_W, TBL_O, TBL_IN, NUM_TBL };
@@ -126,6 +131,7 @@ struct dmu_plan_s {
   int launches = 0;
   long long timeout_ns = 2000000000LL;
   bool cta_pair = true;  // tensor-core launches on CTA pairs (256 x 256 tiles)
+  bool half_store = true;  // half-stored symmetric Gram-space matrices
 
   unsigned int* status_dev() const { return reinterpret_cast<unsigned int*>(ws + off_status); }
   float* inv_dev() const { return reinterpret_cast<float*>(ws + off_inv); }
@@ -206,7 +212,8 @@ int tiles_for(int M, int N, bool sym, int* tm, int* tn, int bm = BM) {
 // ---------------------------------------------------------------- tc launches
 struct Prob {
   GemmProblem g;
-  int amap, bmap;  // plan map indices
+  int amap, bmap;      // plan map indices
+  int amap_t = -1, bmap_t = -1;  // transposed-read maps of half-stored operands
 };
 
 dmu_status run_tc(dmu_plan p, std::vector<Prob>& probs, int na, int nb, int kind, cudaStream_t s) {
@@ -217,13 +224,16 @@ dmu_status run_tc(dmu_plan p, std::vector<Prob>& probs, int na, int nb, int kind
     std::vector<int> used;
     int nprob = 0, tiles = 0;
     while (i < probs.size() && nprob < MAX_PROBS) {
+      std::vector<int> want = {probs[i].amap, probs[i].bmap};
+      if (probs[i].amap_t >= 0) want.push_back(probs[i].amap_t);
+      if (probs[i].bmap_t >= 0) want.push_back(probs[i].bmap_t);
       int need = 0;
-      bool fa = false, fb = false;
-      for (int u : used) {
-        fa |= (u == probs[i].amap);
-        fb |= (u == probs[i].bmap);
+      for (size_t w = 0; w < want.size(); ++w) {
+        bool seen = false;
+        for (int u : used) seen |= (u == want[w]);
+        for (size_t v = 0; v < w; ++v) seen |= (want[v] == want[w]);
+        need += seen ? 0 : 1;
       }
-      need = (fa ? 0 : 1) + (fb || probs[i].bmap == probs[i].amap ? 0 : 1);
       if ((int)used.size() + need > MAX_MAPS) break;
       auto slot = [&](int pm) {
         for (size_t k = 0; k < used.size(); ++k)
@@ -234,6 +244,8 @@ dmu_status run_tc(dmu_plan p, std::vector<Prob>& probs, int na, int nb, int kind
       GemmProblem g = probs[i].g;
       g.a_map = slot(probs[i].amap);
       g.b_map = slot(probs[i].bmap);
+      g.a_map_t = probs[i].amap_t >= 0 ? slot(probs[i].amap_t) : g.a_map;
+      g.b_map_t = probs[i].bmap_t >= 0 ? slot(probs[i].bmap_t) : g.b_map;
       g.tiles_per_mat = tiles_for(g.M, g.N, g.sym != 0, &g.tiles_m, &g.tiles_n, p->cta_pair ? 256 : BM);
       g.tile_begin = tiles;
       tiles += g.count * g.tiles_per_mat;
@@ -303,6 +315,10 @@ Prob gram_prob(dmu_plan p, int c, int a_slot, int b_slot, int terms, float alpha
   g.ld = gc.ldg;
   g.mat_stride = gc.m * gc.ldg;
   pr.amap = pr.bmap = gc.map;
+  if (gc.half) {
+    g.half_a = g.half_b = g.half_out = 1;
+    pr.amap_t = pr.bmap_t = gc.map_t;
+  }
   return pr;
 }
 
@@ -408,6 +424,10 @@ Prob gram_prob_h(dmu_plan p, int c, int a_slot, int b_slot, float alpha, float b
   g.ld = gc.ldg;
   g.mat_stride = gc.m * gc.ldg;
   pr.amap = pr.bmap = gc.map;
+  if (gc.half) {
+    g.half_a = g.half_b = g.half_out = 1;
+    pr.amap_t = pr.bmap_t = gc.map_t;
+  }
   return pr;
 }
 
@@ -526,6 +546,7 @@ dmu_status gram_bf16(dmu_plan p, const float co[3], int steps, cudaStream_t s) {
     g.ld = gc.ldg;
     g.mat_stride = gc.m * gc.ldg;
     pr.amap = pr.bmap = b.tall ? b.map_mn : b.map_k;
+    g.half_out = gc.half ? 1 : 0;
     syrk.push_back(pr);
   }
   dmu_status st = run_tc(p, syrk, 1, 1, KIND_BF16, s);
@@ -722,6 +743,7 @@ dmu_status dmu_plan_create(const dmu_shape* shapes, int count, dmu_dtype dtype, 
   p->shapes.assign(shapes, shapes + count);
   p->esize = dtype == DMU_BF16 ? 2 : 4;
   if (const char* e = std::getenv("DMU_CTA_PAIR")) p->cta_pair = std::atoi(e) != 0;
+  if (const char* e = std::getenv("DMU_HALF")) p->half_store = std::atoi(e) != 0;
 
   int ndev = 0;
   if (cudaGetDeviceCount(&ndev) == cudaSuccess && ndev > 0) {
@@ -767,6 +789,7 @@ dmu_status dmu_plan_create(const dmu_shape* shapes, int count, dmu_dtype dtype, 
           else
             g.prec = prec;
           g.kind = g.prec == DMU_PREC_TF32 ? KIND_TF32 : (g.prec == DMU_PREC_F16 ? KIND_F16 : KIND_BF16);
+          g.half = g.kind != KIND_TF32 && p->half_store;
         }
         cidx[b.m] = (int)p->classes.size();
         p->classes.push_back(g);
@@ -910,19 +933,31 @@ dmu_status dmu_set_workspace(dmu_plan p, void* dev_ptr, size_t bytes) {
         p->maps.push_back(mp);
       } else {
         const uint64_t s1 = (uint64_t)g.ldg * 2, s2 = (uint64_t)g.m * g.ldg * 2;
+        const CUtensorMapDataType dt =
+            g.kind == KIND_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
         st = encode_map(&mg, p->ws + g.off, (uint64_t)g.m, (uint64_t)g.m, (uint64_t)NUM_SLOTS * g.count, s1,
-                        s2, 64, 128,
-                        g.kind == KIND_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+                        s2, 64, 128, dt);
         if (st != DMU_OK) return st;
         g.map = (int)p->maps.size();
         p->maps.push_back(mg);
+        CUtensorMap mt;  // transposed reads of half-stored blocks
+        st = encode_map(&mt, p->ws + g.off, (uint64_t)g.m, (uint64_t)g.m, (uint64_t)NUM_SLOTS * g.count, s1,
+                        s2, 64, 64, dt);
+        if (st != DMU_OK) return st;
+        g.map_t = (int)p->maps.size();
+        p->maps.push_back(mt);
         if (g.kind == KIND_F16) {
-          CUtensorMap mp;
+          CUtensorMap mp, mpt;
           st = encode_map(&mp, p->ws + g.off_pf, (uint64_t)g.m, (uint64_t)g.m, (uint64_t)2 * g.count, s1, s2, 64,
                           128);
           if (st != DMU_OK) return st;
           g.map_pf = (int)p->maps.size();
           p->maps.push_back(mp);
+          st = encode_map(&mpt, p->ws + g.off_pf, (uint64_t)g.m, (uint64_t)g.m, (uint64_t)2 * g.count, s1, s2, 64,
+                          64);
+          if (st != DMU_OK) return st;
+          g.map_pf_t = (int)p->maps.size();
+          p->maps.push_back(mpt);
         }
       }
     }
@@ -1035,6 +1070,10 @@ dmu_status dmu_apply_update(dmu_plan p, void* const* weights, float lr, float* c
       g.w_cols = b.cols;
       pr.amap = gc.kind != KIND_BF16 ? gc.map_pf : gc.map;
       pr.bmap = b.tall ? b.map_k : b.map_mn;
+      if (gc.half) {
+        g.half_a = 1;
+        pr.amap_t = gc.kind != KIND_BF16 ? gc.map_pf_t : gc.map_t;
+      }
       probs.push_back(pr);
     }
     return run_tc(p, probs, 2, 1, KIND_BF16, s);
@@ -1131,16 +1170,17 @@ dmu_status dmu_debug_gram(dmu_plan p, int which, int index, float* out, void* st
   const size_t moff = (size_t)(bk->cls_off + local) * gc.m * gc.ldg;
   int q = which;
   if (which == 7) q = p->p_final == 0 ? 3 : 4;
+  const int hf = gc.half ? 1 : 0;
   if (p->dtype == DMU_BF16 && gc.kind == KIND_F16) {
     if (which == 7) {
       CUDA_TRY(launch_pair_to_f32(p->pf_bf16(bk->cls, 0) + moff, p->pf_bf16(bk->cls, 1) + moff, gc.m, gc.m,
-                                  gc.ldg, out, s));
+                                  gc.ldg, out, s, hf));
     } else {
       const int slots[5] = {SLOT_G_HI, SLOT_R_HI, SLOT_T_HI, SLOT_PA_HI, SLOT_PB_HI};
       const int sh = slots[q];
       CUDA_TRY(launch_pair_h_to_f32(p->slot_bf16(bk->cls, sh) + moff,
                                     sh == SLOT_R_HI ? nullptr : p->slot_bf16(bk->cls, sh + 1) + moff, gc.m, gc.m,
-                                    gc.ldg, 1.f / half_slot_scale(sh), out, s));
+                                    gc.ldg, 1.f / half_slot_scale(sh), out, s, hf));
     }
   } else if (p->dtype == DMU_BF16 && gc.kind == KIND_TF32) {
     if (which == 7) {
@@ -1155,7 +1195,7 @@ dmu_status dmu_debug_gram(dmu_plan p, int which, int index, float* out, void* st
     const bool has_lo = !(sh == SLOT_R_HI && gc.prec == DMU_PREC_FAST);
     CUDA_TRY(launch_pair_to_f32(p->slot_bf16(bk->cls, sh) + moff,
                                 has_lo ? p->slot_bf16(bk->cls, sh + 1) + moff : nullptr, gc.m, gc.m, gc.ldg,
-                                out, s));
+                                out, s, hf));
   } else {
     CUDA_TRY(launch_f32_copy2d(p->slot_f32(bk->cls, q) + moff, gc.m, gc.m, gc.ldg, out, s));
   }

@@ -73,7 +73,7 @@ def test_gram_intermediates_k1_k2(prec, tol):
     for i in range(len(shapes)):
         r0 = plan.debug(1, i).cpu().numpy()
         p1 = plan.debug(7, i).cpu().numpy()
-        assert np.array_equal(p1, p1.T)
+        _assert_symmetric(p1)
         assert rel(r0, traces[i][0]["R"]) < tol, ("R0", shapes[i], rel(r0, traces[i][0]["R"]))
         assert rel(p1, traces[i][0]["P"]) < tol, ("P1", shapes[i], rel(p1, traces[i][0]["P"]))
     # two steps: G_1, T_0, R_1, P_2
@@ -82,7 +82,7 @@ def test_gram_intermediates_k1_k2(prec, tol):
         tr = traces[i]
         got = {k: plan.debug(j, i).cpu().numpy() for k, j in (("G", 0), ("R", 1), ("T", 2), ("P", 7))}
         for k in got:
-            assert np.array_equal(got[k], got[k].T), (k, shapes[i])
+            _assert_symmetric(got[k], (k, shapes[i]))
         assert rel(got["T"], tr[0]["T"]) < tol, ("T0", shapes[i], rel(got["T"], tr[0]["T"]))
         assert rel(got["G"], tr[1]["G"]) < tol, ("G1", shapes[i], rel(got["G"], tr[1]["G"]))
         assert rel(got["R"], tr[1]["R"]) < tol, ("R1", shapes[i], rel(got["R"], tr[1]["R"]))
@@ -93,9 +93,20 @@ def _bf16(x):
     return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16).double().numpy()
 
 
+def _mirrored(d):
+    """A symmetric product as the kernels store it: the upper triangle, and
+    its mirror image below (whether the lower blocks are written or read
+    back as transposed upper blocks)."""
+    return np.triu(d) + np.triu(d, 1).T
+
+
+def _assert_symmetric(x, what=None):
+    assert np.array_equal(x, x.T), what
+
+
 def _emul_product(a, b, prec):
-    """The upper-triangle, mirrored bf16 product each precision mode issues,
-    in fp64 from the GPU's own operands (hi + lo pairs)."""
+    """The half-stored bf16 product each precision mode issues, in fp64 from
+    the GPU's own operands (hi + lo pairs)."""
     ah, bh = _bf16(a), _bf16(b)
     al, bl = _bf16(a - ah), _bf16(b - bh)
     d = ah @ bh
@@ -103,7 +114,7 @@ def _emul_product(a, b, prec):
         d = d + al @ bh
     if prec in ("split3",):
         d = d + ah @ bl + al @ bh
-    return np.triu(d) + np.triu(d, 1).T
+    return _mirrored(d)
 
 
 @pytest.mark.parametrize("prec", ["fast", "split2", "split3"])
@@ -112,7 +123,7 @@ def test_products_match_emulation(prec):
     terms the mode issues, on the operands read back from the GPU: checks
     the kernel, not the method's conditioning."""
     a, b, c = dmu.QUINTIC
-    shapes = [(128, 512), (384, 384), (520, 200)]
+    shapes = [(128, 512), (384, 384), (520, 200), (300, 700)]
     w, grads, plan = _plan_inputs(shapes, 13, prec=prec)
     plan.momentum_normalize(grads, None, beta=0.0, eps=EPS)
     plan.gram_ns_batched(None, dmu.QUINTIC, 2)
@@ -144,13 +155,14 @@ def test_tf32_f16_products_accuracy(prec):
     for i in range(len(shapes)):
         d = {k: plan.debug(j, i).cpu().numpy().astype(np.float64) for k, j in
              (("G", 0), ("R", 1), ("PA", 3), ("P", 7))}
+        store = _mirrored
         gg = d["G"] @ d["G"]
-        r_ref = b * d["G"] + c * (np.triu(gg) + np.triu(gg, 1).T)
+        r_ref = b * d["G"] + c * store(gg)
         assert rel(d["R"], r_ref) < 1e-3, ("R", shapes[i], rel(d["R"], r_ref))
         rp = d["R"] @ d["PA"]
-        p_ref = a * d["PA"] + (np.triu(rp) + np.triu(rp, 1).T)
+        p_ref = a * d["PA"] + store(rp)
         assert rel(d["P"], p_ref) < 1e-3, ("P", shapes[i], rel(d["P"], p_ref))
-        assert np.array_equal(d["P"], d["P"].T)
+        _assert_symmetric(d["P"])
 
 
 @pytest.mark.parametrize("prec", ["tf32", "f16", "auto"])
@@ -308,6 +320,21 @@ def test_plan_errors_on_gpu():
     st = lib.dmu_gram_ns_batched(plan.handle, None, ctypes.cast(bad, ctypes.c_void_p), 1,
                                  ctypes.cast(co, ctypes.c_void_p), 5, None)
     assert st == dmu.ERR_NOT_PLANNED
+
+
+@pytest.mark.parametrize("prec", ["auto", "split3"])
+def test_half_and_full_storage_agree(prec, monkeypatch):
+    """Half-stored symmetric matrices (upper blocks only, lower blocks read
+    transposed) must give bitwise the results of fully mirrored storage."""
+    shapes = [(1100, 3000), (3000, 1100), (520, 200), (700, 700)]
+    w = synth.custom("half", shapes, seed=31)
+    monkeypatch.setenv("DMU_HALF", "1")
+    a = run_step(w, prec=prec)
+    monkeypatch.setenv("DMU_HALF", "0")
+    b = run_step(w, prec=prec)
+    for i in range(w.count):
+        assert torch.equal(a["o"][i], b["o"][i]), shapes[i]
+        assert torch.equal(a["w_after"][i], b["w_after"][i]), shapes[i]
 
 
 @pytest.mark.parametrize("prec", ["auto", "split3", "tf32"])
