@@ -514,13 +514,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
       for (int t = blockIdx.x; ok && t < p.total_tiles; t += gridDim.x) {
         const TileCoord tc = decode_tile<BM>(p, t);
         const GemmProblem& pr = p.prob[tc.pi];
+        // Per-tile operand parameters, read from the parameter space once.
         const CUtensorMap* am = &p.maps[pr.a_map];
         const CUtensorMap* bm = &p.maps[pr.b_map];
+        const CUtensorMap* am_t = pr.half_a ? &p.maps[pr.a_map_t] : am;
+        const CUtensorMap* bm_t = pr.half_b ? &p.maps[pr.b_map_t] : bm;
         const int na = (NA > 1 && (pr.terms & TERM_LH)) ? 2 : 1;
         const int nb = (NB > 1 && (pr.terms & TERM_HL)) ? 2 : 1;
         const uint32_t bytes = na * A_PART_BYTES + nb * B_PART_BYTES;
         const int nk = (pr.K + BKE - 1) / BKE;
         const int arow = tc.bi * BM, brow = tc.bj * BN;
+        const int thr_a = pr.half_a ? arow / HALF_BLOCK : 0, thr_b = pr.half_b ? brow / HALF_BLOCK : 0;
+        const bool a_mn = pr.a_mn != 0, b_mn = pr.b_mn != 0;
+        const int za0 = pr.a_z[0] + tc.mat, za1 = pr.a_z[1] + tc.mat;
+        const int zb0 = pr.b_z[0] + tc.mat, zb1 = pr.b_z[1] + tc.mat;
         for (int kb = 0; kb < nk; ++kb) {
           if (!wait_bar(empty_bar(stage), phase ^ 1u, abort_flag, p)) {
             ok = false;
@@ -534,14 +541,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
           const uint32_t sa = ring + stage * Cfg::STAGE_BYTES;
           const uint32_t sb = sa + NA * A_PART_BYTES;
           const int ktile = k0 / HALF_BLOCK;
-          const bool a_t = pr.half_a && (arow / HALF_BLOCK) > ktile;  // read the transposed block
-          const bool b_t = pr.half_b && (brow / HALF_BLOCK) > ktile;
-          const CUtensorMap* am_k = a_t ? &p.maps[pr.a_map_t] : am;
-          const CUtensorMap* bm_k = b_t ? &p.maps[pr.b_map_t] : bm;
+          const bool a_t = ktile < thr_a;  // read the transposed block
+          const bool b_t = ktile < thr_b;
+          const CUtensorMap* am_k = a_t ? am_t : am;
+          const CUtensorMap* bm_k = b_t ? bm_t : bm;
           for (int part = 0; part < na; ++part) {
             const uint32_t dst = sa + part * A_PART_BYTES;
-            const int z = pr.a_z[part] + tc.mat;
-            if (!pr.a_mn && !a_t) {
+            const int z = part ? za1 : za0;
+            if (!a_mn && !a_t) {
               ptx::tma_load_3d(dst, am_k, fb, k0, arow, z);
             } else {
               ptx::tma_load_3d(dst, am_k, fb, arow, k0, z);
@@ -550,8 +557,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
           }
           for (int part = 0; part < nb; ++part) {
             const uint32_t dst = sb + part * B_PART_BYTES;
-            const int z = pr.b_z[part] + tc.mat;
-            if (!pr.b_mn && !b_t) {
+            const int z = part ? zb1 : zb0;
+            if (!b_mn && !b_t) {
               ptx::tma_load_3d(dst, bm_k, fb, k0, brow, z);
               ptx::tma_load_3d(dst + 16384, bm_k, fb, k0, brow + 128, z);
             } else {
@@ -599,8 +606,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
         }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        const uint32_t a_sbo = 1024u, b_sbo = 1024u;
-        const int arow_blk = (tc.bi * BM) / HALF_BLOCK, brow_blk = (tc.bj * BN) / HALF_BLOCK;
+        // Per-tile MMA parameters in registers: the K loop issues MMAs from
+        // precomputed descriptor halves only.
+        const int terms = pr.terms, pr_a_mn = pr.a_mn, pr_b_mn = pr.b_mn;
+        const int thr_a = pr.half_a ? (tc.bi * BM) / HALF_BLOCK : 0;
+        const int thr_b = pr.half_b ? (tc.bj * BN) / HALF_BLOCK : 0;
+        const uint32_t idesc0 = ptx::make_idesc(BM, BN, 0, 0, OPFMT);
+        const uint64_t hi_k = ptx::make_sw128_desc(0u, 16u, 1024u), hi_mn = ptx::make_sw128_desc(0u, 8192u, 1024u);
         uint32_t accumulate = 0;
         for (int kb = 0; kb < nk; ++kb) {
           if (!wait_bar(full_bar(stage), phase, abort_flag, p)) {
@@ -609,33 +621,32 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
           }
           ptx::tc_fence_after();
           const int ktile = (kb * BKE) / HALF_BLOCK;
-          const int a_mn = pr.a_mn | ((pr.half_a && arow_blk > ktile) ? 1 : 0);
-          const int b_mn = pr.b_mn | ((pr.half_b && brow_blk > ktile) ? 1 : 0);
-          const uint32_t idesc = ptx::make_idesc(BM, BN, a_mn, b_mn, OPFMT);
-          const uint32_t a_lbo = a_mn ? 8192u : 16u, b_lbo = b_mn ? 8192u : 16u;
-          const uint32_t a_kstep = a_mn ? 2048u : 32u, b_kstep = b_mn ? 2048u : 32u;
+          const uint32_t a_mn = (uint32_t)(pr_a_mn | (ktile < thr_a ? 1 : 0));
+          const uint32_t b_mn = (uint32_t)(pr_b_mn | (ktile < thr_b ? 1 : 0));
+          const uint32_t idesc = idesc0 | (a_mn << 15) | (b_mn << 16);
+          const uint64_t a_hi = a_mn ? hi_mn : hi_k, b_hi = b_mn ? hi_mn : hi_k;
+          const uint32_t a_ks = a_mn ? 2048u : 32u, b_ks = b_mn ? 2048u : 32u;
           const uint32_t sa = ring + stage * Cfg::STAGE_BYTES;
           const uint32_t sb = sa + NA * A_PART_BYTES;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {  // 4 MMAs x 32 bytes of K per 128-byte row
 #pragma unroll
             for (int term = 0; term < 3; ++term) {
-              const int bit = 1 << term;
-              if (!(pr.terms & bit)) continue;
               if (term == 1 && NB < 2) continue;
               if (term == 2 && NA < 2) continue;
-              const uint32_t pa = sa + (term == 2 ? A_PART_BYTES : 0);
-              const uint32_t pb = sb + (term == 1 ? B_PART_BYTES : 0);
-              const uint64_t ad = ptx::make_sw128_desc(pa + kk * a_kstep, a_lbo, a_sbo);
-              const uint64_t bd = ptx::make_sw128_desc(pb + kk * b_kstep, b_lbo, b_sbo);
+              if (!(terms & (1 << term))) continue;
+              const uint32_t pa = sa + (term == 2 ? A_PART_BYTES : 0) + kk * a_ks;
+              const uint32_t pb = sb + (term == 1 ? B_PART_BYTES : 0) + kk * b_ks;
+              const uint64_t ad = a_hi | (uint64_t)((pa >> 4) & 0x3FFFu);
+              const uint64_t bd = b_hi | (uint64_t)((pb >> 4) & 0x3FFFu);
               if (KIND == KIND_TF32)
                 ptx::mma_tf32(d_tmem, ad, bd, idesc, accumulate);
               else
                 ptx::mma_bf16(d_tmem, ad, bd, idesc, accumulate);
               accumulate = 1;
-              issued = true;
             }
           }
+          issued = true;
           ptx::mma_commit(empty_bar(stage));
           if (++stage == S) {
             stage = 0;
@@ -722,13 +733,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
 constexpr int BM2 = 256;
 constexpr int HALF_BYTES = 128 * 128;  // 128 rows x 128-byte K row
 
-// K atoms (128-byte rows) per stage: measured on the GPU, every stage
-// boundary costs ~700 cycles of MMA-pipe time beyond the MMAs themselves,
-// so the one-MMA-per-slice configurations take two atoms (8 MMAs) per
-// stage; the split configurations already issue 8-12 MMAs per atom.
+// K atoms (128-byte rows) per stage.  Measured on the GPU, each stage
+// boundary (commit, barrier wait, fence) costs several hundred cycles of the
+// issuing thread beyond the MMAs, so the one-MMA-per-slice configurations
+// take three atoms (12 MMAs, two 96 KB stages) per stage; the split
+// configurations already issue 8-12 MMAs per atom.
 template <int NA, int NB>
 struct Tc2Cfg {
-  static constexpr int KAT = (NA + NB <= 2) ? 2 : 1;
+  static constexpr int KAT = (NA + NB <= 2) ? 3 : 1;
   static constexpr int STAGE_BYTES = (NA + NB) * HALF_BYTES * KAT;
   static constexpr int STAGES = (200 * 1024) / STAGE_BYTES;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
@@ -824,15 +836,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       for (int t = pair; ok && t < p.total_tiles; t += npairs) {
         const TileCoord tc = decode_tile<BM2>(p, t);
         const GemmProblem& pr = p.prob[tc.pi];
+        // Per-tile operand parameters, read from the parameter space once:
+        // the K loop below issues only TMA copies and barrier operations.
         const CUtensorMap* am = &p.maps[pr.a_map];
         const CUtensorMap* bm = &p.maps[pr.b_map];
+        const CUtensorMap* am_t = pr.half_a ? &p.maps[pr.a_map_t] : am;
+        const CUtensorMap* bm_t = pr.half_b ? &p.maps[pr.b_map_t] : bm;
+        const int thr_a = pr.half_a ? tc.bi : 0, thr_b = pr.half_b ? tc.bj : 0;
+        const bool a_mn = pr.a_mn != 0, b_mn = pr.b_mn != 0;
+        const int za0 = pr.a_z[0] + tc.mat, za1 = pr.a_z[1] + tc.mat;
+        const int zb0 = pr.b_z[0] + tc.mat, zb1 = pr.b_z[1] + tc.mat;
         const int na = (NA > 1 && (pr.terms & TERM_LH)) ? 2 : 1;
         const int nb = (NB > 1 && (pr.terms & TERM_HL)) ? 2 : 1;
         const uint32_t bytes_pair = 2u * (uint32_t)(na + nb) * HALF_BYTES * KATOMS;
         const int nk = (pr.K + BKE - 1) / BKE;
         const int arow = tc.bi * BM2 + (int)rank * 128, brow = tc.bj * BN + (int)rank * 128;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!wait_bar_cluster(empty_bar(stage), phase ^ 1u, abort_flag, p)) {
+          if (!wait_bar(empty_bar(stage), phase ^ 1u, abort_flag, p)) {
             ok = false;
             break;
           }
@@ -845,17 +865,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
           // stage layout: [A parts][B parts], each part KATOMS 16 KB atoms
           const uint32_t sa = ring + stage * Cfg::STAGE_BYTES;
           const uint32_t sb = sa + NA * KATOMS * HALF_BYTES;
+#pragma unroll
           for (int at = 0; at < KATOMS; ++at) {
             const int k0 = kb * BKE + at * ATOM_E;
             const int ktile = k0 / HALF_BLOCK;
-            const bool a_t = pr.half_a && tc.bi > ktile;  // rows of block bi, K in an earlier block
-            const bool b_t = pr.half_b && tc.bj > ktile;
-            const CUtensorMap* am_k = a_t ? &p.maps[pr.a_map_t] : am;
-            const CUtensorMap* bm_k = b_t ? &p.maps[pr.b_map_t] : bm;
+            const bool a_t = ktile < thr_a;  // rows of block bi, K in an earlier block
+            const bool b_t = ktile < thr_b;
+            const CUtensorMap* am_k = a_t ? am_t : am;
+            const CUtensorMap* bm_k = b_t ? bm_t : bm;
             for (int part = 0; part < na; ++part) {
               const uint32_t dst = sa + (part * KATOMS + at) * HALF_BYTES;
-              const int z = pr.a_z[part] + tc.mat;
-              if (!pr.a_mn && !a_t) {
+              const int z = part ? za1 : za0;
+              if (!a_mn && !a_t) {
                 ptx::tma_load_3d_pair(dst, am_k, fb_leader, k0, arow, z);
               } else {
                 ptx::tma_load_3d_pair(dst, am_k, fb_leader, arow, k0, z);
@@ -864,8 +885,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
             }
             for (int part = 0; part < nb; ++part) {
               const uint32_t dst = sb + (part * KATOMS + at) * HALF_BYTES;
-              const int z = pr.b_z[part] + tc.mat;
-              if (!pr.b_mn && !b_t) {
+              const int z = part ? zb1 : zb0;
+              if (!b_mn && !b_t) {
                 ptx::tma_load_3d_pair(dst, bm_k, fb_leader, k0, brow, z);
               } else {
                 ptx::tma_load_3d_pair(dst, bm_k, fb_leader, brow, k0, z);
@@ -914,8 +935,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
         uint32_t accumulate = 0;
+        const int terms = pr.terms, pr_a_mn = pr.a_mn, pr_b_mn = pr.b_mn;
+        const int thr_a = pr.half_a ? tc.bi : 0, thr_b = pr.half_b ? tc.bj : 0;
+        const uint32_t idesc0 = ptx::make_idesc(BM2, BN, 0, 0, OPFMT);
+        const uint64_t hi_k = ptx::make_sw128_desc(0u, 16u, 1024u), hi_mn = ptx::make_sw128_desc(0u, 8192u, 1024u);
         for (int kb = 0; kb < nk; ++kb) {
-          if (!wait_bar_cluster(full_bar(stage), phase, abort_flag, p)) {
+          if (!wait_bar(full_bar(stage), phase, abort_flag, p)) {
             ok = false;
             break;
           }
@@ -923,31 +948,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
           const uint32_t sa = ring + stage * Cfg::STAGE_BYTES;
           const uint32_t sb = sa + NA * KATOMS * HALF_BYTES;
 #pragma unroll
-          for (int kq = 0; kq < 4 * KATOMS; ++kq) {
-            const int at = kq >> 2, kk = kq & 3;
+          for (int at = 0; at < KATOMS; ++at) {
             const int ktile = (kb * BKE + at * ATOM_E) / HALF_BLOCK;
-            const int a_mn = pr.a_mn | ((pr.half_a && tc.bi > ktile) ? 1 : 0);
-            const int b_mn = pr.b_mn | ((pr.half_b && tc.bj > ktile) ? 1 : 0);
-            const uint32_t idesc = ptx::make_idesc(BM2, BN, a_mn, b_mn, OPFMT);
-            const uint32_t a_lbo = a_mn ? 8192u : 16u, b_lbo = b_mn ? 8192u : 16u;
-            const uint32_t a_kstep = a_mn ? 2048u : 32u, b_kstep = b_mn ? 2048u : 32u;
+            const uint32_t a_mn = (uint32_t)(pr_a_mn | (ktile < thr_a ? 1 : 0));
+            const uint32_t b_mn = (uint32_t)(pr_b_mn | (ktile < thr_b ? 1 : 0));
+            const uint32_t idesc = idesc0 | (a_mn << 15) | (b_mn << 16);
+            const uint64_t a_hi = a_mn ? hi_mn : hi_k, b_hi = b_mn ? hi_mn : hi_k;
+            const uint32_t a_ks = a_mn ? 2048u : 32u, b_ks = b_mn ? 2048u : 32u;
 #pragma unroll
-            for (int term = 0; term < 3; ++term) {
-              if (!(pr.terms & (1 << term))) continue;
-              if (term == 1 && NB < 2) continue;
-              if (term == 2 && NA < 2) continue;
-              const uint32_t pa = sa + ((term == 2 ? KATOMS : 0) + at) * HALF_BYTES;
-              const uint32_t pb = sb + ((term == 1 ? KATOMS : 0) + at) * HALF_BYTES;
-              const uint64_t ad = ptx::make_sw128_desc(pa + kk * a_kstep, a_lbo, 1024u);
-              const uint64_t bd = ptx::make_sw128_desc(pb + kk * b_kstep, b_lbo, 1024u);
-              if (KIND == KIND_TF32)
-                ptx::mma2_tf32(d_tmem, ad, bd, idesc, accumulate);
-              else
-                ptx::mma2_f16(d_tmem, ad, bd, idesc, accumulate);
-              accumulate = 1;
-              issued = true;
+            for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+              for (int term = 0; term < 3; ++term) {
+                if (term == 1 && NB < 2) continue;
+                if (term == 2 && NA < 2) continue;
+                if (!(terms & (1 << term))) continue;
+                const uint32_t pa = sa + ((term == 2 ? KATOMS : 0) + at) * HALF_BYTES + kk * a_ks;
+                const uint32_t pb = sb + ((term == 1 ? KATOMS : 0) + at) * HALF_BYTES + kk * b_ks;
+                const uint64_t ad = a_hi | (uint64_t)((pa >> 4) & 0x3FFFu);
+                const uint64_t bd = b_hi | (uint64_t)((pb >> 4) & 0x3FFFu);
+                if (KIND == KIND_TF32)
+                  ptx::mma2_tf32(d_tmem, ad, bd, idesc, accumulate);
+                else
+                  ptx::mma2_f16(d_tmem, ad, bd, idesc, accumulate);
+                accumulate = 1;
+              }
             }
           }
+          issued = true;
           ptx::mma2_commit_both(empty_bar(stage));
           if (++stage == S) {
             stage = 0;
