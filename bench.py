@@ -46,6 +46,56 @@ def alg_flops(shapes, k=K_STEPS):
     return tot
 
 
+def gemm_alg_bytes(shapes, k=K_STEPS):
+    """Algorithmic DRAM bytes of the tensor-core launches of one step, every
+    operand read once and every result written once (half-stored symmetric
+    m x m matrices, m^2/2 elements; 16-bit operands, 32-bit hi/lo pairs):
+    SYRK reads Mb (2 B/elem) and writes G (4 B); each of the 4K-3 symmetric
+    products reads two 16-bit operands and a pair Cin and writes a pair;
+    the final reads the P pair and Mb and reads and writes W (bf16)."""
+    tot = 0.0
+    for r, c in shapes:
+        m, e = min(r, c), float(r) * c
+        half = 0.5 * m * m
+        tot += 2 * e + 4 * half                 # SYRK
+        tot += (4 * k - 3) * 12 * half          # products
+        tot += 4 * half + 6 * e                 # final + update
+    return tot
+
+
+# DRAM traffic of the tensor-core kernel measured by ncu (one pass:
+# gpu__time_duration.sum, dram__bytes_read.sum, dram__bytes_write.sum; see
+# profiles/k_gemm_tc2_qwen7b_x28_launch_list.md) for the kernel sources
+# whose sha256 is recorded here.  The figure is reported only while
+# gemm_tc.cu + plan.cu still hash to it: a changed kernel reports null.
+TRAFFIC_CAPTURE = {
+    "sources": ["gram_newton_schulz_b200/csrc/gemm_tc.cu", "gram_newton_schulz_b200/csrc/plan.cu"],
+    "sha256": "35d178b6b405d7b9c62a31188e2ca566963c5218e6502316d736e08c95cf4411",
+    "workload": "qwen2.5-7b-layer-set-x28",
+    "dram_bytes_per_step": 282.3e9,
+    "launches_per_step": 30,
+}
+
+
+def captured_traffic(workload_name):
+    """Measured DRAM bytes per tensor-core launch, or None when the capture
+    does not apply (other workload, or kernel sources changed since)."""
+    import hashlib
+    cap = TRAFFIC_CAPTURE
+    if workload_name != cap["workload"]:
+        return None
+    h = hashlib.sha256()
+    for rel in cap["sources"]:
+        path = os.path.join(ROOT, rel)
+        if not os.path.exists(path):
+            return None
+        with open(path, "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest() != cap["sha256"]:
+        return None
+    return cap["dram_bytes_per_step"] / cap["launches_per_step"]
+
+
 def momentum_bytes(shapes, grad_bytes=2):
     """HBM bytes of the momentum pass: read G and M, write M and Mb."""
     e = sum(r * c for r, c in shapes)
@@ -270,6 +320,7 @@ def main():
     barrier()
     torch.cuda.synchronize(dev)
     launches = 0
+    tc_total = 0  # tensor-core launches (Gram recursion + final update)
     for k in range(K):
         ev[k][0].record(stream)
         plan.momentum_normalize(grads, moms, beta=w.beta, eps=1e-7)
@@ -277,9 +328,11 @@ def main():
         ev[k][1].record(stream)
         plan.gram_ns_batched(None, dmu.QUINTIC, K_STEPS)
         launches += plan.last_launch_count()
+        tc_total += plan.last_launch_count()
         ev[k][2].record(stream)
         plan.apply_update(weights, lr=w.lr)
         launches += plan.last_launch_count()
+        tc_total += plan.last_launch_count()
         ev[k][3].record(stream)
     torch.cuda.synchronize(dev)
     barrier()
@@ -288,6 +341,10 @@ def main():
     t_mom = sum(e[0].elapsed_time(e[1]) for e in ev)
     t_gram = sum(e[1].elapsed_time(e[2]) for e in ev)
     t_upd = sum(e[2].elapsed_time(e[3]) for e in ev)
+    tc_launches = tc_total / K
+    # per-rank launches are those of the captured run only for the whole
+    # layer set at the default precision
+    traffic = captured_traffic(w_full.name) if args.shard == "replica" and args.prec == "auto" else None
     step_ms = owners.max_over_ranks(total_ms / K, device=dev)
     status = plan.read_status()
 
@@ -384,8 +441,10 @@ def main():
             "split_ms": {"momentum": round(t_mom / K, 3), "gram": round(t_gram / K, 3),
                          "update": round(t_upd / K, 3)},
             "roofline": {"bound": "tensor", "achieved": round(achieved_tf, 1), "peak": peak_tf,
-                         "unit": "TFLOP/s", "frac": round(achieved_tf / peak_tf, 4), "traffic": None,
-                         "kernel": "k_gemm_tc (all Gram-space and final launches)",
+                         "unit": "TFLOP/s", "frac": round(achieved_tf / peak_tf, 4),
+                         "traffic": traffic,
+                         "alg_bytes_per_launch": round(gemm_alg_bytes(w.shapes) / max(tc_launches, 1)),
+                         "kernel": "k_gemm_tc2 (all Gram-space and final launches)",
                          "peak_kind": f"{peak_kind} bf16 sustained"},
             "hbm_kernel": {"kernel": "k_momentum", "achieved": round(mom_gbs, 1), "peak": hbm,
                            "unit": "GB/s", "frac": round(mom_gbs / hbm, 4), "peak_kind": peak_kind},

@@ -51,3 +51,23 @@ def test_reference_arm_prints_one_json_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["unit"] == "ms" and d["higher_is_better"] is False
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_gemm_alg_bytes_closed_form():
+    # one 2x4 matrix, K = 5: SYRK 2*8 + 4*2, products 17*12*2, final 4*2 + 6*8
+    assert bench.gemm_alg_bytes([(2, 4)]) == (16 + 8) + 17 * 24 + (8 + 48)
+    assert bench.gemm_alg_bytes([(4, 2)]) == bench.gemm_alg_bytes([(2, 4)])
+
+
+def test_captured_traffic_applies_only_to_its_sources(monkeypatch):
+    cap = dict(bench.TRAFFIC_CAPTURE)
+    assert bench.captured_traffic("uniform-64x512x2048") is None
+    monkeypatch.setattr(bench, "TRAFFIC_CAPTURE", dict(cap, sha256="0" * 64))
+    assert bench.captured_traffic(cap["workload"]) is None
+    import hashlib
+    h = hashlib.sha256()
+    for rel in cap["sources"]:
+        with open(os.path.join(ROOT, rel), "rb") as fh:
+            h.update(fh.read())
+    monkeypatch.setattr(bench, "TRAFFIC_CAPTURE", dict(cap, sha256=h.hexdigest()))
+    assert bench.captured_traffic(cap["workload"]) == cap["dram_bytes_per_step"] / cap["launches_per_step"]
