@@ -10,10 +10,14 @@ flush is needed between steps.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...   # the fp64 oracle on host cores
 
-Multi-GPU (torchrun, one process per GPU): every rank owns a full layer set
-of its own (owner-sharded by matrix, no collective on the data path), so
-per-GPU work is fixed (weak scaling); the step time is the max over ranks.
-Prints one JSON line on rank 0.
+Multi-GPU (torchrun, one process per GPU), two modes:
+* ``--shard replica`` (default): every rank owns a full layer set of its
+  own, with no collective on the data path.  Per-GPU work is fixed (weak
+  scaling).
+* ``--shard owner``: the ranks split one layer set by LPT owners and
+  exchange gradients and weights over NCCL.  Each owner bucket gets one
+  reduce in and one broadcast out (strong scaling).
+The step time is the max over ranks.  Prints one JSON line on rank 0.
 """
 from __future__ import annotations
 
@@ -239,6 +243,115 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_owner(args, w_full, dev, world, rank, local, barrier):
+    """Owner-sharded data-parallel step (DMuon page, section 2.1): every rank
+    holds the gradients and weights of the whole layer set; one reduce per
+    owner bucket brings the gradients to their owners, each owner updates its
+    matrices, one broadcast per bucket returns the weights.  Total work is
+    fixed as ranks are added (strong scaling)."""
+    import torch
+    from gram_newton_schulz_b200 import dmu, dp, owners, synth
+
+    osd = dp.OwnerShardedStep(w_full.shapes, dtype=w_full.dtype, prec=args.prec, device=dev)
+    b = osd.buckets
+    wdt = torch.bfloat16 if w_full.dtype == "bf16" else torch.float32
+    gflat, wflat = b.alloc(wdt, dev), b.alloc(wdt, dev)
+    for i in range(w_full.count):
+        b.view(gflat, i).copy_(synth.gradients(w_full, dev, indices=[i])[0])
+        b.view(wflat, i).copy_(synth.weights(w_full, dev, indices=[i])[0])
+    owned = osd.owned_shapes()
+    moms = [torch.zeros(s, dtype=torch.float32, device=dev) for s in owned]
+    kw = dict(beta=w_full.beta, lr=w_full.lr, eps=1e-7, coeffs=dmu.QUINTIC, steps=K_STEPS)
+    for _ in range(args.warmup):
+        osd.step(gflat, wflat, moms, **kw)
+    torch.cuda.synchronize(dev)
+    plan = osd.compute.plan
+    if plan is not None and plan.read_status() != 0:
+        raise SystemExit("device status word set during warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(dev)
+    launches = tc = 0
+    for k in range(K):
+        osd.step(gflat, wflat, moms, events=ev[k], **kw)
+        launches += osd.compute.launches
+        tc += osd.compute.tc_launches
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    step_ms = owners.max_over_ranks(ev[0][0].elapsed_time(ev[K - 1][3]) / K, device=dev)
+    t_in = sum(e[0].elapsed_time(e[1]) for e in ev) / K
+    t_cmp = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+    t_out = sum(e[2].elapsed_time(e[3]) for e in ev) / K
+    t_cmp_max = owners.max_over_ranks(t_cmp, device=dev)
+    status = plan.read_status() if plan is not None else 0
+
+    # e2e through the public API with host buffers: each step uploads this
+    # rank's whole local gradient from pinned memory and reads the whole
+    # updated model back.
+    e2e = None
+    if not args.no_e2e:
+        E = args.e2e_steps
+        h_g = [t.to("cpu").pin_memory() for t in gflat]
+        h_w = [t.to("cpu").pin_memory() for t in wflat]
+        h2d = sum(t.numel() * t.element_size() for t in h_g)
+        d2h = sum(t.numel() * t.element_size() for t in h_w)
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(E):
+            for hg, g in zip(h_g, gflat):
+                g.copy_(hg, non_blocking=True)
+            osd.step(gflat, wflat, moms, **kw)
+            for hw, x in zip(h_w, wflat):
+                hw.copy_(x, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        barrier()
+        e2e = {"value": round(owners.max_over_ranks(e0.elapsed_time(e1) / E, device=dev), 3), "unit": "ms",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "overlap": "none: copy in, step, copy out in order on one stream"}
+
+    peaks, peak_kind = load_peaks()
+    peak_tf = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    job_flops = alg_flops(w_full.shapes)
+    achieved_tf = alg_flops(owned) / (t_cmp / 1e3) / 1e12 if owned else 0.0
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(step_ms, 3), "unit": "ms", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": round(step_ms, 3), "higher_is_better": False,
+            "scaling": "strong", "vs_baseline": None,
+            "dtype": "bf16" if w_full.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": {"workload": w_full.name, "matrices": w_full.count, "matrices_total": w_full.count,
+                       "K": K_STEPS, "coeffs": [3.4445, -4.7750, 2.0315], "precision": args.prec,
+                       "parallelism": f"owner x{world}: LPT owners, reduce in / broadcast out over "
+                                      f"{'NCCL' if world > 1 else 'nothing (1 rank)'}",
+                       "l2": "inputs larger than L2 (no flush needed)"},
+            "throughput": {"matrices_per_s": round(w_full.count / (step_ms / 1e3), 1),
+                           "alg_tflops": round(job_flops / (step_ms / 1e3) / 1e12, 1),
+                           "alg_tflops_frac_per_gpu": round(job_flops / world / (step_ms / 1e3) / 1e12 / peak_tf, 4)},
+            "split_ms": {"exchange_in": round(t_in, 3), "compute": round(t_cmp, 3),
+                         "compute_max_over_ranks": round(t_cmp_max, 3), "exchange_out": round(t_out, 3)},
+            "roofline": {"bound": "tensor", "achieved": round(achieved_tf, 1), "peak": peak_tf,
+                         "unit": "TFLOP/s", "frac": round(achieved_tf / peak_tf, 4), "traffic": None,
+                         "kernel": "rank 0's whole owned update (momentum + Gram + final)",
+                         "peak_kind": f"{peak_kind} bf16 sustained"},
+            "gpu_launches": launches,
+            "status_word": status,
+            "clocks": clk,
+            "e2e": e2e,
+            "cpu_baseline": None,
+        }
+        print(json.dumps(line), flush=True)
+    osd.close()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -248,7 +361,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--shard", default="replica", choices=["replica", "owner"],
                     help="replica: every rank owns a full layer set (weak scaling); owner: the ranks "
-                         "split one layer set by LPT owner assignment (strong scaling)")
+                         "split one layer set by LPT owners, gradients reduced to owners and weights "
+                         "broadcast back over NCCL (strong scaling)")
     ap.add_argument("--shapes", default=None,
                     help="custom spiked bf16 workload for profiling, e.g. 3584x3584*8,512x3584*4")
     ap.add_argument("--prec", default="auto")
@@ -285,10 +399,12 @@ def main():
 
     from gram_newton_schulz_b200 import owners
     w_full = custom_workload(args.shapes) if args.shapes else synth.workload(args.workload)
-    if args.shard == "owner" and world > 1:
-        mine = owners.owned_indices(owners.assign_shapes(w_full.shapes, world), rank)
-    else:
-        mine = list(range(w_full.count))
+    if args.shard == "owner":
+        run_owner(args, w_full, dev, world, rank, local, barrier)
+        if world > 1:
+            dist.destroy_process_group()
+        return
+    mine = list(range(w_full.count))
     w = synth.Workload(w_full.name, w_full.seed, w_full.dtype, tuple(w_full.shapes[i] for i in mine),
                        w_full.dist, w_full.var, w_full.rank, w_full.beta, w_full.lr)
     grads = synth.gradients(w_full, dev, indices=mine)
@@ -344,13 +460,13 @@ def main():
     tc_launches = tc_total / K
     # per-rank launches are those of the captured run only for the whole
     # layer set at the default precision
-    traffic = captured_traffic(w_full.name) if args.shard == "replica" and args.prec == "auto" else None
+    traffic = captured_traffic(w_full.name) if args.prec == "auto" else None
     step_ms = owners.max_over_ranks(total_ms / K, device=dev)
     status = plan.read_status()
 
     peaks, peak_kind = load_peaks()
     flops = alg_flops(w.shapes)
-    job_shapes = w_full.shapes if args.shard == "owner" else w_full.shapes * world
+    job_shapes = w_full.shapes * world
     job_flops = alg_flops(job_shapes)
     tc_s = (t_gram + t_upd) / K / 1e3
     achieved_tf = flops / tc_s / 1e12
@@ -428,12 +544,11 @@ def main():
         line = {
             "metric": METRIC, "value": round(step_ms, 3), "unit": "ms", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": round(step_ms, 3), "higher_is_better": False,
-            "scaling": "strong" if args.shard == "owner" else "weak", "vs_baseline": None,
+            "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
             "config": {"workload": w_full.name, "matrices": w_full.count, "matrices_total": len(job_shapes),
                        "K": K_STEPS, "coeffs": [3.4445, -4.7750, 2.0315], "precision": args.prec,
-                       "parallelism": (f"owner x{world} (LPT owners of one layer set)" if args.shard == "owner"
-                                       else f"replica x{world} (one owned layer set per rank)"),
+                       "parallelism": f"replica x{world} (one owned layer set per rank)",
                        "l2": "inputs larger than L2 (no flush needed)"},
             "throughput": {"matrices_per_s": round(len(job_shapes) / (step_ms / 1e3), 1),
                            "alg_tflops": round(job_flops / (step_ms / 1e3) / 1e12, 1),

@@ -1,0 +1,215 @@
+"""Owner-sharded data-parallel step (DMuon page, section 2.1) on CPU ranks.
+
+The exchange logic of `gram_newton_schulz_b200.dp` runs here over gloo
+(127.0.0.1) with world sizes 2 and 3. The device compute is replaced by the
+fp64 oracle, since tests may import it and the product path may not. The
+tests check:
+
+* bucket layout: every matrix in exactly one owner bucket, views on
+  256-byte boundaries, no overlap;
+* after one step, every rank holds the weights the oracle gives for the
+  mean gradient, bit for bit. The gradients are chosen so that their float32
+  sums are exact in any order;
+* the owner's momentum is the oracle's, and each rank computes exactly its
+  owned matrices;
+* a rank that dies before the exchange surfaces on the other rank as an
+  error from the collective (short process-group timeout), not a hang.
+"""
+import datetime
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from gram_newton_schulz_b200 import dp
+from oracle import gram_ns
+
+SHAPES = [(8, 24), (24, 8), (16, 16), (4, 32), (12, 20), (8, 8), (32, 16)]
+BETA, LR, EPS = 0.9, 0.05, 1e-7
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _grad(i, rank):
+    """Per-rank gradient of matrix i: multiples of 2^-6 in [-2, 2], so float32
+    sums over a few ranks are exact in any order."""
+    rows, cols = SHAPES[i]
+    g = np.random.default_rng(1000 * i + rank).integers(-128, 129, size=(rows, cols))
+    return (g / 64.0).astype(np.float32)
+
+
+def _weight(i):
+    rows, cols = SHAPES[i]
+    return np.random.default_rng(77 + i).standard_normal((rows, cols)).astype(np.float32)
+
+
+def _momentum0(i):
+    rows, cols = SHAPES[i]
+    return (np.random.default_rng(300 + i).integers(-64, 65, size=(rows, cols)) / 32.0).astype(np.float32)
+
+
+class OracleCompute:
+    """Test stand-in for the device compute: the fp64 oracle per owned matrix."""
+
+    def __init__(self, indices):
+        self.indices = list(indices)
+        self.calls = []
+
+    def __call__(self, grads, momenta, weights, *, beta, lr, eps, coeffs, steps):
+        self.calls.append(list(self.indices))
+        for g, m, w in zip(grads, momenta, weights):
+            m_new, _, w_new = gram_ns.muon_step(w.double().numpy(), m.double().numpy(), g.double().numpy(),
+                                                beta=beta, lr=lr, eps=eps, coeffs=coeffs, steps=steps)
+            m.copy_(torch.from_numpy(m_new))
+            w.copy_(torch.from_numpy(w_new))
+
+
+def _expected(world):
+    """Weights and momenta after one step, from the mean gradient."""
+    out_w, out_m = [], []
+    for i in range(len(SHAPES)):
+        s = np.zeros(SHAPES[i], dtype=np.float32)
+        for r in range(world):
+            s = s + _grad(i, r)
+        mean = (s / np.float32(world)).astype(np.float32)
+        m_new, _, w_new = gram_ns.muon_step(_weight(i).astype(np.float64), _momentum0(i).astype(np.float64),
+                                            mean.astype(np.float64), beta=BETA, lr=LR, eps=EPS)
+        out_w.append(w_new.astype(np.float32))
+        out_m.append(m_new.astype(np.float32))
+    return out_w, out_m
+
+
+def _step_worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        buckets = dp.OwnerBuckets(SHAPES, world)
+        compute = OracleCompute(buckets.members[rank])
+        step = dp.OwnerShardedStep(SHAPES, compute=compute)
+        gf = buckets.alloc(torch.float32, "cpu")
+        wf = buckets.alloc(torch.float32, "cpu")
+        for i in range(len(SHAPES)):
+            buckets.view(gf, i).copy_(torch.from_numpy(_grad(i, rank)))
+            buckets.view(wf, i).copy_(torch.from_numpy(_weight(i)))
+        moms = [torch.from_numpy(_momentum0(i)).clone() for i in step.mine]
+        step.step(gf, wf, moms, beta=BETA, lr=LR, eps=EPS)
+        q.put((rank, list(step.mine), compute.calls,
+               [buckets.view(wf, i).numpy().copy() for i in range(len(SHAPES))],
+               [m.numpy().copy() for m in moms]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_owner_buckets_layout():
+    for world in (1, 2, 3, 4):
+        b = dp.OwnerBuckets(SHAPES, world)
+        seen = sorted(i for r in range(world) for i in b.members[r])
+        assert seen == list(range(len(SHAPES)))
+        for r in range(world):
+            spans = sorted((b.offset[i], b.offset[i] + SHAPES[i][0] * SHAPES[i][1]) for i in b.members[r])
+            for (s0, e0), (s1, _) in zip(spans, spans[1:]):
+                assert e0 <= s1
+            assert all(s % dp.ALIGN_ELEMS == 0 for s, _ in spans)
+            assert not spans or spans[-1][1] <= b.sizes[r]
+        flats = b.alloc(torch.float32, "cpu")
+        for i, v in enumerate(b.views(flats)):
+            assert tuple(v.shape) == SHAPES[i] and v.is_contiguous()
+            assert (v.data_ptr() - flats[b.owner[i]].data_ptr()) % 256 == 0
+
+
+def test_single_process_step_matches_oracle():
+    compute = OracleCompute(range(len(SHAPES)))
+    step = dp.OwnerShardedStep(SHAPES, compute=compute)
+    assert step.world == 1 and step.mine == list(range(len(SHAPES)))
+    b = step.buckets
+    gf, wf = b.alloc(torch.float32, "cpu"), b.alloc(torch.float32, "cpu")
+    for i in range(len(SHAPES)):
+        b.view(gf, i).copy_(torch.from_numpy(_grad(i, 0)))
+        b.view(wf, i).copy_(torch.from_numpy(_weight(i)))
+    moms = [torch.from_numpy(_momentum0(i)).clone() for i in step.mine]
+    step.step(gf, wf, moms, beta=BETA, lr=LR, eps=EPS)
+    ew, em = _expected(1)
+    for i in range(len(SHAPES)):
+        assert np.array_equal(b.view(wf, i).numpy(), ew[i])
+        assert np.array_equal(moms[i].numpy(), em[i])
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_gloo_owner_step_matches_oracle(world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_step_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    try:
+        results = sorted([q.get(timeout=180) for _ in range(world)], key=lambda t: t[0])
+    finally:
+        for p in procs:
+            p.join(timeout=60)
+            if p.is_alive():
+                p.kill()
+    for p in procs:
+        assert p.exitcode == 0
+    ew, em = _expected(world)
+    owned = []
+    for rank, mine, calls, weights, moms in results:
+        assert calls == [mine]  # one compute call, over the owned matrices only
+        owned += mine
+        for i in range(len(SHAPES)):
+            assert np.array_equal(weights[i], ew[i]), (rank, i)
+        for k, i in enumerate(mine):
+            assert np.array_equal(moms[k], em[i]), (rank, i)
+    assert sorted(owned) == list(range(len(SHAPES)))
+
+
+def _dying_worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    if rank == 1:
+        q.put((rank, "left"))
+        q.close()
+        q.join_thread()
+        os._exit(0)  # leaves between steps, before the exchange
+    buckets = dp.OwnerBuckets(SHAPES, world)
+    step = dp.OwnerShardedStep(SHAPES, compute=OracleCompute(buckets.members[rank]))
+    gf, wf = buckets.alloc(torch.float32, "cpu"), buckets.alloc(torch.float32, "cpu")
+    moms = [torch.zeros(SHAPES[i]) for i in step.mine]
+    try:
+        step.step(gf, wf, moms)
+        q.put((rank, "no error"))
+    except Exception as e:  # the collective reports the missing peer
+        q.put((rank, "error: " + type(e).__name__))
+    q.close()
+    q.join_thread()
+    os._exit(0)
+
+
+def test_gloo_missing_rank_is_an_error_not_a_hang():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_dying_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    try:
+        got = dict(q.get(timeout=120) for _ in range(2))
+    finally:
+        for p in procs:
+            p.join(timeout=30)
+            if p.is_alive():
+                p.kill()
+    assert got[1] == "left"
+    assert got[0].startswith("error"), got[0]

@@ -1,0 +1,41 @@
+"""The owner-sharded step's device path on one GPU (world size 1, so there
+are no collectives): the compute must run on views of the per-owner flat
+buffers, and must agree bit for bit with the same update through
+`dmu.Plan.step` on separate tensors."""
+import pytest
+import torch
+
+from gram_newton_schulz_b200 import dmu, dp, synth
+
+pytestmark = pytest.mark.gpu
+
+
+def test_owner_step_on_flat_buffers_matches_plan_step():
+    shapes = [(512, 2048), (2048, 512), (384, 384), (256, 1024), (1024, 1024)]
+    w = synth.custom("dp-check", shapes, seed=11)
+    dev = torch.device("cuda", 0)
+    grads = synth.gradients(w, dev)
+    weights = synth.weights(w, dev)
+
+    osd = dp.OwnerShardedStep(shapes, device=dev)
+    assert osd.world == 1 and osd.mine == list(range(len(shapes)))
+    b = osd.buckets
+    gflat, wflat = b.alloc(torch.bfloat16, dev), b.alloc(torch.bfloat16, dev)
+    for i in range(len(shapes)):
+        b.view(gflat, i).copy_(grads[i])
+        b.view(wflat, i).copy_(weights[i])
+    moms_a = [torch.zeros(s, dtype=torch.float32, device=dev) for s in shapes]
+    moms_b = [torch.zeros(s, dtype=torch.float32, device=dev) for s in shapes]
+    plan = dmu.Plan(shapes, device=dev)
+    w_ref = [x.clone() for x in weights]
+    for _ in range(2):
+        osd.step(gflat, wflat, moms_a, beta=0.95, lr=0.02)
+        plan.step(grads, moms_b, w_ref, beta=0.95, lr=0.02)
+    torch.cuda.synchronize()
+    assert osd.compute.launches > 0 and osd.compute.tc_launches > 0
+    for i in range(len(shapes)):
+        assert torch.equal(b.view(wflat, i), w_ref[i]), i
+        assert torch.equal(moms_a[i], moms_b[i]), i
+    assert osd.compute.plan.read_status() == 0
+    osd.close()
+    plan.close()
