@@ -12,7 +12,11 @@ float64, with ``numpy.matmul`` as the only library primitive.
 Pins (``tests/test_oracle_pins.py``): SVD polar factor, spectral closed
 form, Gram-form == rectangular form, transpose / scale / orthogonal
 invariance, the quintic singular-value band, and exact rational special
-cases.  No function here is "parity unpinned".
+cases.  ``demuon.py`` (one DeMuon iteration over N agents) is pinned in
+``tests/test_demuon_oracle.py``: the single-agent reduction to Muon, the
+gradient-tracking mean invariant, one-step consensus on the complete
+graph, a hand-computed scalar case, and the ring's closed-form mixing rate.
+No function here is "parity unpinned".
 """
 
 from .gram_ns import (  # noqa: F401
