@@ -48,7 +48,11 @@ SIGNATURES = {
     "dmu_get_schedule": (ctypes.c_int, [_VP]),
     "dmu_momentum_norm_static": (ctypes.c_int, [_VP, _VP, _VP, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
                                                 ctypes.c_float, ctypes.c_float, _VP, _VP]),
+    "dmu_demuon_track": (ctypes.c_int, [ctypes.c_int, ctypes.c_int64, _VP, ctypes.c_float, _VP, _VP, _VP, _VP,
+                                        _VP, _VP]),
+    "dmu_demuon_mix": (ctypes.c_int, [ctypes.c_int, ctypes.c_int64, _VP, ctypes.c_float, _VP, _VP, _VP, _VP]),
 }
+DEMUON_MAX_AGENTS = 16
 
 
 class Shape(ctypes.Structure):
@@ -231,3 +235,46 @@ class Plan:
 
     def last_launch_count(self) -> int:
         return int(self.lib.dmu_last_launch_count(self.handle))
+
+
+# ---------------------------------------------------------------- DeMuon
+def _mix_array(mix, n: int):
+    flat = [float(x) for row in mix for x in row]
+    if len(flat) != n * n:
+        raise ValueError(f"mix must be {n} x {n}")
+    return (ctypes.c_float * (n * n))(*flat)
+
+
+def _flat_args(tensors, what: str, dtype, numel: int):
+    import torch
+    for t in tensors:
+        if t.dtype != dtype or not t.is_contiguous() or t.numel() < numel or not t.is_cuda:
+            raise ValueError(f"{what}: expected contiguous CUDA {dtype} tensors of at least {numel} elements")
+    return _ptr_array([t.data_ptr() for t in tensors])
+
+
+def demuon_track(mix, theta: float, grads, momenta, v_in, v_out, v_bf16, numel: Optional[int] = None,
+                 stream=None):
+    """dmu_demuon_track on per-agent flat tensors: M and V fp32, grads and
+    the msgn input bf16; ``mix`` is n x n (row i: what agent i applies)."""
+    import torch
+    lib = load()
+    n = len(grads)
+    numel = grads[0].numel() if numel is None else int(numel)
+    args = [_flat_args(grads, "grads", torch.bfloat16, numel), _flat_args(momenta, "momenta", torch.float32, numel),
+            _flat_args(v_in, "v_in", torch.float32, numel), _flat_args(v_out, "v_out", torch.float32, numel),
+            _flat_args(v_bf16, "v_bf16", torch.bfloat16, numel)]
+    _check(lib.dmu_demuon_track(n, numel, ctypes.cast(_mix_array(mix, n), _VP), float(theta),
+                                *[ctypes.cast(a, _VP) for a in args], _stream_handle(stream, grads[0].device)))
+
+
+def demuon_mix(mix, eta: float, x_in, o, x_out, numel: Optional[int] = None, stream=None):
+    """dmu_demuon_mix on per-agent flat fp32 tensors: X_i' = sum_j w_ij (X_j - eta O_j)."""
+    import torch
+    lib = load()
+    n = len(x_in)
+    numel = x_in[0].numel() if numel is None else int(numel)
+    args = [_flat_args(x_in, "x_in", torch.float32, numel), _flat_args(o, "o", torch.float32, numel),
+            _flat_args(x_out, "x_out", torch.float32, numel)]
+    _check(lib.dmu_demuon_mix(n, numel, ctypes.cast(_mix_array(mix, n), _VP), float(eta),
+                              *[ctypes.cast(a, _VP) for a in args], _stream_handle(stream, x_in[0].device)))

@@ -245,6 +245,48 @@ DMU_API dmu_status dmu_momentum_norm_static(const void* grad, float* momentum, v
                                             int64_t rows, int64_t cols, dmu_dtype dtype, float beta,
                                             float eps, float* inv_norm_out, void* stream);
 
+/* ---------------------------------------------------------------- DeMuon
+ * Decentralised Muon over a communication graph of N agents (DeMuon
+ * technical summary, "Methodology", 1. DeMuon: local momentum, gradient
+ * tracking, and iterates updated from the neighbours' msgn steps).  Each
+ * agent i keeps, per weight matrix, a momentum estimate M_i, a tracked
+ * gradient V_i and an iterate X_i.  One iteration with mixing weights w_ij:
+ *
+ *   M_i' = (1 - theta) M_i + theta G_i          dmu_demuon_track
+ *   V_i' = sum_j w_ij V_j + M_i' - M_i          dmu_demuon_track
+ *   O_j  = msgn(bf16(V_j'))                     a plan over all agents' matrices:
+ *                                               dmu_momentum_normalize (beta 0),
+ *                                               dmu_gram_ns_batched,
+ *                                               dmu_apply_update (out_o only)
+ *   X_i' = sum_j w_ij (X_j - eta O_j)           dmu_demuon_mix
+ *
+ * The page names these sequences and operations but prints no formulas; the
+ * recursions above are the plain gradient-tracking reading.
+ *
+ * Layout: every agent's state for all its matrices is one flat array of
+ * `numel` elements (fp32 for M, V, X, O; bf16 for G and the msgn input),
+ * the same element order in every agent; the kernels treat it as a vector.
+ * `mix` is a HOST array of n_agents x n_agents fp32 weights, row-major, row
+ * i holding the weights agent i applies to every agent's values.  The
+ * pointer arguments are HOST arrays of n_agents DEVICE pointers, each
+ * 16-byte aligned.  Outputs must not alias inputs of another role (every
+ * output element reads all agents' inputs): v_out vs v_in, x_out vs x_in
+ * and o.  Sums over agents run in agent order, so results are
+ * deterministic.  Errors: n_agents outside [1, DMU_DEMUON_MAX_AGENTS], a
+ * null or misaligned pointer, aliasing, non-finite weights, theta outside
+ * [0, 1] or a non-finite eta return DMU_ERR_INVALID_ARG before any launch.
+ * Both calls are stream-ordered and do not synchronise. */
+#define DMU_DEMUON_MAX_AGENTS 16
+
+DMU_API dmu_status dmu_demuon_track(int n_agents, int64_t numel, const float* mix, float theta,
+                                    const void* const* grads, float* const* momenta,
+                                    const float* const* v_in, float* const* v_out, void* const* v_bf16,
+                                    void* stream);
+
+DMU_API dmu_status dmu_demuon_mix(int n_agents, int64_t numel, const float* mix, float eta,
+                                  const float* const* x_in, const float* const* o, float* const* x_out,
+                                  void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -146,3 +146,58 @@ def test_binding_rejects_mismatched_tensors():
         p._check_tensors([Fake()], "grads", torch.bfloat16)
     with pytest.raises(ValueError):
         p._check_tensors([], "grads", torch.bfloat16)
+
+
+def test_demuon_argument_errors_before_any_launch():
+    """dmu_demuon_track / dmu_demuon_mix validate everything on the host;
+    these calls return before any CUDA call, so they need no GPU.  The fake
+    device pointers are never dereferenced."""
+    lib = dmu.load()
+    vp = ctypes.c_void_p
+
+    def ptrs(*vals):
+        arr = (ctypes.c_void_p * len(vals))(*vals)
+        return ctypes.cast(arr, vp), arr
+
+    mix2 = (ctypes.c_float * 4)(0.5, 0.5, 0.5, 0.5)
+    m2 = ctypes.cast(mix2, vp)
+    a, ka = ptrs(0x1000, 0x2000)
+    b, kb = ptrs(0x3000, 0x4000)
+    c, kc = ptrs(0x5000, 0x6000)
+    d, kd = ptrs(0x7000, 0x8000)
+    e, ke = ptrs(0x9000, 0xa000)
+    track = lib.dmu_demuon_track
+    mixf = lib.dmu_demuon_mix
+    assert track(0, 16, m2, 0.1, a, b, c, d, e, None) == dmu.ERR_INVALID_ARG      # no agents
+    assert track(17, 16, m2, 0.1, a, b, c, d, e, None) == dmu.ERR_INVALID_ARG     # too many agents
+    assert track(2, -1, m2, 0.1, a, b, c, d, e, None) == dmu.ERR_INVALID_ARG      # negative size
+    assert track(2, 16, None, 0.1, a, b, c, d, e, None) == dmu.ERR_INVALID_ARG    # no weights
+    assert track(2, 16, m2, 1.5, a, b, c, d, e, None) == dmu.ERR_INVALID_ARG      # theta > 1
+    assert track(2, 16, m2, float("nan"), a, b, c, d, e, None) == dmu.ERR_INVALID_ARG
+    assert track(2, 16, m2, 0.1, a, b, c, c, e, None) == dmu.ERR_INVALID_ARG      # v_out aliases v_in
+    assert b"alias" in lib.dmu_last_error()
+    odd, ko = ptrs(0x1004, 0x2000)
+    assert track(2, 16, m2, 0.1, odd, b, c, d, e, None) == dmu.ERR_INVALID_ARG    # misaligned
+    assert b"16-byte" in lib.dmu_last_error()
+    nul, kn = ptrs(0x1000, 0)
+    assert track(2, 16, m2, 0.1, nul, b, c, d, e, None) == dmu.ERR_INVALID_ARG    # null pointer
+    bad = (ctypes.c_float * 4)(0.5, float("inf"), 0.5, 0.5)
+    assert track(2, 16, ctypes.cast(bad, vp), 0.1, a, b, c, d, e, None) == dmu.ERR_INVALID_ARG
+    assert mixf(2, 16, m2, float("inf"), a, b, c, None) == dmu.ERR_INVALID_ARG    # eta not finite
+    assert mixf(2, 16, m2, 0.1, a, b, a, None) == dmu.ERR_INVALID_ARG             # x_out aliases x_in
+    assert mixf(2, 16, m2, 0.1, a, b, b, None) == dmu.ERR_INVALID_ARG             # x_out aliases o
+    assert mixf(2, 16, m2, 0.1, odd, b, c, None) == dmu.ERR_INVALID_ARG
+    assert mixf(0, 16, m2, 0.1, a, b, c, None) == dmu.ERR_INVALID_ARG
+    # zero elements is valid and launches nothing
+    assert track(2, 0, m2, 0.1, a, b, c, d, e, None) == dmu.OK
+    assert mixf(2, 0, m2, 0.1, a, b, c, None) == dmu.OK
+
+
+def test_demuon_mixing_matrices_match_the_oracle():
+    import numpy as np
+    from gram_newton_schulz_b200 import demuon
+    from oracle import demuon as odm
+    for topo in ("complete", "ring", "exponential"):
+        for n in (1, 2, 3, 4, 6, 8, 16):
+            np.testing.assert_allclose(np.array(demuon.mixing_matrix(topo, n)), odm.mixing_matrix(topo, n),
+                                       rtol=0, atol=1e-15)
