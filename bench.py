@@ -352,6 +352,68 @@ def run_owner(args, w_full, dev, world, rank, local, barrier):
     osd.close()
 
 
+def run_demuon(args, w_full, dev, local):
+    """DeMuon iteration over N simulated agents (``--demuon N``), each agent
+    holding the workload's matrices: tracking kernel, msgn through one plan
+    over all agents' matrices, mixing kernel.  One JSON line; the
+    elementwise kernels are reported against the HBM roofline."""
+    import torch
+    from gram_newton_schulz_b200 import demuon, synth
+
+    n = args.demuon
+    dm = demuon.DeMuon(w_full.shapes, n, topology=args.topology, theta=0.1, eta=0.02, device=dev)
+    for a in range(n):
+        for k in range(w_full.count):
+            dm.grad(a, k).copy_(synth.gradients(w_full, dev, indices=[k])[0])
+            dm.iterate(a, k).copy_(synth.weights(w_full, dev, indices=[k])[0].float())
+    dm.plan.momentum_normalize(dm._vb_views, None, beta=0.0)
+    schedule = "cta_pair" if (args.no_autotune or dm.plan.autotune() == 1) else "single_cta"
+    for _ in range(args.warmup):
+        dm.step()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize(dev)
+    for k in range(K):
+        dm.step(events=ev[k])
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    step_ms = ev[0][0].elapsed_time(ev[K - 1][3]) / K
+    t_track = sum(e[0].elapsed_time(e[1]) for e in ev) / K
+    t_msgn = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+    t_mix = sum(e[2].elapsed_time(e[3]) for e in ev) / K
+    peaks, peak_kind = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    elems = n * dm.numel
+    track_gbs = elems * 20 / (t_track / 1e3) / 1e9  # G 2 + M 4 + V 4 read; M 4 + V 4 + bf16 V 2 written
+    mix_gbs = elems * 12 / (t_mix / 1e3) / 1e9      # X 4 + O 4 read; X 4 written
+    line = {
+        "metric": f"DeMuon iteration ms ({n} simulated agents, {args.topology} graph)",
+        "value": round(step_ms, 3), "unit": "ms", "n_gpus": 1, "steps": K, "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 3), "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w_full.name, "agents": n, "topology": args.topology,
+                   "mixing_rate": None, "matrices_per_agent": w_full.count, "theta": 0.1, "eta": 0.02,
+                   "schedule": schedule},
+        "split_ms": {"track": round(t_track, 3), "msgn": round(t_msgn, 3), "mix": round(t_mix, 3)},
+        "roofline": {"bound": "hbm", "achieved": round(track_gbs, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(track_gbs / hbm, 4), "traffic": None, "kernel": "k_demuon_track",
+                     "peak_kind": peak_kind},
+        "mix_kernel": {"kernel": "k_demuon_mix", "achieved": round(mix_gbs, 1), "peak": hbm, "unit": "GB/s",
+                       "frac": round(mix_gbs / hbm, 4)},
+        "gpu_launches": None, "clocks": clk, "e2e": None, "cpu_baseline": None,
+    }
+    import numpy as np
+    w = np.array(dm.mix)
+    s = np.linalg.svd(w, compute_uv=False)
+    line["config"]["mixing_rate"] = round(float(s[1]) if len(s) > 1 else 0.0, 6)
+    print(json.dumps(line), flush=True)
+    dm.close()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -369,6 +431,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--demuon", type=int, default=0,
+                    help="time a DeMuon iteration over this many simulated agents instead of the Muon step")
+    ap.add_argument("--topology", default="ring", choices=["ring", "exponential", "complete"])
     ap.add_argument("--no-autotune", action="store_true",
                     help="keep the default CTA-pair schedule instead of timing both")
     ap.add_argument("--ref-budget", type=float, default=10.0)
@@ -401,6 +466,11 @@ def main():
 
     from gram_newton_schulz_b200 import owners
     w_full = custom_workload(args.shapes) if args.shapes else synth.workload(args.workload)
+    if args.demuon:
+        if world > 1:
+            raise SystemExit("--demuon simulates its agents on one GPU")
+        run_demuon(args, w_full, dev, local)
+        return
     if args.shard == "owner":
         run_owner(args, w_full, dev, world, rank, local, barrier)
         if world > 1:
