@@ -74,9 +74,9 @@ def gemm_alg_bytes(shapes, k=K_STEPS):
 # gemm_tc.cu + plan.cu still hash to it: a changed kernel reports null.
 TRAFFIC_CAPTURE = {
     "sources": ["gram_newton_schulz_b200/csrc/gemm_tc.cu", "gram_newton_schulz_b200/csrc/plan.cu"],
-    "sha256": "35d178b6b405d7b9c62a31188e2ca566963c5218e6502316d736e08c95cf4411",
+    "sha256": "0dc3541f061fdc6ac259bc07ecc570725a0297d200a218144ac21f0ad0039325",
     "workload": "qwen2.5-7b-layer-set-x28",
-    "dram_bytes_per_step": 282.3e9,
+    "dram_bytes_per_step": 394.27e9,
     "launches_per_step": 30,
 }
 

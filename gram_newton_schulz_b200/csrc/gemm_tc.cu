@@ -163,6 +163,19 @@ __device__ __forceinline__ void store_pair(__nv_bfloat16* hi, __nv_bfloat16* lo,
 // Columns per epilogue chunk (one tcgen05.ld of 32 lanes x CW columns).
 constexpr int CW = 16;
 
+// 16-byte global load that asks L2 to fetch the surrounding 256 bytes from
+// DRAM.  An epilogue thread reads its row 32 bytes per chunk, a chunk at a
+// time; with the hint the first chunk brings the warp's whole 256-byte row
+// segment in at once, instead of one 32-byte sector at a time.
+__device__ __forceinline__ uint4 ld_row16(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p)
+               : "memory");
+  return r;
+}
+
 // One CW-column chunk of a Gram-space output tile for the thread's row i.
 // Input and outputs are bf16 hi/lo pairs (FMT_PAIR) or fp32 (FMT_F32).
 // `tri`: store only i <= j and mirror (symmetric outputs, except the
@@ -212,8 +225,8 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
       uint4 uh[CW / 8], ul[CW / 8];
 #pragma unroll
       for (int q = 0; q < CW / 8; ++q) {
-        uh[q] = ph[q];
-        ul[q] = pl[q];
+        uh[q] = ld_row16(ph + q);
+        ul[q] = ld_row16(pl + q);
       }
 #pragma unroll
       for (int q = 0; q < CW / 8; ++q) {
@@ -236,9 +249,9 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
 #pragma unroll
       for (int q = 0; q < CW / 8; ++q) {
         float fh[8], fl[8];
-        unpack8(ph[q], fh);
+        unpack8(ld_row16(ph + q), fh);
         if (pl) {
-          unpack8(pl[q], fl);
+          unpack8(ld_row16(pl + q), fl);
         } else {
 #pragma unroll
           for (int e = 0; e < 8; ++e) fl[e] = 0.f;
@@ -385,7 +398,7 @@ __device__ __forceinline__ void epi_update_chunk(const GemmProblem& pr, int mat,
           uint4* pw = reinterpret_cast<uint4*>(w + rowoff + col0);
           uint4 wv[CW / 8];
 #pragma unroll
-          for (int q = 0; q < CW / 8; ++q) wv[q] = pw[q];
+          for (int q = 0; q < CW / 8; ++q) wv[q] = ld_row16(pw + q);
 #pragma unroll
           for (int q = 0; q < CW / 8; ++q) {
             float f[8];
@@ -1050,10 +1063,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
 // arrives on; the wait gives up after timeout_ns and sets DMU_FLAG_TIMEOUT.
 __global__ void k_wait_selftest(unsigned int* status, long long timeout_ns) {
   __shared__ __align__(8) uint64_t bar;
-  __shared__ int abort_flag;
   if (threadIdx.x == 0) {
     ptx::mbar_init(ptx::smem_u32(&bar), 1);
-    abort_flag = 0;
     ptx::fence_mbar_init();
   }
   __syncthreads();
