@@ -50,6 +50,30 @@ def alg_flops(shapes, k=K_STEPS):
     return tot
 
 
+def executed_flops(shapes, k=K_STEPS, tile=256):
+    """MMA flops the default (AUTO) precision actually issues in one step.
+
+    Per matrix (m = min, n = max):
+    * SYRK: one bf16 MMA per K slice over the upper 256 x 256 tiles.
+    * 4K - 3 symmetric products over the same tiles: one scaled-fp16 MMA per
+      K slice for m >= 1024 (F16 class), three bf16 MMAs (hi.hi + hi.lo +
+      lo.hi) below (SPLIT3).
+    * The final: hi and lo of P, two MMAs over every m x n tile.
+    Diagonal tiles are computed whole.  Tiles are counted as full 256 x 256
+    blocks; ragged edges are ignored."""
+    tot = 0.0
+    for r, c in shapes:
+        m, n = min(r, c), max(r, c)
+        tb = -(-m // tile)
+        upper = tb * (tb + 1) // 2 * tile * tile          # elements of the upper tiles
+        mm = min(m, tb * tile)
+        terms = 1 if m >= 1024 else 3
+        tot += 2.0 * upper * n                              # SYRK
+        tot += (4 * k - 3) * terms * 2.0 * upper * mm       # products, K = m
+        tot += 2 * 2.0 * m * m * n                          # final, two terms
+    return tot
+
+
 def gemm_alg_bytes(shapes, k=K_STEPS):
     """Algorithmic DRAM bytes of the tensor-core launches of one step, every
     operand read once and every result written once (half-stored symmetric
@@ -531,6 +555,7 @@ def main():
     torch.cuda.synchronize(dev)
     barrier()
     eager_ms = ev[0][0].elapsed_time(ev[K - 1][3]) / K
+    per_step = [e[0].elapsed_time(e[3]) for e in ev]
     t_mom = sum(e[0].elapsed_time(e[1]) for e in ev)
     t_gram = sum(e[1].elapsed_time(e[2]) for e in ev)
     t_upd = sum(e[2].elapsed_time(e[3]) for e in ev)
@@ -663,7 +688,10 @@ def main():
                        "parallelism": f"replica x{world} (one owned layer set per rank)",
                        "schedule": schedule, "launch": graph_note,
                        "l2": "inputs larger than L2 (no flush needed)"},
-            "throughput": {"matrices_per_s": round(len(job_shapes) / (step_ms / 1e3), 1),
+            "step_ms_stats": {"median": round(statistics.median(per_step), 3), "min": round(min(per_step), 3),
+                              "max": round(max(per_step), 3), "of": "eager steps"},
+            "throughput": {"executed_tflops": round(executed_flops(job_shapes) / (step_ms / 1e3) / 1e12, 1),
+                           "matrices_per_s": round(len(job_shapes) / (step_ms / 1e3), 1),
                            "alg_tflops": round(job_flops / (step_ms / 1e3) / 1e12, 1),
                            "alg_tflops_frac_per_gpu": round(job_flops / world / (step_ms / 1e3) / 1e12 / peak_tf, 4)},
             "split_ms": {"momentum": round(t_mom / K, 3), "gram": round(t_gram / K, 3),

@@ -71,3 +71,14 @@ def test_captured_traffic_applies_only_to_its_sources(monkeypatch):
             h.update(fh.read())
     monkeypatch.setattr(bench, "TRAFFIC_CAPTURE", dict(cap, sha256=h.hexdigest()))
     assert bench.captured_traffic(cap["workload"]) == cap["dram_bytes_per_step"] / cap["launches_per_step"]
+
+
+def test_executed_flops_counts_issued_mma_work():
+    # one 256 x 512 matrix: one 256 x 256 upper tile, SPLIT3 (3 MMAs) below m = 1024
+    up = 256 * 256
+    assert bench.executed_flops([(256, 512)]) == 2 * up * 512 + 17 * 3 * 2 * up * 256 + 4 * 256 * 256 * 512
+    # m = 1024: 4 x 4 blocks, 10 upper tiles, one F16 MMA per K slice
+    up = 10 * 256 * 256
+    assert bench.executed_flops([(1024, 4096)]) == 2 * up * 4096 + 17 * 1 * 2 * up * 1024 + 4 * 1024 * 1024 * 4096
+    w = synth.workload("qwen2.5-7b-layer-set-x28")
+    assert 1.2 < bench.executed_flops(w.shapes) / bench.alg_flops(w.shapes) < 1.45
