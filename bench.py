@@ -570,13 +570,29 @@ def main():
     graph_note = "off (--no-graph)"
     total_ms = eager_ms
     if not args.no_graph:
+        g = None
         try:
             g = torch.cuda.CUDAGraph()
             torch.cuda.synchronize(dev)
-            with torch.cuda.graph(g):
+            # thread_local: a communicator's watchdog thread may poll its
+            # events while this thread captures
+            with torch.cuda.graph(g, capture_error_mode="thread_local"):
                 step()
             g.replay()
             torch.cuda.synchronize(dev)
+            graph_note = "captured step replayed (CUDA graph)"
+        except Exception as e:  # capture refused: keep the eager number, say why
+            graph_note = f"capture failed, eager timing: {type(e).__name__}: {str(e)[:120]}"
+            g = None
+        # every rank takes the same path: graph timing only if all captured
+        all_ok = g is not None
+        if world > 1:
+            flag = torch.tensor([1 if all_ok else 0], dtype=torch.int32, device=dev)
+            dist.all_reduce(flag, op=dist.ReduceOp.MIN)
+            all_ok = bool(flag.item())
+            if not all_ok and g is not None:
+                graph_note = "another rank's capture failed, eager timing"
+        if all_ok:
             gev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
             barrier()
             torch.cuda.synchronize(dev)
@@ -587,11 +603,7 @@ def main():
             torch.cuda.synchronize(dev)
             barrier()
             total_ms = gev[0].elapsed_time(gev[1]) / K
-            graph_note = "captured step replayed (CUDA graph)"
-            del g
-        except Exception as e:  # capture refused: keep the eager number, say why
-            graph_note = f"capture failed, eager timing: {type(e).__name__}: {str(e)[:120]}"
-            total_ms = eager_ms
+        del g
     clk = clocks.stop()
     total_ms *= K
     # per-rank launches are those of the captured run only for the whole
