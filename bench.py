@@ -382,7 +382,7 @@ def run_demuon(args, w_full, dev, local):
     over all agents' matrices, mixing kernel.  One JSON line; the
     elementwise kernels are reported against the HBM roofline."""
     import torch
-    from gram_newton_schulz_b200 import demuon, synth
+    from gram_newton_schulz_b200 import demuon, dmu, synth
 
     n = args.demuon
     dm = demuon.DeMuon(w_full.shapes, n, topology=args.topology, theta=0.1, eta=0.02, device=dev)
@@ -391,7 +391,7 @@ def run_demuon(args, w_full, dev, local):
             dm.grad(a, k).copy_(synth.gradients(w_full, dev, indices=[k])[0])
             dm.iterate(a, k).copy_(synth.weights(w_full, dev, indices=[k])[0].float())
     dm.plan.momentum_normalize(dm._vb_views, None, beta=0.0)
-    schedule = "cta_pair" if (args.no_autotune or dm.plan.autotune() == 1) else "single_cta"
+    schedule = "cta_pair" if args.no_autotune else dmu.SCHEDULES[dm.plan.autotune()]
     for _ in range(args.warmup):
         dm.step()
     torch.cuda.synchronize(dev)
@@ -523,7 +523,7 @@ def main():
     # on this plan's own data and keep the faster (both give bitwise-equal
     # results).  It needs the momentum image, so one momentum pass first.
     plan.momentum_normalize(grads, moms, beta=w.beta, eps=1e-7)
-    schedule = "cta_pair" if (args.no_autotune or plan.autotune() == 1) else "single_cta"
+    schedule = "cta_pair" if args.no_autotune else dmu.SCHEDULES[plan.autotune()]
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)

@@ -141,7 +141,9 @@ struct SimtProblem {
 };
 
 // ---------------------------------------------------------------- launchers
-cudaError_t launch_gemm_tc(const GemmParams& p, int na, int nb, int kind, int num_sms, cudaStream_t s);
+// Single-CTA tensor-core launch: 128 x tbn tiles, tbn = 256 or 128.
+cudaError_t launch_gemm_tc(const GemmParams& p, int na, int nb, int kind, int num_sms, int tbn,
+                           cudaStream_t s);
 // CTA-pair variant: 256 x 256 tiles (tiles_* of every problem computed with
 // a 256-row block), clusters of 2 CTAs, tcgen05.mma.cta_group::2.
 cudaError_t launch_gemm_tc2(const GemmParams& p, int na, int nb, int kind, int num_sms, cudaStream_t s);

@@ -32,13 +32,15 @@
 
 namespace dmu {
 
-template <int NA, int NB>
+template <int NA, int NB, int TBN = BN>
 struct TcCfg {  // stage geometry is the same for both operand kinds
-  static constexpr int STAGE_BYTES = NA * A_PART_BYTES + NB * B_PART_BYTES;
+  static constexpr int B_PART = TBN * BK * 2;  // TBN rows of one 128-byte K row
+  static constexpr int STAGE_BYTES = NA * A_PART_BYTES + NB * B_PART;
   static constexpr int STAGES = (200 * 1024) / STAGE_BYTES;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
-  static_assert(STAGES >= 2, "at least two stages");
+  static_assert(STAGES >= 2 && STAGES <= 13, "stage count (barrier area holds 13)");
+  static_assert(TBN == 128 || TBN == 256, "tile width");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 
@@ -46,7 +48,7 @@ struct TileCoord {
   int pi, mat, bi, bj;
 };
 
-template <int TBM>
+template <int TBM, int TBN = BN>
 __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int t) {
   TileCoord c;
   int pi = 0;
@@ -60,10 +62,10 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int t) {
     bi = tl % pr.tiles_m;
     bj = tl / pr.tiles_m;
   } else {
-    // column block bj holds row blocks 0 .. min(tiles_m, ((bj+1)*BN-1)/TBM + 1) - 1
+    // column block bj holds row blocks 0 .. min(tiles_m, ((bj+1)*TBN-1)/TBM + 1) - 1
     bj = 0;
     for (;;) {
-      int cnt = min(pr.tiles_m, ((bj + 1) * BN - 1) / TBM + 1);
+      int cnt = min(pr.tiles_m, ((bj + 1) * TBN - 1) / TBM + 1);
       if (tl < cnt) break;
       tl -= cnt;
       ++bj;
@@ -465,9 +467,9 @@ __device__ __forceinline__ void epi_update_chunk(const GemmProblem& pr, int mat,
 }
 
 // ------------------------------------------------------------- kernel
-template <int NA, int NB, int KIND>
+template <int NA, int NB, int KIND, int TBN>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_constant__ GemmParams p) {
-  using Cfg = TcCfg<NA, NB>;
+  using Cfg = TcCfg<NA, NB, TBN>;
   constexpr int BKE = KIND == KIND_TF32 ? 32 : 64;  // elements per 128-byte K-block row
   constexpr int OPFMT = KIND == KIND_TF32 ? 2 : (KIND == KIND_F16 ? 0 : 1);  // idesc A/B format code
   constexpr int S = Cfg::STAGES;
@@ -525,7 +527,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
       bool ok = true;
       uint32_t issued_mask = 0, issued_par = 0;  // per stage: a load was issued, its phase parity
       for (int t = blockIdx.x; ok && t < p.total_tiles; t += gridDim.x) {
-        const TileCoord tc = decode_tile<BM>(p, t);
+        const TileCoord tc = decode_tile<BM, TBN>(p, t);
         const GemmProblem& pr = p.prob[tc.pi];
         // Per-tile operand parameters, read from the parameter space once.
         const CUtensorMap* am = &p.maps[pr.a_map];
@@ -534,9 +536,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
         const CUtensorMap* bm_t = pr.half_b ? &p.maps[pr.b_map_t] : bm;
         const int na = (NA > 1 && (pr.terms & TERM_LH)) ? 2 : 1;
         const int nb = (NB > 1 && (pr.terms & TERM_HL)) ? 2 : 1;
-        const uint32_t bytes = na * A_PART_BYTES + nb * B_PART_BYTES;
+        const uint32_t bytes = na * A_PART_BYTES + nb * Cfg::B_PART;
         const int nk = (pr.K + BKE - 1) / BKE;
-        const int arow = tc.bi * BM, brow = tc.bj * BN;
+        const int arow = tc.bi * BM, brow = tc.bj * TBN;
         const int thr_a = pr.half_a ? arow / HALF_BLOCK : 0, thr_b = pr.half_b ? brow / HALF_BLOCK : 0;
         const bool a_mn = pr.a_mn != 0, b_mn = pr.b_mn != 0;
         const int za0 = pr.a_z[0] + tc.mat, za1 = pr.a_z[1] + tc.mat;
@@ -569,14 +571,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
             }
           }
           for (int part = 0; part < nb; ++part) {
-            const uint32_t dst = sb + part * B_PART_BYTES;
+            const uint32_t dst = sb + part * Cfg::B_PART;
             const int z = part ? zb1 : zb0;
             if (!b_mn && !b_t) {
-              ptx::tma_load_3d(dst, bm_k, fb, k0, brow, z);
-              ptx::tma_load_3d(dst + 16384, bm_k, fb, k0, brow + 128, z);
+#pragma unroll
+              for (int c = 0; c < TBN / 128; ++c) ptx::tma_load_3d(dst + 16384 * c, bm_k, fb, k0, brow + 128 * c, z);
             } else {
 #pragma unroll
-              for (int c = 0; c < 4; ++c) ptx::tma_load_3d(dst + 8192 * c, bm_k, fb, brow + 64 * c, k0, z);
+              for (int c = 0; c < TBN / 64; ++c) ptx::tma_load_3d(dst + 8192 * c, bm_k, fb, brow + 64 * c, k0, z);
             }
           }
           if (++stage == S) {
@@ -610,7 +612,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
       bool ok = true;
       bool issued = false;
       for (int t = blockIdx.x; ok && t < p.total_tiles; t += gridDim.x) {
-        const TileCoord tc = decode_tile<BM>(p, t);
+        const TileCoord tc = decode_tile<BM, TBN>(p, t);
         const GemmProblem& pr = p.prob[tc.pi];
         const int nk = (pr.K + BKE - 1) / BKE;
         if (!wait_bar(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p)) {
@@ -618,13 +620,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
           break;
         }
         ptx::tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * TBN);
         // Per-tile MMA parameters in registers: the K loop issues MMAs from
         // precomputed descriptor halves only.
         const int terms = pr.terms, pr_a_mn = pr.a_mn, pr_b_mn = pr.b_mn;
         const int thr_a = pr.half_a ? (tc.bi * BM) / HALF_BLOCK : 0;
-        const int thr_b = pr.half_b ? (tc.bj * BN) / HALF_BLOCK : 0;
-        const uint32_t idesc0 = ptx::make_idesc(BM, BN, 0, 0, OPFMT);
+        const int thr_b = pr.half_b ? (tc.bj * TBN) / HALF_BLOCK : 0;
+        const uint32_t idesc0 = ptx::make_idesc(BM, TBN, 0, 0, OPFMT);
         const uint64_t hi_k = ptx::make_sw128_desc(0u, 16u, 1024u), hi_mn = ptx::make_sw128_desc(0u, 8192u, 1024u);
         uint32_t accumulate = 0;
         for (int kb = 0; kb < nk; ++kb) {
@@ -649,7 +651,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
               if (term == 2 && NA < 2) continue;
               if (!(terms & (1 << term))) continue;
               const uint32_t pa = sa + (term == 2 ? A_PART_BYTES : 0) + kk * a_ks;
-              const uint32_t pb = sb + (term == 1 ? B_PART_BYTES : 0) + kk * b_ks;
+              const uint32_t pb = sb + (term == 1 ? Cfg::B_PART : 0) + kk * b_ks;
               const uint64_t ad = a_hi | (uint64_t)((pa >> 4) & 0x3FFFu);
               const uint64_t bd = b_hi | (uint64_t)((pb >> 4) & 0x3FFFu);
               if (KIND == KIND_TF32)
@@ -686,12 +688,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
   } else {
     // ------------------------------------------------ epilogue (warps 2..9)
     const int q = warp & 3;                        // TMEM lane quarter this warp may access
-    const int ch_begin = ((warp - 2) >> 2) * (BN / 2 / CW);  // column half of the tile
-    const int ch_end = ch_begin + BN / 2 / CW;
+    const int ch_begin = ((warp - 2) >> 2) * (TBN / 2 / CW);  // column half of the tile
+    const int ch_end = ch_begin + TBN / 2 / CW;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
-      const TileCoord tc = decode_tile<BM>(p, t);
+      const TileCoord tc = decode_tile<BM, TBN>(p, t);
       const GemmProblem& pr = p.prob[tc.pi];
       int ok = 1;
       if (lane == 0) ok = wait_bar(tfull_bar(acc), acc_phase, abort_flag, p) ? 1 : 0;
@@ -699,15 +701,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
       if (!ok) break;
       ptx::tc_fence_after();
       const int row_lo = tc.bi * BM + q * 32;
-      const bool tri = pr.sym && (!pr.half_out || (tc.bi * BM) / HALF_BLOCK == tc.bj);
+      const bool tri = pr.sym && (!pr.half_out || (tc.bi * BM) / HALF_BLOCK == (tc.bj * TBN) / HALF_BLOCK);
       const int i = row_lo + lane;
       for (int ch = ch_begin; ch < ch_end; ++ch) {
-        const int col0 = tc.bj * BN + ch * CW;
+        const int col0 = tc.bj * TBN + ch * CW;
         if (col0 >= pr.N) break;
         if (tri && col0 + CW - 1 < row_lo) continue;  // chunk strictly below the diagonal
         if (row_lo >= pr.M) break;
         uint32_t r[CW];
-        ptx::tmem_ld16(tmem_base + (uint32_t)(acc * BN + ch * CW) + ((uint32_t)(q * 32) << 16), r);
+        ptx::tmem_ld16(tmem_base + (uint32_t)(acc * TBN + ch * CW) + ((uint32_t)(q * 32) << 16), r);
         ptx::tmem_wait_ld();
         if (pr.epi == EPI_GRAM)
           epi_gram_chunk(pr, tc.mat, i, col0, r, tri);
@@ -1086,10 +1088,10 @@ cudaError_t launch_wait_selftest(unsigned int* status, long long timeout_ns, cud
   return cudaGetLastError();
 }
 
-template <int NA, int NB, int KIND>
+template <int NA, int NB, int KIND, int TBN>
 static cudaError_t configure_one() {
-  return cudaFuncSetAttribute(k_gemm_tc<NA, NB, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              TcCfg<NA, NB>::SMEM_BYTES);
+  return cudaFuncSetAttribute(k_gemm_tc<NA, NB, KIND, TBN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              TcCfg<NA, NB, TBN>::SMEM_BYTES);
 }
 
 template <int NA, int NB, int KIND>
@@ -1100,11 +1102,16 @@ static cudaError_t configure_two() {
 
 cudaError_t gemm_tc_configure() {
   cudaError_t e;
-  if ((e = configure_one<1, 1, KIND_BF16>()) != cudaSuccess) return e;
-  if ((e = configure_one<2, 1, KIND_BF16>()) != cudaSuccess) return e;
-  if ((e = configure_one<2, 2, KIND_BF16>()) != cudaSuccess) return e;
-  if ((e = configure_one<1, 1, KIND_TF32>()) != cudaSuccess) return e;
-  if ((e = configure_one<1, 1, KIND_F16>()) != cudaSuccess) return e;
+  if ((e = configure_one<1, 1, KIND_BF16, 256>()) != cudaSuccess) return e;
+  if ((e = configure_one<1, 1, KIND_BF16, 128>()) != cudaSuccess) return e;
+  if ((e = configure_one<2, 1, KIND_BF16, 256>()) != cudaSuccess) return e;
+  if ((e = configure_one<2, 1, KIND_BF16, 128>()) != cudaSuccess) return e;
+  if ((e = configure_one<2, 2, KIND_BF16, 256>()) != cudaSuccess) return e;
+  if ((e = configure_one<2, 2, KIND_BF16, 128>()) != cudaSuccess) return e;
+  if ((e = configure_one<1, 1, KIND_TF32, 256>()) != cudaSuccess) return e;
+  if ((e = configure_one<1, 1, KIND_TF32, 128>()) != cudaSuccess) return e;
+  if ((e = configure_one<1, 1, KIND_F16, 256>()) != cudaSuccess) return e;
+  if ((e = configure_one<1, 1, KIND_F16, 128>()) != cudaSuccess) return e;
   if ((e = configure_two<1, 1, KIND_BF16>()) != cudaSuccess) return e;
   if ((e = configure_two<2, 1, KIND_BF16>()) != cudaSuccess) return e;
   if ((e = configure_two<2, 2, KIND_BF16>()) != cudaSuccess) return e;
@@ -1121,10 +1128,13 @@ int gemm_tc_stages(int na, int nb) {
 }
 
 template <int NA, int NB, int KIND>
-static cudaError_t launch_one(const GemmParams& p, int num_sms, cudaStream_t s) {
+static cudaError_t launch_one(const GemmParams& p, int num_sms, int tbn, cudaStream_t s) {
   const int grid = p.total_tiles < num_sms ? p.total_tiles : num_sms;
   if (grid <= 0) return cudaSuccess;
-  k_gemm_tc<NA, NB, KIND><<<grid, GEMM_THREADS, TcCfg<NA, NB>::SMEM_BYTES, s>>>(p);
+  if (tbn == 128)
+    k_gemm_tc<NA, NB, KIND, 128><<<grid, GEMM_THREADS, TcCfg<NA, NB, 128>::SMEM_BYTES, s>>>(p);
+  else
+    k_gemm_tc<NA, NB, KIND, 256><<<grid, GEMM_THREADS, TcCfg<NA, NB, 256>::SMEM_BYTES, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -1152,18 +1162,20 @@ cudaError_t launch_gemm_tc2(const GemmParams& p, int na, int nb, int kind, int n
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_gemm_tc(const GemmParams& p, int na, int nb, int kind, int num_sms, cudaStream_t s) {
+cudaError_t launch_gemm_tc(const GemmParams& p, int na, int nb, int kind, int num_sms, int tbn,
+                           cudaStream_t s) {
+  if (tbn != 128 && tbn != 256) return cudaErrorInvalidValue;
   if (kind == KIND_TF32) {
-    if (na == 1 && nb == 1) return launch_one<1, 1, KIND_TF32>(p, num_sms, s);
+    if (na == 1 && nb == 1) return launch_one<1, 1, KIND_TF32>(p, num_sms, tbn, s);
     return cudaErrorInvalidValue;
   }
   if (kind == KIND_F16) {
-    if (na == 1 && nb == 1) return launch_one<1, 1, KIND_F16>(p, num_sms, s);
+    if (na == 1 && nb == 1) return launch_one<1, 1, KIND_F16>(p, num_sms, tbn, s);
     return cudaErrorInvalidValue;
   }
-  if (na == 1 && nb == 1) return launch_one<1, 1, KIND_BF16>(p, num_sms, s);
-  if (na == 2 && nb == 1) return launch_one<2, 1, KIND_BF16>(p, num_sms, s);
-  if (na == 2 && nb == 2) return launch_one<2, 2, KIND_BF16>(p, num_sms, s);
+  if (na == 1 && nb == 1) return launch_one<1, 1, KIND_BF16>(p, num_sms, tbn, s);
+  if (na == 2 && nb == 1) return launch_one<2, 1, KIND_BF16>(p, num_sms, tbn, s);
+  if (na == 2 && nb == 2) return launch_one<2, 2, KIND_BF16>(p, num_sms, tbn, s);
   return cudaErrorInvalidValue;
 }
 

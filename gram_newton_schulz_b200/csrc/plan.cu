@@ -130,7 +130,9 @@ struct dmu_plan_s {
   float eps = 1e-7f;
   int launches = 0;
   long long timeout_ns = 2000000000LL;
-  bool cta_pair = true;  // tensor-core launches on CTA pairs (256 x 256 tiles)
+  // tensor-core tile schedule: 1 = CTA pairs (256 x 256 tiles), 0 = single
+  // CTAs (128 x 256), 2 = single CTAs (128 x 128, for many small matrices)
+  int sched = 1;
   bool half_store = true;  // half-stored symmetric Gram-space matrices
 
   unsigned int* status_dev() const { return reinterpret_cast<unsigned int*>(ws + off_status); }
@@ -197,13 +199,13 @@ bool aligned16(const void* const* ptrs, int n) {
 // Tile grid of one problem for row blocks of `bm` (128: one CTA per tile;
 // 256: a CTA pair per tile) and column blocks of BN; symmetric problems keep
 // only the tiles that touch the upper triangle (same rule as the kernels).
-int tiles_for(int M, int N, bool sym, int* tm, int* tn, int bm = BM) {
+int tiles_for(int M, int N, bool sym, int* tm, int* tn, int bm = BM, int bn = BN) {
   *tm = (M + bm - 1) / bm;
-  *tn = (N + BN - 1) / BN;
+  *tn = (N + bn - 1) / bn;
   if (!sym) return (*tm) * (*tn);
   int t = 0;
   for (int bj = 0; bj < *tn; ++bj) {
-    int c = ((bj + 1) * BN - 1) / bm + 1;
+    int c = ((bj + 1) * bn - 1) / bm + 1;
     t += c < *tm ? c : *tm;
   }
   return t;
@@ -246,7 +248,8 @@ dmu_status run_tc(dmu_plan p, std::vector<Prob>& probs, int na, int nb, int kind
       g.b_map = slot(probs[i].bmap);
       g.a_map_t = probs[i].amap_t >= 0 ? slot(probs[i].amap_t) : g.a_map;
       g.b_map_t = probs[i].bmap_t >= 0 ? slot(probs[i].bmap_t) : g.b_map;
-      g.tiles_per_mat = tiles_for(g.M, g.N, g.sym != 0, &g.tiles_m, &g.tiles_n, p->cta_pair ? 256 : BM);
+      g.tiles_per_mat = tiles_for(g.M, g.N, g.sym != 0, &g.tiles_m, &g.tiles_n, p->sched == 1 ? 256 : BM,
+                                  p->sched == 2 ? 128 : BN);
       g.tile_begin = tiles;
       tiles += g.count * g.tiles_per_mat;
       gp.prob[nprob++] = g;
@@ -257,10 +260,10 @@ dmu_status run_tc(dmu_plan p, std::vector<Prob>& probs, int na, int nb, int kind
     gp.total_tiles = tiles;
     gp.status = p->status_dev();
     gp.timeout_ns = p->timeout_ns;
-    if (p->cta_pair)
+    if (p->sched == 1)
       CUDA_TRY(launch_gemm_tc2(gp, na, nb, kind, p->num_sms, s));
     else
-      CUDA_TRY(launch_gemm_tc(gp, na, nb, kind, p->num_sms, s));
+      CUDA_TRY(launch_gemm_tc(gp, na, nb, kind, p->num_sms, p->sched == 2 ? 128 : 256, s));
     p->launches++;
   }
   return DMU_OK;
@@ -742,7 +745,11 @@ dmu_status dmu_plan_create(const dmu_shape* shapes, int count, dmu_dtype dtype, 
   p->count = count;
   p->shapes.assign(shapes, shapes + count);
   p->esize = dtype == DMU_BF16 ? 2 : 4;
-  if (const char* e = std::getenv("DMU_CTA_PAIR")) p->cta_pair = std::atoi(e) != 0;
+  if (const char* e = std::getenv("DMU_CTA_PAIR")) p->sched = std::atoi(e) != 0 ? 1 : 0;
+  if (const char* e = std::getenv("DMU_SCHEDULE")) {
+    const int v = std::atoi(e);
+    if (v >= 0 && v <= 2) p->sched = v;
+  }
   if (const char* e = std::getenv("DMU_HALF")) p->half_store = std::atoi(e) != 0;
 
   int ndev = 0;
@@ -1227,7 +1234,7 @@ static std::string schedule_key(dmu_plan p) {
   return k.str();
 }
 
-int dmu_get_schedule(dmu_plan p) { return p ? (p->cta_pair ? 1 : 0) : -1; }
+int dmu_get_schedule(dmu_plan p) { return p ? p->sched : -1; }
 
 dmu_status dmu_autotune(dmu_plan p, const char* cache_path, void* stream) {
   g_err.clear();
@@ -1244,21 +1251,21 @@ dmu_status dmu_autotune(dmu_plan p, const char* cache_path, void* stream) {
     while (std::getline(in, line)) {
       std::istringstream ls(line);
       std::string k;
-      int pair = -1;
-      if ((ls >> k >> pair) && k == key && (pair == 0 || pair == 1)) {
-        p->cta_pair = pair == 1;
+      int sched = -1;
+      if ((ls >> k >> sched) && k == key && sched >= 0 && sched <= 2) {
+        p->sched = sched;
         return DMU_OK;
       }
     }
   }
   const float co[3] = {3.4445f, -4.7750f, 2.0315f};
-  float ms[2] = {0.f, 0.f};
+  float ms[3] = {0.f, 0.f, 0.f};
   cudaEvent_t e0, e1;
   CUDA_TRY(cudaEventCreate(&e0));
   CUDA_TRY(cudaEventCreate(&e1));
-  const bool keep = p->cta_pair;
-  for (int variant = 0; variant < 2; ++variant) {
-    p->cta_pair = variant == 1;
+  const int keep = p->sched;
+  for (int variant = 0; variant < 3; ++variant) {
+    p->sched = variant;
     st = gram_bf16(p, co, 5, s);  // warm-up
     for (int rep = 0; st == DMU_OK && rep < 3; ++rep) {
       CUDA_TRY(cudaEventRecord(e0, s));
@@ -1270,7 +1277,7 @@ dmu_status dmu_autotune(dmu_plan p, const char* cache_path, void* stream) {
       ms[variant] = rep == 0 ? t : std::min(ms[variant], t);
     }
     if (st != DMU_OK) {
-      p->cta_pair = keep;
+      p->sched = keep;
       cudaEventDestroy(e0);
       cudaEventDestroy(e1);
       return st;
@@ -1278,11 +1285,17 @@ dmu_status dmu_autotune(dmu_plan p, const char* cache_path, void* stream) {
   }
   cudaEventDestroy(e0);
   cudaEventDestroy(e1);
-  p->cta_pair = ms[1] <= ms[0];
+  // the CTA-pair schedule wins ties, then 128 x 256 single CTAs
+  int best = 1;
+  if (ms[0] < ms[best]) best = 0;
+  if (ms[2] < ms[best]) best = 2;
+  p->sched = best;
   p->have_p = true;
   if (cache_path) {
     std::ofstream out(cache_path, std::ios::app);
-    if (out) out << key << " " << (p->cta_pair ? 1 : 0) << " pair_ms=" << ms[1] << " single_ms=" << ms[0] << "\n";
+    if (out)
+      out << key << " " << best << " pair_ms=" << ms[1] << " single_ms=" << ms[0] << " single128_ms=" << ms[2]
+          << "\n";
   }
   return DMU_OK;
 }

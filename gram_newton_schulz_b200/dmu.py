@@ -28,6 +28,7 @@ STATUS_NAMES = ["OK", "INVALID_ARG", "UNSUPPORTED", "WORKSPACE", "CUDA", "NONFIN
 DTYPES = {"bf16": 0, "f32": 1}
 PRECS = {"auto": 0, "fast": 1, "split2": 2, "split3": 3, "tf32": 4, "f16": 5}
 FLAG_NONFINITE, FLAG_TIMEOUT = 1, 2
+SCHEDULES = {0: "single_cta", 1: "cta_pair", 2: "single_cta_n128"}
 
 # name -> (restype, argtypes); every symbol of include/dmu.h
 _VP = ctypes.c_void_p
@@ -204,8 +205,9 @@ class Plan:
         self.apply_update(weights, lr, out_o, stream)
 
     def autotune(self, cache_path: Optional[str] = None, stream=None) -> int:
-        """Choose the faster tensor-core schedule by measurement (needs a prior
-        momentum_normalize); returns 1 for CTA pairs, 0 for single CTAs."""
+        """Choose the fastest tensor-core schedule by measurement (needs a prior
+        momentum_normalize); returns 1 for CTA pairs (256 x 256 tiles), 0 for
+        single CTAs with 128 x 256 tiles, 2 for single CTAs with 128 x 128."""
         _check(self.lib.dmu_autotune(self.handle, cache_path.encode() if cache_path else None,
                                      _stream_handle(stream, self.device)))
         return int(self.lib.dmu_get_schedule(self.handle))

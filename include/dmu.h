@@ -49,9 +49,13 @@
  *     vectorised paths (misaligned pointers take a scalar path).
  *   - Threads: a plan must not be used by two host threads at once.
  *   - Schedule: tensor-core launches run on CTA pairs (256 x 256 tiles,
- *     tcgen05.mma.cta_group::2) unless the environment variable
- *     DMU_CTA_PAIR=0 is set when the plan is created (one CTA per
- *     128 x 256 tile).
+ *     tcgen05.mma.cta_group::2) by default.  Two single-CTA schedules
+ *     exist: 128 x 256 tiles, and 128 x 128 tiles for many small matrices.
+ *     dmu_autotune picks one by measurement.  At plan creation the
+ *     environment variable DMU_SCHEDULE=0|1|2 (0 = 128 x 256 single CTAs,
+ *     1 = CTA pairs, 2 = 128 x 128 single CTAs) overrides the default, and
+ *     so does DMU_CTA_PAIR=0|1.  Every schedule accumulates each element
+ *     over K in the same order, so all give bitwise-equal results.
  */
 #ifndef DMU_H
 #define DMU_H
@@ -194,18 +198,20 @@ DMU_API dmu_status dmu_read_status(dmu_plan plan, uint32_t* flags);
  * Synchronises `stream`. */
 DMU_API dmu_status dmu_debug_gram(dmu_plan plan, int which, int index, float* out, void* stream);
 
-/* Pick the faster tensor-core schedule for this plan by measurement (DMuon
+/* Pick the fastest tensor-core schedule for this plan by measurement (DMuon
  * page, section 2.4: per-shape kernel configurations are tuned once and
  * cached).  Times the whole Gram recursion (K = 5) with CTA-pair kernels
- * (256 x 256 tiles) and with single-CTA kernels (128 x 256 tiles) on the
- * data left by dmu_momentum_normalize, keeps the faster, and appends the
+ * (256 x 256 tiles) and with single-CTA kernels (128 x 256 and 128 x 128
+ * tiles) on the data left by dmu_momentum_normalize, keeps the fastest
+ * (CTA pairs win ties), and appends the
  * choice to the text file `cache_path` (may be NULL: no cache).  A cached
  * entry for the same device, shapes, dtype and precision is reused without
  * timing.  Synchronises `stream`; overwrites the plan's Gram-space state.
  * Errors: NOT_PLANNED (no dmu_momentum_normalize yet), CUDA. */
 DMU_API dmu_status dmu_autotune(dmu_plan plan, const char* cache_path, void* stream);
 
-/* Current schedule of the plan: 1 = CTA pairs, 0 = single CTA. */
+/* Current schedule of the plan: 1 = CTA pairs (256 x 256), 0 = single
+ * CTAs (128 x 256), 2 = single CTAs (128 x 128); -1 for a NULL plan. */
 DMU_API int dmu_get_schedule(dmu_plan plan);
 
 /* Number of kernel launches the last compute call enqueued. */

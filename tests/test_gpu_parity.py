@@ -340,17 +340,18 @@ def test_half_and_full_storage_agree(prec, monkeypatch):
 @pytest.mark.parametrize("prec", ["auto", "split3", "tf32"])
 def test_cta_pair_and_single_cta_agree(prec, monkeypatch):
     """The CTA-pair kernels (256 x 256 tiles, cta_group::2) and the single-CTA
-    kernels (128 x 256 tiles) accumulate every element over K in the same
-    order, so they must give bitwise-equal results."""
-    shapes = [(1100, 3000), (3000, 1100), (512, 2048), (520, 200), (384, 384)]
+    kernels (128 x 256 and 128 x 128 tiles) accumulate every element over K
+    in the same order, so they must give bitwise-equal results."""
+    shapes = [(1100, 3000), (3000, 1100), (512, 2048), (520, 200), (384, 384), (128, 512), (100, 300)]
     w = synth.custom("pair", shapes, seed=29)
-    monkeypatch.setenv("DMU_CTA_PAIR", "1")
+    monkeypatch.setenv("DMU_SCHEDULE", "1")
     a = run_step(w, prec=prec)
-    monkeypatch.setenv("DMU_CTA_PAIR", "0")
-    b = run_step(w, prec=prec)
-    for i in range(w.count):
-        assert torch.equal(a["o"][i], b["o"][i]), shapes[i]
-        assert torch.equal(a["w_after"][i], b["w_after"][i]), shapes[i]
+    for sched in ("0", "2"):
+        monkeypatch.setenv("DMU_SCHEDULE", sched)
+        b = run_step(w, prec=prec)
+        for i in range(w.count):
+            assert torch.equal(a["o"][i], b["o"][i]), (sched, shapes[i])
+            assert torch.equal(a["w_after"][i], b["w_after"][i]), (sched, shapes[i])
 
 
 def test_autotune_picks_and_caches_schedule(tmp_path):
@@ -361,9 +362,9 @@ def test_autotune_picks_and_caches_schedule(tmp_path):
     plan = dmu.Plan(shapes)
     plan.momentum_normalize(grads, None, beta=0.0)
     choice = plan.autotune(cache)
-    assert choice in (0, 1)
+    assert choice in (0, 1, 2)
     text = open(cache).read()
-    assert "pair_ms=" in text and "single_ms=" in text
+    assert "pair_ms=" in text and "single_ms=" in text and "single128_ms=" in text
     # a second plan with the same shapes reuses the cached choice
     plan2 = dmu.Plan(shapes)
     plan2.momentum_normalize(grads, None, beta=0.0)
