@@ -98,9 +98,9 @@ def gemm_alg_bytes(shapes, k=K_STEPS):
 # gemm_tc.cu + plan.cu still hash to it: a changed kernel reports null.
 TRAFFIC_CAPTURE = {
     "sources": ["gram_newton_schulz_b200/csrc/gemm_tc.cu", "gram_newton_schulz_b200/csrc/plan.cu"],
-    "sha256": "0dc3541f061fdc6ac259bc07ecc570725a0297d200a218144ac21f0ad0039325",
+    "sha256": "420df83e0f5cc7e0185ec55d7839f0b29986d77e621a90e3308b7ff88620bf05",
     "workload": "qwen2.5-7b-layer-set-x28",
-    "dram_bytes_per_step": 394.27e9,
+    "dram_bytes_per_step": 259.92e9,
     "launches_per_step": 30,
 }
 
