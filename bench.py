@@ -276,7 +276,8 @@ def run_owner(args, w_full, dev, world, rank, local, barrier):
     import torch
     from gram_newton_schulz_b200 import dmu, dp, owners, synth
 
-    osd = dp.OwnerShardedStep(w_full.shapes, dtype=w_full.dtype, prec=args.prec, device=dev)
+    measured = dp.shared_costs(w_full.shapes) if args.measured_owners else None
+    osd = dp.OwnerShardedStep(w_full.shapes, dtype=w_full.dtype, prec=args.prec, device=dev, measured=measured)
     b = osd.buckets
     wdt = torch.bfloat16 if w_full.dtype == "bf16" else torch.float32
     gflat, wflat = b.alloc(wdt, dev), b.alloc(wdt, dev)
@@ -356,6 +357,7 @@ def run_owner(args, w_full, dev, world, rank, local, barrier):
                        "K": K_STEPS, "coeffs": [3.4445, -4.7750, 2.0315], "precision": args.prec,
                        "parallelism": f"owner x{world}: LPT owners, reduce in / broadcast out over "
                                       f"{'NCCL' if world > 1 else 'nothing (1 rank)'}",
+                       "owner_costs": "measured per shape on rank 0" if args.measured_owners else "flop model",
                        "l2": "inputs larger than L2 (no flush needed)"},
             "throughput": {"matrices_per_s": round(w_full.count / (step_ms / 1e3), 1),
                            "alg_tflops": round(job_flops / (step_ms / 1e3) / 1e12, 1),
@@ -455,6 +457,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--measured-owners", action="store_true",
+                    help="owner mode: LPT on per-shape costs measured on rank 0 instead of the flop model")
     ap.add_argument("--demuon", type=int, default=0,
                     help="time a DeMuon iteration over this many simulated agents instead of the Muon step")
     ap.add_argument("--topology", default="ring", choices=["ring", "exponential", "complete"])

@@ -78,6 +78,20 @@ class OwnerBuckets:
         return [self.view(flats, i) for i in range(len(self.shapes))]
 
 
+def shared_costs(shapes, measure=None, group=None, src: int = 0) -> Dict[Tuple[int, int], float]:
+    """Per-shape costs that every rank agrees on: rank ``src`` measures
+    them (``owners.measure_costs`` on its GPU by default) and broadcasts the
+    table, so LPT gives the same owners everywhere."""
+    import torch.distributed as dist
+    if measure is None:
+        measure = owners.measure_costs
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size(group) == 1:
+        return dict(measure(shapes))
+    box = [dict(measure(shapes)) if dist.get_rank(group) == src else None]
+    dist.broadcast_object_list(box, src=src, group=group)
+    return box[0]
+
+
 class PlanCompute:
     """The owned matrices' update on the GPU: one `dmu.Plan` over them."""
 

@@ -9,8 +9,9 @@ fallback: longest-processing-time-first (LPT) list scheduling on a per-matrix
 cost, which is within 4/3 of the optimal makespan.
 
 The cost of a matrix is the step's algorithmic flop count (Gram SYRK, the
-symmetric products of K steps and the final product) unless measured costs
-are supplied.  Host logic only: no device work happens here.
+symmetric products of K steps and the final product).  `measure_costs`
+returns measured per-shape costs instead, timed through the library on the
+GPU; they override the flop model.  Everything else here is host logic.
 """
 from __future__ import annotations
 
@@ -73,3 +74,34 @@ def max_over_ranks(value: float, device=None) -> float:
     t = torch.tensor([float(value)], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def measure_costs(shapes: Sequence[Tuple[int, int]], device=None, reps: int = 2,
+                  max_per_shape: int = 4) -> Dict[Tuple[int, int], float]:
+    """Measured cost (ms per matrix) of one full update for every distinct
+    shape, timed on this GPU with CUDA events.  This is the per-shape
+    profiling that the DMuon page's load balancer feeds its assignment
+    with (section 2.3).  Each shape gets a plan over up to ``max_per_shape``
+    copies, so batching is part of the cost, and a synthetic bf16 gradient.
+    Device work only through the library."""
+    import torch
+    from . import dmu, synth
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    out: Dict[Tuple[int, int], float] = {}
+    for shape in sorted({(int(r), int(c)) for r, c in shapes}):
+        k = min(max_per_shape, sum(1 for s in shapes if (int(s[0]), int(s[1])) == shape))
+        w = synth.custom("cost", [shape] * k, seed=17)
+        grads = synth.gradients(w, dev)
+        weights = synth.weights(w, dev)
+        moms = [torch.zeros(shape, dtype=torch.float32, device=dev) for _ in range(k)]
+        plan = dmu.Plan([shape] * k, device=dev)
+        plan.step(grads, moms, weights, lr=0.0)  # warm-up, uploads the pointer tables
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            plan.step(grads, moms, weights, lr=0.0)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        out[shape] = e0.elapsed_time(e1) / reps / k
+        plan.close()
+    return out

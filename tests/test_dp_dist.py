@@ -213,3 +213,38 @@ def test_gloo_missing_rank_is_an_error_not_a_hang():
                 p.kill()
     assert got[1] == "left"
     assert got[0].startswith("error"), got[0]
+
+
+def _cost_worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        # every rank "measures" something different; only rank 0's table counts
+        fake = lambda shapes: {tuple(s): float(s[0] * s[1]) * (1.0 + rank) for s in shapes}  # noqa: E731
+        costs = dp.shared_costs(SHAPES, measure=fake)
+        step = dp.OwnerShardedStep(SHAPES, compute=OracleCompute([]), measured=costs)
+        q.put((rank, sorted(costs.items()), list(step.buckets.owner)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_measured_costs_are_shared_so_owners_agree():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_cost_worker, args=(r, 3, port, q)) for r in range(3)]
+    for p in procs:
+        p.start()
+    try:
+        res = [q.get(timeout=180) for _ in range(3)]
+    finally:
+        for p in procs:
+            p.join(timeout=60)
+            if p.is_alive():
+                p.kill()
+    costs = {r: c for r, c, _ in res}
+    owners_ = {r: o for r, _, o in res}
+    assert costs[0] == costs[1] == costs[2]
+    assert dict(costs[0])[(8, 24)] == 8 * 24 * 1.0  # rank 0's measurement
+    assert owners_[0] == owners_[1] == owners_[2]

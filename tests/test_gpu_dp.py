@@ -39,3 +39,14 @@ def test_owner_step_on_flat_buffers_matches_plan_step():
     assert osd.compute.plan.read_status() == 0
     osd.close()
     plan.close()
+
+
+def test_measured_costs_order_shapes_by_work():
+    from gram_newton_schulz_b200 import owners
+    shapes = [(256, 1024), (1024, 4096), (1024, 4096), (512, 512)]
+    costs = owners.measure_costs(shapes)
+    assert set(costs) == {(256, 1024), (1024, 4096), (512, 512)}
+    assert all(c > 0 for c in costs.values())
+    assert costs[(1024, 4096)] > costs[(256, 1024)]
+    own = owners.assign_shapes(shapes, 2, measured=costs)
+    assert sorted(set(own)) == [0, 1]
