@@ -76,20 +76,23 @@ def max_over_ranks(value: float, device=None) -> float:
     return float(t.item())
 
 
-def measure_costs(shapes: Sequence[Tuple[int, int]], device=None, reps: int = 2,
-                  max_per_shape: int = 4) -> Dict[Tuple[int, int], float]:
+def measure_costs(shapes: Sequence[Tuple[int, int]], device=None, reps: int = 3,
+                  batch: int = 4) -> Dict[Tuple[int, int], float]:
     """Measured cost (ms per matrix) of one full update for every distinct
     shape, timed on this GPU with CUDA events.  This is the per-shape
     profiling that the DMuon page's load balancer feeds its assignment
-    with (section 2.3).  Each shape gets a plan over up to ``max_per_shape``
-    copies, so batching is part of the cost, and a synthetic bf16 gradient.
-    Device work only through the library."""
+    with (section 2.3).
+
+    Each shape is timed in batches of ``batch`` and ``2 * batch`` copies.
+    The cost is the difference divided by ``batch``: the marginal cost of
+    one more matrix in a batched step.  Fixed per-launch overheads, which a
+    rank pays once whatever it owns, then cancel.  Synthetic bf16
+    gradients; device work only through the library."""
     import torch
     from . import dmu, synth
     dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
-    out: Dict[Tuple[int, int], float] = {}
-    for shape in sorted({(int(r), int(c)) for r, c in shapes}):
-        k = min(max_per_shape, sum(1 for s in shapes if (int(s[0]), int(s[1])) == shape))
+
+    def step_ms(shape, k):
         w = synth.custom("cost", [shape] * k, seed=17)
         grads = synth.gradients(w, dev)
         weights = synth.weights(w, dev)
@@ -102,6 +105,14 @@ def measure_costs(shapes: Sequence[Tuple[int, int]], device=None, reps: int = 2,
             plan.step(grads, moms, weights, lr=0.0)
         e1.record()
         torch.cuda.synchronize(dev)
-        out[shape] = e0.elapsed_time(e1) / reps / k
         plan.close()
+        return e0.elapsed_time(e1) / reps
+
+    out: Dict[Tuple[int, int], float] = {}
+    distinct = sorted({(int(r), int(c)) for r, c in shapes})
+    step_ms(distinct[0], 1)  # first-use costs (module load, clocks) outside the measurements
+    for shape in distinct:
+        t1 = step_ms(shape, batch)
+        t2 = step_ms(shape, 2 * batch)
+        out[shape] = max((t2 - t1) / batch, 1e-6)
     return out
