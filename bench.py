@@ -527,7 +527,10 @@ def main():
     # on this plan's own data and keep the faster (both give bitwise-equal
     # results).  It needs the momentum image, so one momentum pass first.
     plan.momentum_normalize(grads, moms, beta=w.beta, eps=1e-7)
-    schedule = "cta_pair" if args.no_autotune else dmu.SCHEDULES[plan.autotune()]
+    if w.dtype != "bf16":
+        schedule = "simt_fp32"  # fp32 plans run the FFMA path; nothing to tune
+    else:
+        schedule = "cta_pair" if args.no_autotune else dmu.SCHEDULES[plan.autotune()]
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
