@@ -277,7 +277,8 @@ def run_owner(args, w_full, dev, world, rank, local, barrier):
     from gram_newton_schulz_b200 import dmu, dp, owners, synth
 
     measured = dp.shared_costs(w_full.shapes) if args.measured_owners else None
-    osd = dp.OwnerShardedStep(w_full.shapes, dtype=w_full.dtype, prec=args.prec, device=dev, measured=measured)
+    osd = dp.OwnerShardedStep(w_full.shapes, dtype=w_full.dtype, prec=args.prec, device=dev, measured=measured,
+                              method=args.owner_method)
     b = osd.buckets
     wdt = torch.bfloat16 if w_full.dtype == "bf16" else torch.float32
     gflat, wflat = b.alloc(wdt, dev), b.alloc(wdt, dev)
@@ -358,6 +359,7 @@ def run_owner(args, w_full, dev, world, rank, local, barrier):
                        "parallelism": f"owner x{world}: LPT owners, reduce in / broadcast out over "
                                       f"{'NCCL' if world > 1 else 'nothing (1 rank)'}",
                        "owner_costs": "measured per shape on rank 0" if args.measured_owners else "flop model",
+                       "owner_method": args.owner_method,
                        "l2": "inputs larger than L2 (no flush needed)"},
             "throughput": {"matrices_per_s": round(w_full.count / (step_ms / 1e3), 1),
                            "alg_tflops": round(job_flops / (step_ms / 1e3) / 1e12, 1),
@@ -457,6 +459,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--owner-method", default="milp", choices=["milp", "lpt"],
+                    help="owner mode: exact MILP over per-cost counts (LPT fallback) or greedy LPT")
     ap.add_argument("--measured-owners", action="store_true",
                     help="owner mode: LPT on per-shape costs measured on rank 0 instead of the flop model")
     ap.add_argument("--demuon", type=int, default=0,

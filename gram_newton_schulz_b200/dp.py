@@ -48,10 +48,16 @@ class OwnerBuckets:
     bucket.  The same on every rank: LPT is deterministic."""
 
     def __init__(self, shapes: Sequence[Tuple[int, int]], world: int,
-                 measured: Optional[Dict[Tuple[int, int], float]] = None):
+                 measured: Optional[Dict[Tuple[int, int], float]] = None, method: str = "lpt",
+                 owner: Optional[Sequence[int]] = None):
         self.shapes = [(int(r), int(c)) for r, c in shapes]
         self.world = int(world)
-        self.owner = owners.assign_shapes(self.shapes, self.world, measured=measured)
+        if owner is not None:
+            if len(owner) != len(self.shapes) or any(not 0 <= int(o) < self.world for o in owner):
+                raise ValueError("owner: one rank in [0, world) per matrix")
+            self.owner = [int(o) for o in owner]
+        else:
+            self.owner = owners.assign_shapes(self.shapes, self.world, measured=measured, method=method)
         self.members: List[List[int]] = [owners.owned_indices(self.owner, r) for r in range(self.world)]
         self.offset = [0] * len(self.shapes)
         self.sizes = [0] * self.world
@@ -128,13 +134,21 @@ class OwnerShardedStep:
     """
 
     def __init__(self, shapes, *, group=None, compute=None, dtype="bf16", prec="auto",
-                 device=None, measured=None):
+                 device=None, measured=None, method: str = "lpt"):
         import torch.distributed as dist
         self.group = group
         self.dist = dist.is_available() and dist.is_initialized()
         self.world = dist.get_world_size(group) if self.dist else 1
         self.rank = dist.get_rank(group) if self.dist else 0
-        self.buckets = OwnerBuckets(shapes, self.world, measured=measured)
+        owner = None
+        if self.world > 1:
+            # rank 0 decides and every rank takes its answer, so the owners
+            # agree even if a solver's result depended on the process
+            box = [owners.assign_shapes(shapes, self.world, measured=measured, method=method)
+                   if self.rank == 0 else None]
+            dist.broadcast_object_list(box, src=0, group=group)
+            owner = box[0]
+        self.buckets = OwnerBuckets(shapes, self.world, measured=measured, method=method, owner=owner)
         self.mine = self.buckets.members[self.rank]
         owned = [self.buckets.shapes[i] for i in self.mine]
         self.compute = compute if compute is not None else PlanCompute(owned, dtype, prec, device)

@@ -4,9 +4,10 @@ DMuon page, section 2.1 (owner-centric execution): every weight matrix has
 exactly one owner rank, which keeps its optimizer state and runs its update
 once.  Section 2.3 (computation-aware load balancing): owners are chosen to
 minimise the predicted makespan -- by an MILP, with a greedy heuristic as
-the fallback for large search spaces.  This module implements the greedy
-fallback: longest-processing-time-first (LPT) list scheduling on a per-matrix
-cost, which is within 4/3 of the optimal makespan.
+the fallback for large search spaces.  This module implements both: the
+greedy fallback, longest-processing-time-first (LPT) list scheduling on a
+per-matrix cost (within 4/3 of the optimal makespan), and `milp_assign`,
+an exact mixed-integer program over per-cost counts.
 
 The cost of a matrix is the step's algorithmic flop count (Gram SYRK, the
 symmetric products of K steps and the final product).  `measure_costs`
@@ -42,6 +43,67 @@ def lpt_assign(costs: Sequence[float], n_ranks: int) -> List[int]:
     return owner
 
 
+def milp_assign(costs: Sequence[float], n_ranks: int, time_limit: float = 5.0,
+                max_vars: int = 4000) -> List[int]:
+    """Owners that minimise the makespan, by a mixed-integer program (DMuon
+    page, section 2.3), with LPT as the fallback for large search spaces.
+
+    Matrices of equal cost are interchangeable, so the program has one
+    integer count y[s, r] per distinct cost s and rank r:
+
+        minimise T  subject to  sum_r y[s, r] = n_s  for every s,
+                                sum_s c_s y[s, r] <= T  for every rank r,
+
+    solved by scipy's HiGHS interface within ``time_limit`` seconds.  The
+    counts are then dealt to the matrices of each cost in index order.  The
+    program's answer is kept only when its makespan is not worse than
+    LPT's.  With more than ``max_vars`` variables, or without a solution in
+    time, the result is LPT's."""
+    import numpy as np
+    from scipy.optimize import Bounds, LinearConstraint, milp
+
+    lpt = lpt_assign(costs, n_ranks)
+    if n_ranks == 1 or not costs:
+        return lpt
+    groups: Dict[float, List[int]] = {}
+    for i, c in enumerate(costs):
+        groups.setdefault(float(c), []).append(i)
+    keys = sorted(groups, reverse=True)
+    n_s, n_r = len(keys), n_ranks
+    nv = n_s * n_r + 1
+    if nv > max_vars:
+        return lpt
+    obj = np.zeros(nv)
+    obj[-1] = 1.0
+    a_eq = np.zeros((n_s, nv))
+    counts = np.array([len(groups[k]) for k in keys], dtype=float)
+    for si in range(n_s):
+        a_eq[si, si * n_r:(si + 1) * n_r] = 1.0
+    a_ub = np.zeros((n_r, nv))
+    for r in range(n_r):
+        for si, k in enumerate(keys):
+            a_ub[r, si * n_r + r] = k
+        a_ub[r, -1] = -1.0
+    lb = np.zeros(nv)
+    ub = np.concatenate([np.repeat(counts, n_r), [np.inf]])
+    integrality = np.concatenate([np.ones(nv - 1), [0]])
+    res = milp(obj, constraints=[LinearConstraint(a_eq, counts, counts), LinearConstraint(a_ub, -np.inf, 0.0)],
+               integrality=integrality, bounds=Bounds(lb, ub), options={"time_limit": float(time_limit)})
+    if res.x is None:
+        return lpt
+    y = np.rint(res.x[:-1]).astype(int).reshape(n_s, n_r)
+    if not all(int(y[si].sum()) == len(groups[k]) for si, k in enumerate(keys)) or (y < 0).any():
+        return lpt
+    owner = [0] * len(costs)
+    for si, k in enumerate(keys):
+        ids, pos = groups[k], 0
+        for r in range(n_r):
+            for _ in range(int(y[si, r])):
+                owner[ids[pos]] = r
+                pos += 1
+    return owner if makespan(costs, owner, n_ranks) <= makespan(costs, lpt, n_ranks) else lpt
+
+
 def makespan(costs: Sequence[float], owner: Sequence[int], n_ranks: int) -> float:
     loads = [0.0] * n_ranks
     for c, r in zip(costs, owner):
@@ -54,13 +116,18 @@ def owned_indices(owner: Sequence[int], rank: int) -> List[int]:
 
 
 def assign_shapes(shapes: Sequence[Tuple[int, int]], n_ranks: int, steps: int = 5,
-                  measured: Optional[Dict[Tuple[int, int], float]] = None) -> List[int]:
+                  measured: Optional[Dict[Tuple[int, int], float]] = None, method: str = "lpt") -> List[int]:
     """Owners for a list of (rows, cols); ``measured`` maps a shape to its
-    measured per-matrix cost and overrides the flop model for that shape."""
+    measured per-matrix cost and overrides the flop model for that shape.
+    ``method``: "lpt" (greedy) or "milp" (exact program, LPT fallback)."""
     costs = []
     for r, c in shapes:
         key = (int(r), int(c))
         costs.append(measured[key] if measured and key in measured else matrix_cost(r, c, steps))
+    if method == "milp":
+        return milp_assign(costs, n_ranks)
+    if method != "lpt":
+        raise ValueError(f"unknown owner method {method!r}")
     return lpt_assign(costs, n_ranks)
 
 

@@ -184,13 +184,15 @@ def _dying_worker(rank, world, port, q):
         q.join_thread()
         os._exit(0)  # leaves between steps, before the exchange
     buckets = dp.OwnerBuckets(SHAPES, world)
-    step = dp.OwnerShardedStep(SHAPES, compute=OracleCompute(buckets.members[rank]))
-    gf, wf = buckets.alloc(torch.float32, "cpu"), buckets.alloc(torch.float32, "cpu")
-    moms = [torch.zeros(SHAPES[i]) for i in step.mine]
     try:
+        # the owner table is broadcast from rank 0 when the step is built,
+        # and the exchange follows: either collective reports the missing peer
+        step = dp.OwnerShardedStep(SHAPES, compute=OracleCompute(buckets.members[rank]))
+        gf, wf = buckets.alloc(torch.float32, "cpu"), buckets.alloc(torch.float32, "cpu")
+        moms = [torch.zeros(SHAPES[i]) for i in step.mine]
         step.step(gf, wf, moms)
         q.put((rank, "no error"))
-    except Exception as e:  # the collective reports the missing peer
+    except Exception as e:
         q.put((rank, "error: " + type(e).__name__))
     q.close()
     q.join_thread()

@@ -107,3 +107,29 @@ def test_two_gloo_ranks_cover_every_matrix_once():
     for rank, covered, same, mx in results:
         assert covered and same
         assert mx == 11.0
+
+
+@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("n", [2, 3])
+def test_milp_reaches_the_optimum_on_small_instances(seed, n):
+    g = torch.Generator().manual_seed(100 + seed)
+    base = (torch.rand(3, generator=g) * 10 + 1).tolist()
+    costs = [base[int(i)] for i in torch.randint(0, 3, (7,), generator=g)]  # repeated costs, as shapes repeat
+    own = owners.milp_assign(costs, n)
+    assert sorted(set(own)) <= list(range(n)) and len(own) == len(costs)
+    assert owners.makespan(costs, own, n) == pytest.approx(_opt_makespan(costs, n), rel=1e-9)
+    assert owners.makespan(costs, own, n) <= owners.makespan(costs, owners.lpt_assign(costs, n), n) + 1e-9
+    assert own == owners.milp_assign(costs, n)
+
+
+def test_milp_on_the_layer_set_is_valid_and_no_worse_than_lpt():
+    w = synth.workload("qwen2.5-7b-layer-set-x28")
+    costs = [owners.matrix_cost(r, c) for r, c in w.shapes]
+    for n in (2, 3, 5, 8):
+        own = owners.assign_shapes(w.shapes, n, method="milp")
+        assert len(own) == w.count and sorted(set(own)) == list(range(n))
+        assert owners.makespan(costs, own, n) <= owners.makespan(costs, owners.lpt_assign(costs, n), n) + 1e-6
+    with pytest.raises(ValueError):
+        owners.assign_shapes(w.shapes, 2, method="annealing")
+    # too many variables: the greedy fallback
+    assert owners.milp_assign(costs, 8, max_vars=10) == owners.lpt_assign(costs, 8)
