@@ -267,6 +267,27 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def all_ranks_ok(ok: bool, dev, world: int) -> bool:
+    """True only if every rank reports ok (MIN all-reduce), so that all
+    ranks take the same branch before the next collective."""
+    if world <= 1:
+        return ok
+    import torch
+    import torch.distributed as dist
+    flag = torch.tensor([1 if ok else 0], dtype=torch.int32, device=dev)
+    dist.all_reduce(flag, op=dist.ReduceOp.MIN)
+    return bool(flag.item())
+
+
+def pin_copies(tensors):
+    """Pinned host copies of device tensors, or (None, reason) when the host
+    cannot pin that much memory."""
+    try:
+        return [t.to("cpu").pin_memory() for t in tensors], None
+    except RuntimeError as e:  # host out of pinnable memory
+        return None, f"{type(e).__name__}: {str(e)[:100]}"
+
+
 def run_owner(args, w_full, dev, world, rank, local, barrier):
     """Owner-sharded data-parallel step (DMuon page, section 2.1): every rank
     holds the gradients and weights of the whole layer set; one reduce per
@@ -321,10 +342,15 @@ def run_owner(args, w_full, dev, world, rank, local, barrier):
     # rank's whole local gradient from pinned memory and reads the whole
     # updated model back.
     e2e = None
+    h_g = h_w = None
     if not args.no_e2e:
+        h_g, why = pin_copies(gflat)
+        if h_g is not None:
+            h_w, why = pin_copies(wflat)
+        if not all_ranks_ok(h_w is not None, dev, world):
+            e2e = {"value": None, "unit": "ms", "note": f"host buffers not pinned on some rank: {why}"}
+    if not args.no_e2e and e2e is None:
         E = args.e2e_steps
-        h_g = [t.to("cpu").pin_memory() for t in gflat]
-        h_w = [t.to("cpu").pin_memory() for t in wflat]
         h2d = sum(t.numel() * t.element_size() for t in h_g)
         d2h = sum(t.numel() * t.element_size() for t in h_w)
         barrier()
@@ -644,10 +670,15 @@ def main():
     # waits for that download.  All copies of every timed step are inside
     # the timed region.
     e2e = None
+    h_grads = h_w = None
     if not args.no_e2e:
+        h_grads, why = pin_copies(grads)
+        if h_grads is not None:
+            h_w, why = pin_copies(weights)
+        if not all_ranks_ok(h_w is not None, dev, world):
+            e2e = {"value": None, "unit": "ms", "note": f"host buffers not pinned on some rank: {why}"}
+    if not args.no_e2e and e2e is None:
         E = args.e2e_steps
-        h_grads = [g.to("cpu").pin_memory() for g in grads]
-        h_w = [x.to("cpu").pin_memory() for x in weights]
         g_buf = [grads, [torch.empty_like(g) for g in grads]]
         h2d = sum(t.numel() * t.element_size() for t in h_grads)
         d2h = sum(t.numel() * t.element_size() for t in h_w)
