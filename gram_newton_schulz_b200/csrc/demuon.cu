@@ -234,11 +234,17 @@ extern "C" DMU_API dmu_status dmu_demuon_track(int n_agents, int64_t numel, cons
     }
   }
   for (int i = 0; i < n_agents; ++i)
-    for (int j = 0; j < n_agents; ++j)
+    for (int j = 0; j < n_agents; ++j) {
       if (a.v_out[i] == a.v_in[j]) {
         set_last_error("v_out must not alias v_in: every output reads all agents' v_in");
         return DMU_ERR_INVALID_ARG;
       }
+      if (a.v_out[i] == a.m[j] || (const void*)a.vb[i] == (const void*)a.g[j] ||
+          (const void*)a.vb[i] == (const void*)a.m[j] || (const void*)a.v_out[i] == (const void*)a.vb[j]) {
+        set_last_error("v_out, v_bf16 and momenta must be distinct arrays, and v_bf16 must not alias grads");
+        return DMU_ERR_INVALID_ARG;
+      }
+    }
   for (int i = n_agents; i < DEMUON_MAX; ++i) {
     a.g[i] = nullptr;
     a.m[i] = a.v_out[i] = nullptr;

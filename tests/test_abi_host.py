@@ -176,6 +176,9 @@ def test_demuon_argument_errors_before_any_launch():
     assert track(2, 16, m2, float("nan"), a, b, c, d, e, None) == dmu.ERR_INVALID_ARG
     assert track(2, 16, m2, 0.1, a, b, c, c, e, None) == dmu.ERR_INVALID_ARG      # v_out aliases v_in
     assert b"alias" in lib.dmu_last_error()
+    assert track(2, 16, m2, 0.1, a, b, c, b, e, None) == dmu.ERR_INVALID_ARG      # v_out aliases momenta
+    assert track(2, 16, m2, 0.1, a, b, c, d, a, None) == dmu.ERR_INVALID_ARG      # v_bf16 aliases grads
+    assert track(2, 16, m2, 0.1, a, b, c, d, d, None) == dmu.ERR_INVALID_ARG      # v_bf16 aliases v_out
     odd, ko = ptrs(0x1004, 0x2000)
     assert track(2, 16, m2, 0.1, odd, b, c, d, e, None) == dmu.ERR_INVALID_ARG    # misaligned
     assert b"16-byte" in lib.dmu_last_error()
