@@ -621,13 +621,9 @@ def main():
             graph_note = f"capture failed, eager timing: {type(e).__name__}: {str(e)[:120]}"
             g = None
         # every rank takes the same path: graph timing only if all captured
-        all_ok = g is not None
-        if world > 1:
-            flag = torch.tensor([1 if all_ok else 0], dtype=torch.int32, device=dev)
-            dist.all_reduce(flag, op=dist.ReduceOp.MIN)
-            all_ok = bool(flag.item())
-            if not all_ok and g is not None:
-                graph_note = "another rank's capture failed, eager timing"
+        all_ok = all_ranks_ok(g is not None, dev, world)
+        if not all_ok and g is not None:
+            graph_note = "another rank's capture failed, eager timing"
         if all_ok:
             gev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
             barrier()

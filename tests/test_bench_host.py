@@ -82,3 +82,56 @@ def test_executed_flops_counts_issued_mma_work():
     assert bench.executed_flops([(1024, 4096)]) == 2 * up * 4096 + 17 * 1 * 2 * up * 1024 + 4 * 1024 * 1024 * 4096
     w = synth.workload("qwen2.5-7b-layer-set-x28")
     assert 1.2 < bench.executed_flops(w.shapes) / bench.alg_flops(w.shapes) < 1.45
+
+
+def _agree_worker(rank, world, port, q):
+    import datetime
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        all_true = bench.all_ranks_ok(True, "cpu", world)
+        one_false = bench.all_ranks_ok(rank != 1, "cpu", world)
+        q.put((rank, all_true, one_false))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_all_ranks_ok_is_a_min_over_ranks():
+    """bench.py decides the graph-timed and e2e legs collectively: one rank's
+    failure turns the leg off everywhere, so no rank waits alone in a
+    collective.  Three gloo ranks on 127.0.0.1."""
+    import socket
+    import torch.multiprocessing as mp
+    sock = socket.socket()
+    sock.bind(("127.0.0.1", 0))
+    port = sock.getsockname()[1]
+    sock.close()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_agree_worker, args=(r, 3, port, q)) for r in range(3)]
+    for p in procs:
+        p.start()
+    try:
+        res = [q.get(timeout=120) for _ in range(3)]
+    finally:
+        for p in procs:
+            p.join(timeout=60)
+            if p.is_alive():
+                p.kill()
+    assert all(a is True and b is False for _, a, b in res)
+    assert bench.all_ranks_ok(False, "cpu", 1) is False and bench.all_ranks_ok(True, "cpu", 1) is True
+
+
+def test_pin_copies_reports_failure_instead_of_raising(monkeypatch):
+    import torch
+
+    class Bad:
+        def to(self, *_):
+            raise RuntimeError("cannot pin")
+
+    out, why = bench.pin_copies([Bad()])
+    assert out is None and "cannot pin" in why
+    ok, why = bench.pin_copies([torch.zeros(3)]) if torch.cuda.is_available() else ([None], None)
+    assert why is None
