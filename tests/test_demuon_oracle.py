@@ -193,3 +193,14 @@ def test_pins_accept_the_oracle_and_reject_every_mutant():
     assert _pins_hold(lambda *a: _step(*a))  # the unmutated copy passes too
     for bug in ["swapped W index", "flipped tracking sign", "msgn of the old V", "update not mixed"]:
         assert not _pins_hold(lambda *a, b=bug: _step(*a, bug=b)), bug
+
+
+@pytest.mark.parametrize("n", [3, 5, 8, 13, 16])
+def test_exponential_mixing_rate_closed_form(n):
+    """The exponential graph's W is circulant with equal weights on the
+    offsets {0} and {2^k < n}; its eigenvalues are the averages of the
+    matching roots of unity, and W is normal, so its singular values are
+    their moduli."""
+    hops = [0] + [1 << k for k in range(n.bit_length()) if (1 << k) < n]
+    eig = [abs(sum(np.exp(-2j * np.pi * h * k / n) for h in hops)) / len(hops) for k in range(1, n)]
+    assert demuon.mixing_rate(demuon.mixing_matrix("exponential", n)) == pytest.approx(max(eig), abs=1e-12)

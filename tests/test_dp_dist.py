@@ -250,3 +250,47 @@ def test_measured_costs_are_shared_so_owners_agree():
     assert costs[0] == costs[1] == costs[2]
     assert dict(costs[0])[(8, 24)] == 8 * 24 * 1.0  # rank 0's measurement
     assert owners_[0] == owners_[1] == owners_[2]
+
+
+def _sparse_worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        shapes = SHAPES[:3]  # fewer matrices than ranks: some ranks own nothing
+        step = dp.OwnerShardedStep(shapes, compute=OracleCompute([]))
+        step.compute.indices = list(step.mine)
+        b = step.buckets
+        gf, wf = b.alloc(torch.float32, "cpu"), b.alloc(torch.float32, "cpu")
+        for i in range(len(shapes)):
+            b.view(gf, i).copy_(torch.from_numpy(_grad(i, rank)))
+            b.view(wf, i).copy_(torch.from_numpy(_weight(i)))
+        moms = [torch.from_numpy(_momentum0(i)).clone() for i in step.mine]
+        step.step(gf, wf, moms, beta=BETA, lr=LR, eps=EPS)
+        q.put((rank, list(step.mine), [b.view(wf, i).numpy().copy() for i in range(len(shapes))]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_more_ranks_than_matrices():
+    world = 5
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_sparse_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    try:
+        res = [q.get(timeout=180) for _ in range(world)]
+    finally:
+        for p in procs:
+            p.join(timeout=60)
+            if p.is_alive():
+                p.kill()
+    ew, _ = _expected(world)
+    owned = sorted(i for _, mine, _ in res for i in mine)
+    assert owned == [0, 1, 2]
+    assert sum(1 for _, mine, _ in res if not mine) == world - 3
+    for rank, mine, weights in res:
+        for i in range(3):
+            assert np.array_equal(weights[i], ew[i]), (rank, i)
