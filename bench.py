@@ -254,12 +254,19 @@ def run_reference(args):
         total, threads, sample, _ = oracle_sample_seconds(w.shapes, budget_s=args.ref_budget)
         if k >= args.warmup:
             vals.append(total * 1e3)
-    v = statistics.median(vals)
+    # The job of an N-GPU run is N layer sets (one per rank, weak scaling);
+    # the host cores do all of them, so the per-set time is scaled by N.
+    world = max(1, int(os.environ.get("WORLD_SIZE", "1")))
+    v = statistics.median(vals) * world
+    if world > 1:
+        sample += f"; times {world} layer sets, the job of {world} ranks"
     line = {
-        "impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "ms", "n_gpus": args.gpus,
+        "impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "ms", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(v, 3), "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "matrices": w.count, "K": K_STEPS, "coeffs": [3.4445, -4.7750, 2.0315]},
+        "config": {"workload": w.name, "matrices": w.count, "matrices_total": w.count * world, "K": K_STEPS,
+                   "coeffs": [3.4445, -4.7750, 2.0315], "precision": "f64 oracle",
+                   "parallelism": f"replica x{world}, all on the host cores"},
         "cpu_baseline": {"value": round(v, 3), "unit": "ms", "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": round(v, 3), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
