@@ -27,6 +27,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -151,7 +152,7 @@ class ClockSampler:
 
     def start(self):
         try:
-            out_dir = os.path.join(ROOT, "gpurun_out")
+            out_dir = os.environ.get("DMU_CLOCKS_DIR") or tempfile.gettempdir()
             os.makedirs(out_dir, exist_ok=True)
             self.path = os.path.join(out_dir, f"clocks_rank{self.index}.csv")
             self.fh = open(self.path, "w")
