@@ -18,7 +18,8 @@ Each pin is independent of the oracle's own arithmetic:
 ``test_pins_catch_planted_mistakes`` plants plausible mistakes in copies of
 the oracle (a dropped term, a flipped sign, swapped coefficients, a missing
 step, a transposed iterate, a missing normalisation) and checks that a pin
-fails for every one of them.
+fails for every one of them; ``test_gram_pin_catches_planted_mistakes`` does
+the same for the Gram-space form (a one-sided G update, an unaccumulated P).
 """
 import json
 import math
@@ -211,7 +212,13 @@ def test_bf16_bits_conversion():
 # ---------------------------------------------------------------- mutations
 def _pins_pass(mod):
     """Run the spectral, polar and special-case pins against a module-like
-    object that provides ``orthogonalize`` with the oracle's signature."""
+    object that provides ``orthogonalize`` with the oracle's signature.
+    Diverging mutants overflow; that is their expected failure, not a warning."""
+    with np.errstate(over="ignore", invalid="ignore"):
+        return _pins_pass_inner(mod)
+
+
+def _pins_pass_inner(mod):
     try:
         rng = np.random.default_rng(42)
         for shape in [(5, 9), (9, 5), (6, 6)]:
@@ -313,3 +320,43 @@ def test_pins_catch_planted_mistakes():
 
     # Not a mistake: the Gram matrix on the other side is equivalent.
     assert _pins_pass(_Mutant(_rect_right_gram))
+
+
+# Mistakes planted in the Gram-space form: the Gram == rectangular pin, with
+# the rectangular form pinned to the SVD above, must reject every one.
+def _gram_pin_passes(gram_fn):
+    for shape in [(8, 8), (12, 30)]:
+        rng = np.random.default_rng(shape[0] * 7 + shape[1])
+        x0 = oracle.frobenius_normalize(rng.standard_normal(shape), 0.0)
+        try:
+            with np.errstate(over="ignore", invalid="ignore"):
+                ok = _rel(gram_fn(x0), oracle.ns_rectangular(x0)) < 1e-12
+            if not ok:
+                return False
+        except ValueError:
+            return False
+    return True
+
+
+def _gram_variant(one_sided=False, p_not_accumulated=False, right_gram=False, p_right=False):
+    def fn(x0, coeffs=oracle.QUINTIC, steps=5):
+        a, b, c = coeffs
+        g = x0.T @ x0 if right_gram else x0 @ x0.T
+        eye = np.eye(g.shape[0])
+        p = eye.copy()
+        for _ in range(steps):
+            q = a * eye + b * g + c * (g @ g)
+            g = q @ g if one_sided else q @ g @ q
+            p = q if p_not_accumulated else (p @ q if p_right else q @ p)
+        return x0 @ p if right_gram else p @ x0
+    return fn
+
+
+def test_gram_pin_catches_planted_mistakes():
+    assert _gram_pin_passes(oracle.ns_gram)
+    assert not _gram_pin_passes(_gram_variant(one_sided=True)), "G <- Q G"
+    assert not _gram_pin_passes(_gram_variant(p_not_accumulated=True)), "P <- Q"
+    # Not mistakes: every Q_k is a polynomial in G_0, so P Q == Q P, and the
+    # right-side Gram X0^T X0 with O = X0 P gives the same iterate.
+    assert _gram_pin_passes(_gram_variant(p_right=True))
+    assert _gram_pin_passes(_gram_variant(right_gram=True))
