@@ -278,10 +278,11 @@ DMU_API dmu_status dmu_momentum_norm_static(const void* grad, float* momentum, v
  * 16-byte aligned.  Outputs must not alias inputs of another role (every
  * output element reads all agents' inputs): v_out vs v_in, x_out vs x_in
  * and o; v_out, v_bf16 and momenta are distinct arrays, and v_bf16 does
- * not alias grads (momenta are updated in place).  Sums over agents run in agent order, so results are
- * deterministic.  Errors: n_agents outside [1, DMU_DEMUON_MAX_AGENTS], a
- * null or misaligned pointer, aliasing, non-finite weights, theta outside
- * [0, 1] or a non-finite eta return DMU_ERR_INVALID_ARG before any launch.
+ * not alias grads (momenta are updated in place).  Sums over agents run
+ * in agent order, so results are deterministic.  Errors: n_agents outside
+ * [1, DMU_DEMUON_MAX_AGENTS], a null or misaligned pointer, aliasing,
+ * non-finite weights, theta outside [0, 1] or a non-finite eta return
+ * DMU_ERR_INVALID_ARG before any launch.
  * Both calls are stream-ordered and do not synchronise. */
 #define DMU_DEMUON_MAX_AGENTS 16
 
