@@ -26,7 +26,15 @@ def f(x, co):
 
 
 def main():
-    out = {"coeffs": [str(c) for c in COEFFS], "quintic": {}, "cubic": {}}
+    out = {
+        "source": ("scalar Newton-Schulz polynomial f(s) = a s + b s^3 + c s^5 iterated 5 times, "
+                   "exact in rationals; the iteration approximates msgn (DeMuon technical summary, "
+                   "Methodology 1, matrix orthogonalisation) and acts on each singular value alone"),
+        "generator": "tests/golden/make_quintic_exact.py",
+        "coeffs": [str(c) for c in COEFFS],
+        "quintic": {},
+        "cubic": {},
+    }
     for p in POINTS:
         x = Fraction(p)
         seq, y = [], x
