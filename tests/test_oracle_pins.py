@@ -10,7 +10,9 @@ Each pin is independent of the oracle's own arithmetic:
   the scalar polynomial;
 * exact rational special cases (row vector, diagonal matrix) against
   ``tests/golden/quintic_exact.json`` (written with Python fractions);
-* Gram form == rectangular form (DMuon page, section 2.2);
+* Gram form == rectangular form (DMuon page, section 2.2), and every
+  intermediate of the Gram trace (G_k, R_k, T_k, P_k) against products of
+  the rectangular iterates X_k, X_{k+1};
 * invariances: transpose, positive scale, orthogonal conjugation;
 * the singular-value band of five quintic steps;
 * closed-form values of the momentum and of the update scale.
@@ -360,3 +362,38 @@ def test_gram_pin_catches_planted_mistakes():
     # right-side Gram X0^T X0 with O = X0 P gives the same iterate.
     assert _gram_pin_passes(_gram_variant(p_right=True))
     assert _gram_pin_passes(_gram_variant(right_gram=True))
+
+
+# Every intermediate of the Gram trace (which the GPU stage checks compare
+# against) is fixed by the rectangular iterates X_k, themselves pinned to
+# the SVD: G_k = X_k X_k^T, T_k = Q_k G_k = X_{k+1} X_k^T,
+# R_k X_k = X_{k+1} - a X_k and P_{k+1} X_0 = X_{k+1}.
+def _trace_pinned(trace, x0, a=A):
+    xs = [oracle.ns_rectangular(x0, steps=k) for k in range(len(trace) + 1)]
+    for k, st in enumerate(trace):
+        checks = [
+            (st["G"], xs[k] @ xs[k].T),
+            (st["T"], xs[k + 1] @ xs[k].T),
+            (st["R"] @ xs[k], xs[k + 1] - a * xs[k]),
+            (st["P"] @ x0, xs[k + 1]),
+        ]
+        for got, want in checks:
+            if not _rel(got, want) < 1e-11:
+                return False
+    return True
+
+
+@pytest.mark.parametrize("shape", [(10, 23), (16, 16), (1, 9)])
+def test_gram_trace_matches_rectangular_iterates(shape):
+    rng = np.random.default_rng(sum(shape))
+    x0 = oracle.frobenius_normalize(rng.standard_normal(shape), 0.0)
+    trace = oracle.gram_trace(x0)
+    assert _trace_pinned(trace, x0)
+    # a T that drops its a G term, or a G advanced one-sidedly, is rejected
+    bad_t = [dict(st, T=st["R"] @ st["G"]) for st in trace]
+    assert not _trace_pinned(bad_t, x0)
+    bad_g = [dict(st) for st in trace]
+    for k in range(1, len(bad_g)):
+        q = A * np.eye(shape[0]) + bad_g[k - 1]["R"]
+        bad_g[k]["G"] = q @ trace[k - 1]["G"]
+    assert not _trace_pinned(bad_g, x0)
