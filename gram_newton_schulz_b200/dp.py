@@ -107,7 +107,7 @@ class PlanCompute:
         self.launches = 0      # kernel launches of the last call
         self.tc_launches = 0   # of which tensor-core (Gram recursion + final update)
 
-    def __call__(self, grads, momenta, weights, *, beta, lr, eps, coeffs, steps):
+    def __call__(self, grads, momenta, weights, *, beta, lr, eps, coeffs, steps, out_o=None):
         self.launches = self.tc_launches = 0
         if self.plan is None:
             return
@@ -115,7 +115,7 @@ class PlanCompute:
         n0 = self.plan.last_launch_count()
         self.plan.gram_ns_batched(None, coeffs, steps)
         n1 = self.plan.last_launch_count()
-        self.plan.apply_update(weights, lr)
+        self.plan.apply_update(weights, lr, out_o=out_o)
         n2 = self.plan.last_launch_count()
         self.launches, self.tc_launches = n0 + n1 + n2, n1 + n2
 
@@ -157,14 +157,15 @@ class OwnerShardedStep:
         return [self.buckets.shapes[i] for i in self.mine]
 
     def step(self, grad_flats: list, weight_flats: list, momenta: list, *, beta=0.95, lr=0.02,
-             eps=1e-7, coeffs=(3.4445, -4.7750, 2.0315), steps=5, events=None):
+             eps=1e-7, coeffs=(3.4445, -4.7750, 2.0315), steps=5, events=None, out_o=None):
         """grad_flats / weight_flats: the per-owner flat buffers of
         `OwnerBuckets.alloc`, on every rank; momenta: fp32 tensors of the owned
         matrices, in `self.mine` order.  On return every rank's weight buffers
         hold the updated weights (the broadcasts are waited on, which on GPUs
         orders the current stream after them).  ``events``: four CUDA events
         recorded on the current stream at the start, after the exchange in,
-        after the compute and after the exchange out."""
+        after the compute and after the exchange out.  ``out_o``: optional
+        fp32 tensors (owned matrices, `self.mine` order) that receive O."""
         import torch.distributed as dist
         if len(momenta) != len(self.mine):
             raise ValueError(f"expected {len(self.mine)} momenta, got {len(momenta)}")
@@ -180,7 +181,8 @@ class OwnerShardedStep:
             events[1].record()
         grads = [b.view(grad_flats, i) for i in self.mine]
         weights = [b.view(weight_flats, i) for i in self.mine]
-        self.compute(grads, momenta, weights, beta=beta, lr=lr, eps=eps, coeffs=coeffs, steps=steps)
+        kw = {} if out_o is None else {"out_o": out_o}
+        self.compute(grads, momenta, weights, beta=beta, lr=lr, eps=eps, coeffs=coeffs, steps=steps, **kw)
         if events is not None:
             events[2].record()
         if self.world > 1:

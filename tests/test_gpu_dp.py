@@ -1,11 +1,17 @@
 """The owner-sharded step's device path on one GPU (world size 1, so there
 are no collectives): the compute must run on views of the per-owner flat
-buffers, and must agree bit for bit with the same update through
-`dmu.Plan.step` on separate tensors."""
+buffers; its O must match the fp64 oracle's Muon step (2e-2 relative
+Frobenius error) and its W write must be within one bf16 ulp of
+bf16(W - lr * scale * O); and it must agree bit for bit with the same
+update through `dmu.Plan.step` on separate tensors.  (DMuon page, section
+2.1: the owner runs the whole update of the matrices it owns.)"""
+import numpy as np
 import pytest
 import torch
 
+import oracle
 from gram_newton_schulz_b200 import dmu, dp, synth
+from gpu_util import check_update_within_ulp, f64, rel
 
 pytestmark = pytest.mark.gpu
 
@@ -39,6 +45,40 @@ def test_owner_step_on_flat_buffers_matches_plan_step():
     assert osd.compute.plan.read_status() == 0
     osd.close()
     plan.close()
+
+
+def test_owner_step_matches_oracle():
+    """Two owner-sharded steps on flat buffers; after the second, O of every
+    matrix against the oracle on the accumulated momentum, W against O."""
+    shapes = [(512, 2048), (2048, 512), (384, 384), (1024, 4096), (4096, 1024), (300, 700)]
+    w = synth.custom("dp-oracle", shapes, seed=12)
+    dev = torch.device("cuda", 0)
+    grads = synth.gradients(w, dev)
+    weights = synth.weights(w, dev)
+    osd = dp.OwnerShardedStep(shapes, device=dev)
+    b = osd.buckets
+    gflat, wflat = b.alloc(torch.bfloat16, dev), b.alloc(torch.bfloat16, dev)
+    for i in range(len(shapes)):
+        b.view(gflat, i).copy_(grads[i])
+        b.view(wflat, i).copy_(weights[i])
+    moms = [torch.zeros(s, dtype=torch.float32, device=dev) for s in shapes]
+    outs = [torch.empty(s, dtype=torch.float32, device=dev) for s in shapes]
+    osd.step(gflat, wflat, moms, beta=0.95, lr=0.02)
+    w_mid = [b.view(wflat, i).clone() for i in range(len(shapes))]
+    osd.step(gflat, wflat, moms, beta=0.95, lr=0.02, out_o=outs)
+    torch.cuda.synchronize()
+    assert osd.compute.plan.read_status() == 0
+    for i, (r, c) in enumerate(shapes):
+        g = f64(grads[i])
+        m_ref = oracle.momentum(oracle.momentum(np.zeros_like(g), g, 0.95), g, 0.95)
+        np.testing.assert_allclose(f64(moms[i]), m_ref, rtol=2.0 ** -22, atol=0)
+        # the oracle's Muon step on the momentum the device holds
+        _, o_ref, _ = oracle.muon_step(f64(w_mid[i]), 0.95 * g, g, beta=1.0, lr=0.02)
+        e = rel(f64(outs[i]), o_ref)
+        assert e < 2e-2, (r, c, e)
+        u = check_update_within_ulp(w_mid[i], b.view(wflat, i), outs[i], r, c, 0.02)
+        assert u <= 1.0, (r, c, u)
+    osd.close()
 
 
 def test_measured_costs_order_shapes_by_work():
