@@ -13,9 +13,11 @@
 //
 // Every GPU that loads the library holds the 64 KB array until the process
 // exits.  In host code the array's name is only a host-side stand-in, so its
-// device address is looked up with cudaGetSymbolAddress once per device, on
-// the first call made with that device current.
-#include <mutex>
+// device address is looked up with cudaGetSymbolAddress on every call, with
+// the caller's device current: the lookup allocates nothing, and a fresh
+// lookup stays right when the device's context was reset and the module
+// loaded again at another address.  The first call on a device may load the
+// module, so it belongs before any stream capture.
 
 #include "dmu_internal.h"
 
@@ -28,14 +30,10 @@ namespace {
 constexpr int SCR_CHUNK = 16384;        // elements per partial sum
 constexpr int SCR_MAX_CHUNKS = 16384;   // partial sums held by the static scratch
 constexpr long long SCR_MAX_ELEMS = (long long)SCR_CHUNK * SCR_MAX_CHUNKS;  // 2^28 elements
-constexpr int SCR_MAX_DEVICES = 64;
 
 // The scratch: written chunk by chunk before it is read in the same call, so
 // it never needs clearing; calls that overlap on the GPU race on it.
 static __device__ __align__(256) float g_scratch_partial[SCR_MAX_CHUNKS];
-
-float* g_scratch_dev[SCR_MAX_DEVICES] = {};
-std::mutex g_scratch_mu;
 
 __device__ __forceinline__ void grad8(const void* g, int f32, long long idx, float* v) {
   if (f32) {
@@ -136,17 +134,13 @@ __global__ void k_norm_static(const float* __restrict__ partial, int nchunks, fl
   if (lane == 0) inv_out[0] = (float)(1.0 / (sqrt(s) + (double)eps));
 }
 
-// Device address of the static scratch on the current device (looked up
-// once per device; cudaGetSymbolAddress allocates nothing).
-cudaError_t scratch_address(int dev, float** out) {
-  std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (!g_scratch_dev[dev]) {
-    void* p = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&p, g_scratch_partial);
-    if (e != cudaSuccess) return e;
-    g_scratch_dev[dev] = reinterpret_cast<float*>(p);
-  }
-  *out = g_scratch_dev[dev];
+// Device address of the static scratch in the current device's context
+// (cudaGetSymbolAddress allocates nothing).
+cudaError_t scratch_address(float** out) {
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_scratch_partial);
+  if (e != cudaSuccess) return e;
+  *out = reinterpret_cast<float*>(p);
   return cudaSuccess;
 }
 
@@ -177,11 +171,11 @@ extern "C" DMU_API dmu_status dmu_momentum_norm_static(const void* grad, float* 
     dmu::set_last_error("matrix too large for the static scratch: at most 268435456 (2^28) elements");
     return DMU_ERR_UNSUPPORTED;
   }
-  int dev = 0;
+  int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
-  if (e == cudaSuccess && (dev < 0 || dev >= SCR_MAX_DEVICES)) e = cudaErrorInvalidDevice;
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   float* scratch = nullptr;
-  if (e == cudaSuccess) e = scratch_address(dev, &scratch);
+  if (e == cudaSuccess) e = scratch_address(&scratch);
   if (e != cudaSuccess) {
     dmu::set_last_error(cudaGetErrorString(e));
     return DMU_ERR_CUDA;
@@ -190,8 +184,6 @@ extern "C" DMU_API dmu_status dmu_momentum_norm_static(const void* grad, float* 
   const int vec = (n % 8 == 0) && !(reinterpret_cast<uintptr_t>(grad) & 15) &&
                   !(reinterpret_cast<uintptr_t>(momentum) & 15) && !(reinterpret_cast<uintptr_t>(image_out) & 15);
   const int nchunks = (int)((n + SCR_CHUNK - 1) / SCR_CHUNK);
-  int sms = 148;
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   int grid = sms * 8;
   if (grid > nchunks) grid = nchunks;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

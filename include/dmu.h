@@ -98,8 +98,11 @@ typedef enum {
  * turns the antisymmetric part of the operand rounding error into a
  * symmetric one; with one bf16 MMA per product that error shifts the small
  * eigenvalues of G enough to miss 2e-2 on spiked inputs, so:
- *   FAST   : one bf16 MMA per product (hi x hi)        -- low precision;
- *   SPLIT2 : two MMAs per product (hi x hi + lo x hi)  -- low precision;
+ *   FAST   : one bf16 MMA per product (hi x hi)        -- low precision:
+ *            misses the 2e-2 bound on spiked inputs (measured 0.07-0.17
+ *            relative error on rank-8 spiked 128x512 .. 512x2048);
+ *   SPLIT2 : two MMAs per product (hi x hi + lo x hi)  -- low precision:
+ *            misses 2e-2 on the same inputs (0.06-0.14);
  *   SPLIT3 : three MMAs per product (hi x hi + hi x lo + lo x hi);
  *   TF32   : Gram-space state in fp32, one kind::tf32 MMA per product
  *            (half the bf16 rate; 10-bit operand mantissa);
@@ -241,9 +244,10 @@ DMU_API void dmu_plan_destroy(dmu_plan plan);
  *                  dtype (bf16 image for DMU_BF16); may be NULL;
  *   inv_norm_out : device, one float, receives 1/(||M||_F + eps).
  * Limit: rows*cols <= 2^28 (268435456); larger returns DMU_ERR_UNSUPPORTED
- * before any launch.  The first call on a device (with that device
- * current) looks up the array's device address; make that first call
- * before any stream capture.  Every call on a device shares the array:
+ * before any launch.  Every call looks up the array's device address in
+ * the current device's context (the lookup allocates nothing); the first
+ * call on a device may load the library's device code, so make that first
+ * call before any stream capture.  Every call on a device shares the array:
  * calls that overlap on the GPU race and must be ordered by the caller.
  * The array needs no clearing (each call writes every slot it reads).
  * Allocates nothing (no cudaMalloc, cudaFree or allocating library call). */

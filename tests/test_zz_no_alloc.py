@@ -23,11 +23,14 @@ pytestmark = pytest.mark.gpu
 BETA, EPS = 0.95, 1e-7
 
 
-def _static_call(lib, g, mom, img, inv, dtype_code):
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _static_call(lib, g, mom, img, inv, dtype_code, beta=BETA):
     r, c = g.shape
     return lib.dmu_momentum_norm_static(
-        ctypes.c_void_p(g.data_ptr()), ctypes.c_void_p(mom.data_ptr()) if mom is not None else None,
-        ctypes.c_void_p(img.data_ptr()), r, c, dtype_code, BETA, EPS, ctypes.c_void_p(inv.data_ptr()),
+        _ptr(g), _ptr(mom), _ptr(img), r, c, dtype_code, beta, EPS, _ptr(inv),
         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
@@ -58,6 +61,54 @@ def test_static_scratch_matches_plan_path_two_calls(dtype):
         assert float(inv_b[0]) == pytest.approx(float(inv_a[0]), rel=1e-6)
         x = mom_b.double().cpu().numpy()
         assert float(inv_b[0]) == pytest.approx(1.0 / (np.linalg.norm(x) + EPS), rel=2e-6)
+
+
+@pytest.mark.parametrize("drop", ["momentum", "image"])
+def test_static_scratch_optional_outputs(drop):
+    """momentum = NULL: M = G and no state is written; image_out = NULL: only
+    the norm is produced.  Compared with the plan path at beta = 0 (M = G)."""
+    lib = dmu.load()
+    shape = (1024, 768)
+    w = synth.custom("noalloc-opt", [shape], seed=97)
+    g = synth.gradients(w, "cuda")[0]
+    plan = dmu.Plan([shape])
+    plan.momentum_normalize([g], None, beta=0.0, eps=EPS)
+    inv_a = plan.debug(6)
+    img_a = plan.debug(5, 0)
+    for _ in range(2):
+        if drop == "momentum":
+            img_b = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+            st = _static_call(lib, g, None, img_b, inv_b := torch.full((1,), -1.0, device="cuda"), 0)
+        else:
+            mom = torch.zeros(shape, device="cuda")
+            img_b = None
+            st = _static_call(lib, g, mom, None, inv_b := torch.full((1,), -1.0, device="cuda"), 0)
+        assert st == dmu.OK, lib.dmu_last_error()
+        torch.cuda.synchronize()
+        if img_b is not None:
+            assert torch.equal(img_a, img_b.float())
+        else:
+            assert torch.equal(mom, g.float())  # beta * 0 + G
+        assert float(inv_b[0]) == pytest.approx(float(inv_a[0]), rel=1e-6)
+
+
+def test_static_call_allocates_no_device_memory():
+    """Free device memory is the same before and after a warmed-up call."""
+    lib = dmu.load()
+    shape = (2048, 2048)
+    w = synth.custom("noalloc-mem", [shape], seed=98)
+    g = synth.gradients(w, "cuda")[0]
+    mom = torch.zeros(shape, device="cuda")
+    img = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+    inv = torch.empty(1, device="cuda")
+    assert _static_call(lib, g, mom, img, inv, 0) == dmu.OK
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        assert _static_call(lib, g, mom, img, inv, 0) == dmu.OK
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
 
 
 def test_static_scratch_rejects_oversize_and_bad_args():
