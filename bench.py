@@ -38,6 +38,8 @@ METRIC = "Gram-NS optimizer-step ms on 7B-shape layer set; TFLOP/s vs B200 bf16 
 DEFAULT_WORKLOAD = "qwen2.5-7b-layer-set-x28"
 K_STEPS = 5
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# NVIDIA's dense (no 2:4 sparsity) bf16 tensor-core rate of one B200, TFLOP/s
+DATASHEET_DENSE_BF16_TFLOPS = 2250.0
 
 
 def alg_flops(shapes, k=K_STEPS):
@@ -92,9 +94,8 @@ def gemm_alg_bytes(shapes, k=K_STEPS):
 
 
 # DRAM traffic of the tensor-core kernel measured by ncu (one pass:
-# gpu__time_duration.sum, dram__bytes_read.sum, dram__bytes_write.sum; see
-# profiles/k_gemm_tc2_qwen7b_x28_launch_list.md) for the kernel sources
-# whose sha256 is recorded here.  The figure is reported only while
+# gpu__time_duration.sum, dram__bytes_read.sum, dram__bytes_write.sum) for
+# the kernel sources whose sha256 is recorded here.  The figure is reported only while
 # gemm_tc.cu + plan.cu still hash to it: a changed kernel reports null.
 TRAFFIC_CAPTURE = {
     "sources": ["gram_newton_schulz_b200/csrc/gemm_tc.cu", "gram_newton_schulz_b200/csrc/plan.cu"],
@@ -191,9 +192,17 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def oracle_sample_seconds(shapes, budget_s=20.0):
+def oracle_sample_seconds(shapes, budget_s=30.0, per_bucket=2):
     """Time the fp64 oracle (as it stands) on a bounded sample and scale to
-    the full workload by each bucket's fp64 flop count."""
+    the full workload.
+
+    Matrices are drawn round-robin over the shape buckets, cheapest bucket
+    first, up to ``per_bucket`` per bucket, while the predicted cost stays
+    within ``budget_s``.  A bucket with timed matrices is scaled by its own
+    mean time per matrix; a bucket with none by the fp64 flop rate the timed
+    matrices reached.  Returns (seconds for the whole workload, threads,
+    sample description, seconds spent, whether any bucket was extrapolated
+    by flop count)."""
     import numpy as np
     import torch
     from threadpoolctl import threadpool_info
@@ -207,32 +216,35 @@ def oracle_sample_seconds(shapes, budget_s=20.0):
     buckets = {}
     for s in shapes:
         buckets[s] = buckets.get(s, 0) + 1
-    # sample: one matrix of each bucket whose fp64 cost fits the budget,
-    # smallest first; the other buckets are scaled by flop count
     order = sorted(buckets, key=lambda s: rect_flops(*s))
-    w = synth.custom("sample", order, seed=99)
-    timed, spent = {}, 0.0
-    for i, s in enumerate(order):
-        est = rect_flops(*s) / 2e11  # a conservative fp64 rate guess
+    picks = [s for rnd in range(per_bucket) for s in order if buckets[s] > rnd]
+    w = synth.custom("sample", picks, seed=99)
+    timed, spent, rate_guess = {}, 0.0, 2e11  # fp64 flop/s guess before the first timing
+    for i, s in enumerate(picks):
+        est = rect_flops(*s) / rate_guess
         if timed and spent + est > budget_s:
-            break
+            continue
         g = synth.gradient(w, i).to(torch.float64).numpy()
         wt = synth.weight(w, i).to(torch.float64).numpy()
         t0 = time.perf_counter()
         oracle.muon_step(wt, np.zeros_like(g), g, beta=0.95, lr=0.02)
         dt = time.perf_counter() - t0
-        timed[s] = dt
+        timed.setdefault(s, []).append(dt)
         spent += dt
-    rate = sum(rect_flops(*s) for s in timed) / sum(timed.values())
+        rate_guess = sum(rect_flops(*k) * len(v) for k, v in timed.items()) / spent
+    rate = rate_guess
     total = 0.0
     for s, n in buckets.items():
-        total += n * (timed[s] if s in timed else rect_flops(*s) / rate)
+        total += n * (sum(timed[s]) / len(timed[s]) if s in timed else rect_flops(*s) / rate)
+    flop_scaled = any(s not in timed for s in buckets)
+    extrapolated = sum(len(v) for v in timed.values()) < len(shapes)
     threads = max((d.get("num_threads", 1) for d in threadpool_info()), default=os.cpu_count())
-    sample = ("fp64 oracle muon_step timed on one matrix each of " +
-              ", ".join(f"{r}x{c}" for r, c in timed) +
-              ("; other buckets scaled by fp64 flop count" if len(timed) < len(buckets) else "") +
-              f"; scaled to {len(shapes)} matrices")
-    return total, threads, sample, spent
+    sample = ("fp64 oracle muon_step timed on " +
+              ", ".join(f"{len(v)} x {r}x{c}" for (r, c), v in timed.items()) +
+              (f"; buckets {', '.join(f'{r}x{c}' for (r, c) in buckets if (r, c) not in timed)} "
+               f"scaled by the timed fp64 flop rate" if flop_scaled else "") +
+              f"; each bucket scaled to its count, {len(shapes)} matrices in all")
+    return total, threads, sample, spent, extrapolated
 
 
 def custom_workload(spec: str):
@@ -252,7 +264,7 @@ def run_reference(args):
     w = custom_workload(args.shapes) if args.shapes else synth.workload(args.workload)
     vals = []
     for k in range(args.warmup + args.steps):
-        total, threads, sample, _ = oracle_sample_seconds(w.shapes, budget_s=args.ref_budget)
+        total, threads, sample, _, extrap = oracle_sample_seconds(w.shapes, budget_s=args.ref_budget)
         if k >= args.warmup:
             vals.append(total * 1e3)
     # The job of an N-GPU run is N layer sets (one per rank, weak scaling);
@@ -265,10 +277,12 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "ms", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(v, 3), "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "extrapolated": extrap,
         "config": {"workload": w.name, "matrices": w.count, "matrices_total": w.count * world, "K": K_STEPS,
                    "coeffs": [3.4445, -4.7750, 2.0315], "precision": "f64 oracle",
                    "parallelism": f"replica x{world}, all on the host cores"},
-        "cpu_baseline": {"value": round(v, 3), "unit": "ms", "cores": threads, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": round(v, 3), "unit": "ms", "cores": threads, "kind": "oracle", "sample": sample,
+                         "extrapolated": extrap},
         "e2e": {"value": round(v, 3), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -293,6 +307,46 @@ def pin_copies(tensors):
         return [t.to("cpu").pin_memory() for t in tensors], None
     except RuntimeError as e:  # host out of pinnable memory
         return None, f"{type(e).__name__}: {str(e)[:100]}"
+
+
+def host_link_rates(h_in, d_in, h_out, d_out, s_in, s_out, dev):
+    """Copy rates of the e2e leg's own buffers with no compute: pinned host
+    to device alone, device to host alone, and both at once on their two
+    streams (GB/s, bytes over CUDA-event time).  They bound what the e2e
+    step can reach when its copies overlap the compute."""
+    import torch
+
+    def timed(fn):
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        cur = torch.cuda.current_stream(dev)
+        a.record(cur)
+        fn()
+        for st in (s_in, s_out):
+            cur.wait_stream(st)
+        b.record(cur)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / 1e3
+
+    def h2d():
+        s_in.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(s_in):
+            for h, d in zip(h_in, d_in):
+                d.copy_(h, non_blocking=True)
+
+    def d2h():
+        s_out.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(s_out):
+            for h, d in zip(h_out, d_out):
+                h.copy_(d, non_blocking=True)
+
+    bi = sum(t.numel() * t.element_size() for t in h_in)
+    bo = sum(t.numel() * t.element_size() for t in h_out)
+    t_in, t_out = timed(h2d), timed(d2h)
+    t_both = timed(lambda: (h2d(), d2h()))
+    return {"h2d_gbs": round(bi / t_in / 1e9, 1), "d2h_gbs": round(bo / t_out / 1e9, 1),
+            "concurrent_gbs": round((bi + bo) / t_both / 1e9, 1),
+            "bound_ms": round(t_both * 1e3, 3)}
 
 
 def run_owner(args, w_full, dev, world, rank, local, barrier):
@@ -726,13 +780,14 @@ def main():
         barrier()
         e2e_ms = owners.max_over_ranks(e0.elapsed_time(e1) / E, device=dev)
         e2e = {"value": round(e2e_ms, 3), "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "overlap": "H2D of step k+1 and D2H of step k overlap compute (separate copy streams)"}
+               "overlap": "H2D of step k+1 and D2H of step k overlap compute (separate copy streams)",
+               "host_link": host_link_rates(h_grads, grads, h_w, weights, s_in, s_out, dev)}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        total_s, threads, sample, _ = oracle_sample_seconds(w.shapes)
+        total_s, threads, sample, spent, extrap = oracle_sample_seconds(w.shapes)
         cpu = {"value": round(total_s * 1e3, 1), "unit": "ms", "cores": threads, "kind": "oracle",
-               "sample": sample}
+               "sample": sample, "extrapolated": extrap, "seconds_timed": round(spent, 1)}
 
     if rank == 0:
         line = {
@@ -750,7 +805,12 @@ def main():
             "throughput": {"executed_tflops": round(executed_flops(job_shapes) / (step_ms / 1e3) / 1e12, 1),
                            "matrices_per_s": round(len(job_shapes) / (step_ms / 1e3), 1),
                            "alg_tflops": round(job_flops / (step_ms / 1e3) / 1e12, 1),
-                           "alg_tflops_frac_per_gpu": round(job_flops / world / (step_ms / 1e3) / 1e12 / peak_tf, 4)},
+                           "alg_tflops_frac_per_gpu": round(job_flops / world / (step_ms / 1e3) / 1e12 / peak_tf, 4),
+                           "alg_tflops_frac_per_gpu_of": f"{peak_kind} cuBLAS bf16 GEMM, sustained (achievable)",
+                           "alg_tflops_frac_of_datasheet_dense_bf16":
+                               round(job_flops / world / (step_ms / 1e3) / 1e12 / DATASHEET_DENSE_BF16_TFLOPS, 4),
+                           "step_ms_x_median_sm_ghz": (round(step_ms * clk["sm_mhz"] / 1e3, 2)
+                                                       if clk and clk.get("sm_mhz") else None)},
             "split_ms": {"momentum": round(t_mom / K, 3), "gram": round(t_gram / K, 3),
                          "update": round(t_upd / K, 3)},
             "eager_ms_per_step": round(eager_max, 3),
@@ -759,7 +819,8 @@ def main():
                          "traffic": traffic,
                          "alg_bytes_per_launch": round(gemm_alg_bytes(w.shapes) / max(tc_launches, 1)),
                          "kernel": "k_gemm_tc2 (all Gram-space and final launches)",
-                         "peak_kind": f"{peak_kind} bf16 sustained"},
+                         "peak_kind": f"{peak_kind} cuBLAS bf16 GEMM, sustained (achievable)",
+                         "frac_of_datasheet_dense_bf16": round(achieved_tf / DATASHEET_DENSE_BF16_TFLOPS, 4)},
             "hbm_kernel": {"kernel": "k_momentum", "achieved": round(mom_gbs, 1), "peak": hbm,
                            "unit": "GB/s", "frac": round(mom_gbs / hbm, 4), "peak_kind": peak_kind},
             "gpu_launches": launches,

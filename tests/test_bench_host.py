@@ -35,10 +35,14 @@ def test_custom_workload_parser():
 
 def test_oracle_sample_is_bounded_and_scaled():
     shapes = [(64, 256)] * 3 + [(128, 512)] * 2
-    total, threads, sample, spent = bench.oracle_sample_seconds(shapes, budget_s=5.0)
+    total, threads, sample, spent, extrapolated = bench.oracle_sample_seconds(shapes, budget_s=5.0)
     assert total > 0 and threads >= 1
-    assert "64x256" in sample and "scaled to 5 matrices" in sample
+    # two matrices of each bucket are timed, then each bucket scaled to its count
+    assert "2 x 64x256" in sample and "2 x 128x512" in sample and "5 matrices" in sample
+    assert extrapolated  # 4 of the 5 matrices were timed
     assert spent < 30
+    total1, _, _, _, extrap1 = bench.oracle_sample_seconds([(64, 256)] * 2, budget_s=5.0)
+    assert not extrap1 and total1 > 0
 
 
 def test_reference_arm_prints_one_json_line():
