@@ -131,6 +131,13 @@ def momentum_bytes(shapes, grad_bytes=2):
     return e * (grad_bytes + 4 + 4 + 2)
 
 
+def schedule_summary(sch):
+    """Plan.schedules() as JSON-friendly text: one entry per Gram class (by
+    m) and per final-GEMM bucket (by rows x cols)."""
+    return {"gram": {f"m{m}": v for m, v in sorted(sch["gram"].items())},
+            "final": {f"{r}x{c}": v for (r, c), v in sorted(sch["final"].items())}}
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -482,7 +489,8 @@ def run_demuon(args, w_full, dev, local):
             dm.grad(a, k).copy_(synth.gradients(w_full, dev, indices=[k])[0])
             dm.iterate(a, k).copy_(synth.weights(w_full, dev, indices=[k])[0].float())
     dm.plan.momentum_normalize(dm._vb_views, None, beta=0.0)
-    schedule = "cta_pair" if args.no_autotune else dmu.SCHEDULES[dm.plan.autotune()]
+    schedule = dm.plan.schedules() if args.no_autotune else dm.plan.autotune()
+    schedule = schedule_summary(schedule)
     for _ in range(args.warmup):
         dm.step()
     torch.cuda.synchronize(dev)
@@ -555,7 +563,9 @@ def main():
     ap.add_argument("--topology", default="ring", choices=["ring", "exponential", "complete"])
     ap.add_argument("--no-graph", action="store_true", help="time eager launches only (no CUDA graph replay)")
     ap.add_argument("--no-autotune", action="store_true",
-                    help="keep the default CTA-pair schedule instead of timing both")
+                    help="keep the plan's default schedules instead of timing the candidates")
+    ap.add_argument("--schedule-cache", default=None,
+                    help="schedule cache file for dmu_autotune (read and appended)")
     ap.add_argument("--ref-budget", type=float, default=10.0)
     args = ap.parse_args()
 
@@ -614,14 +624,15 @@ def main():
         n2 = plan.last_launch_count()
         return n0 + n1 + n2
 
-    # Schedule cache: time the recursion with CTA pairs and with single CTAs
-    # on this plan's own data and keep the faster (both give bitwise-equal
-    # results).  It needs the momentum image, so one momentum pass first.
+    # Schedule cache: every Gram class and every bucket's final GEMM is timed
+    # on this plan's own data with each candidate schedule and keeps the
+    # fastest (all candidates give bitwise-equal results).  It needs the
+    # momentum image, so one momentum pass first.
     plan.momentum_normalize(grads, moms, beta=w.beta, eps=1e-7)
     if w.dtype != "bf16":
         schedule = "simt_fp32"  # fp32 plans run the FFMA path; nothing to tune
     else:
-        schedule = "cta_pair" if args.no_autotune else dmu.SCHEDULES[plan.autotune()]
+        schedule = schedule_summary(plan.schedules() if args.no_autotune else plan.autotune(args.schedule_cache))
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
@@ -702,7 +713,9 @@ def main():
     total_ms *= K
     # per-rank launches are those of the captured run only for the whole
     # layer set at the default precision
-    traffic = captured_traffic(w_full.name) if args.prec == "auto" and schedule == "cta_pair" else None
+    all_pairs = all(v == "cta_pair" for part in schedule.values() for v in part.values()) \
+        if isinstance(schedule, dict) else False
+    traffic = captured_traffic(w_full.name) if args.prec == "auto" and all_pairs else None
     step_ms = owners.max_over_ranks(total_ms / K, device=dev)
     eager_max = owners.max_over_ranks(eager_ms, device=dev)
     status = plan.read_status()

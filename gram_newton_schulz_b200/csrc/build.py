@@ -18,7 +18,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 PKG = os.path.dirname(HERE)
 ROOT = os.path.dirname(PKG)
-SOURCES = ["gemm_tc.cu", "kernels_misc.cu", "plan.cu", "noalloc.cu", "demuon.cu"]
+SOURCES = ["gemm_tc.cu", "gram_onchip.cu", "kernels_misc.cu", "plan.cu", "noalloc.cu", "demuon.cu"]
 OUT_DIR = os.path.join(PKG, "_lib")
 OUT = os.path.join(OUT_DIR, "libdmu.so")
 BUILD = os.path.join(ROOT, "_build")

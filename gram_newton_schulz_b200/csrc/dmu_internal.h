@@ -151,9 +151,11 @@ cudaError_t gemm_tc_configure();
 cudaError_t launch_wait_selftest(unsigned int* status, long long timeout_ns, cudaStream_t s);
 int gemm_tc_stages(int na, int nb);
 
+// Per-chunk partial sums: MOM_PARTIALS_PER_CHUNK floats per momentum chunk.
+constexpr int MOM_PARTIALS_PER_CHUNK = 8;
 cudaError_t launch_momentum(const MomChunk* chunks, int nchunks, const MomMat* mats,
                             const void* const* grads, float* const* momenta, int grad_f32,
-                            void* mb, int mb_f32, float beta, float* partial,
+                            void* mb, int mb_f32, float beta, float gscale, float* partial,
                             int vec_ok, int num_sms, cudaStream_t s);
 cudaError_t launch_norm_finalize(const MomMat* mats, int nmats, const float* partial,
                                  float eps, float* inv, unsigned int* status, cudaStream_t s);
@@ -172,4 +174,39 @@ cudaError_t launch_f32_copy2d(const float* src, long long rows, long long cols, 
                               float* out, cudaStream_t s);
 constexpr int HALF_BLOCK = 256;  // block size of half-stored symmetric matrices
 
+}  // namespace dmu
+
+namespace dmu {
+// ---------------------------------------------------------------- on-chip recursion (m <= 128)
+// One shape bucket whose whole Gram recursion runs in one CTA per matrix
+// (SYRK from the momentum image, K steps of the R-form recursion with
+// G/T, R and P held in shared memory as bf16 hi/lo pairs); only the final
+// P is written, as a bf16 hi/lo pair into the class's P slot.
+constexpr int ONCHIP_MAX_M = 128;
+struct OnchipProblem {
+  int count;            // matrices of the bucket
+  int m, n;             // m = min(rows, cols) <= 128, n = max
+  int tall;             // the iterated X is Mb^T (MN-major image reads)
+  int map;              // image tensor map (K-major box 64 x 128, or MN-major 64 x 64)
+  int inv_base;         // index of the bucket's first matrix in `inv`
+  int mat_begin;        // first global matrix index of this problem
+  __nv_bfloat16* p_hi;  // final P of the bucket's first matrix (hi part)
+  __nv_bfloat16* p_lo;
+  long long ld, mat_stride;
+};
+
+struct __align__(64) OnchipParams {
+  CUtensorMap maps[MAX_MAPS];
+  OnchipProblem prob[MAX_PROBS];
+  int nprob;
+  int total;            // matrices over all problems
+  const float* inv;
+  float a, b, c;        // recursion coefficients
+  int steps;            // K >= 1
+  unsigned int* status;
+  long long timeout_ns;
+};
+
+cudaError_t onchip_configure();
+cudaError_t launch_gram_onchip(const OnchipParams& p, int num_sms, cudaStream_t s);
 }  // namespace dmu

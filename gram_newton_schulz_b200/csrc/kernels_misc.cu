@@ -47,67 +47,111 @@ __device__ __forceinline__ void store8_image(void* __restrict__ mb, int mb_f32, 
   }
 }
 
-// Vector path: each thread takes two 8-element vectors per iteration and
-// issues every load (G, M) before any store, so two vectors' loads are in
-// flight per thread; G, M and the image are distinct buffers (restrict).
-__global__ void __launch_bounds__(256, 6) k_momentum(const MomChunk* __restrict__ chunks, int nchunks,
+// M <- beta M + gscale G over one 16384-element chunk per CTA iteration.
+// Each warp owns a fixed 2048-element slice of the chunk and writes its own
+// partial sum of M^2 (partial[chunk * 8 + warp]), so no block-wide barrier
+// stalls the stream at chunk ends, and the partials -- hence the norm --
+// do not depend on the grid size.  Vector path: every thread issues the
+// loads of four 8-element vectors (G, M) before any arithmetic or store.
+// G, M and the image are distinct buffers (restrict).
+constexpr int MOM_WARPS = 8;
+constexpr int MOM_SLICE = MOM_CHUNK / MOM_WARPS;  // 2048 elements per warp
+constexpr int MOM_VEC = 4;                        // vectors in flight per thread
+static_assert(MOM_WARPS == MOM_PARTIALS_PER_CHUNK, "partial sums per chunk");
+
+// Raw 8-element gradient vector: one 16-byte load (bf16) or two (fp32);
+// converted to fp32 only when it is used, so the loads in flight hold 4
+// (bf16) registers per vector.
+template <bool F32> struct GradVec;
+template <> struct GradVec<false> {
+  uint4 u;
+  __device__ __forceinline__ void load(const void* g, long long idx) {
+    u = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(g) + idx));
+  }
+  __device__ __forceinline__ void get(float* out) const {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 t = __bfloat1622float2(h[q]);
+      out[2 * q] = t.x;
+      out[2 * q + 1] = t.y;
+    }
+  }
+};
+template <> struct GradVec<true> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const void* g, long long idx) {
+    const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(g) + idx);
+    a = __ldg(p);
+    b = __ldg(p + 1);
+  }
+  __device__ __forceinline__ void get(float* out) const {
+    out[0] = a.x; out[1] = a.y; out[2] = a.z; out[3] = a.w;
+    out[4] = b.x; out[5] = b.y; out[6] = b.z; out[7] = b.w;
+  }
+};
+
+template <bool F32>
+__global__ void __launch_bounds__(256, 3) k_momentum(const MomChunk* __restrict__ chunks, int nchunks,
                                                   const MomMat* __restrict__ mats,
                                                   const void* const* __restrict__ grads,
-                                                  float* const* __restrict__ momenta, int grad_f32,
-                                                  void* __restrict__ mb, int mb_f32, float beta,
+                                                  float* const* __restrict__ momenta,
+                                                  void* __restrict__ mb, float beta, float gscale,
                                                   float* __restrict__ partial, int vec) {
-  __shared__ float red[8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int c = blockIdx.x; c < nchunks; c += gridDim.x) {
     const MomChunk ch = chunks[c];
-    const MomMat mm = mats[ch.slot];
+    const long long mb_off = mats[ch.slot].mb_off;
     const void* __restrict__ g = grads[ch.slot];
     float* __restrict__ mom = momenta ? momenta[ch.slot] : nullptr;
+    const int s0 = warp * MOM_SLICE;
+    const int s1 = min(ch.len, s0 + MOM_SLICE);
     float ss = 0.f;
     if (vec) {
-      const int stride = blockDim.x * 8;
-      for (int e = threadIdx.x * 8; e < ch.len; e += 2 * stride) {
-        const long long i0 = ch.start + e, i1 = i0 + stride;
-        const bool has1 = e + stride < ch.len;
-        float v0[8], v1[8];
-        float4 m0a, m0b, m1a, m1b;
-        load8_grad(g, grad_f32, i0, v0);
-        if (has1) load8_grad(g, grad_f32, i1, v1);
-        if (mom) {
-          const float4* p0 = reinterpret_cast<const float4*>(mom + i0);
-          m0a = p0[0];
-          m0b = p0[1];
-          if (has1) {
-            const float4* p1 = reinterpret_cast<const float4*>(mom + i1);
-            m1a = p1[0];
-            m1b = p1[1];
-          }
-          v0[0] += beta * m0a.x; v0[1] += beta * m0a.y; v0[2] += beta * m0a.z; v0[3] += beta * m0a.w;
-          v0[4] += beta * m0b.x; v0[5] += beta * m0b.y; v0[6] += beta * m0b.z; v0[7] += beta * m0b.w;
-          float4* q0 = reinterpret_cast<float4*>(mom + i0);
-          q0[0] = make_float4(v0[0], v0[1], v0[2], v0[3]);
-          q0[1] = make_float4(v0[4], v0[5], v0[6], v0[7]);
-          if (has1) {
-            v1[0] += beta * m1a.x; v1[1] += beta * m1a.y; v1[2] += beta * m1a.z; v1[3] += beta * m1a.w;
-            v1[4] += beta * m1b.x; v1[5] += beta * m1b.y; v1[6] += beta * m1b.z; v1[7] += beta * m1b.w;
-            float4* q1 = reinterpret_cast<float4*>(mom + i1);
-            q1[0] = make_float4(v1[0], v1[1], v1[2], v1[3]);
-            q1[1] = make_float4(v1[4], v1[5], v1[6], v1[7]);
+      for (int e = s0 + lane * 8; e < s1; e += 32 * 8 * MOM_VEC) {
+        GradVec<F32> gv[MOM_VEC];
+        float4 ma[MOM_VEC], mc[MOM_VEC];
+#pragma unroll
+        for (int u = 0; u < MOM_VEC; ++u) {
+          const int eu = e + u * 256;
+          if (eu < s1) {
+            gv[u].load(g, ch.start + eu);
+            if (mom) {
+              const float4* pm = reinterpret_cast<const float4*>(mom + ch.start + eu);
+              ma[u] = pm[0];
+              mc[u] = pm[1];
+            }
           }
         }
 #pragma unroll
-        for (int q = 0; q < 8; ++q) ss += v0[q] * v0[q];
-        store8_image(mb, mb_f32, mm.mb_off + i0, v0);  // ldc == cols on the vector path
-        if (has1) {
+        for (int u = 0; u < MOM_VEC; ++u) {
+          const int eu = e + u * 256;
+          if (eu < s1) {
+            const long long i0 = ch.start + eu;
+            float v[8];
+            gv[u].get(v);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) ss += v1[q] * v1[q];
-          store8_image(mb, mb_f32, mm.mb_off + i1, v1);
+            for (int q = 0; q < 8; ++q) v[q] *= gscale;
+            if (mom) {
+              v[0] += beta * ma[u].x; v[1] += beta * ma[u].y; v[2] += beta * ma[u].z; v[3] += beta * ma[u].w;
+              v[4] += beta * mc[u].x; v[5] += beta * mc[u].y; v[6] += beta * mc[u].z; v[7] += beta * mc[u].w;
+              float4* q0 = reinterpret_cast<float4*>(mom + i0);
+              q0[0] = make_float4(v[0], v[1], v[2], v[3]);
+              q0[1] = make_float4(v[4], v[5], v[6], v[7]);
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) ss += v[q] * v[q];
+            store8_image(mb, F32 ? 1 : 0, mb_off + i0, v);  // ldc == cols on the vector path
+          }
         }
       }
     } else {
-      for (int e = threadIdx.x; e < ch.len; e += blockDim.x) {
+      const MomMat mm = mats[ch.slot];
+      for (int e = s0 + lane; e < s1; e += 32) {
         const long long idx = ch.start + e;
-        float v = grad_f32 ? reinterpret_cast<const float*>(g)[idx]
-                           : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(g)[idx]);
+        float v = F32 ? reinterpret_cast<const float*>(g)[idx]
+                      : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(g)[idx]);
+        v *= gscale;
         if (mom) {
           v += beta * mom[idx];
           mom[idx] = v;
@@ -115,24 +159,15 @@ __global__ void __launch_bounds__(256, 6) k_momentum(const MomChunk* __restrict_
         ss += v * v;
         const long long row = idx / mm.cols, col = idx - row * mm.cols;
         const long long o = mm.mb_off + row * mm.ldc + col;
-        if (mb_f32)
+        if (F32)
           reinterpret_cast<float*>(mb)[o] = v;
         else
           reinterpret_cast<__nv_bfloat16*>(mb)[o] = __float2bfloat16_rn(v);
       }
     }
-    // block reduction in a fixed order
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
-    __syncthreads();
-    if (threadIdx.x < 32) {
-      float t = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
-      if (threadIdx.x == 0) partial[c] = t;
-    }
-    __syncthreads();
+    if (lane == 0) partial[(long long)c * MOM_WARPS + warp] = ss;
   }
 }
 
@@ -144,7 +179,8 @@ __global__ void k_norm_finalize(const MomMat* __restrict__ mats, int nmats,
   if (warp >= nmats) return;
   const MomMat mm = mats[warp];
   double s = 0.0;
-  for (int c = mm.chunk_begin + lane; c < mm.chunk_end; c += 32) s += (double)partial[c];
+  for (long long c = (long long)mm.chunk_begin * MOM_WARPS + lane; c < (long long)mm.chunk_end * MOM_WARPS; c += 32)
+    s += (double)partial[c];
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
   if (lane == 0) {
@@ -156,13 +192,17 @@ __global__ void k_norm_finalize(const MomMat* __restrict__ mats, int nmats,
 
 cudaError_t launch_momentum(const MomChunk* chunks, int nchunks, const MomMat* mats,
                             const void* const* grads, float* const* momenta, int grad_f32, void* mb,
-                            int mb_f32, float beta, float* partial, int vec_ok, int num_sms,
+                            int mb_f32, float beta, float gscale, float* partial, int vec_ok, int num_sms,
                             cudaStream_t s) {
   if (nchunks <= 0) return cudaSuccess;
-  int grid = num_sms * 6;
+  int grid = num_sms * 3;  // the resident CTAs per SM of the launch bounds
   if (grid > nchunks) grid = nchunks;
-  k_momentum<<<grid, 256, 0, s>>>(chunks, nchunks, mats, grads, momenta, grad_f32, mb, mb_f32, beta,
-                                  partial, vec_ok);
+  // the image has the gradients' element type (bf16 -> bf16 image, fp32 -> fp32)
+  if (grad_f32 != mb_f32) return cudaErrorInvalidValue;
+  if (grad_f32)
+    k_momentum<true><<<grid, 256, 0, s>>>(chunks, nchunks, mats, grads, momenta, mb, beta, gscale, partial, vec_ok);
+  else
+    k_momentum<false><<<grid, 256, 0, s>>>(chunks, nchunks, mats, grads, momenta, mb, beta, gscale, partial, vec_ok);
   return cudaGetLastError();
 }
 

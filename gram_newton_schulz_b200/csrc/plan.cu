@@ -53,6 +53,7 @@ struct Bucket {
   int64_t ldc = 0;
   int64_t mb_off = 0;  // element offset of the bucket's first image
   int map_k = -1, map_mn = -1;
+  int fsched = -1;     // tile schedule of this bucket's final GEMM (-1: the plan's)
 };
 
 struct GClass {
@@ -69,7 +70,16 @@ struct GClass {
   // through MN-major maps (64 x 64 boxes).
   bool half = false;
   int map_t = -1, map_pf_t = -1;
+  // Tile schedule of this class's Gram recursion: -1 the plan's, 0/1/2 the
+  // staged schedules, SCHED_ONCHIP the whole recursion in one CTA per matrix
+  int sched = -1;
 };
+
+constexpr int SCHED_ONCHIP = 3;
+
+bool onchip_eligible(dmu_dtype dtype, const GClass& g) {
+  return dtype == DMU_BF16 && g.prec == DMU_PREC_SPLIT3 && g.m <= ONCHIP_MAX_M;
+}
 
 enum { TBL_GRADS = 0, TBL_MOMS, TBL_W, TBL_O, TBL_IN, NUM_TBL };
 
@@ -134,6 +144,12 @@ struct dmu_plan_s {
   // CTAs (128 x 256), 2 = single CTAs (128 x 128, for many small matrices)
   int sched = 1;
   bool half_store = true;  // half-stored symmetric Gram-space matrices
+  int tune_class = -1, tune_bucket = -1;  // autotune: run one class / one bucket only
+  int tune_count = 0;                      // autotune: matrices of the tuned bucket's final (0: all)
+
+  int class_sched(int c) const { return classes[c].sched >= 0 ? classes[c].sched : sched; }
+  bool onchip(int c) const { return classes[c].sched == SCHED_ONCHIP; }
+  int final_sched(const Bucket& b) const { return b.fsched >= 0 ? b.fsched : sched; }
 
   unsigned int* status_dev() const { return reinterpret_cast<unsigned int*>(ws + off_status); }
   float* inv_dev() const { return reinterpret_cast<float*>(ws + off_inv); }
@@ -218,7 +234,7 @@ struct Prob {
   int amap_t = -1, bmap_t = -1;  // transposed-read maps of half-stored operands
 };
 
-dmu_status run_tc(dmu_plan p, std::vector<Prob>& probs, int na, int nb, int kind, cudaStream_t s) {
+dmu_status run_tc(dmu_plan p, std::vector<Prob>& probs, int na, int nb, int kind, int sched, cudaStream_t s) {
   size_t i = 0;
   while (i < probs.size()) {
     GemmParams gp;
@@ -248,8 +264,8 @@ dmu_status run_tc(dmu_plan p, std::vector<Prob>& probs, int na, int nb, int kind
       g.b_map = slot(probs[i].bmap);
       g.a_map_t = probs[i].amap_t >= 0 ? slot(probs[i].amap_t) : g.a_map;
       g.b_map_t = probs[i].bmap_t >= 0 ? slot(probs[i].bmap_t) : g.b_map;
-      g.tiles_per_mat = tiles_for(g.M, g.N, g.sym != 0, &g.tiles_m, &g.tiles_n, p->sched == 1 ? 256 : BM,
-                                  p->sched == 2 ? 128 : BN);
+      g.tiles_per_mat = tiles_for(g.M, g.N, g.sym != 0, &g.tiles_m, &g.tiles_n, sched == 1 ? 256 : BM,
+                                  sched == 2 ? 128 : BN);
       g.tile_begin = tiles;
       tiles += g.count * g.tiles_per_mat;
       gp.prob[nprob++] = g;
@@ -260,10 +276,10 @@ dmu_status run_tc(dmu_plan p, std::vector<Prob>& probs, int na, int nb, int kind
     gp.total_tiles = tiles;
     gp.status = p->status_dev();
     gp.timeout_ns = p->timeout_ns;
-    if (p->sched == 1)
+    if (sched == 1)
       CUDA_TRY(launch_gemm_tc2(gp, na, nb, kind, p->num_sms, s));
     else
-      CUDA_TRY(launch_gemm_tc(gp, na, nb, kind, p->num_sms, p->sched == 2 ? 128 : 256, s));
+      CUDA_TRY(launch_gemm_tc(gp, na, nb, kind, p->num_sms, sched == 2 ? 128 : 256, s));
     p->launches++;
   }
   return DMU_OK;
@@ -498,26 +514,89 @@ dmu_status run_products(dmu_plan p, const std::vector<std::pair<Product, bool>>&
                         const float co[3], int p_in, int p_out, cudaStream_t s) {
   const int precs[5] = {DMU_PREC_F16, DMU_PREC_TF32, DMU_PREC_FAST, DMU_PREC_SPLIT2, DMU_PREC_SPLIT3};
   for (int pr : precs) {
-    std::vector<Prob> probs;
-    for (size_t c = 0; c < p->classes.size(); ++c) {
-      if (p->classes[c].prec != pr) continue;
-      for (auto& kd : kinds)
-        if (kd.second) probs.push_back(product(p, (int)c, kd.first, k, last, co, p_in, p_out));
+    for (int sched = 0; sched < SCHED_ONCHIP; ++sched) {
+      std::vector<Prob> probs;
+      for (size_t c = 0; c < p->classes.size(); ++c) {
+        if (p->classes[c].prec != pr || p->class_sched((int)c) != sched) continue;
+        if (p->tune_class >= 0 && (int)c != p->tune_class) continue;
+        for (auto& kd : kinds)
+          if (kd.second) probs.push_back(product(p, (int)c, kd.first, k, last, co, p_in, p_out));
+      }
+      if (probs.empty()) continue;
+      int na, nb, terms, kind;
+      prec_shape(pr, &na, &nb, &terms, &kind);
+      dmu_status st = run_tc(p, probs, na, nb, kind, sched, s);
+      if (st != DMU_OK) return st;
     }
-    if (probs.empty()) continue;
-    int na, nb, terms, kind;
-    prec_shape(pr, &na, &nb, &terms, &kind);
-    dmu_status st = run_tc(p, probs, na, nb, kind, s);
-    if (st != DMU_OK) return st;
   }
   return DMU_OK;
 }
 
+// Classes on the on-chip schedule: one launch (per 8 buckets) runs SYRK and
+// the whole recursion with one CTA per matrix and writes the final P into
+// the class's P slot, where the staged path would have left it.
+dmu_status run_onchip(dmu_plan p, const float co[3], int steps, int p_final, cudaStream_t s) {
+  OnchipParams op;
+  std::memset(&op, 0, sizeof(op));
+  int nmaps = 0;
+  auto flush = [&]() -> dmu_status {
+    if (op.nprob == 0) return DMU_OK;
+    op.inv = p->inv_dev();
+    op.a = co[0];
+    op.b = co[1];
+    op.c = co[2];
+    op.steps = steps;
+    op.status = p->status_dev();
+    op.timeout_ns = p->timeout_ns;
+    CUDA_TRY(launch_gram_onchip(op, p->num_sms, s));
+    p->launches++;
+    std::memset(&op, 0, sizeof(op));
+    nmaps = 0;
+    return DMU_OK;
+  };
+  for (const Bucket& b : p->buckets) {
+    if (!p->onchip(b.cls)) continue;
+    if (p->tune_class >= 0 && b.cls != p->tune_class) continue;
+    if (op.nprob == MAX_PROBS) {
+      dmu_status st = flush();
+      if (st != DMU_OK) return st;
+    }
+    const GClass& gc = p->classes[b.cls];
+    OnchipProblem& q = op.prob[op.nprob++];
+    q.count = b.count;
+    q.m = (int)b.m;
+    q.n = (int)b.n;
+    q.tall = b.tall ? 1 : 0;
+    op.maps[nmaps] = p->maps[b.tall ? b.map_mn : b.map_k];
+    q.map = nmaps++;
+    q.inv_base = b.first_slot;
+    q.mat_begin = op.total;
+    op.total += b.count;
+    const size_t moff = (size_t)b.cls_off * gc.m * gc.ldg;
+    const int hi = p_final == 0 ? SLOT_PA_HI : SLOT_PB_HI;
+    q.p_hi = p->slot_bf16(b.cls, hi) + moff;
+    q.p_lo = p->slot_bf16(b.cls, hi + 1) + moff;
+    q.ld = gc.ldg;
+    q.mat_stride = gc.m * gc.ldg;
+  }
+  return flush();
+}
+
 dmu_status gram_bf16(dmu_plan p, const float co[3], int steps, cudaStream_t s) {
-  // G0 = s^2 X X^T, one problem per shape bucket (SYRK, upper tiles only)
+  // index of the P buffer that holds P_K after `steps` steps (0: A, 1: B)
+  const int p_final = steps >= 1 ? (steps - 1) & 1 : 0;
+  if (steps >= 1) {
+    dmu_status st0 = run_onchip(p, co, steps, p_final, s);
+    if (st0 != DMU_OK) return st0;
+  }
+  // G0 = s^2 X X^T, one problem per shape bucket (SYRK, upper tiles only),
+  // launched with its class's tile schedule
   std::vector<Prob> syrk;
+  std::vector<int> syrk_sched;
   for (const Bucket& b : p->buckets) {
     const GClass& gc = p->classes[b.cls];
+    if (p->tune_class >= 0 && b.cls != p->tune_class) continue;
+    if (steps >= 1 && p->onchip(b.cls)) continue;
     Prob pr;
     std::memset(&pr, 0, sizeof(pr));
     GemmProblem& g = pr.g;
@@ -551,13 +630,22 @@ dmu_status gram_bf16(dmu_plan p, const float co[3], int steps, cudaStream_t s) {
     pr.amap = pr.bmap = b.tall ? b.map_mn : b.map_k;
     g.half_out = gc.half ? 1 : 0;
     syrk.push_back(pr);
+    syrk_sched.push_back(p->onchip(b.cls) ? p->sched : p->class_sched(b.cls));
   }
-  dmu_status st = run_tc(p, syrk, 1, 1, KIND_BF16, s);
-  if (st != DMU_OK) return st;
+  dmu_status st = DMU_OK;
+  for (int sched = 0; sched < SCHED_ONCHIP; ++sched) {
+    std::vector<Prob> group;
+    for (size_t i = 0; i < syrk.size(); ++i)
+      if (syrk_sched[i] == sched) group.push_back(syrk[i]);
+    if (group.empty()) continue;
+    st = run_tc(p, group, 1, 1, KIND_BF16, sched, s);
+    if (st != DMU_OK) return st;
+  }
 
   if (steps == 0) {
     for (size_t c = 0; c < p->classes.size(); ++c) {
       const GClass& gc = p->classes[c];
+      if (p->tune_class >= 0 && (int)c != p->tune_class) continue;
       const bool tf = gc.kind != KIND_BF16;  // TF32 / F16 classes keep the final P in the bf16 pair area
       CUDA_TRY(launch_identity_bf16(tf ? p->pf_bf16((int)c, 0) : p->slot_bf16((int)c, SLOT_PA_HI),
                                     tf ? p->pf_bf16((int)c, 1) : p->slot_bf16((int)c, SLOT_PA_LO),
@@ -582,7 +670,7 @@ dmu_status gram_bf16(dmu_plan p, const float co[3], int steps, cudaStream_t s) {
     }
   }
   p->p_final = p_cur;
-  return DMU_OK;
+  return p_cur == p_final ? DMU_OK : fail(DMU_ERR_CUDA, "internal: final P buffer mismatch");
 }
 
 // ---------------------------------------------------------------- fp32 path
@@ -676,12 +764,13 @@ dmu_status gram_f32(dmu_plan p, const float co[3], int steps, cudaStream_t s) {
   return DMU_OK;
 }
 
-dmu_status run_normalize(dmu_plan p, int tbl, bool with_mom, float beta, float eps, bool vec, cudaStream_t s) {
+dmu_status run_normalize(dmu_plan p, int tbl, bool with_mom, float beta, float gscale, float eps, bool vec,
+                         cudaStream_t s) {
   const bool f32 = p->dtype == DMU_F32;
   CUDA_TRY(launch_momentum(p->chunks_dev(), (int)p->chunks.size(), p->mats_dev(),
                            const_cast<const void* const*>(p->tbl_dev(tbl)),
                            with_mom ? reinterpret_cast<float* const*>(p->tbl_dev(TBL_MOMS)) : nullptr,
-                           f32 ? 1 : 0, p->mb_dev(), f32 ? 1 : 0, beta, p->partial_dev(), vec ? 1 : 0,
+                           f32 ? 1 : 0, p->mb_dev(), f32 ? 1 : 0, beta, gscale, p->partial_dev(), vec ? 1 : 0,
                            p->num_sms, s));
   CUDA_TRY(launch_norm_finalize(p->mats_dev(), p->count, p->partial_dev(), eps, p->inv_dev(),
                                 p->status_dev(), s));
@@ -689,6 +778,66 @@ dmu_status run_normalize(dmu_plan p, int tbl, bool with_mom, float beta, float e
   p->eps = eps;
   p->have_mb = true;
   p->have_p = false;
+  return DMU_OK;
+}
+
+// Final O = P X0 GEMM fused with the weight update, bf16 path: one problem
+// per shape bucket, launched per tile schedule; W and O come from the
+// device pointer tables (TBL_W, TBL_O).
+dmu_status final_launch(dmu_plan p, bool with_w, bool with_o, float lr, cudaStream_t s) {
+  dmu_status st = DMU_OK;
+  std::vector<Prob> probs;
+  std::vector<int> scheds;
+  const int pf_hi = p->p_final == 0 ? SLOT_PA_HI : SLOT_PB_HI;
+  for (const Bucket& b : p->buckets) {
+    const GClass& gc = p->classes[b.cls];
+    if (p->tune_bucket >= 0 && &b != &p->buckets[p->tune_bucket]) continue;
+    Prob pr;
+    std::memset(&pr, 0, sizeof(pr));
+    GemmProblem& g = pr.g;
+    g.count = p->tune_count > 0 ? std::min(p->tune_count, b.count) : b.count;
+    g.M = (int)b.m;
+    g.N = (int)b.n;
+    g.K = (int)b.m;
+    g.sym = 0;
+    g.tiles_per_mat = tiles_for(g.M, g.N, false, &g.tiles_m, &g.tiles_n);
+    g.a_mn = 0;
+    if (gc.kind != KIND_BF16) {
+      g.a_z[0] = b.cls_off;
+      g.a_z[1] = gc.count + b.cls_off;
+    } else {
+      g.a_z[0] = pf_hi * gc.count + b.cls_off;
+      g.a_z[1] = (pf_hi + 1) * gc.count + b.cls_off;
+    }
+    g.b_mn = b.tall ? 0 : 1;
+    g.terms = TERM_HH | TERM_LH;
+    g.epi = EPI_UPDATE;
+    g.alpha = -lr * (float)std::sqrt(std::max(1.0, (double)b.rows / (double)b.cols));
+    g.inv = p->inv_dev();
+    g.inv_base = b.first_slot;
+    g.w_ptrs = with_w ? reinterpret_cast<void* const*>(p->tbl_dev(TBL_W)) : nullptr;
+    g.o_ptrs = with_o ? reinterpret_cast<float* const*>(p->tbl_dev(TBL_O)) : nullptr;
+    g.ptr_base = b.first_slot;
+    g.w_f32 = 0;
+    g.w_transposed = b.tall ? 1 : 0;
+    g.w_cols = b.cols;
+    pr.amap = gc.kind != KIND_BF16 ? gc.map_pf : gc.map;
+    pr.bmap = b.tall ? b.map_k : b.map_mn;
+    if (gc.half) {
+      g.half_a = 1;
+      pr.amap_t = gc.kind != KIND_BF16 ? gc.map_pf_t : gc.map_t;
+    }
+    probs.push_back(pr);
+    scheds.push_back(p->final_sched(b));
+  }
+  for (int sched = 0; sched < SCHED_ONCHIP; ++sched) {
+    std::vector<Prob> group;
+    for (size_t i = 0; i < probs.size(); ++i)
+      if (scheds[i] == sched) group.push_back(probs[i]);
+    if (group.empty()) continue;
+    st = run_tc(p, group, 2, 1, KIND_BF16, sched, s);
+    if (st != DMU_OK) return st;
+  }
   return DMU_OK;
 }
 
@@ -808,6 +957,13 @@ dmu_status dmu_plan_create(const dmu_shape* shapes, int count, dmu_dtype dtype, 
     }
     p->buckets[it->second].mats.push_back(i);
   }
+  // DMU_ONCHIP=1: classes the on-chip recursion covers (split-bf16
+  // precision, m <= 128) start on that schedule
+  if (const char* e = std::getenv("DMU_ONCHIP")) {
+    if (std::atoi(e) != 0)
+      for (GClass& g : p->classes)
+        if (onchip_eligible(dtype, g)) g.sched = SCHED_ONCHIP;
+  }
   p->slot_of.assign(count, 0);
   int slot = 0;
   int64_t mb_elems = 0;
@@ -853,7 +1009,7 @@ dmu_status dmu_plan_create(const dmu_shape* shapes, int count, dmu_dtype dtype, 
   p->off_inv = off;
   off = align_up(off + sizeof(float) * count, 256);
   p->off_partial = off;
-  off = align_up(off + sizeof(float) * p->chunks.size(), 256);
+  off = align_up(off + sizeof(float) * MOM_PARTIALS_PER_CHUNK * p->chunks.size(), 256);
   p->off_chunks = off;
   off = align_up(off + sizeof(MomChunk) * p->chunks.size(), 256);
   p->off_mats = off;
@@ -909,6 +1065,7 @@ dmu_status dmu_set_workspace(dmu_plan p, void* dev_ptr, size_t bytes) {
   p->maps.clear();
   if (p->dtype == DMU_BF16) {
     CUDA_TRY(gemm_tc_configure());
+    CUDA_TRY(onchip_configure());
     for (Bucket& b : p->buckets) {
       CUtensorMap mk, mn;
       void* base = p->mb_dev() + 2 * (size_t)b.mb_off;
@@ -973,12 +1130,13 @@ dmu_status dmu_set_workspace(dmu_plan p, void* dev_ptr, size_t bytes) {
 }
 
 dmu_status dmu_momentum_normalize(dmu_plan p, const void* const* grads, float* const* momenta, float beta,
-                                  float eps, void* stream) {
+                                  float grad_scale, float eps, void* stream) {
   g_err.clear();
   dmu_status st = check_plan(p, true);
   if (st != DMU_OK) return st;
   if (!grads) return fail(DMU_ERR_INVALID_ARG, "grads is NULL");
-  if (!(eps >= 0.f) || !std::isfinite(beta)) return fail(DMU_ERR_INVALID_ARG, "eps must be >= 0 and beta finite");
+  if (!(eps >= 0.f) || !std::isfinite(beta) || !std::isfinite(grad_scale))
+    return fail(DMU_ERR_INVALID_ARG, "eps must be >= 0, beta and grad_scale finite");
   DevGuard dg(p->device);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   p->launches = 0;
@@ -990,7 +1148,7 @@ dmu_status dmu_momentum_normalize(dmu_plan p, const void* const* grads, float* c
     if (st != DMU_OK) return st;
     vec = vec && aligned16(reinterpret_cast<const void* const*>(momenta), p->count);
   }
-  return run_normalize(p, TBL_GRADS, momenta != nullptr, beta, eps, vec, s);
+  return run_normalize(p, TBL_GRADS, momenta != nullptr, beta, grad_scale, eps, vec, s);
 }
 
 dmu_status dmu_gram_ns_batched(dmu_plan p, const void* const* ptrs, const dmu_shape* shapes, int count,
@@ -1012,7 +1170,7 @@ dmu_status dmu_gram_ns_batched(dmu_plan p, const void* const* ptrs, const dmu_sh
   if (ptrs) {
     st = upload_table(p, TBL_IN, ptrs, s);
     if (st != DMU_OK) return st;
-    st = run_normalize(p, TBL_IN, false, 0.f, p->eps, p->vec_shapes && aligned16(ptrs, p->count), s);
+    st = run_normalize(p, TBL_IN, false, 0.f, 1.f, p->eps, p->vec_shapes && aligned16(ptrs, p->count), s);
     if (st != DMU_OK) return st;
   } else if (!p->have_mb) {
     return fail(DMU_ERR_NOT_PLANNED, "no input: call dmu_momentum_normalize first or pass ptrs");
@@ -1041,50 +1199,7 @@ dmu_status dmu_apply_update(dmu_plan p, void* const* weights, float lr, float* c
     if (st != DMU_OK) return st;
   }
   if (!weights && !out_o) return DMU_OK;
-  if (p->dtype == DMU_BF16) {
-    std::vector<Prob> probs;
-    const int pf_hi = p->p_final == 0 ? SLOT_PA_HI : SLOT_PB_HI;
-    for (const Bucket& b : p->buckets) {
-      const GClass& gc = p->classes[b.cls];
-      Prob pr;
-      std::memset(&pr, 0, sizeof(pr));
-      GemmProblem& g = pr.g;
-      g.count = b.count;
-      g.M = (int)b.m;
-      g.N = (int)b.n;
-      g.K = (int)b.m;
-      g.sym = 0;
-      g.tiles_per_mat = tiles_for(g.M, g.N, false, &g.tiles_m, &g.tiles_n);
-      g.a_mn = 0;
-      if (gc.kind != KIND_BF16) {
-        g.a_z[0] = b.cls_off;
-        g.a_z[1] = gc.count + b.cls_off;
-      } else {
-        g.a_z[0] = pf_hi * gc.count + b.cls_off;
-        g.a_z[1] = (pf_hi + 1) * gc.count + b.cls_off;
-      }
-      g.b_mn = b.tall ? 0 : 1;
-      g.terms = TERM_HH | TERM_LH;
-      g.epi = EPI_UPDATE;
-      g.alpha = -lr * (float)std::sqrt(std::max(1.0, (double)b.rows / (double)b.cols));
-      g.inv = p->inv_dev();
-      g.inv_base = b.first_slot;
-      g.w_ptrs = weights ? reinterpret_cast<void* const*>(p->tbl_dev(TBL_W)) : nullptr;
-      g.o_ptrs = out_o ? reinterpret_cast<float* const*>(p->tbl_dev(TBL_O)) : nullptr;
-      g.ptr_base = b.first_slot;
-      g.w_f32 = 0;
-      g.w_transposed = b.tall ? 1 : 0;
-      g.w_cols = b.cols;
-      pr.amap = gc.kind != KIND_BF16 ? gc.map_pf : gc.map;
-      pr.bmap = b.tall ? b.map_k : b.map_mn;
-      if (gc.half) {
-        g.half_a = 1;
-        pr.amap_t = gc.kind != KIND_BF16 ? gc.map_pf_t : gc.map_t;
-      }
-      probs.push_back(pr);
-    }
-    return run_tc(p, probs, 2, 1, KIND_BF16, s);
-  }
+  if (p->dtype == DMU_BF16) return final_launch(p, weights != nullptr, out_o != nullptr, lr, s);
   const int pf = p->p_final == 0 ? FSLOT_PA : FSLOT_PB;
   for (const Bucket& b : p->buckets) {
     const GClass& gc = p->classes[b.cls];
@@ -1174,6 +1289,9 @@ dmu_status dmu_debug_gram(dmu_plan p, int which, int index, float* out, void* st
     return DMU_OK;
   }
   const GClass& gc = p->classes[bk->cls];
+  if (which <= 4 && p->onchip(bk->cls))
+    return fail(DMU_ERR_NOT_PLANNED, "matrix " + std::to_string(index) +
+                                         " runs its recursion on chip: only the final P (which 7) is kept");
   const size_t moff = (size_t)(bk->cls_off + local) * gc.m * gc.ldg;
   int q = which;
   if (which == 7) q = p->p_final == 0 ? 3 : 4;
@@ -1212,29 +1330,69 @@ dmu_status dmu_debug_gram(dmu_plan p, int which, int index, float* out, void* st
 
 int dmu_last_launch_count(dmu_plan p) { return p ? p->launches : 0; }
 
-// Schedule cache (DMuon page, section 2.4: tuned configs are cached and
-// reused).  The key names the device and the plan's shapes, dtype and
-// precision; the value is the chosen schedule and the times that chose it.
-static std::string schedule_key(dmu_plan p) {
+// Schedule cache (DMuon page, section 2.4: kernel configurations are tuned
+// per shape and cached).  Every Gram class (equal m) and every bucket's
+// final GEMM gets its own entry, keyed by the device, the precision and the
+// shapes it covers, so plans that share a class or a bucket share the
+// entry.
+static std::string device_tag(dmu_plan p) {
   cudaDeviceProp prop;
   std::memset(&prop, 0, sizeof(prop));
   cudaGetDeviceProperties(&prop, p->device);
-  std::ostringstream k;
   std::string name = prop.name;
   for (char& c : name)
     if (c == ' ') c = '_';
-  k << name << "/sm" << prop.multiProcessorCount << "/d" << (int)p->dtype << "/p" << (int)p->prec;
-  unsigned long long h = 1469598103934665603ULL;  // FNV-1a over the shape list
-  for (const dmu_shape& sh : p->shapes) {
-    const int64_t v[2] = {sh.rows, sh.cols};
-    const unsigned char* b = reinterpret_cast<const unsigned char*>(v);
-    for (size_t i = 0; i < sizeof(v); ++i) h = (h ^ b[i]) * 1099511628211ULL;
-  }
-  k << "/n" << p->count << "/h" << std::hex << h;
+  std::ostringstream k;
+  k << name << "/sm" << prop.multiProcessorCount;
   return k.str();
 }
 
+static std::string class_key(dmu_plan p, const std::string& dev, int c) {
+  const GClass& g = p->classes[c];
+  std::ostringstream k;
+  k << dev << "/gram/m" << g.m << "/p" << g.prec << "/n" << g.count << "/";
+  for (const Bucket& b : p->buckets)
+    if (b.cls == c) k << b.rows << "x" << b.cols << "*" << b.count << ",";
+  return k.str();
+}
+
+static std::string final_key(dmu_plan p, const std::string& dev, const Bucket& b) {
+  std::ostringstream k;
+  k << dev << "/final/" << b.rows << "x" << b.cols << "/n" << b.count << "/p" << p->classes[b.cls].prec;
+  return k.str();
+}
+
+static std::map<std::string, int> read_cache(const char* path) {
+  std::map<std::string, int> out;
+  if (!path) return out;
+  std::ifstream in(path);
+  std::string line;
+  while (std::getline(in, line)) {
+    std::istringstream ls(line);
+    std::string k;
+    int v = -1;
+    if ((ls >> k >> v) && v >= 0 && v <= SCHED_ONCHIP) out[k] = v;
+  }
+  return out;
+}
+
 int dmu_get_schedule(dmu_plan p) { return p ? p->sched : -1; }
+
+int dmu_get_gram_schedule(dmu_plan p, int index) {
+  if (!p || index < 0 || index >= p->count) return -1;
+  for (const Bucket& b : p->buckets)
+    for (int i : b.mats)
+      if (i == index) return p->class_sched(b.cls);
+  return -1;
+}
+
+int dmu_get_final_schedule(dmu_plan p, int index) {
+  if (!p || index < 0 || index >= p->count) return -1;
+  for (const Bucket& b : p->buckets)
+    for (int i : b.mats)
+      if (i == index) return p->final_sched(b);
+  return -1;
+}
 
 dmu_status dmu_autotune(dmu_plan p, const char* cache_path, void* stream) {
   g_err.clear();
@@ -1244,58 +1402,120 @@ dmu_status dmu_autotune(dmu_plan p, const char* cache_path, void* stream) {
   if (p->dtype != DMU_BF16) return DMU_OK;  // one schedule on the fp32 path
   DevGuard dg(p->device);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const std::string key = schedule_key(p);
-  if (cache_path) {
-    std::ifstream in(cache_path);
-    std::string line;
-    while (std::getline(in, line)) {
-      std::istringstream ls(line);
-      std::string k;
-      int sched = -1;
-      if ((ls >> k >> sched) && k == key && sched >= 0 && sched <= 2) {
-        p->sched = sched;
-        return DMU_OK;
-      }
-    }
-  }
+  const std::string dev = device_tag(p);
+  std::map<std::string, int> cache = read_cache(cache_path);
+  std::vector<std::string> lines;
   const float co[3] = {3.4445f, -4.7750f, 2.0315f};
-  float ms[3] = {0.f, 0.f, 0.f};
   cudaEvent_t e0, e1;
   CUDA_TRY(cudaEventCreate(&e0));
   CUDA_TRY(cudaEventCreate(&e1));
-  const int keep = p->sched;
-  for (int variant = 0; variant < 3; ++variant) {
-    p->sched = variant;
-    st = gram_bf16(p, co, 5, s);  // warm-up
+  // best of three timed runs after one warm-up; a failed run leaves `st` set
+  auto time_min = [&](auto&& run) -> float {
+    float best = 0.f;
+    st = run();
     for (int rep = 0; st == DMU_OK && rep < 3; ++rep) {
-      CUDA_TRY(cudaEventRecord(e0, s));
-      st = gram_bf16(p, co, 5, s);
-      CUDA_TRY(cudaEventRecord(e1, s));
-      CUDA_TRY(cudaEventSynchronize(e1));
+      cudaEventRecord(e0, s);
+      st = run();
+      cudaEventRecord(e1, s);
+      if (cudaEventSynchronize(e1) != cudaSuccess) {
+        st = fail(DMU_ERR_CUDA, "autotune: event synchronisation failed");
+        break;
+      }
       float t = 0.f;
-      CUDA_TRY(cudaEventElapsedTime(&t, e0, e1));
-      ms[variant] = rep == 0 ? t : std::min(ms[variant], t);
+      cudaEventElapsedTime(&t, e0, e1);
+      best = rep == 0 ? t : std::min(best, t);
     }
-    if (st != DMU_OK) {
-      p->sched = keep;
-      cudaEventDestroy(e0);
-      cudaEventDestroy(e1);
-      return st;
+    return best;
+  };
+  const int saved_launches = p->launches;
+
+  // ---- Gram recursion, one class at a time (CTA pairs first: they win ties)
+  for (size_t c = 0; st == DMU_OK && c < p->classes.size(); ++c) {
+    GClass& g = p->classes[c];
+    const std::string key = class_key(p, dev, (int)c);
+    auto hit = cache.find(key);
+    if (hit != cache.end() && (hit->second != SCHED_ONCHIP || onchip_eligible(p->dtype, g))) {
+      g.sched = hit->second;
+      continue;
     }
+    std::vector<int> cand = {1, 0, 2};
+    if (onchip_eligible(p->dtype, g)) cand.push_back(SCHED_ONCHIP);
+    std::ostringstream times;
+    int best = -1;
+    float best_ms = 0.f;
+    p->tune_class = (int)c;
+    for (int sc : cand) {
+      g.sched = sc;
+      const float ms = time_min([&] { return gram_bf16(p, co, 5, s); });
+      if (st != DMU_OK) break;
+      times << " s" << sc << "_ms=" << ms;
+      if (best < 0 || ms < best_ms) {
+        best = sc;
+        best_ms = ms;
+      }
+    }
+    p->tune_class = -1;
+    if (st != DMU_OK) break;
+    g.sched = best;
+    cache[key] = best;
+    lines.push_back(key + " " + std::to_string(best) + times.str());
+  }
+  // the recursion once more with every class on its schedule: P_K for all
+  if (st == DMU_OK) st = gram_bf16(p, co, 5, s);
+
+  // ---- final GEMM + update, one bucket at a time.  Its weight writes go to
+  // the class's G, R and T slots (free after the recursion), never to the
+  // caller's weights; when they cannot hold the whole bucket, the first
+  // matrices that fit are timed.
+  for (size_t bi = 0; st == DMU_OK && bi < p->buckets.size(); ++bi) {
+    Bucket& b = p->buckets[bi];
+    const GClass& g = p->classes[b.cls];
+    const std::string key = final_key(p, dev, b);
+    auto hit = cache.find(key);
+    if (hit != cache.end() && hit->second < SCHED_ONCHIP) {
+      b.fsched = hit->second;
+      continue;
+    }
+    const size_t free_bytes = (size_t)12 * g.count * g.m * g.ldg;  // slots G, R, T of the class
+    const size_t w_bytes = align_up((size_t)b.rows * b.cols * 2, 256);
+    const int n = (int)std::min<size_t>((size_t)b.count, free_bytes / w_bytes);
+    if (n == 0) continue;
+    std::vector<const void*> wt(p->count, nullptr);
+    char* area = p->ws + g.off;
+    for (int k = 0; k < n; ++k) wt[b.mats[k]] = area + (size_t)k * w_bytes;
+    st = upload_table(p, TBL_W, wt.data(), s, true);
+    if (st != DMU_OK) break;
+    p->tune_bucket = (int)bi;
+    p->tune_count = n;
+    std::ostringstream times;
+    int best = -1;
+    float best_ms = 0.f;
+    for (int sc : {1, 0, 2}) {
+      b.fsched = sc;
+      const float ms = time_min([&] { return final_launch(p, true, false, 0.f, s); });
+      if (st != DMU_OK) break;
+      times << " s" << sc << "_ms=" << ms;
+      if (best < 0 || ms < best_ms) {
+        best = sc;
+        best_ms = ms;
+      }
+    }
+    p->tune_bucket = -1;
+    p->tune_count = 0;
+    p->tbl_valid[TBL_W] = false;  // the caller's table is uploaded again by the next update
+    if (st != DMU_OK) break;
+    b.fsched = best;
+    cache[key] = best;
+    lines.push_back(key + " " + std::to_string(best) + times.str() + " timed_matrices=" + std::to_string(n));
   }
   cudaEventDestroy(e0);
   cudaEventDestroy(e1);
-  // the CTA-pair schedule wins ties, then 128 x 256 single CTAs
-  int best = 1;
-  if (ms[0] < ms[best]) best = 0;
-  if (ms[2] < ms[best]) best = 2;
-  p->sched = best;
-  p->have_p = true;
-  if (cache_path) {
+  p->launches = saved_launches;
+  if (st != DMU_OK) return st;
+  p->have_p = true;  // P_K of the quintic K = 5 recursion on every class
+  if (cache_path && !lines.empty()) {
     std::ofstream out(cache_path, std::ios::app);
-    if (out)
-      out << key << " " << best << " pair_ms=" << ms[1] << " single_ms=" << ms[0] << " single128_ms=" << ms[2]
-          << "\n";
+    for (const std::string& l : lines) out << l << "\n";
   }
   return DMU_OK;
 }

@@ -28,7 +28,7 @@ STATUS_NAMES = ["OK", "INVALID_ARG", "UNSUPPORTED", "WORKSPACE", "CUDA", "NONFIN
 DTYPES = {"bf16": 0, "f32": 1}
 PRECS = {"auto": 0, "fast": 1, "split2": 2, "split3": 3, "tf32": 4, "f16": 5}
 FLAG_NONFINITE, FLAG_TIMEOUT = 1, 2
-SCHEDULES = {0: "single_cta", 1: "cta_pair", 2: "single_cta_n128"}
+SCHEDULES = {0: "single_cta", 1: "cta_pair", 2: "single_cta_n128", 3: "onchip"}
 
 # name -> (restype, argtypes); every symbol of include/dmu.h
 _VP = ctypes.c_void_p
@@ -36,7 +36,7 @@ SIGNATURES = {
     "dmu_plan_create": (ctypes.c_int, [_VP, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.POINTER(_VP)]),
     "dmu_workspace_bytes": (ctypes.c_size_t, [_VP]),
     "dmu_set_workspace": (ctypes.c_int, [_VP, _VP, ctypes.c_size_t]),
-    "dmu_momentum_normalize": (ctypes.c_int, [_VP, _VP, _VP, ctypes.c_float, ctypes.c_float, _VP]),
+    "dmu_momentum_normalize": (ctypes.c_int, [_VP, _VP, _VP, ctypes.c_float, ctypes.c_float, ctypes.c_float, _VP]),
     "dmu_gram_ns_batched": (ctypes.c_int, [_VP, _VP, _VP, ctypes.c_int, _VP, ctypes.c_int, _VP]),
     "dmu_apply_update": (ctypes.c_int, [_VP, _VP, ctypes.c_float, _VP, _VP]),
     "dmu_read_status": (ctypes.c_int, [_VP, ctypes.POINTER(ctypes.c_uint32)]),
@@ -47,6 +47,8 @@ SIGNATURES = {
     "dmu_plan_destroy": (None, [_VP]),
     "dmu_autotune": (ctypes.c_int, [_VP, ctypes.c_char_p, _VP]),
     "dmu_get_schedule": (ctypes.c_int, [_VP]),
+    "dmu_get_gram_schedule": (ctypes.c_int, [_VP, ctypes.c_int]),
+    "dmu_get_final_schedule": (ctypes.c_int, [_VP, ctypes.c_int]),
     "dmu_momentum_norm_static": (ctypes.c_int, [_VP, _VP, _VP, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
                                                 ctypes.c_float, ctypes.c_float, _VP, _VP]),
     "dmu_demuon_track": (ctypes.c_int, [ctypes.c_int, ctypes.c_int64, _VP, ctypes.c_float, _VP, _VP, _VP, _VP,
@@ -155,7 +157,8 @@ class Plan:
         import torch
         return torch.bfloat16 if self.dtype == "bf16" else torch.float32
 
-    def momentum_normalize(self, grads, momenta=None, beta: float = 0.95, eps: float = 1e-7, stream=None):
+    def momentum_normalize(self, grads, momenta=None, beta: float = 0.95, eps: float = 1e-7, stream=None,
+                           grad_scale: float = 1.0):
         import torch
         self._check_tensors(grads, "grads", self._wdtype())
         g = _ptr_array([t.data_ptr() for t in grads])
@@ -165,7 +168,8 @@ class Plan:
             m = _ptr_array([t.data_ptr() for t in momenta])
         _check(self.lib.dmu_momentum_normalize(self.handle, ctypes.cast(g, _VP),
                                                ctypes.cast(m, _VP) if m is not None else None,
-                                               float(beta), float(eps), _stream_handle(stream, self.device)))
+                                               float(beta), float(grad_scale), float(eps),
+                                               _stream_handle(stream, self.device)))
 
     def gram_ns_batched(self, ptrs=None, coeffs=QUINTIC, steps: int = 5, stream=None):
         arr = None
@@ -204,13 +208,22 @@ class Plan:
         self.gram_ns_batched(None, coeffs, steps, stream)
         self.apply_update(weights, lr, out_o, stream)
 
-    def autotune(self, cache_path: Optional[str] = None, stream=None) -> int:
-        """Choose the fastest tensor-core schedule by measurement (needs a prior
-        momentum_normalize); returns 1 for CTA pairs (256 x 256 tiles), 0 for
-        single CTAs with 128 x 256 tiles, 2 for single CTAs with 128 x 128."""
+    def autotune(self, cache_path: Optional[str] = None, stream=None) -> dict:
+        """Choose, by measurement, the schedule of every Gram class and of
+        every bucket's final GEMM (needs a prior momentum_normalize); returns
+        `schedules()`."""
         _check(self.lib.dmu_autotune(self.handle, cache_path.encode() if cache_path else None,
                                      _stream_handle(stream, self.device)))
-        return int(self.lib.dmu_get_schedule(self.handle))
+        return self.schedules()
+
+    def schedules(self) -> dict:
+        """{"gram": {m: name}, "final": {(rows, cols): name}} with the
+        schedule names of SCHEDULES."""
+        gram, final = {}, {}
+        for i, (r, c) in enumerate(self.shapes):
+            gram[min(r, c)] = SCHEDULES.get(int(self.lib.dmu_get_gram_schedule(self.handle, i)), "?")
+            final[(r, c)] = SCHEDULES.get(int(self.lib.dmu_get_final_schedule(self.handle, i)), "?")
+        return {"gram": gram, "final": final}
 
     def read_status(self) -> int:
         flags = ctypes.c_uint32(0)

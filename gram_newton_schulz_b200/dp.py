@@ -12,7 +12,8 @@ One exchange step per optimizer step, as collectives over the process group
 
 * **In.** One `reduce` (sum) per owner bucket to that owner. A bucket is the
   flat buffer that holds the gradients of all matrices one rank owns. The
-  owner divides its bucket by the world size to get the mean gradient.
+  owner's momentum pass reads the sum scaled by 1 / world size, the mean
+  gradient, with no separate pass over the bucket.
 * **Compute.** The owner runs momentum, Gram Newton-Schulz and the fused
   weight update on its own matrices only.
 * **Out.** One `broadcast` per owner bucket of the updated weights from
@@ -107,11 +108,11 @@ class PlanCompute:
         self.launches = 0      # kernel launches of the last call
         self.tc_launches = 0   # of which tensor-core (Gram recursion + final update)
 
-    def __call__(self, grads, momenta, weights, *, beta, lr, eps, coeffs, steps, out_o=None):
+    def __call__(self, grads, momenta, weights, *, beta, lr, eps, coeffs, steps, grad_scale=1.0, out_o=None):
         self.launches = self.tc_launches = 0
         if self.plan is None:
             return
-        self.plan.momentum_normalize(grads, momenta, beta, eps)
+        self.plan.momentum_normalize(grads, momenta, beta, eps, grad_scale=grad_scale)
         n0 = self.plan.last_launch_count()
         self.plan.gram_ns_batched(None, coeffs, steps)
         n1 = self.plan.last_launch_count()
@@ -176,13 +177,15 @@ class OwnerShardedStep:
             works = [dist.reduce(grad_flats[r], dst=r, op=dist.ReduceOp.SUM, group=self.group, async_op=True)
                      for r in range(self.world)]
             works[self.rank].wait()
-            grad_flats[self.rank].div_(self.world)
         if events is not None:
             events[1].record()
         grads = [b.view(grad_flats, i) for i in self.mine]
         weights = [b.view(weight_flats, i) for i in self.mine]
         kw = {} if out_o is None else {"out_o": out_o}
-        self.compute(grads, momenta, weights, beta=beta, lr=lr, eps=eps, coeffs=coeffs, steps=steps, **kw)
+        # the owner's bucket holds the sum of the ranks' gradients; the
+        # momentum pass scales it to the mean as it reads it
+        self.compute(grads, momenta, weights, beta=beta, lr=lr, eps=eps, coeffs=coeffs, steps=steps,
+                     grad_scale=1.0 / self.world, **kw)
         if events is not None:
             events[2].record()
         if self.world > 1:

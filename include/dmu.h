@@ -152,13 +152,18 @@ DMU_API dmu_status dmu_set_workspace(dmu_plan plan, void* dev_ptr, size_t bytes)
 /* Step 1 + the norm of step 3, for all matrices of the plan.
  *   grads[i]   : device pointer, rows*cols elements of the plan dtype.
  *   momenta[i] : device pointer, rows*cols fp32, updated in place
- *                (M <- beta*M + G).  momenta == NULL means "no state":
- *                M = G and nothing is written back.
+ *                (M <- beta*M + grad_scale*G).  momenta == NULL means "no
+ *                state": M = grad_scale*G and nothing is written back.
+ *   grad_scale : factor on the gradient, applied in the same pass (1 for
+ *                the plain update; 1/N turns the sum of N data-parallel
+ *                gradients into their mean without a separate pass).
+ * Errors: INVALID_ARG for a NULL grads array or pointer, eps < 0, or a
+ * non-finite beta or grad_scale; WORKSPACE; CUDA.
  * Writes the bf16 (or fp32) image of M and 1/(||M||_F + eps) for every
  * matrix into the workspace.  Source: DMuon page, section 1. */
 DMU_API dmu_status dmu_momentum_normalize(dmu_plan plan, const void* const* grads,
-                                  float* const* momenta, float beta, float eps,
-                                  void* stream);
+                                  float* const* momenta, float beta, float grad_scale,
+                                  float eps, void* stream);
 
 /* Steps 2-4: the Gram Newton-Schulz recursion, batched over all matrices.
  *   ptrs   : NULL to use the matrices left by dmu_momentum_normalize; or
@@ -213,9 +218,19 @@ DMU_API dmu_status dmu_debug_gram(dmu_plan plan, int which, int index, float* ou
  * Errors: NOT_PLANNED (no dmu_momentum_normalize yet), CUDA. */
 DMU_API dmu_status dmu_autotune(dmu_plan plan, const char* cache_path, void* stream);
 
-/* Current schedule of the plan: 1 = CTA pairs (256 x 256), 0 = single
- * CTAs (128 x 256), 2 = single CTAs (128 x 128); -1 for a NULL plan. */
+/* The plan's default tile schedule: 1 = CTA pairs (256 x 256), 0 = single
+ * CTAs (128 x 256), 2 = single CTAs (128 x 128); -1 for a NULL plan.
+ * Classes and buckets that dmu_autotune (or DMU_ONCHIP) gave their own
+ * schedule report it through the two calls below. */
 DMU_API int dmu_get_schedule(dmu_plan plan);
+
+/* Schedule of the Gram recursion of matrix `index`'s class (all matrices
+ * with its m): 0, 1, 2 as above, or 3 = the whole recursion on chip (one
+ * CTA per matrix, m <= 128, split-bf16 precision).  -1 for a bad argument. */
+DMU_API int dmu_get_gram_schedule(dmu_plan plan, int index);
+
+/* Tile schedule (0, 1, 2) of the final GEMM of matrix `index`'s bucket. */
+DMU_API int dmu_get_final_schedule(dmu_plan plan, int index);
 
 /* Number of kernel launches the last compute call enqueued. */
 DMU_API int dmu_last_launch_count(dmu_plan plan);

@@ -43,7 +43,7 @@ int main(void) {
   CHECK(dmu_workspace_bytes(NULL) == 0);
   CHECK(dmu_get_schedule(NULL) == -1);
   CHECK(dmu_set_workspace(NULL, NULL, 0) == DMU_ERR_INVALID_ARG);
-  CHECK(dmu_momentum_normalize(NULL, NULL, NULL, 0.9f, 1e-7f, NULL) == DMU_ERR_INVALID_ARG);
+  CHECK(dmu_momentum_normalize(NULL, NULL, NULL, 0.9f, 1.0f, 1e-7f, NULL) == DMU_ERR_INVALID_ARG);
   CHECK(dmu_apply_update(NULL, NULL, 0.02f, NULL, NULL) == DMU_ERR_INVALID_ARG);
   dmu_plan_destroy(NULL);
 

@@ -67,7 +67,7 @@ def test_argument_errors():
     assert lib.dmu_plan_create(p, 1, 0, 0, 0, None) == dmu.ERR_INVALID_ARG
     # calls on a NULL plan
     assert lib.dmu_set_workspace(None, None, 0) == dmu.ERR_INVALID_ARG
-    assert lib.dmu_momentum_normalize(None, None, None, 0.9, 1e-7, None) == dmu.ERR_INVALID_ARG
+    assert lib.dmu_momentum_normalize(None, None, None, 0.9, 1.0, 1e-7, None) == dmu.ERR_INVALID_ARG
     co = (ctypes.c_float * 3)(*dmu.QUINTIC)
     assert lib.dmu_gram_ns_batched(None, None, p, 1, ctypes.cast(co, ctypes.c_void_p), 5, None) == dmu.ERR_INVALID_ARG
     assert lib.dmu_apply_update(None, None, 0.02, None, None) == dmu.ERR_INVALID_ARG
@@ -111,7 +111,7 @@ def test_host_only_plan_layout_qwen7b():
     assert 50e9 < total < 60e9
     # no device: setting a workspace or computing fails cleanly
     assert lib.dmu_set_workspace(h, ctypes.c_void_p(256), total) == dmu.ERR_CUDA
-    assert lib.dmu_momentum_normalize(h, None, None, 0.9, 1e-7, None) == dmu.ERR_WORKSPACE
+    assert lib.dmu_momentum_normalize(h, None, None, 0.9, 1.0, 1e-7, None) == dmu.ERR_WORKSPACE
     lib.dmu_plan_destroy(h)
 
 
@@ -204,3 +204,28 @@ def test_demuon_mixing_matrices_match_the_oracle():
         for n in (1, 2, 3, 4, 6, 8, 16):
             np.testing.assert_allclose(np.array(demuon.mixing_matrix(topo, n)), odm.mixing_matrix(topo, n),
                                        rtol=0, atol=1e-15)
+
+
+def test_per_class_schedule_queries(monkeypatch):
+    """Planning alone (no device needed): with DMU_ONCHIP=1 the split-bf16
+    classes with m <= 128 start on the on-chip schedule (3), the others and
+    every final GEMM on the plan default (CTA pairs, 1)."""
+    lib = dmu.load()
+    monkeypatch.setenv("DMU_ONCHIP", "1")
+    monkeypatch.delenv("DMU_SCHEDULE", raising=False)
+    monkeypatch.delenv("DMU_CTA_PAIR", raising=False)
+    pairs = [(128, 512), (512, 128), (256, 1024), (64, 64), (2048, 1024)]
+    st, h, keep = _create(pairs)
+    assert st == dmu.OK
+    assert [lib.dmu_get_gram_schedule(h, i) for i in range(5)] == [3, 3, 1, 3, 1]
+    assert [lib.dmu_get_final_schedule(h, i) for i in range(5)] == [1] * 5
+    assert lib.dmu_get_gram_schedule(h, 5) == -1 and lib.dmu_get_final_schedule(h, -1) == -1
+    assert lib.dmu_get_gram_schedule(None, 0) == -1
+    lib.dmu_plan_destroy(h)
+    st, h, keep = _create(pairs, prec=1)  # FAST precision: nothing runs on chip
+    assert st == dmu.OK and lib.dmu_get_gram_schedule(h, 0) == 1
+    lib.dmu_plan_destroy(h)
+    monkeypatch.setenv("DMU_ONCHIP", "0")
+    st, h, keep = _create(pairs)
+    assert st == dmu.OK and lib.dmu_get_gram_schedule(h, 0) == 1
+    lib.dmu_plan_destroy(h)

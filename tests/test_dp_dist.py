@@ -65,9 +65,10 @@ class OracleCompute:
         self.indices = list(indices)
         self.calls = []
 
-    def __call__(self, grads, momenta, weights, *, beta, lr, eps, coeffs, steps):
+    def __call__(self, grads, momenta, weights, *, beta, lr, eps, coeffs, steps, grad_scale=1.0):
         self.calls.append(list(self.indices))
         for g, m, w in zip(grads, momenta, weights):
+            g = g * np.float32(grad_scale)  # fp32 product, as the momentum pass forms it
             m_new, _, w_new = gram_ns.muon_step(w.double().numpy(), m.double().numpy(), g.double().numpy(),
                                                 beta=beta, lr=lr, eps=eps, coeffs=coeffs, steps=steps)
             m.copy_(torch.from_numpy(m_new))
@@ -81,7 +82,8 @@ def _expected(world):
         s = np.zeros(SHAPES[i], dtype=np.float32)
         for r in range(world):
             s = s + _grad(i, r)
-        mean = (s / np.float32(world)).astype(np.float32)
+        # the mean as the owner's momentum pass forms it: the fp32 sum times 1/N in fp32
+        mean = (s * np.float32(1.0 / world)).astype(np.float32)
         m_new, _, w_new = gram_ns.muon_step(_weight(i).astype(np.float64), _momentum0(i).astype(np.float64),
                                             mean.astype(np.float64), beta=BETA, lr=LR, eps=EPS)
         out_w.append(w_new.astype(np.float32))
