@@ -60,7 +60,8 @@ def executed_flops(shapes, k=K_STEPS, tile=256):
     * 4K - 3 symmetric products over the same tiles: one scaled-fp16 MMA per
       K slice for m >= 1024 (F16 class), three bf16 MMAs (hi.hi + hi.lo +
       lo.hi) below (SPLIT3).
-    * The final: hi and lo of P, two MMAs over every m x n tile.
+    * The final over every m x n tile: one fp16 MMA per K slice for the F16
+      class (P as one fp16 operand), two below (P as an fp16 hi/lo pair).
     Diagonal tiles are computed whole.  Tiles are counted as full 256 x 256
     blocks; ragged edges are ignored."""
     tot = 0.0
@@ -72,7 +73,7 @@ def executed_flops(shapes, k=K_STEPS, tile=256):
         terms = 1 if m >= 1024 else 3
         tot += 2.0 * upper * n                              # SYRK
         tot += (4 * k - 3) * terms * 2.0 * upper * mm       # products, K = m
-        tot += 2 * 2.0 * m * m * n                          # final, two terms
+        tot += (1 if m >= 1024 else 2) * 2.0 * m * m * n    # final
     return tot
 
 
@@ -82,14 +83,15 @@ def gemm_alg_bytes(shapes, k=K_STEPS):
     m x m matrices, m^2/2 elements; 16-bit operands, 32-bit hi/lo pairs):
     SYRK reads Mb (2 B/elem) and writes G (4 B); each of the 4K-3 symmetric
     products reads two 16-bit operands and a pair Cin and writes a pair;
-    the final reads the P pair and Mb and reads and writes W (bf16)."""
+    the final reads P (one fp16 operand for m >= 1024, an fp16 pair below)
+    and the image, and reads and writes W (bf16)."""
     tot = 0.0
     for r, c in shapes:
         m, e = min(r, c), float(r) * c
         half = 0.5 * m * m
         tot += 2 * e + 4 * half                 # SYRK
         tot += (4 * k - 3) * 12 * half          # products
-        tot += 4 * half + 6 * e                 # final + update
+        tot += (2 if m >= 1024 else 4) * half + 6 * e  # final + update
     return tot
 
 
@@ -125,10 +127,12 @@ def captured_traffic(workload_name):
     return cap["dram_bytes_per_step"] / cap["launches_per_step"]
 
 
-def momentum_bytes(shapes, grad_bytes=2):
-    """HBM bytes of the momentum pass: read G and M, write M and Mb."""
+def momentum_bytes(shapes, grad_bytes=2, image16=False):
+    """HBM bytes of the momentum phase: read G and M, write M and the bf16
+    image; with ``image16`` also the in-place conversion of the image to
+    scaled fp16 (read 2, write 2)."""
     e = sum(r * c for r, c in shapes)
-    return e * (grad_bytes + 4 + 4 + 2)
+    return e * (grad_bytes + 4 + 4 + 2 + (4 if image16 else 0))
 
 
 def schedule_summary(sch):
@@ -728,7 +732,7 @@ def main():
     achieved_tf = flops / tc_s / 1e12
     peak_tf = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     mom_s = t_mom / K / 1e3
-    mom_gbs = momentum_bytes(w.shapes) / mom_s / 1e9
+    mom_gbs = momentum_bytes(w.shapes, image16=w.dtype == "bf16") / mom_s / 1e9
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
 
     # End to end through the public API with host buffers: every step copies
@@ -834,7 +838,8 @@ def main():
                          "kernel": "k_gemm_tc2 (all Gram-space and final launches)",
                          "peak_kind": f"{peak_kind} cuBLAS bf16 GEMM, sustained (achievable)",
                          "frac_of_datasheet_dense_bf16": round(achieved_tf / DATASHEET_DENSE_BF16_TFLOPS, 4)},
-            "hbm_kernel": {"kernel": "k_momentum", "achieved": round(mom_gbs, 1), "peak": hbm,
+            "hbm_kernel": {"kernel": "k_momentum + k_norm_finalize + k_image16 (the momentum phase)",
+                           "achieved": round(mom_gbs, 1), "peak": hbm,
                            "unit": "GB/s", "frac": round(mom_gbs / hbm, 4), "peak_kind": peak_kind},
             "gpu_launches": launches,
             "status_word": status,

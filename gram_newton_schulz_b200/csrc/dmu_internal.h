@@ -3,6 +3,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -158,10 +159,13 @@ cudaError_t launch_momentum(const MomChunk* chunks, int nchunks, const MomMat* m
                             void* mb, int mb_f32, float beta, float gscale, float* partial,
                             int vec_ok, int num_sms, cudaStream_t s);
 cudaError_t launch_norm_finalize(const MomMat* mats, int nmats, const float* partial,
-                                 float eps, float* inv, unsigned int* status, cudaStream_t s);
+                                 float eps, float* inv, float* iscale, float* inv_img, unsigned int* status,
+                                 cudaStream_t s);
+cudaError_t launch_image16(const MomChunk* chunks, int nchunks, const MomMat* mats, void* mb, const float* iscale,
+                           int vec_ok, int num_sms, cudaStream_t s);
 cudaError_t launch_simt_gemm(const SimtProblem& p, cudaStream_t s);
-cudaError_t launch_identity_bf16(__nv_bfloat16* hi, __nv_bfloat16* lo, int count, int m,
-                                 long long ld, long long mat_stride, cudaStream_t s);
+cudaError_t launch_identity16(void* hi, void* lo, int count, int m, long long ld, long long mat_stride, int f16,
+                              cudaStream_t s);
 cudaError_t launch_identity_f32(float* p, int count, int m, long long ld, long long mat_stride,
                                 cudaStream_t s);
 // Test-hook conversions; `half` reads a half-stored symmetric matrix
@@ -181,7 +185,7 @@ namespace dmu {
 // One shape bucket whose whole Gram recursion runs in one CTA per matrix
 // (SYRK from the momentum image, K steps of the R-form recursion with
 // G/T, R and P held in shared memory as bf16 hi/lo pairs); only the final
-// P is written, as a bf16 hi/lo pair into the class's P slot.
+// P is written, as an fp16 hi/lo pair into the class's final-P area.
 constexpr int ONCHIP_MAX_M = 128;
 struct OnchipProblem {
   int count;            // matrices of the bucket
@@ -190,8 +194,8 @@ struct OnchipProblem {
   int map;              // image tensor map (K-major box 64 x 128, or MN-major 64 x 64)
   int inv_base;         // index of the bucket's first matrix in `inv`
   int mat_begin;        // first global matrix index of this problem
-  __nv_bfloat16* p_hi;  // final P of the bucket's first matrix (hi part)
-  __nv_bfloat16* p_lo;
+  __half* p_hi;         // final P of the bucket's first matrix, fp16 hi/lo pair
+  __half* p_lo;
   long long ld, mat_stride;
 };
 

@@ -1112,11 +1112,14 @@ cudaError_t gemm_tc_configure() {
   if ((e = configure_one<1, 1, KIND_TF32, 128>()) != cudaSuccess) return e;
   if ((e = configure_one<1, 1, KIND_F16, 256>()) != cudaSuccess) return e;
   if ((e = configure_one<1, 1, KIND_F16, 128>()) != cudaSuccess) return e;
+  if ((e = configure_one<2, 1, KIND_F16, 256>()) != cudaSuccess) return e;
+  if ((e = configure_one<2, 1, KIND_F16, 128>()) != cudaSuccess) return e;
   if ((e = configure_two<1, 1, KIND_BF16>()) != cudaSuccess) return e;
   if ((e = configure_two<2, 1, KIND_BF16>()) != cudaSuccess) return e;
   if ((e = configure_two<2, 2, KIND_BF16>()) != cudaSuccess) return e;
   if ((e = configure_two<1, 1, KIND_TF32>()) != cudaSuccess) return e;
   if ((e = configure_two<1, 1, KIND_F16>()) != cudaSuccess) return e;
+  if ((e = configure_two<2, 1, KIND_F16>()) != cudaSuccess) return e;
   return cudaSuccess;
 }
 
@@ -1154,6 +1157,7 @@ cudaError_t launch_gemm_tc2(const GemmParams& p, int na, int nb, int kind, int n
   }
   if (kind == KIND_F16) {
     if (na == 1 && nb == 1) return launch_two<1, 1, KIND_F16>(p, num_sms, s);
+    if (na == 2 && nb == 1) return launch_two<2, 1, KIND_F16>(p, num_sms, s);
     return cudaErrorInvalidValue;
   }
   if (na == 1 && nb == 1) return launch_two<1, 1, KIND_BF16>(p, num_sms, s);
@@ -1171,6 +1175,7 @@ cudaError_t launch_gemm_tc(const GemmParams& p, int na, int nb, int kind, int nu
   }
   if (kind == KIND_F16) {
     if (na == 1 && nb == 1) return launch_one<1, 1, KIND_F16>(p, num_sms, tbn, s);
+    if (na == 2 && nb == 1) return launch_one<2, 1, KIND_F16>(p, num_sms, tbn, s);
     return cudaErrorInvalidValue;
   }
   if (na == 1 && nb == 1) return launch_one<1, 1, KIND_BF16>(p, num_sms, tbn, s);

@@ -14,8 +14,10 @@
 //           T = a G + R G          (k < K-1)
 //           P' = a P + R P         (k >= 1)
 //           G' = a T + T R         (k < K-1)
-//   only P_K leaves the SM: a bf16 hi/lo pair in the class's P slot, where
-//   the final O = P X0 GEMM (fused with the weight update) reads it.
+//   only P_K leaves the SM: an fp16 hi/lo pair in the class's final-P area,
+//   where the final O = P X0 GEMM (fused with the weight update) reads it.
+// X is the fp16 image 2^e M (scale folded into `inv`), so the Gram matrix
+// is one kind::f16 MMA per K slice on fp16 operands.
 //
 // Precision is the split-bf16 class of the staged path (three MMAs per
 // product: hi*hi + hi*lo + lo*hi), with the same K order, the same epilogue
@@ -110,8 +112,8 @@ struct EpiArgs {
   int cin;        // buffer or -1
   int out;        // buffer, or -1 for the global P slot
   int out2;       // buffer, -1 none, -2 the global P slot
-  __nv_bfloat16* g_hi;  // global P of this matrix (out == -1 or out2 == -2)
-  __nv_bfloat16* g_lo;
+  __half* g_hi;  // global P of this matrix, fp16 pair (out == -1 or out2 == -2)
+  __half* g_lo;
   long long ld;
 };
 
@@ -135,9 +137,28 @@ __device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
   }
 }
 
+__device__ __forceinline__ void split8_h(const float* v, uint4& hi, uint4& lo) {
+  __half2* h = reinterpret_cast<__half2*>(&hi);
+  __half2* l = reinterpret_cast<__half2*>(&lo);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const __half h0 = __float2half_rn(v[2 * q]);
+    const __half h1 = __float2half_rn(v[2 * q + 1]);
+    h[q] = __halves2half2(h0, h1);
+    l[q] = __halves2half2(__float2half_rn(v[2 * q] - __half2float(h0)),
+                          __float2half_rn(v[2 * q + 1] - __half2float(h1)));
+  }
+}
+
+__device__ __forceinline__ void st_pair_h(__half* hi, __half* lo, long long o, float v) {
+  const __half h = __float2half_rn(v);
+  hi[o] = h;
+  lo[o] = __float2half_rn(v - __half2float(h));
+}
+
 // Stores of one chunk (row i, columns col0 .. col0 + 15, only j < m) to a
-// shared-memory pair `buf` or to a global pair (hi, lo, row stride ld).
-__device__ __forceinline__ void store_chunk(uint8_t* buf, __nv_bfloat16* ghi, __nv_bfloat16* glo, long long ld,
+// shared-memory bf16 pair `buf` or to a global fp16 pair (hi, lo, stride ld).
+__device__ __forceinline__ void store_chunk(uint8_t* buf, __half* ghi, __half* glo, long long ld,
                                             int m, int i, int col0, const float (&v)[OC_CW]) {
   const bool full = col0 + OC_CW <= m;
   const bool all_upper = i <= col0;
@@ -145,12 +166,13 @@ __device__ __forceinline__ void store_chunk(uint8_t* buf, __nv_bfloat16* ghi, __
 #pragma unroll
     for (int q = 0; q < OC_CW / 8; ++q) {
       uint4 h, l;
-      split8(v + 8 * q, h, l);
       if (buf) {
+        split8(v + 8 * q, h, l);
         const uint32_t o = oc_off(i, col0 + 8 * q);
         *reinterpret_cast<uint4*>(buf + o) = h;
         *reinterpret_cast<uint4*>(buf + OC_PART + o) = l;
       } else {
+        split8_h(v + 8 * q, h, l);
         *reinterpret_cast<uint4*>(ghi + i * ld + col0 + 8 * q) = h;
         *reinterpret_cast<uint4*>(glo + i * ld + col0 + 8 * q) = l;
       }
@@ -160,13 +182,10 @@ __device__ __forceinline__ void store_chunk(uint8_t* buf, __nv_bfloat16* ghi, __
     for (int c = 0; c < OC_CW; ++c) {
       const int j = col0 + c;
       if (j < m && i <= j) {
-        if (buf) {
+        if (buf)
           st_pair_smem(buf, i, j, v[c]);
-        } else {
-          const __nv_bfloat16 h = __float2bfloat16_rn(v[c]);
-          ghi[i * ld + j] = h;
-          glo[i * ld + j] = __float2bfloat16_rn(v[c] - bf(h));
-        }
+        else
+          st_pair_h(ghi, glo, i * ld + j, v[c]);
       }
     }
   }
@@ -175,13 +194,10 @@ __device__ __forceinline__ void store_chunk(uint8_t* buf, __nv_bfloat16* ghi, __
   for (int c = 0; c < OC_CW; ++c) {
     const int j = col0 + c;
     if (j < m && i < j) {
-      if (buf) {
+      if (buf)
         st_pair_smem(buf, j, i, v[c]);
-      } else {
-        const __nv_bfloat16 h = __float2bfloat16_rn(v[c]);
-        ghi[j * ld + i] = h;
-        glo[j * ld + i] = __float2bfloat16_rn(v[c] - bf(h));
-      }
+      else
+        st_pair_h(ghi, glo, j * ld + i, v[c]);
     }
   }
 }
@@ -392,7 +408,7 @@ __global__ void __launch_bounds__(OC_THREADS, 1) k_gram_onchip(const __grid_cons
         // G' of step K-2, whose epilogue was waited for before step K-1)
         const int nk = (pr.n + 63) / 64;
         const uint32_t mn = pr.tall ? 1u : 0u;
-        const uint32_t idesc = ptx::make_idesc(128, 128, mn, mn, 1);
+        const uint32_t idesc = ptx::make_idesc(128, 128, mn, mn, 0);  // fp16 image operands
         const uint64_t hi_d = mn ? ptx::make_sw128_desc(0u, 8192u, 1024u) : ptx::make_sw128_desc(0u, 16u, 1024u);
         const uint32_t ks = mn ? 2048u : 32u;
         uint32_t accumulate = 0;
@@ -475,8 +491,8 @@ __global__ void __launch_bounds__(OC_THREADS, 1) k_gram_onchip(const __grid_cons
       const OnchipProblem& pr = p.prob[find_prob(p, t)];
       const int mat = t - pr.mat_begin;
       const int m = pr.m;
-      __nv_bfloat16* g_hi = pr.p_hi + mat * pr.mat_stride;
-      __nv_bfloat16* g_lo = pr.p_lo + mat * pr.mat_stride;
+      __half* g_hi = pr.p_hi + mat * pr.mat_stride;
+      __half* g_lo = pr.p_lo + mat * pr.mat_stride;
       const float s = p.inv[pr.inv_base + mat];
       // ---- G0 = s^2 X X^T
       if (!wait_acc(0)) break;

@@ -171,9 +171,13 @@ __global__ void __launch_bounds__(256, 3) k_momentum(const MomChunk* __restrict_
   }
 }
 
+// Also the power-of-two scale 2^e of the fp16 image (when `iscale` is
+// given): 2^e ||M||_F <= 2^15, so every entry of 2^e M is below fp16's
+// largest finite value, and entries down to ||M||_F 2^-29 stay normal;
+// inv_img = inv 2^-e reads the scaled image back as X0.
 __global__ void k_norm_finalize(const MomMat* __restrict__ mats, int nmats,
                                 const float* __restrict__ partial, float eps, float* __restrict__ inv,
-                                unsigned int* status) {
+                                float* __restrict__ iscale, float* __restrict__ inv_img, unsigned int* status) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= nmats) return;
@@ -186,8 +190,63 @@ __global__ void k_norm_finalize(const MomMat* __restrict__ mats, int nmats,
   if (lane == 0) {
     const double nrm = sqrt(s);
     if (!isfinite(s)) atomicOr(status, DMU_FLAG_NONFINITE);
-    inv[warp] = (float)(1.0 / (nrm + (double)eps));
+    const float iv = (float)(1.0 / (nrm + (double)eps));
+    inv[warp] = iv;
+    if (iscale) {
+      int e = 0;
+      if (nrm > 0.0 && isfinite(nrm)) e = 15 - (int)ceil(log2(nrm));
+      e = max(-100, min(100, e));
+      iscale[warp] = ldexpf(1.f, e);
+      inv_img[warp] = ldexpf(iv, -e);
+    }
   }
+}
+
+// The bf16 image of M, converted in place to fp16 scaled by 2^e per matrix
+// (exact for every entry in fp16's normal range; the fp16 image feeds the
+// kind::f16 MMAs of the Gram matrix and of the final product).  Same chunk
+// walk as the momentum pass.
+__global__ void __launch_bounds__(256) k_image16(const MomChunk* __restrict__ chunks, int nchunks,
+                                                 const MomMat* __restrict__ mats, void* __restrict__ mb,
+                                                 const float* __restrict__ iscale, int vec) {
+  for (int c = blockIdx.x; c < nchunks; c += gridDim.x) {
+    const MomChunk ch = chunks[c];
+    const MomMat mm = mats[ch.slot];
+    const float sc = iscale[ch.slot];
+    if (vec) {
+      uint4* base = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(mb) + mm.mb_off + ch.start);
+      const int nv = ch.len >> 3;
+      for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+        uint4 u = base[v];
+        __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+        uint4 o;
+        __half2* oh = reinterpret_cast<__half2*>(&o);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __bfloat1622float2(h[q]);
+          oh[q] = __floats2half2_rn(f.x * sc, f.y * sc);
+        }
+        base[v] = o;
+      }
+    } else {
+      for (int e = threadIdx.x; e < ch.len; e += blockDim.x) {
+        const long long idx = ch.start + e;
+        const long long row = idx / mm.cols, col = idx - row * mm.cols;
+        __nv_bfloat16* p = reinterpret_cast<__nv_bfloat16*>(mb) + mm.mb_off + row * mm.ldc + col;
+        const __half hv = __float2half_rn(__bfloat162float(*p) * sc);
+        *reinterpret_cast<__half*>(p) = hv;
+      }
+    }
+  }
+}
+
+cudaError_t launch_image16(const MomChunk* chunks, int nchunks, const MomMat* mats, void* mb, const float* iscale,
+                           int vec_ok, int num_sms, cudaStream_t s) {
+  if (nchunks <= 0) return cudaSuccess;
+  int grid = num_sms * 8;
+  if (grid > nchunks) grid = nchunks;
+  k_image16<<<grid, 256, 0, s>>>(chunks, nchunks, mats, mb, iscale, vec_ok);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_momentum(const MomChunk* chunks, int nchunks, const MomMat* mats,
@@ -207,24 +266,27 @@ cudaError_t launch_momentum(const MomChunk* chunks, int nchunks, const MomMat* m
 }
 
 cudaError_t launch_norm_finalize(const MomMat* mats, int nmats, const float* partial, float eps,
-                                 float* inv, unsigned int* status, cudaStream_t s) {
+                                 float* inv, float* iscale, float* inv_img, unsigned int* status, cudaStream_t s) {
   if (nmats <= 0) return cudaSuccess;
   const int threads = 256, per = threads / 32;
-  k_norm_finalize<<<(nmats + per - 1) / per, threads, 0, s>>>(mats, nmats, partial, eps, inv, status);
+  k_norm_finalize<<<(nmats + per - 1) / per, threads, 0, s>>>(mats, nmats, partial, eps, inv, iscale, inv_img,
+                                                             status);
   return cudaGetLastError();
 }
 
 // ------------------------------------------------------------- helpers
-__global__ void k_identity_bf16(__nv_bfloat16* hi, __nv_bfloat16* lo, int count, int m, long long ld,
-                                long long mat_stride) {
+// Identity as a 16-bit hi/lo pair; `one` is the bit pattern of 1.0 in the
+// pair's format (0x3F80 bf16, 0x3C00 fp16).
+__global__ void k_identity16(uint16_t* hi, uint16_t* lo, int count, int m, long long ld, long long mat_stride,
+                             uint16_t one) {
   const long long total = (long long)count * m * m;
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
        e += (long long)gridDim.x * blockDim.x) {
     const long long mat = e / ((long long)m * m);
     const long long r = (e / m) % m, c = e % m;
     const long long o = mat * mat_stride + r * ld + c;
-    hi[o] = __float2bfloat16_rn(r == c ? 1.f : 0.f);
-    lo[o] = __float2bfloat16_rn(0.f);
+    hi[o] = r == c ? one : (uint16_t)0;
+    lo[o] = 0;
   }
 }
 
@@ -283,9 +345,11 @@ static int grid_for(long long total) {
   return (int)g;
 }
 
-cudaError_t launch_identity_bf16(__nv_bfloat16* hi, __nv_bfloat16* lo, int count, int m, long long ld,
-                                 long long mat_stride, cudaStream_t s) {
-  k_identity_bf16<<<grid_for((long long)count * m * m), 256, 0, s>>>(hi, lo, count, m, ld, mat_stride);
+cudaError_t launch_identity16(void* hi, void* lo, int count, int m, long long ld, long long mat_stride, int f16,
+                              cudaStream_t s) {
+  k_identity16<<<grid_for((long long)count * m * m), 256, 0, s>>>(
+      reinterpret_cast<uint16_t*>(hi), reinterpret_cast<uint16_t*>(lo), count, m, ld, mat_stride,
+      f16 ? (uint16_t)0x3C00 : (uint16_t)0x3F80);
   return cudaGetLastError();
 }
 cudaError_t launch_identity_f32(float* p, int count, int m, long long ld, long long mat_stride,

@@ -60,11 +60,11 @@ struct GClass {
   int64_t m = 0, ldg = 0;
   int count = 0;
   size_t off = 0;     // byte offset in the workspace
-  size_t off_pf = 0;  // TF32 classes: bf16 hi/lo pair of the final P
+  size_t off_pf = 0;  // all but F16 classes: the final P as an fp16 hi/lo pair
   int prec = DMU_PREC_FAST;
   int kind = KIND_BF16;
   int map = -1;       // TMA map over the Gram slots (bf16 pairs or fp32)
-  int map_pf = -1;    // TF32 classes: bf16 map over the final-P pair
+  int map_pf = -1;    // all but F16 classes: fp16 map over the final-P pair
   // Half storage (all but TF32 classes): symmetric Gram-space matrices keep
   // only their upper 256 x 256 blocks; lower blocks are read transposed
   // through MN-major maps (64 x 64 boxes).
@@ -126,7 +126,8 @@ struct dmu_plan_s {
   bool vec_shapes = true;
   size_t esize = 2;
   // workspace layout (bytes)
-  size_t off_status = 0, off_inv = 0, off_partial = 0, off_chunks = 0, off_mats = 0, off_tbl = 0,
+  size_t off_status = 0, off_inv = 0, off_iscale = 0, off_invimg = 0, off_partial = 0, off_chunks = 0,
+         off_mats = 0, off_tbl = 0,
          off_mb = 0, off_gram = 0, total = 0;
   char* ws = nullptr;
   size_t ws_bytes = 0;
@@ -153,6 +154,11 @@ struct dmu_plan_s {
 
   unsigned int* status_dev() const { return reinterpret_cast<unsigned int*>(ws + off_status); }
   float* inv_dev() const { return reinterpret_cast<float*>(ws + off_inv); }
+  // bf16 plans: per-matrix scale 2^e of the fp16 image, and inv * 2^-e
+  float* iscale_dev() const { return reinterpret_cast<float*>(ws + off_iscale); }
+  float* invimg_dev() const { return reinterpret_cast<float*>(ws + off_invimg); }
+  // the scale the tensor-core kernels apply to image products
+  const float* inv_kernel() const { return dtype == DMU_BF16 ? invimg_dev() : inv_dev(); }
   float* partial_dev() const { return reinterpret_cast<float*>(ws + off_partial); }
   const MomChunk* chunks_dev() const { return reinterpret_cast<const MomChunk*>(ws + off_chunks); }
   const MomMat* mats_dev() const { return reinterpret_cast<const MomMat*>(ws + off_mats); }
@@ -167,8 +173,8 @@ struct dmu_plan_s {
     const GClass& g = classes[c];
     return reinterpret_cast<float*>(ws + g.off) + (size_t)slot * g.count * g.m * g.ldg;
   }
-  // TF32 classes: half 0 = hi, 1 = lo of the final P
-  __nv_bfloat16* pf_bf16(int c, int half) const {
+  // final P of non-F16 classes as an fp16 pair: half 0 = hi, 1 = lo
+  __nv_bfloat16* pf_bf16(int c, int half) const {  // 16-bit storage; the bits are fp16
     const GClass& g = classes[c];
     return reinterpret_cast<__nv_bfloat16*>(ws + g.off_pf) + (size_t)half * g.count * g.m * g.ldg;
   }
@@ -296,6 +302,10 @@ void prec_shape(int prec, int* na, int* nb, int* terms, int* kind) {
   }
 }
 
+// Output slot meaning "the final P, as an fp16 hi/lo pair in the class's
+// final-P area" (classes other than F16, whose P slots are fp16 already).
+constexpr int OUT_PF = -2;
+
 // A Gram-space product over all matrices of class c:
 //   out = alpha * (A B) + beta * Cin + gamma * I   [, out2 = out + gamma2 * I]
 Prob gram_prob(dmu_plan p, int c, int a_slot, int b_slot, int terms, float alpha, float beta,
@@ -325,9 +335,19 @@ Prob gram_prob(dmu_plan p, int c, int a_slot, int b_slot, int terms, float alpha
     g.cin_hi = p->slot_bf16(c, cin_slot);
     g.cin_lo = p->slot_bf16(c, cin_slot + 1);
   }
-  g.out_hi = p->slot_bf16(c, out_slot);
-  g.out_lo = out_lo ? p->slot_bf16(c, out_slot + 1) : nullptr;
-  if (out2_slot >= 0) {
+  if (out_slot == OUT_PF) {
+    g.out_fmt = FMT_PAIR_H;
+    g.out_hi = p->pf_bf16(c, 0);
+    g.out_lo = p->pf_bf16(c, 1);
+  } else {
+    g.out_hi = p->slot_bf16(c, out_slot);
+    g.out_lo = out_lo ? p->slot_bf16(c, out_slot + 1) : nullptr;
+  }
+  if (out2_slot == OUT_PF) {
+    g.out2_fmt = FMT_PAIR_H;
+    g.out2_hi = p->pf_bf16(c, 0);
+    g.out2_lo = p->pf_bf16(c, 1);
+  } else if (out2_slot >= 0) {
     g.out2_hi = p->slot_bf16(c, out2_slot);
     g.out2_lo = p->slot_bf16(c, out2_slot + 1);
   }
@@ -341,13 +361,12 @@ Prob gram_prob(dmu_plan p, int c, int a_slot, int b_slot, int terms, float alpha
   return pr;
 }
 
-// TF32 classes: fp32 slots; out_slot == OUT_PF writes the final P as a
-// bf16 hi/lo pair (the operand of the final bf16 GEMM).
-constexpr int OUT_PF = -2;
+// TF32 classes: fp32 slots; out_slot == OUT_PF writes the final P as an
+// fp16 hi/lo pair (the operand of the final fp16 GEMM).
 
 void set_f32_out(dmu_plan p, int c, int slot, int* fmt, float** f, __nv_bfloat16** hi, __nv_bfloat16** lo) {
   if (slot == OUT_PF) {
-    *fmt = FMT_PAIR;
+    *fmt = FMT_PAIR_H;
     *hi = p->pf_bf16(c, 0);
     *lo = p->pf_bf16(c, 1);
   } else if (slot >= 0) {
@@ -394,12 +413,7 @@ Prob gram_prob_f32(dmu_plan p, int c, int a_slot, int b_slot, float alpha, float
 float half_slot_scale(int slot) { return slot >= SLOT_PA_HI ? 1.f : 256.f; }
 
 void set_h_out(dmu_plan p, int c, int slot, int* fmt, __nv_bfloat16** hi, __nv_bfloat16** lo, float* scale) {
-  if (slot == OUT_PF) {
-    *fmt = FMT_PAIR;
-    *hi = p->pf_bf16(c, 0);
-    *lo = p->pf_bf16(c, 1);
-    *scale = 1.f;
-  } else if (slot >= 0) {
+  if (slot >= 0) {
     *fmt = FMT_PAIR_H;
     *hi = p->slot_bf16(c, slot);  // fp16 bits; same element size as bf16
     *lo = p->slot_bf16(c, slot + 1);
@@ -464,11 +478,11 @@ Prob product(dmu_plan p, int c, Product what, int k, bool last, const float co[3
       case PROD_R:
         // R is only ever an MMA operand (hi): its lo half is not stored
         return gram_prob_h(p, c, SLOT_G_HI, SLOT_G_HI, co[2], co[1], SLOT_G_HI, SLOT_R_HI,
-                           k == 0 ? (last ? OUT_PF : SLOT_PA_HI) : -1, co[0], false);
+                           k == 0 ? SLOT_PA_HI : -1, co[0], false);
       case PROD_T:
         return gram_prob_h(p, c, SLOT_R_HI, SLOT_G_HI, 1.f, co[0], SLOT_G_HI, SLOT_T_HI, -1, 0.f);
       case PROD_P:
-        return gram_prob_h(p, c, SLOT_R_HI, hin, 1.f, co[0], hin, last ? OUT_PF : hout, -1, 0.f);
+        return gram_prob_h(p, c, SLOT_R_HI, hin, 1.f, co[0], hin, hout, -1, 0.f);
       case PROD_G:
       default:
         return gram_prob_h(p, c, SLOT_T_HI, SLOT_R_HI, 1.f, co[0], SLOT_T_HI, SLOT_G_HI, -1, 0.f);
@@ -495,13 +509,13 @@ Prob product(dmu_plan p, int c, Product what, int k, bool last, const float co[3
   switch (what) {
     case PROD_R:
       return gram_prob(p, c, SLOT_G_HI, SLOT_G_HI, terms, co[2], co[1], SLOT_G_HI, SLOT_R_HI, r_lo,
-                       k == 0 ? PA : -1, co[0]);
+                       k == 0 ? (last ? OUT_PF : PA) : -1, co[0]);
     case PROD_T:
       return gram_prob(p, c, SLOT_R_HI, SLOT_G_HI, terms, 1.f, co[0], SLOT_G_HI, SLOT_T_HI, true, -1, 0.f);
     case PROD_P:
       if (gc.prec == DMU_PREC_SPLIT2)
-        return gram_prob(p, c, pin, SLOT_R_HI, terms, 1.f, co[0], pin, pout, true, -1, 0.f);
-      return gram_prob(p, c, SLOT_R_HI, pin, terms, 1.f, co[0], pin, pout, true, -1, 0.f);
+        return gram_prob(p, c, pin, SLOT_R_HI, terms, 1.f, co[0], pin, last ? OUT_PF : pout, true, -1, 0.f);
+      return gram_prob(p, c, SLOT_R_HI, pin, terms, 1.f, co[0], pin, last ? OUT_PF : pout, true, -1, 0.f);
     case PROD_G:
     default:
       return gram_prob(p, c, SLOT_T_HI, SLOT_R_HI, terms, 1.f, co[0], SLOT_T_HI, SLOT_G_HI, true, -1, 0.f);
@@ -541,7 +555,7 @@ dmu_status run_onchip(dmu_plan p, const float co[3], int steps, int p_final, cud
   int nmaps = 0;
   auto flush = [&]() -> dmu_status {
     if (op.nprob == 0) return DMU_OK;
-    op.inv = p->inv_dev();
+    op.inv = p->inv_kernel();
     op.a = co[0];
     op.b = co[1];
     op.c = co[2];
@@ -573,9 +587,9 @@ dmu_status run_onchip(dmu_plan p, const float co[3], int steps, int p_final, cud
     q.mat_begin = op.total;
     op.total += b.count;
     const size_t moff = (size_t)b.cls_off * gc.m * gc.ldg;
-    const int hi = p_final == 0 ? SLOT_PA_HI : SLOT_PB_HI;
-    q.p_hi = p->slot_bf16(b.cls, hi) + moff;
-    q.p_lo = p->slot_bf16(b.cls, hi + 1) + moff;
+    (void)p_final;  // the final P goes to the class's fp16 final-P area
+    q.p_hi = reinterpret_cast<__half*>(p->pf_bf16(b.cls, 0) + moff);
+    q.p_lo = reinterpret_cast<__half*>(p->pf_bf16(b.cls, 1) + moff);
     q.ld = gc.ldg;
     q.mat_stride = gc.m * gc.ldg;
   }
@@ -610,7 +624,7 @@ dmu_status gram_bf16(dmu_plan p, const float co[3], int steps, cudaStream_t s) {
     g.epi = EPI_GRAM;
     g.alpha_mode = ALPHA_INV2;
     g.alpha = 1.f;
-    g.inv = p->inv_dev();
+    g.inv = p->inv_kernel();
     g.inv_base = b.first_slot;
     const size_t moff = (size_t)b.cls_off * gc.m * gc.ldg;
     if (gc.kind == KIND_TF32) {
@@ -638,7 +652,7 @@ dmu_status gram_bf16(dmu_plan p, const float co[3], int steps, cudaStream_t s) {
     for (size_t i = 0; i < syrk.size(); ++i)
       if (syrk_sched[i] == sched) group.push_back(syrk[i]);
     if (group.empty()) continue;
-    st = run_tc(p, group, 1, 1, KIND_BF16, sched, s);
+    st = run_tc(p, group, 1, 1, KIND_F16, sched, s);  // the fp16 image of X
     if (st != DMU_OK) return st;
   }
 
@@ -646,10 +660,12 @@ dmu_status gram_bf16(dmu_plan p, const float co[3], int steps, cudaStream_t s) {
     for (size_t c = 0; c < p->classes.size(); ++c) {
       const GClass& gc = p->classes[c];
       if (p->tune_class >= 0 && (int)c != p->tune_class) continue;
-      const bool tf = gc.kind != KIND_BF16;  // TF32 / F16 classes keep the final P in the bf16 pair area
-      CUDA_TRY(launch_identity_bf16(tf ? p->pf_bf16((int)c, 0) : p->slot_bf16((int)c, SLOT_PA_HI),
-                                    tf ? p->pf_bf16((int)c, 1) : p->slot_bf16((int)c, SLOT_PA_LO),
-                                    gc.count, (int)gc.m, gc.ldg, gc.m * gc.ldg, s));
+      // P_0 = I as an fp16 pair: in P buffer A for F16 classes, in the
+      // final-P area for the others
+      const bool f16 = gc.kind == KIND_F16;
+      CUDA_TRY(launch_identity16(f16 ? p->slot_bf16((int)c, SLOT_PA_HI) : p->pf_bf16((int)c, 0),
+                                 f16 ? p->slot_bf16((int)c, SLOT_PA_LO) : p->pf_bf16((int)c, 1),
+                                 gc.count, (int)gc.m, gc.ldg, gc.m * gc.ldg, 1, s));
       p->launches++;
     }
     p->p_final = 0;
@@ -773,8 +789,15 @@ dmu_status run_normalize(dmu_plan p, int tbl, bool with_mom, float beta, float g
                            f32 ? 1 : 0, p->mb_dev(), f32 ? 1 : 0, beta, gscale, p->partial_dev(), vec ? 1 : 0,
                            p->num_sms, s));
   CUDA_TRY(launch_norm_finalize(p->mats_dev(), p->count, p->partial_dev(), eps, p->inv_dev(),
+                                f32 ? nullptr : p->iscale_dev(), f32 ? nullptr : p->invimg_dev(),
                                 p->status_dev(), s));
   p->launches += 2;
+  if (!f32) {
+    // the bf16 image becomes 2^e M in fp16, in place (the tensor-core operand)
+    CUDA_TRY(launch_image16(p->chunks_dev(), (int)p->chunks.size(), p->mats_dev(), p->mb_dev(), p->iscale_dev(),
+                            p->vec_shapes ? 1 : 0, p->num_sms, s));
+    p->launches++;
+  }
   p->eps = eps;
   p->have_mb = true;
   p->have_p = false;
@@ -802,18 +825,19 @@ dmu_status final_launch(dmu_plan p, bool with_w, bool with_o, float lr, cudaStre
     g.sym = 0;
     g.tiles_per_mat = tiles_for(g.M, g.N, false, &g.tiles_m, &g.tiles_n);
     g.a_mn = 0;
-    if (gc.kind != KIND_BF16) {
+    const bool f16 = gc.kind == KIND_F16;
+    if (f16) {  // P in fp16 at scale 1, one MMA per K slice (hi only)
+      g.a_z[0] = g.a_z[1] = pf_hi * gc.count + b.cls_off;
+      g.terms = TERM_HH;
+    } else {    // the fp16 hi/lo pair of the final-P area, two MMAs
       g.a_z[0] = b.cls_off;
       g.a_z[1] = gc.count + b.cls_off;
-    } else {
-      g.a_z[0] = pf_hi * gc.count + b.cls_off;
-      g.a_z[1] = (pf_hi + 1) * gc.count + b.cls_off;
+      g.terms = TERM_HH | TERM_LH;
     }
     g.b_mn = b.tall ? 0 : 1;
-    g.terms = TERM_HH | TERM_LH;
     g.epi = EPI_UPDATE;
     g.alpha = -lr * (float)std::sqrt(std::max(1.0, (double)b.rows / (double)b.cols));
-    g.inv = p->inv_dev();
+    g.inv = p->inv_kernel();
     g.inv_base = b.first_slot;
     g.w_ptrs = with_w ? reinterpret_cast<void* const*>(p->tbl_dev(TBL_W)) : nullptr;
     g.o_ptrs = with_o ? reinterpret_cast<float* const*>(p->tbl_dev(TBL_O)) : nullptr;
@@ -821,11 +845,11 @@ dmu_status final_launch(dmu_plan p, bool with_w, bool with_o, float lr, cudaStre
     g.w_f32 = 0;
     g.w_transposed = b.tall ? 1 : 0;
     g.w_cols = b.cols;
-    pr.amap = gc.kind != KIND_BF16 ? gc.map_pf : gc.map;
+    pr.amap = f16 ? gc.map : gc.map_pf;
     pr.bmap = b.tall ? b.map_k : b.map_mn;
     if (gc.half) {
       g.half_a = 1;
-      pr.amap_t = gc.kind != KIND_BF16 ? gc.map_pf_t : gc.map_t;
+      pr.amap_t = f16 ? gc.map_t : gc.map_pf_t;
     }
     probs.push_back(pr);
     scheds.push_back(p->final_sched(b));
@@ -835,7 +859,7 @@ dmu_status final_launch(dmu_plan p, bool with_w, bool with_o, float lr, cudaStre
     for (size_t i = 0; i < probs.size(); ++i)
       if (scheds[i] == sched) group.push_back(probs[i]);
     if (group.empty()) continue;
-    st = run_tc(p, group, 2, 1, KIND_BF16, sched, s);
+    st = run_tc(p, group, 2, 1, KIND_F16, sched, s);
     if (st != DMU_OK) return st;
   }
   return DMU_OK;
@@ -1008,6 +1032,10 @@ dmu_status dmu_plan_create(const dmu_shape* shapes, int count, dmu_dtype dtype, 
   off = align_up(off + 16, 256);
   p->off_inv = off;
   off = align_up(off + sizeof(float) * count, 256);
+  p->off_iscale = off;
+  off = align_up(off + sizeof(float) * count, 256);
+  p->off_invimg = off;
+  off = align_up(off + sizeof(float) * count, 256);
   p->off_partial = off;
   off = align_up(off + sizeof(float) * MOM_PARTIALS_PER_CHUNK * p->chunks.size(), 256);
   p->off_chunks = off;
@@ -1028,12 +1056,12 @@ dmu_status dmu_plan_create(const dmu_shape* shapes, int count, dmu_dtype dtype, 
       off = align_up(off + 4 * (size_t)NUM_FSLOTS * elems, 1024);
       g.off_pf = off;
       off = align_up(off + 2 * 2 * elems, 1024);
-    } else if (g.kind == KIND_F16) {
+    } else if (g.kind == KIND_F16) {  // its final P stays in its fp16 P slots
+      off = align_up(off + 2 * (size_t)NUM_SLOTS * elems, 1024);
+    } else {
       off = align_up(off + 2 * (size_t)NUM_SLOTS * elems, 1024);
       g.off_pf = off;
       off = align_up(off + 2 * 2 * elems, 1024);
-    } else {
-      off = align_up(off + 2 * (size_t)NUM_SLOTS * elems, 1024);
     }
   }
   p->total = off;
@@ -1070,9 +1098,12 @@ dmu_status dmu_set_workspace(dmu_plan p, void* dev_ptr, size_t bytes) {
       CUtensorMap mk, mn;
       void* base = p->mb_dev() + 2 * (size_t)b.mb_off;
       const uint64_t s1 = (uint64_t)b.ldc * 2, s2 = (uint64_t)b.rows * b.ldc * 2;
-      st = encode_map(&mk, base, (uint64_t)b.cols, (uint64_t)b.rows, (uint64_t)b.count, s1, s2, 64, 128);
+      // the image is read as fp16 (2^e M, converted in place after the norm)
+      st = encode_map(&mk, base, (uint64_t)b.cols, (uint64_t)b.rows, (uint64_t)b.count, s1, s2, 64, 128,
+                      CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
       if (st != DMU_OK) return st;
-      st = encode_map(&mn, base, (uint64_t)b.cols, (uint64_t)b.rows, (uint64_t)b.count, s1, s2, 64, 64);
+      st = encode_map(&mn, base, (uint64_t)b.cols, (uint64_t)b.rows, (uint64_t)b.count, s1, s2, 64, 64,
+                      CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
       if (st != DMU_OK) return st;
       b.map_k = (int)p->maps.size();
       p->maps.push_back(mk);
@@ -1091,7 +1122,7 @@ dmu_status dmu_set_workspace(dmu_plan p, void* dev_ptr, size_t bytes) {
         CUtensorMap mp;
         const uint64_t t1 = (uint64_t)g.ldg * 2, t2 = (uint64_t)g.m * g.ldg * 2;
         st = encode_map(&mp, p->ws + g.off_pf, (uint64_t)g.m, (uint64_t)g.m, (uint64_t)2 * g.count, t1, t2, 64,
-                        128);
+                        128, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
         if (st != DMU_OK) return st;
         g.map_pf = (int)p->maps.size();
         p->maps.push_back(mp);
@@ -1110,15 +1141,15 @@ dmu_status dmu_set_workspace(dmu_plan p, void* dev_ptr, size_t bytes) {
         if (st != DMU_OK) return st;
         g.map_t = (int)p->maps.size();
         p->maps.push_back(mt);
-        if (g.kind == KIND_F16) {
+        if (g.kind != KIND_F16) {  // the fp16 final-P pair of bf16-pair classes (half-stored)
           CUtensorMap mp, mpt;
           st = encode_map(&mp, p->ws + g.off_pf, (uint64_t)g.m, (uint64_t)g.m, (uint64_t)2 * g.count, s1, s2, 64,
-                          128);
+                          128, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
           if (st != DMU_OK) return st;
           g.map_pf = (int)p->maps.size();
           p->maps.push_back(mp);
           st = encode_map(&mpt, p->ws + g.off_pf, (uint64_t)g.m, (uint64_t)g.m, (uint64_t)2 * g.count, s1, s2, 64,
-                          64);
+                          64, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
           if (st != DMU_OK) return st;
           g.map_pf_t = (int)p->maps.size();
           p->maps.push_back(mpt);
@@ -1254,7 +1285,7 @@ dmu_status dmu_debug_gram(dmu_plan p, int which, int index, float* out, void* st
   dmu_status st = check_plan(p, true);
   if (st != DMU_OK) return st;
   if (!out) return fail(DMU_ERR_INVALID_ARG, "out is NULL");
-  if (which < 0 || which > 8) return fail(DMU_ERR_INVALID_ARG, "which must be in [0, 8]");
+  if (which < 0 || which > 9) return fail(DMU_ERR_INVALID_ARG, "which must be in [0, 9]");
   if (which < 6 && (index < 0 || index >= p->count)) return fail(DMU_ERR_INVALID_ARG, "index out of range");
   if (which == 7 && (index < 0 || index >= p->count)) return fail(DMU_ERR_INVALID_ARG, "index out of range");
   DevGuard dg(p->device);
@@ -1266,8 +1297,10 @@ dmu_status dmu_debug_gram(dmu_plan p, int which, int index, float* out, void* st
     CUDA_TRY(cudaStreamSynchronize(s));
     return DMU_OK;
   }
-  if (which == 6) {
-    CUDA_TRY(cudaMemcpyAsync(out, p->inv_dev(), sizeof(float) * p->count, cudaMemcpyDeviceToDevice, s));
+  if (which == 6 || which == 9) {
+    const float* src = which == 6 ? p->inv_dev() : p->iscale_dev();
+    if (which == 9 && p->dtype != DMU_BF16) return fail(DMU_ERR_INVALID_ARG, "fp32 plans keep no image scale");
+    CUDA_TRY(cudaMemcpyAsync(out, src, sizeof(float) * p->count, cudaMemcpyDeviceToDevice, s));
     CUDA_TRY(cudaStreamSynchronize(s));
     return DMU_OK;
   }
@@ -1278,9 +1311,12 @@ dmu_status dmu_debug_gram(dmu_plan p, int which, int index, float* out, void* st
   const int local = slot - bk->first_slot;
   if (which == 5) {
     const MomMat& mm = p->mats[slot];
-    if (p->dtype == DMU_BF16) {
-      CUDA_TRY(launch_pair_to_f32(reinterpret_cast<const __nv_bfloat16*>(p->mb_dev()) + mm.mb_off, nullptr,
-                                  mm.rows, mm.cols, mm.ldc, out, s));
+    if (p->dtype == DMU_BF16) {  // the fp16 image 2^e M, scaled back
+      float sc = 1.f;
+      CUDA_TRY(cudaMemcpyAsync(&sc, p->iscale_dev() + slot, sizeof(float), cudaMemcpyDeviceToHost, s));
+      CUDA_TRY(cudaStreamSynchronize(s));
+      CUDA_TRY(launch_pair_h_to_f32(reinterpret_cast<const uint16_t*>(p->mb_dev()) + mm.mb_off, nullptr, mm.rows,
+                                    mm.cols, mm.ldc, 1.f / sc, out, s));
     } else {
       CUDA_TRY(launch_f32_copy2d(reinterpret_cast<const float*>(p->mb_dev()) + mm.mb_off, mm.rows, mm.cols,
                                  mm.ldc, out, s));
@@ -1296,11 +1332,12 @@ dmu_status dmu_debug_gram(dmu_plan p, int which, int index, float* out, void* st
   int q = which;
   if (which == 7) q = p->p_final == 0 ? 3 : 4;
   const int hf = gc.half ? 1 : 0;
-  if (p->dtype == DMU_BF16 && gc.kind == KIND_F16) {
-    if (which == 7) {
-      CUDA_TRY(launch_pair_to_f32(p->pf_bf16(bk->cls, 0) + moff, p->pf_bf16(bk->cls, 1) + moff, gc.m, gc.m,
-                                  gc.ldg, out, s, hf));
-    } else {
+  if (p->dtype == DMU_BF16 && which == 7 && gc.kind != KIND_F16) {
+    // the final P of other classes: the fp16 pair in the final-P area
+    CUDA_TRY(launch_pair_h_to_f32(p->pf_bf16(bk->cls, 0) + moff, p->pf_bf16(bk->cls, 1) + moff, gc.m, gc.m, gc.ldg,
+                                  1.f, out, s, hf));
+  } else if (p->dtype == DMU_BF16 && gc.kind == KIND_F16) {
+    {
       const int slots[5] = {SLOT_G_HI, SLOT_R_HI, SLOT_T_HI, SLOT_PA_HI, SLOT_PB_HI};
       const int sh = slots[q];
       CUDA_TRY(launch_pair_h_to_f32(p->slot_bf16(bk->cls, sh) + moff,
@@ -1308,12 +1345,7 @@ dmu_status dmu_debug_gram(dmu_plan p, int which, int index, float* out, void* st
                                     gc.ldg, 1.f / half_slot_scale(sh), out, s, hf));
     }
   } else if (p->dtype == DMU_BF16 && gc.kind == KIND_TF32) {
-    if (which == 7) {
-      CUDA_TRY(launch_pair_to_f32(p->pf_bf16(bk->cls, 0) + moff, p->pf_bf16(bk->cls, 1) + moff, gc.m, gc.m,
-                                  gc.ldg, out, s));
-    } else {
-      CUDA_TRY(launch_f32_copy2d(p->slot_f32(bk->cls, q) + moff, gc.m, gc.m, gc.ldg, out, s));
-    }
+    CUDA_TRY(launch_f32_copy2d(p->slot_f32(bk->cls, q) + moff, gc.m, gc.m, gc.ldg, out, s));
   } else if (p->dtype == DMU_BF16) {
     const int slots[5] = {SLOT_G_HI, SLOT_R_HI, SLOT_T_HI, SLOT_PA_HI, SLOT_PB_HI};
     const int sh = slots[q];

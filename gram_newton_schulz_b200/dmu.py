@@ -237,7 +237,7 @@ class Plan:
         import torch
         if which == 8:
             out = torch.empty(1, dtype=torch.float32, device=self.device)
-        elif which == 6:
+        elif which in (6, 9):
             out = torch.empty(self.count, dtype=torch.float32, device=self.device)
         elif which == 5:
             out = torch.empty(self.shapes[index], dtype=torch.float32, device=self.device)

@@ -92,8 +92,12 @@ typedef enum {
 } dmu_dtype;
 
 /* Precision of the Gram-space products on the bf16 path.  Gram-space
- * matrices are always stored as a bf16 pair (hi, lo = bf16(x - hi)) and
- * the final P X0 product always uses both halves of P.  Each symmetric
+ * matrices are stored as a 16-bit pair (hi, lo = round(x - hi)).  The image
+ * of M that the Gram matrix and the final product read is M rounded to bf16
+ * and held in fp16 at a power-of-two scale 2^e (exact for every entry in
+ * fp16's normal range); the final P X0 product multiplies it by P as one
+ * fp16 operand (F16 classes) or as an fp16 hi/lo pair (other classes).
+ * Each symmetric
  * product is computed on its upper-triangle tiles and mirrored, which
  * turns the antisymmetric part of the operand rounding error into a
  * symmetric one; with one bf16 MMA per product that error shifts the small
@@ -195,14 +199,18 @@ DMU_API dmu_status dmu_read_status(dmu_plan plan, uint32_t* flags);
 /* Test hook: write one workspace quantity as fp32 into `out` (device).
  *   which 0..4 : Gram-space matrix G, R, T, P(buffer A), P(buffer B) of
  *                matrix `index` (m*m floats, hi + lo combined);
- *   which 5    : the normalised input image Mb of matrix `index`
- *                (rows*cols floats, unscaled);
+ *   which 5    : the input image of matrix `index` (rows*cols floats, in
+ *                M's units): on the bf16 path M rounded to bf16, then held
+ *                as fp16 at the power-of-two scale of which 9;
  *   which 6    : 1/(||M||_F + eps) of every matrix (count floats);
  *   which 7    : the final P of matrix `index` (m*m floats);
  *   which 8    : bounded-wait self-test, writes nothing to `out`: a kernel
  *                waits `index` microseconds (1..1e6) on a barrier that
  *                nothing completes, gives up, and sets DMU_FLAG_TIMEOUT
- *                (read it with dmu_read_status).
+ *                (read it with dmu_read_status);
+ *   which 9    : bf16 plans: the scale 2^e of every matrix's fp16 image
+ *                (count floats), chosen so that 2^e ||M||_F is in
+ *                (2^14, 2^15].
  * Synchronises `stream`. */
 DMU_API dmu_status dmu_debug_gram(dmu_plan plan, int which, int index, float* out, void* stream);
 

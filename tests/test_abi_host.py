@@ -91,9 +91,12 @@ def _ws_expected(shapes, nslots, esize=2, auto_tf32=True):
         classes[m] = classes.get(m, 0) + 1
     for m, n in classes.items():
         ldg = -(-m // 8) * 8 if esize == 2 else m
-        if esize == 2 and auto_tf32 and m >= 1024:
-            gram += 12 * n * m * ldg  # 5 fp32 slots + final-P bf16 pair = 24 B = 12 bf16 elements
+        if esize == 2 and auto_tf32 and m < 1024:
+            # split-bf16 classes: 10 slots + the final P as an fp16 pair
+            gram += (nslots + 2) * n * m * ldg
         else:
+            # scaled-fp16 classes (m >= 1024) keep their final P in their own
+            # fp16 P slots; fp32 plans have 5 fp32 slots
             gram += nslots * n * m * ldg
     return esize * (mb + gram)
 
@@ -108,7 +111,7 @@ def test_host_only_plan_layout_qwen7b():
     expect = _ws_expected(w.shapes, 10)
     # tables, per-chunk partial sums and alignment add a little on top
     assert expect <= total <= expect * 1.002
-    assert 50e9 < total < 60e9
+    assert 45e9 < total < 52e9
     # no device: setting a workspace or computing fails cleanly
     assert lib.dmu_set_workspace(h, ctypes.c_void_p(256), total) == dmu.ERR_CUDA
     assert lib.dmu_momentum_normalize(h, None, None, 0.9, 1.0, 1e-7, None) == dmu.ERR_WORKSPACE

@@ -41,12 +41,15 @@ def test_syrk_and_final_gemm_k0(prec):
     outs = [torch.empty(s, dtype=torch.float32, device="cuda") for s in w.shapes]
     plan.apply_update(None, lr=LR, out_o=outs)
     inv = plan.debug(6).cpu().numpy().astype(np.float64)
+    isc = plan.debug(9).cpu().numpy().astype(np.float64)
     for i, (r, c) in enumerate(w.shapes):
         x = f64(grads[i])
         nrm = np.linalg.norm(x)
         assert inv[i] == pytest.approx(1.0 / (nrm + EPS), rel=2e-6)
+        # the image is M = G in fp16 at scale 2^e, with 2^e ||M|| in (2^14, 2^15]
+        assert np.log2(isc[i]) == np.round(np.log2(isc[i])) and 2 ** 14 < isc[i] * nrm <= 2 ** 15
         mb = plan.debug(5, i).cpu().numpy()
-        np.testing.assert_array_equal(mb, x)  # bf16 image of M = G exactly
+        np.testing.assert_array_equal(mb, (x * isc[i]).astype(np.float16).astype(np.float64) / isc[i])
         xo = x.T if r > c else x
         g_ref = (xo @ xo.T) * float(inv[i]) ** 2
         g = plan.debug(0, i).cpu().numpy().astype(np.float64)
@@ -129,7 +132,7 @@ def test_products_match_emulation(prec):
     plan.gram_ns_batched(None, dmu.QUINTIC, 2)
     for i in range(len(shapes)):
         d = {k: plan.debug(j, i).cpu().numpy().astype(np.float64) for k, j in
-             (("G", 0), ("R", 1), ("PA", 3), ("PB", 4))}
+             (("G", 0), ("R", 1), ("PA", 3), ("PB", 7))}  # P_2, the final P (fp16 pair)
         r_ref = b * d["G"] + c * _emul_product(d["G"], d["G"], prec)
         # fp32 accumulation and hi/lo storage leave ~1e-5; a wrong term is >= 1e-3
         tol = 1e-4

@@ -27,6 +27,14 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else None
 
 
+def _as_plan_image(img, sc):
+    """A bf16 image as the plan path holds it: fp16 at scale sc (fp32 images
+    are kept as they are)."""
+    if img.dtype == torch.float32:
+        return img
+    return (img.float() * sc).half().float() / sc
+
+
 def _static_call(lib, g, mom, img, inv, dtype_code, beta=BETA):
     r, c = g.shape
     return lib.dmu_momentum_norm_static(
@@ -49,6 +57,7 @@ def test_static_scratch_matches_plan_path_two_calls(dtype):
         plan.momentum_normalize([g], [mom_a], beta=BETA, eps=EPS)
         inv_a = plan.debug(6)
         img_a = plan.debug(5, 0)
+        sc = float(plan.debug(9)[0]) if dtype == "bf16" else 1.0
 
         mom_b = m0.clone()
         img_b = torch.empty(shape, dtype=tdt, device="cuda")
@@ -57,7 +66,9 @@ def test_static_scratch_matches_plan_path_two_calls(dtype):
         assert st == dmu.OK, lib.dmu_last_error()
         torch.cuda.synchronize()
         assert torch.equal(mom_a, mom_b)
-        assert torch.equal(img_a, img_b.float())
+        # the plan keeps its bf16 image as fp16 scaled by 2^e; the same values
+        # up to fp16's rounding of entries below its normal range
+        assert torch.equal(img_a, _as_plan_image(img_b, sc))
         assert float(inv_b[0]) == pytest.approx(float(inv_a[0]), rel=1e-6)
         x = mom_b.double().cpu().numpy()
         assert float(inv_b[0]) == pytest.approx(1.0 / (np.linalg.norm(x) + EPS), rel=2e-6)
@@ -75,6 +86,7 @@ def test_static_scratch_optional_outputs(drop):
     plan.momentum_normalize([g], None, beta=0.0, eps=EPS)
     inv_a = plan.debug(6)
     img_a = plan.debug(5, 0)
+    sc = float(plan.debug(9)[0])
     for _ in range(2):
         if drop == "momentum":
             img_b = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
@@ -86,7 +98,7 @@ def test_static_scratch_optional_outputs(drop):
         assert st == dmu.OK, lib.dmu_last_error()
         torch.cuda.synchronize()
         if img_b is not None:
-            assert torch.equal(img_a, img_b.float())
+            assert torch.equal(img_a, _as_plan_image(img_b, sc))
         else:
             assert torch.equal(mom, g.float())  # beta * 0 + G
         assert float(inv_b[0]) == pytest.approx(float(inv_a[0]), rel=1e-6)
