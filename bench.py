@@ -11,12 +11,13 @@ flush is needed between steps.
     python bench.py --impl reference ...   # the fp64 oracle on host cores
 
 Multi-GPU (torchrun, one process per GPU), two modes:
-* ``--shard replica`` (default): every rank owns a full layer set of its
-  own, with no collective on the data path.  Per-GPU work is fixed (weak
+* ``--shard owner`` (the default under several ranks): the ranks split one
+  layer set by LPT owners and exchange gradients and weights over NCCL: one
+  reduce in per owner bucket, and each owner's weights broadcast back in
+  two publish groups, the first while the second computes (strong
   scaling).
-* ``--shard owner``: the ranks split one layer set by LPT owners and
-  exchange gradients and weights over NCCL.  Each owner bucket gets one
-  reduce in and one broadcast out (strong scaling).
+* ``--shard replica``: every rank owns a full layer set of its own, with no
+  collective on the data path.  Per-GPU work is fixed (weak scaling).
 The step time is the max over ranks.  Prints one JSON line on rank 0.
 """
 from __future__ import annotations
@@ -280,18 +281,25 @@ def run_reference(args):
             vals.append(total * 1e3)
     # The job of an N-GPU run is N layer sets (one per rank, weak scaling);
     # the host cores do all of them, so the per-set time is scaled by N.
+    # The job mirrors the GPU arm's: under several ranks the default (owner)
+    # mode updates ONE layer set across the ranks (strong scaling); replica
+    # mode updates one layer set per rank, N sets in all, all of which the
+    # host cores do here.
     world = max(1, int(os.environ.get("WORLD_SIZE", "1")))
-    v = statistics.median(vals) * world
-    if world > 1:
-        sample += f"; times {world} layer sets, the job of {world} ranks"
+    replica = args.shard == "replica" or world == 1
+    sets = world if replica else 1
+    v = statistics.median(vals) * sets
+    if sets > 1:
+        sample += f"; times {sets} layer sets, the job of {world} replica ranks"
     line = {
         "impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "ms", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(v, 3), "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "scaling": "weak" if replica else "strong", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "extrapolated": extrap,
-        "config": {"workload": w.name, "matrices": w.count, "matrices_total": w.count * world, "K": K_STEPS,
+        "config": {"workload": w.name, "matrices": w.count, "matrices_total": w.count * sets, "K": K_STEPS,
                    "coeffs": [3.4445, -4.7750, 2.0315], "precision": "f64 oracle",
-                   "parallelism": f"replica x{world}, all on the host cores"},
+                   "parallelism": (f"replica x{world}" if replica else f"owner x{world}") +
+                                  ", all on the host cores"},
         "cpu_baseline": {"value": round(v, 3), "unit": "ms", "cores": threads, "kind": "oracle", "sample": sample,
                          "extrapolated": extrap},
         "e2e": {"value": round(v, 3), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -384,8 +392,7 @@ def run_owner(args, w_full, dev, world, rank, local, barrier):
     for _ in range(args.warmup):
         osd.step(gflat, wflat, moms, **kw)
     torch.cuda.synchronize(dev)
-    plan = osd.compute.plan
-    if plan is not None and plan.read_status() != 0:
+    if osd.read_status() != 0:
         raise SystemExit("device status word set during warm-up")
 
     K = args.steps
@@ -398,8 +405,8 @@ def run_owner(args, w_full, dev, world, rank, local, barrier):
     launches = tc = 0
     for k in range(K):
         osd.step(gflat, wflat, moms, events=ev[k], **kw)
-        launches += osd.compute.launches
-        tc += osd.compute.tc_launches
+        launches += osd.launches
+        tc += osd.tc_launches
     torch.cuda.synchronize(dev)
     barrier()
     clk = clocks.stop()
@@ -408,7 +415,7 @@ def run_owner(args, w_full, dev, world, rank, local, barrier):
     t_cmp = sum(e[1].elapsed_time(e[2]) for e in ev) / K
     t_out = sum(e[2].elapsed_time(e[3]) for e in ev) / K
     t_cmp_max = owners.max_over_ranks(t_cmp, device=dev)
-    status = plan.read_status() if plan is not None else 0
+    status = osd.read_status()
 
     # e2e through the public API with host buffers: each step uploads this
     # rank's whole local gradient from pinned memory and reads the whole
@@ -548,18 +555,20 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="dmu", choices=["dmu", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
-    ap.add_argument("--shard", default="replica", choices=["replica", "owner"],
-                    help="replica: every rank owns a full layer set (weak scaling); owner: the ranks "
-                         "split one layer set by LPT owners, gradients reduced to owners and weights "
-                         "broadcast back over NCCL (strong scaling)")
+    ap.add_argument("--shard", default="auto", choices=["auto", "replica", "owner"],
+                    help="owner: the ranks split one layer set by LPT owners, gradients reduced to owners "
+                         "and weights broadcast back over NCCL (strong scaling); replica: every rank owns a "
+                         "full layer set (weak scaling); auto (default): owner under several ranks, the "
+                         "plain single-GPU step otherwise")
     ap.add_argument("--shapes", default=None,
                     help="custom spiked bf16 workload for profiling, e.g. 3584x3584*8,512x3584*4")
     ap.add_argument("--prec", default="auto")
     ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--owner-method", default="milp", choices=["milp", "lpt"],
-                    help="owner mode: exact MILP over per-cost counts (LPT fallback) or greedy LPT")
+    ap.add_argument("--owner-method", default="lpt", choices=["lpt", "milp"],
+                    help="owner mode: greedy LPT on the per-matrix cost (default), or an exact MILP over "
+                         "per-cost counts with LPT as its fallback")
     ap.add_argument("--measured-owners", action="store_true",
                     help="owner mode: LPT on per-shape costs measured on rank 0 instead of the flop model")
     ap.add_argument("--demuon", type=int, default=0,
@@ -605,7 +614,7 @@ def main():
             raise SystemExit("--demuon simulates its agents on one GPU")
         run_demuon(args, w_full, dev, local)
         return
-    if args.shard == "owner":
+    if args.shard == "owner" or (args.shard == "auto" and world > 1):
         run_owner(args, w_full, dev, world, rank, local, barrier)
         if world > 1:
             dist.destroy_process_group()

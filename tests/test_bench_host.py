@@ -147,15 +147,21 @@ def test_pin_copies_reports_failure_instead_of_raising(monkeypatch):
 
 
 def test_reference_arm_under_two_ranks():
-    """Rank 0 alone runs the oracle for the whole job (two layer sets under
-    two ranks); the other rank exits 0 without work or output."""
+    """Rank 0 alone runs the oracle for the whole job -- one layer set split
+    over the ranks in the default owner mode, two layer sets in replica
+    mode; the other rank exits 0 without work or output."""
     base = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1", "--warmup", "0",
             "--shapes", "64x256*2", "--ref-budget", "2"]
     env0 = dict(os.environ, WORLD_SIZE="2", RANK="0", LOCAL_RANK="0")
     out = subprocess.run(base, capture_output=True, text=True, timeout=300, cwd=ROOT, env=env0)
     assert out.returncode == 0, out.stderr
     d = json.loads([l for l in out.stdout.splitlines() if l.strip()][0])
-    assert d["n_gpus"] == 2 and d["config"]["matrices_total"] == 4 and "2 ranks" in d["cpu_baseline"]["sample"]
+    assert d["n_gpus"] == 2 and d["config"]["matrices_total"] == 2 and d["scaling"] == "strong"
+    out = subprocess.run(base + ["--shard", "replica"], capture_output=True, text=True, timeout=300, cwd=ROOT,
+                         env=env0)
+    assert out.returncode == 0, out.stderr
+    d = json.loads([l for l in out.stdout.splitlines() if l.strip()][0])
+    assert d["config"]["matrices_total"] == 4 and "2 replica ranks" in d["cpu_baseline"]["sample"]
     env1 = dict(os.environ, WORLD_SIZE="2", RANK="1", LOCAL_RANK="1")
     out1 = subprocess.run(base, capture_output=True, text=True, timeout=300, cwd=ROOT, env=env1)
     assert out1.returncode == 0 and out1.stdout.strip() == ""

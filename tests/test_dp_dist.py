@@ -11,7 +11,10 @@ tests check:
   mean gradient, bit for bit. The gradients are chosen so that their float32
   sums are exact in any order;
 * the owner's momentum is the oracle's, and each rank computes exactly its
-  owned matrices;
+  owned matrices, in two publish groups;
+* the collectives are issued in the same order on every rank: all reduces,
+  then each group's broadcasts right after that group's compute, so a
+  group's publish overlaps the next group's compute;
 * a rank that dies before the exchange surfaces on the other rank as an
   error from the collective (short process-group timeout), not a hang.
 """
@@ -59,14 +62,18 @@ def _momentum0(i):
 
 
 class OracleCompute:
-    """Test stand-in for the device compute: the fp64 oracle per owned matrix."""
+    """Test stand-in for the device compute: the fp64 oracle per owned
+    matrix.  ``log`` records ("compute", matrices) per call."""
 
-    def __init__(self, indices):
-        self.indices = list(indices)
-        self.calls = []
+    def __init__(self, log=None):
+        self.log = log if log is not None else []
+
+    @property
+    def calls(self):
+        return [n for kind, n in self.log if kind == "compute"]
 
     def __call__(self, grads, momenta, weights, *, beta, lr, eps, coeffs, steps, grad_scale=1.0):
-        self.calls.append(list(self.indices))
+        self.log.append(("compute", len(grads)))
         for g, m, w in zip(grads, momenta, weights):
             g = g * np.float32(grad_scale)  # fp32 product, as the momentum pass forms it
             m_new, _, w_new = gram_ns.muon_step(w.double().numpy(), m.double().numpy(), g.double().numpy(),
@@ -96,17 +103,33 @@ def _step_worker(rank, world, port, q):
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
-        buckets = dp.OwnerBuckets(SHAPES, world)
-        compute = OracleCompute(buckets.members[rank])
+        log = []
+        compute = OracleCompute(log)
         step = dp.OwnerShardedStep(SHAPES, compute=compute)
+        buckets = step.buckets
         gf = buckets.alloc(torch.float32, "cpu")
         wf = buckets.alloc(torch.float32, "cpu")
         for i in range(len(SHAPES)):
             buckets.view(gf, i).copy_(torch.from_numpy(_grad(i, rank)))
             buckets.view(wf, i).copy_(torch.from_numpy(_weight(i)))
         moms = [torch.from_numpy(_momentum0(i)).clone() for i in step.mine]
-        step.step(gf, wf, moms, beta=BETA, lr=LR, eps=EPS)
-        q.put((rank, list(step.mine), compute.calls,
+        # record the order in which the step issues its collectives
+        real_reduce, real_bcast = dist.reduce, dist.broadcast
+
+        def reduce(t, dst, **kw):
+            log.append(("reduce", dst))
+            return real_reduce(t, dst, **kw)
+
+        def broadcast(t, src, **kw):
+            log.append(("bcast", src))
+            return real_bcast(t, src, **kw)
+
+        dist.reduce, dist.broadcast = reduce, broadcast
+        try:
+            step.step(gf, wf, moms, beta=BETA, lr=LR, eps=EPS)
+        finally:
+            dist.reduce, dist.broadcast = real_reduce, real_bcast
+        q.put((rank, list(step.mine), log, [len(g) for g in step.publish],
                [buckets.view(wf, i).numpy().copy() for i in range(len(SHAPES))],
                [m.numpy().copy() for m in moms]))
     finally:
@@ -131,9 +154,10 @@ def test_owner_buckets_layout():
 
 
 def test_single_process_step_matches_oracle():
-    compute = OracleCompute(range(len(SHAPES)))
+    compute = OracleCompute()
     step = dp.OwnerShardedStep(SHAPES, compute=compute)
-    assert step.world == 1 and step.mine == list(range(len(SHAPES)))
+    assert step.world == 1 and sorted(step.mine) == list(range(len(SHAPES)))
+    assert len(compute.calls) == 0 and [len(g) for g in step.publish] != [len(SHAPES), 0]
     b = step.buckets
     gf, wf = b.alloc(torch.float32, "cpu"), b.alloc(torch.float32, "cpu")
     for i in range(len(SHAPES)):
@@ -141,10 +165,36 @@ def test_single_process_step_matches_oracle():
         b.view(wf, i).copy_(torch.from_numpy(_weight(i)))
     moms = [torch.from_numpy(_momentum0(i)).clone() for i in step.mine]
     step.step(gf, wf, moms, beta=BETA, lr=LR, eps=EPS)
+    assert compute.calls == [len(g) for g in step.publish]  # one call per publish group
     ew, em = _expected(1)
     for i in range(len(SHAPES)):
         assert np.array_equal(b.view(wf, i).numpy(), ew[i])
-        assert np.array_equal(moms[i].numpy(), em[i])
+    for k, i in enumerate(step.mine):
+        assert np.array_equal(moms[k].numpy(), em[i])
+
+
+def test_publish_groups_balance_cost():
+    """Each rank's owned matrices split into two publish groups of about
+    equal flop cost (LPT over the groups), each in its own bucket."""
+    from gram_newton_schulz_b200 import owners
+    for world in (1, 2, 3):
+        b = dp.OwnerBuckets(SHAPES, world, groups=2)
+        assert len(b.sizes) == 2 * world
+        for r in range(world):
+            g0, g1 = b.group_members[r]
+            assert sorted(g0 + g1) == sorted(b.members[r]) and b.members[r] == g0 + g1
+            c0 = sum(owners.matrix_cost(*SHAPES[i]) for i in g0)
+            c1 = sum(owners.matrix_cost(*SHAPES[i]) for i in g1)
+            if g0 and g1:
+                assert max(c0, c1) <= min(c0, c1) + max(owners.matrix_cost(*SHAPES[i]) for i in g0 + g1)
+        flats = b.alloc(torch.float32, "cpu")
+        seen = set()
+        for i, v in enumerate(b.views(flats)):
+            assert tuple(v.shape) == SHAPES[i]
+            k = b.bucket(b.owner[i], b.group[i])
+            assert (v.data_ptr() - flats[k].data_ptr()) % 256 == 0
+            seen.add((k, b.offset[i]))
+        assert len(seen) == len(SHAPES)
 
 
 @pytest.mark.parametrize("world", [2, 3])
@@ -166,8 +216,16 @@ def test_gloo_owner_step_matches_oracle(world):
         assert p.exitcode == 0
     ew, em = _expected(world)
     owned = []
-    for rank, mine, calls, weights, moms in results:
-        assert calls == [mine]  # one compute call, over the owned matrices only
+    for rank, mine, log, groups, weights, moms in results:
+        # reduces of all 2 * world buckets first; then per publish group: its
+        # compute (if the group has matrices), then one broadcast per rank
+        expect = [("reduce", b // 2) for b in range(2 * world)]
+        for g in range(2):
+            if groups[g]:
+                expect.append(("compute", groups[g]))
+            expect += [("bcast", r) for r in range(world)]
+        assert log == expect, (rank, log)
+        assert sum(groups) == len(mine)
         owned += mine
         for i in range(len(SHAPES)):
             assert np.array_equal(weights[i], ew[i]), (rank, i)
@@ -185,11 +243,11 @@ def _dying_worker(rank, world, port, q):
         q.close()
         q.join_thread()
         os._exit(0)  # leaves between steps, before the exchange
-    buckets = dp.OwnerBuckets(SHAPES, world)
     try:
         # the owner table is broadcast from rank 0 when the step is built,
         # and the exchange follows: either collective reports the missing peer
-        step = dp.OwnerShardedStep(SHAPES, compute=OracleCompute(buckets.members[rank]))
+        step = dp.OwnerShardedStep(SHAPES, compute=OracleCompute())
+        buckets = step.buckets
         gf, wf = buckets.alloc(torch.float32, "cpu"), buckets.alloc(torch.float32, "cpu")
         moms = [torch.zeros(SHAPES[i]) for i in step.mine]
         step.step(gf, wf, moms)
@@ -227,7 +285,7 @@ def _cost_worker(rank, world, port, q):
         # every rank "measures" something different; only rank 0's table counts
         fake = lambda shapes: {tuple(s): float(s[0] * s[1]) * (1.0 + rank) for s in shapes}  # noqa: E731
         costs = dp.shared_costs(SHAPES, measure=fake)
-        step = dp.OwnerShardedStep(SHAPES, compute=OracleCompute([]), measured=costs)
+        step = dp.OwnerShardedStep(SHAPES, compute=OracleCompute(), measured=costs)
         q.put((rank, sorted(costs.items()), list(step.buckets.owner)))
     finally:
         dist.destroy_process_group()
@@ -260,8 +318,7 @@ def _sparse_worker(rank, world, port, q):
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
         shapes = SHAPES[:3]  # fewer matrices than ranks: some ranks own nothing
-        step = dp.OwnerShardedStep(shapes, compute=OracleCompute([]))
-        step.compute.indices = list(step.mine)
+        step = dp.OwnerShardedStep(shapes, compute=OracleCompute())
         b = step.buckets
         gf, wf = b.alloc(torch.float32, "cpu"), b.alloc(torch.float32, "cpu")
         for i in range(len(shapes)):

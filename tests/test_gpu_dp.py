@@ -24,13 +24,13 @@ def test_owner_step_on_flat_buffers_matches_plan_step():
     weights = synth.weights(w, dev)
 
     osd = dp.OwnerShardedStep(shapes, device=dev)
-    assert osd.world == 1 and osd.mine == list(range(len(shapes)))
+    assert osd.world == 1 and sorted(osd.mine) == list(range(len(shapes)))
     b = osd.buckets
     gflat, wflat = b.alloc(torch.bfloat16, dev), b.alloc(torch.bfloat16, dev)
     for i in range(len(shapes)):
         b.view(gflat, i).copy_(grads[i])
         b.view(wflat, i).copy_(weights[i])
-    moms_a = [torch.zeros(s, dtype=torch.float32, device=dev) for s in shapes]
+    moms_a = [torch.zeros(shapes[i], dtype=torch.float32, device=dev) for i in osd.mine]
     moms_b = [torch.zeros(s, dtype=torch.float32, device=dev) for s in shapes]
     plan = dmu.Plan(shapes, device=dev)
     w_ref = [x.clone() for x in weights]
@@ -38,11 +38,12 @@ def test_owner_step_on_flat_buffers_matches_plan_step():
         osd.step(gflat, wflat, moms_a, beta=0.95, lr=0.02)
         plan.step(grads, moms_b, w_ref, beta=0.95, lr=0.02)
     torch.cuda.synchronize()
-    assert osd.compute.launches > 0 and osd.compute.tc_launches > 0
+    assert osd.launches > 0 and osd.tc_launches > 0
     for i in range(len(shapes)):
         assert torch.equal(b.view(wflat, i), w_ref[i]), i
-        assert torch.equal(moms_a[i], moms_b[i]), i
-    assert osd.compute.plan.read_status() == 0
+    for k, i in enumerate(osd.mine):
+        assert torch.equal(moms_a[k], moms_b[i]), i
+    assert osd.read_status() == 0
     osd.close()
     plan.close()
 
@@ -61,17 +62,20 @@ def test_owner_step_matches_oracle():
     for i in range(len(shapes)):
         b.view(gflat, i).copy_(grads[i])
         b.view(wflat, i).copy_(weights[i])
-    moms = [torch.zeros(s, dtype=torch.float32, device=dev) for s in shapes]
-    outs = [torch.empty(s, dtype=torch.float32, device=dev) for s in shapes]
+    # momenta and O in the step's owned order
+    moms = [torch.zeros(shapes[i], dtype=torch.float32, device=dev) for i in osd.mine]
+    outs_m = [torch.empty(shapes[i], dtype=torch.float32, device=dev) for i in osd.mine]
     osd.step(gflat, wflat, moms, beta=0.95, lr=0.02)
     w_mid = [b.view(wflat, i).clone() for i in range(len(shapes))]
-    osd.step(gflat, wflat, moms, beta=0.95, lr=0.02, out_o=outs)
+    osd.step(gflat, wflat, moms, beta=0.95, lr=0.02, out_o=outs_m)
     torch.cuda.synchronize()
-    assert osd.compute.plan.read_status() == 0
+    assert osd.read_status() == 0
+    pos = {i: k for k, i in enumerate(osd.mine)}
+    outs = [outs_m[pos[i]] for i in range(len(shapes))]
     for i, (r, c) in enumerate(shapes):
         g = f64(grads[i])
         m_ref = oracle.momentum(oracle.momentum(np.zeros_like(g), g, 0.95), g, 0.95)
-        np.testing.assert_allclose(f64(moms[i]), m_ref, rtol=2.0 ** -22, atol=0)
+        np.testing.assert_allclose(f64(moms[pos[i]]), m_ref, rtol=2.0 ** -22, atol=0)
         # the oracle's Muon step on the momentum the device holds
         _, o_ref, _ = oracle.muon_step(f64(w_mid[i]), 0.95 * g, g, beta=1.0, lr=0.02)
         e = rel(f64(outs[i]), o_ref)
