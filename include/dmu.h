@@ -214,16 +214,24 @@ DMU_API dmu_status dmu_read_status(dmu_plan plan, uint32_t* flags);
  * Synchronises `stream`. */
 DMU_API dmu_status dmu_debug_gram(dmu_plan plan, int which, int index, float* out, void* stream);
 
-/* Pick the fastest tensor-core schedule for this plan by measurement (DMuon
- * page, section 2.4: per-shape kernel configurations are tuned once and
- * cached).  Times the whole Gram recursion (K = 5) with CTA-pair kernels
- * (256 x 256 tiles) and with single-CTA kernels (128 x 256 and 128 x 128
- * tiles) on the data left by dmu_momentum_normalize, keeps the fastest
- * (CTA pairs win ties), and appends the
- * choice to the text file `cache_path` (may be NULL: no cache).  A cached
- * entry for the same device, shapes, dtype and precision is reused without
- * timing.  Synchronises `stream`; overwrites the plan's Gram-space state.
- * Errors: NOT_PLANNED (no dmu_momentum_normalize yet), CUDA. */
+/* Pick the fastest schedule per shape by measurement (DMuon page, section
+ * 2.4: per-shape kernel configurations are tuned once and cached).
+ *   - Every Gram class (all matrices with one m) is timed alone over the
+ *     whole quintic recursion (K = 5) with CTA pairs (256 x 256 tiles),
+ *     single CTAs (128 x 256 and 128 x 128 tiles) and, for split-bf16
+ *     classes with m <= 128, the on-chip recursion; CTA pairs win ties.
+ *   - Every shape bucket's final GEMM + update is then timed alone with the
+ *     three tile schedules.  Its weight writes go to the class's free
+ *     Gram-space scratch, never to the caller's weights (buckets whose
+ *     weights do not fit there are timed on the first matrices that do).
+ * Times run on the data left by dmu_momentum_normalize.  Each choice is
+ * appended to the text file `cache_path` (may be NULL: no cache) as one
+ * line "<key> <schedule> <times...>"; the key names the device, the
+ * precision and the shapes of the class or bucket, so any plan with the
+ * same class or bucket reuses the entry without timing.  Synchronises
+ * `stream`; overwrites the plan's Gram-space state and leaves P_K of the
+ * quintic K = 5 recursion for dmu_apply_update.  Errors: NOT_PLANNED (no
+ * dmu_momentum_normalize yet), CUDA. */
 DMU_API dmu_status dmu_autotune(dmu_plan plan, const char* cache_path, void* stream);
 
 /* The plan's default tile schedule: 1 = CTA pairs (256 x 256), 0 = single
