@@ -33,6 +33,15 @@ __device__ __forceinline__ void load8_grad(const void* g, int f32, long long idx
   }
 }
 
+// fp16 image entries: 2^e v rounded to fp16 (sc = 2^e)
+__device__ __forceinline__ void store8_image_h(void* __restrict__ mb, long long o, const float* v, float sc) {
+  uint4 u;
+  __half2* h = reinterpret_cast<__half2*>(&u);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) h[q] = __floats2half2_rn(v[2 * q] * sc, v[2 * q + 1] * sc);
+  *reinterpret_cast<uint4*>(reinterpret_cast<__half*>(mb) + o) = u;
+}
+
 __device__ __forceinline__ void store8_image(void* __restrict__ mb, int mb_f32, long long o, const float* v) {
   if (mb_f32) {
     float4* d = reinterpret_cast<float4*>(reinterpret_cast<float*>(mb) + o);
@@ -91,17 +100,23 @@ template <> struct GradVec<true> {
   }
 };
 
+// Image: fp32 plans write M itself; bf16 plans write fp16(2^e M) with the
+// scale 2^e the previous call chose for this matrix (iscale), or nothing
+// when there is none yet -- k_norm_finalize then flags the matrix and
+// k_image_fix writes its image.
 template <bool F32>
 __global__ void __launch_bounds__(256, 3) k_momentum(const MomChunk* __restrict__ chunks, int nchunks,
                                                   const MomMat* __restrict__ mats,
                                                   const void* const* __restrict__ grads,
                                                   float* const* __restrict__ momenta,
                                                   void* __restrict__ mb, float beta, float gscale,
+                                                  const float* __restrict__ iscale,
                                                   float* __restrict__ partial, int vec) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int c = blockIdx.x; c < nchunks; c += gridDim.x) {
     const MomChunk ch = chunks[c];
     const long long mb_off = mats[ch.slot].mb_off;
+    const float sc = F32 ? 1.f : iscale[ch.slot];
     const void* __restrict__ g = grads[ch.slot];
     float* __restrict__ mom = momenta ? momenta[ch.slot] : nullptr;
     const int s0 = warp * MOM_SLICE;
@@ -141,7 +156,10 @@ __global__ void __launch_bounds__(256, 3) k_momentum(const MomChunk* __restrict_
             }
 #pragma unroll
             for (int q = 0; q < 8; ++q) ss += v[q] * v[q];
-            store8_image(mb, F32 ? 1 : 0, mb_off + i0, v);  // ldc == cols on the vector path
+            if (F32)
+              store8_image(mb, 1, mb_off + i0, v);  // ldc == cols on the vector path
+            else if (sc > 0.f)
+              store8_image_h(mb, mb_off + i0, v, sc);
           }
         }
       }
@@ -161,8 +179,8 @@ __global__ void __launch_bounds__(256, 3) k_momentum(const MomChunk* __restrict_
         const long long o = mm.mb_off + row * mm.ldc + col;
         if (F32)
           reinterpret_cast<float*>(mb)[o] = v;
-        else
-          reinterpret_cast<__nv_bfloat16*>(mb)[o] = __float2bfloat16_rn(v);
+        else if (sc > 0.f)
+          reinterpret_cast<__half*>(mb)[o] = __float2half_rn(v * sc);
       }
     }
 #pragma unroll
@@ -171,13 +189,18 @@ __global__ void __launch_bounds__(256, 3) k_momentum(const MomChunk* __restrict_
   }
 }
 
-// Also the power-of-two scale 2^e of the fp16 image (when `iscale` is
-// given): 2^e ||M||_F <= 2^15, so every entry of 2^e M is below fp16's
-// largest finite value, and entries down to ||M||_F 2^-29 stay normal;
-// inv_img = inv 2^-e reads the scaled image back as X0.
+// bf16 plans also keep the power-of-two scale 2^e of each matrix's fp16
+// image (iscale): the previous call's scale stays while 2^e ||M||_F lies in
+// (2^9, 2^15] -- every entry of 2^e M is then below fp16's largest finite
+// value, and entries down to ||M||_F 2^-23 stay in fp16's normal range --
+// so a steady run writes the image in the momentum pass alone.  Otherwise
+// (first call, or the norm moved 8x) a new scale with 2^e ||M||_F in
+// (2^11, 2^12] is chosen and the matrix is flagged for k_image_fix.
+// inv_img = inv 2^-e reads the image back as X0.
 __global__ void k_norm_finalize(const MomMat* __restrict__ mats, int nmats,
                                 const float* __restrict__ partial, float eps, float* __restrict__ inv,
-                                float* __restrict__ iscale, float* __restrict__ inv_img, unsigned int* status) {
+                                float* __restrict__ iscale, float* __restrict__ inv_img, int* __restrict__ fix,
+                                unsigned int* status) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= nmats) return;
@@ -193,84 +216,105 @@ __global__ void k_norm_finalize(const MomMat* __restrict__ mats, int nmats,
     const float iv = (float)(1.0 / (nrm + (double)eps));
     inv[warp] = iv;
     if (iscale) {
-      int e = 0;
-      if (nrm > 0.0 && isfinite(nrm)) e = 15 - (int)ceil(log2(nrm));
-      e = max(-100, min(100, e));
-      iscale[warp] = ldexpf(1.f, e);
-      inv_img[warp] = ldexpf(iv, -e);
+      const float prev = iscale[warp];
+      const double scaled = (double)prev * nrm;
+      const bool keep = prev > 0.f && isfinite(nrm) && scaled > 512.0 && scaled <= 32768.0;
+      float sc = prev;
+      if (!keep) {
+        int e = 0;
+        if (nrm > 0.0 && isfinite(nrm)) e = 12 - (int)ceil(log2(nrm));
+        e = max(-100, min(100, e));
+        sc = ldexpf(1.f, e);
+        iscale[warp] = sc;
+      }
+      fix[warp] = keep ? 0 : 1;
+      inv_img[warp] = iv / sc;  // exact: sc is a power of two
     }
   }
 }
 
-// The bf16 image of M, converted in place to fp16 scaled by 2^e per matrix
-// (exact for every entry in fp16's normal range; the fp16 image feeds the
-// kind::f16 MMAs of the Gram matrix and of the final product).  Same chunk
-// walk as the momentum pass.
-__global__ void __launch_bounds__(256) k_image16(const MomChunk* __restrict__ chunks, int nchunks,
-                                                 const MomMat* __restrict__ mats, void* __restrict__ mb,
-                                                 const float* __restrict__ iscale, int vec) {
+// The fp16 image 2^e M of the matrices k_norm_finalize flagged, recomputed
+// from their source: M as the momentum pass left it, or, without momentum
+// state, gscale * G exactly as the momentum pass formed it.  Chunks of
+// matrices that keep their scale return at once.
+__global__ void __launch_bounds__(256) k_image_fix(const MomChunk* __restrict__ chunks, int nchunks,
+                                                   const MomMat* __restrict__ mats,
+                                                   const void* const* __restrict__ grads,
+                                                   float* const* __restrict__ momenta, float gscale,
+                                                   void* __restrict__ mb, const float* __restrict__ iscale,
+                                                   const int* __restrict__ fix, int vec) {
   for (int c = blockIdx.x; c < nchunks; c += gridDim.x) {
     const MomChunk ch = chunks[c];
+    if (!fix[ch.slot]) continue;
     const MomMat mm = mats[ch.slot];
     const float sc = iscale[ch.slot];
+    const __nv_bfloat16* g = reinterpret_cast<const __nv_bfloat16*>(grads[ch.slot]);
+    const float* mom = momenta ? momenta[ch.slot] : nullptr;
     if (vec) {
-      uint4* base = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(mb) + mm.mb_off + ch.start);
-      const int nv = ch.len >> 3;
-      for (int v = threadIdx.x; v < nv; v += blockDim.x) {
-        uint4 u = base[v];
-        __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
-        uint4 o;
-        __half2* oh = reinterpret_cast<__half2*>(&o);
+      for (int e = threadIdx.x * 8; e < ch.len; e += blockDim.x * 8) {
+        const long long i0 = ch.start + e;
+        float v[8];
+        if (mom) {
+          const float4* pm = reinterpret_cast<const float4*>(mom + i0);
+          const float4 a = pm[0], b = pm[1];
+          v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+          v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+        } else {
+          GradVec<false> gv;
+          gv.load(g, i0);
+          gv.get(v);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 f = __bfloat1622float2(h[q]);
-          oh[q] = __floats2half2_rn(f.x * sc, f.y * sc);
+          for (int q = 0; q < 8; ++q) v[q] *= gscale;
         }
-        base[v] = o;
+        store8_image_h(mb, mm.mb_off + i0, v, sc);  // ldc == cols on the vector path
       }
     } else {
       for (int e = threadIdx.x; e < ch.len; e += blockDim.x) {
         const long long idx = ch.start + e;
+        const float v = mom ? mom[idx] : __bfloat162float(g[idx]) * gscale;
         const long long row = idx / mm.cols, col = idx - row * mm.cols;
-        __nv_bfloat16* p = reinterpret_cast<__nv_bfloat16*>(mb) + mm.mb_off + row * mm.ldc + col;
-        const __half hv = __float2half_rn(__bfloat162float(*p) * sc);
-        *reinterpret_cast<__half*>(p) = hv;
+        reinterpret_cast<__half*>(mb)[mm.mb_off + row * mm.ldc + col] = __float2half_rn(v * sc);
       }
     }
   }
 }
 
-cudaError_t launch_image16(const MomChunk* chunks, int nchunks, const MomMat* mats, void* mb, const float* iscale,
-                           int vec_ok, int num_sms, cudaStream_t s) {
+cudaError_t launch_image_fix(const MomChunk* chunks, int nchunks, const MomMat* mats, const void* const* grads,
+                             float* const* momenta, float gscale, void* mb, const float* iscale, const int* fix,
+                             int vec_ok, int num_sms, cudaStream_t s) {
   if (nchunks <= 0) return cudaSuccess;
   int grid = num_sms * 8;
   if (grid > nchunks) grid = nchunks;
-  k_image16<<<grid, 256, 0, s>>>(chunks, nchunks, mats, mb, iscale, vec_ok);
+  k_image_fix<<<grid, 256, 0, s>>>(chunks, nchunks, mats, grads, momenta, gscale, mb, iscale, fix, vec_ok);
   return cudaGetLastError();
 }
 
 cudaError_t launch_momentum(const MomChunk* chunks, int nchunks, const MomMat* mats,
                             const void* const* grads, float* const* momenta, int grad_f32, void* mb,
-                            int mb_f32, float beta, float gscale, float* partial, int vec_ok, int num_sms,
-                            cudaStream_t s) {
+                            int mb_f32, float beta, float gscale, const float* iscale, float* partial, int vec_ok,
+                            int num_sms, cudaStream_t s) {
   if (nchunks <= 0) return cudaSuccess;
   int grid = num_sms * 3;  // the resident CTAs per SM of the launch bounds
   if (grid > nchunks) grid = nchunks;
-  // the image has the gradients' element type (bf16 -> bf16 image, fp32 -> fp32)
+  // the image has the gradients' element type for fp32 plans (fp32 -> fp32);
+  // bf16 plans write fp16 at the kept scale
   if (grad_f32 != mb_f32) return cudaErrorInvalidValue;
   if (grad_f32)
-    k_momentum<true><<<grid, 256, 0, s>>>(chunks, nchunks, mats, grads, momenta, mb, beta, gscale, partial, vec_ok);
+    k_momentum<true><<<grid, 256, 0, s>>>(chunks, nchunks, mats, grads, momenta, mb, beta, gscale, nullptr, partial,
+                                          vec_ok);
   else
-    k_momentum<false><<<grid, 256, 0, s>>>(chunks, nchunks, mats, grads, momenta, mb, beta, gscale, partial, vec_ok);
+    k_momentum<false><<<grid, 256, 0, s>>>(chunks, nchunks, mats, grads, momenta, mb, beta, gscale, iscale, partial,
+                                           vec_ok);
   return cudaGetLastError();
 }
 
 cudaError_t launch_norm_finalize(const MomMat* mats, int nmats, const float* partial, float eps,
-                                 float* inv, float* iscale, float* inv_img, unsigned int* status, cudaStream_t s) {
+                                 float* inv, float* iscale, float* inv_img, int* fix, unsigned int* status,
+                                 cudaStream_t s) {
   if (nmats <= 0) return cudaSuccess;
   const int threads = 256, per = threads / 32;
   k_norm_finalize<<<(nmats + per - 1) / per, threads, 0, s>>>(mats, nmats, partial, eps, inv, iscale, inv_img,
-                                                             status);
+                                                             fix, status);
   return cudaGetLastError();
 }
 

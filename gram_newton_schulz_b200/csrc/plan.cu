@@ -126,8 +126,8 @@ struct dmu_plan_s {
   bool vec_shapes = true;
   size_t esize = 2;
   // workspace layout (bytes)
-  size_t off_status = 0, off_inv = 0, off_iscale = 0, off_invimg = 0, off_partial = 0, off_chunks = 0,
-         off_mats = 0, off_tbl = 0,
+  size_t off_status = 0, off_inv = 0, off_iscale = 0, off_invimg = 0, off_fix = 0, off_partial = 0,
+         off_chunks = 0, off_mats = 0, off_tbl = 0,
          off_mb = 0, off_gram = 0, total = 0;
   char* ws = nullptr;
   size_t ws_bytes = 0;
@@ -157,6 +157,7 @@ struct dmu_plan_s {
   // bf16 plans: per-matrix scale 2^e of the fp16 image, and inv * 2^-e
   float* iscale_dev() const { return reinterpret_cast<float*>(ws + off_iscale); }
   float* invimg_dev() const { return reinterpret_cast<float*>(ws + off_invimg); }
+  int* fix_dev() const { return reinterpret_cast<int*>(ws + off_fix); }  // image needs rewriting
   // the scale the tensor-core kernels apply to image products
   const float* inv_kernel() const { return dtype == DMU_BF16 ? invimg_dev() : inv_dev(); }
   float* partial_dev() const { return reinterpret_cast<float*>(ws + off_partial); }
@@ -783,19 +784,21 @@ dmu_status gram_f32(dmu_plan p, const float co[3], int steps, cudaStream_t s) {
 dmu_status run_normalize(dmu_plan p, int tbl, bool with_mom, float beta, float gscale, float eps, bool vec,
                          cudaStream_t s) {
   const bool f32 = p->dtype == DMU_F32;
-  CUDA_TRY(launch_momentum(p->chunks_dev(), (int)p->chunks.size(), p->mats_dev(),
-                           const_cast<const void* const*>(p->tbl_dev(tbl)),
-                           with_mom ? reinterpret_cast<float* const*>(p->tbl_dev(TBL_MOMS)) : nullptr,
-                           f32 ? 1 : 0, p->mb_dev(), f32 ? 1 : 0, beta, gscale, p->partial_dev(), vec ? 1 : 0,
-                           p->num_sms, s));
+  const void* const* src = const_cast<const void* const*>(p->tbl_dev(tbl));
+  float* const* moms = with_mom ? reinterpret_cast<float* const*>(p->tbl_dev(TBL_MOMS)) : nullptr;
+  // bf16 plans: the image is fp16(2^e M) at the scale the previous call kept
+  // for each matrix; matrices whose scale no longer fits (or that have none
+  // yet) are rewritten by the fix-up pass, which reads M (or the gradient)
+  CUDA_TRY(launch_momentum(p->chunks_dev(), (int)p->chunks.size(), p->mats_dev(), src, moms, f32 ? 1 : 0,
+                           p->mb_dev(), f32 ? 1 : 0, beta, gscale, f32 ? nullptr : p->iscale_dev(),
+                           p->partial_dev(), vec ? 1 : 0, p->num_sms, s));
   CUDA_TRY(launch_norm_finalize(p->mats_dev(), p->count, p->partial_dev(), eps, p->inv_dev(),
                                 f32 ? nullptr : p->iscale_dev(), f32 ? nullptr : p->invimg_dev(),
-                                p->status_dev(), s));
+                                f32 ? nullptr : p->fix_dev(), p->status_dev(), s));
   p->launches += 2;
   if (!f32) {
-    // the bf16 image becomes 2^e M in fp16, in place (the tensor-core operand)
-    CUDA_TRY(launch_image16(p->chunks_dev(), (int)p->chunks.size(), p->mats_dev(), p->mb_dev(), p->iscale_dev(),
-                            p->vec_shapes ? 1 : 0, p->num_sms, s));
+    CUDA_TRY(launch_image_fix(p->chunks_dev(), (int)p->chunks.size(), p->mats_dev(), src, moms, gscale, p->mb_dev(),
+                              p->iscale_dev(), p->fix_dev(), vec ? 1 : 0, p->num_sms, s));
     p->launches++;
   }
   p->eps = eps;
@@ -1036,6 +1039,8 @@ dmu_status dmu_plan_create(const dmu_shape* shapes, int count, dmu_dtype dtype, 
   off = align_up(off + sizeof(float) * count, 256);
   p->off_invimg = off;
   off = align_up(off + sizeof(float) * count, 256);
+  p->off_fix = off;
+  off = align_up(off + sizeof(int) * count, 256);
   p->off_partial = off;
   off = align_up(off + sizeof(float) * MOM_PARTIALS_PER_CHUNK * p->chunks.size(), 256);
   p->off_chunks = off;
@@ -1086,6 +1091,8 @@ dmu_status dmu_set_workspace(dmu_plan p, void* dev_ptr, size_t bytes) {
   for (int t = 0; t < NUM_TBL; ++t) p->tbl_valid[t] = false;
   p->have_mb = p->have_p = false;
   CUDA_TRY(cudaMemset(p->ws + p->off_status, 0, 16));
+  // no image scale yet: the first momentum call writes every image in its fix-up pass
+  CUDA_TRY(cudaMemset(p->ws + p->off_iscale, 0, sizeof(float) * p->count));
   CUDA_TRY(cudaMemcpy(p->ws + p->off_chunks, p->chunks.data(), sizeof(MomChunk) * p->chunks.size(),
                       cudaMemcpyHostToDevice));
   CUDA_TRY(cudaMemcpy(p->ws + p->off_mats, p->mats.data(), sizeof(MomMat) * p->mats.size(),

@@ -93,9 +93,9 @@ typedef enum {
 
 /* Precision of the Gram-space products on the bf16 path.  Gram-space
  * matrices are stored as a 16-bit pair (hi, lo = round(x - hi)).  The image
- * of M that the Gram matrix and the final product read is M rounded to bf16
- * and held in fp16 at a power-of-two scale 2^e (exact for every entry in
- * fp16's normal range); the final P X0 product multiplies it by P as one
+ * of M that the Gram matrix and the final product read is fp16(2^e M) at a
+ * power-of-two scale 2^e per matrix (for bf16 gradients and a first step,
+ * exactly M); the final P X0 product multiplies it by P as one
  * fp16 operand (F16 classes) or as an fp16 hi/lo pair (other classes).
  * Each symmetric
  * product is computed on its upper-triangle tiles and mirrored, which
@@ -200,8 +200,8 @@ DMU_API dmu_status dmu_read_status(dmu_plan plan, uint32_t* flags);
  *   which 0..4 : Gram-space matrix G, R, T, P(buffer A), P(buffer B) of
  *                matrix `index` (m*m floats, hi + lo combined);
  *   which 5    : the input image of matrix `index` (rows*cols floats, in
- *                M's units): on the bf16 path M rounded to bf16, then held
- *                as fp16 at the power-of-two scale of which 9;
+ *                M's units): on the bf16 path fp16(2^e M), read back with
+ *                the power-of-two scale 2^e of which 9;
  *   which 6    : 1/(||M||_F + eps) of every matrix (count floats);
  *   which 7    : the final P of matrix `index` (m*m floats);
  *   which 8    : bounded-wait self-test, writes nothing to `out`: a kernel
@@ -209,8 +209,10 @@ DMU_API dmu_status dmu_read_status(dmu_plan plan, uint32_t* flags);
  *                nothing completes, gives up, and sets DMU_FLAG_TIMEOUT
  *                (read it with dmu_read_status);
  *   which 9    : bf16 plans: the scale 2^e of every matrix's fp16 image
- *                (count floats), chosen so that 2^e ||M||_F is in
- *                (2^14, 2^15].
+ *                (count floats).  A matrix keeps its scale from call to
+ *                call while 2^e ||M||_F stays in (2^9, 2^15]; otherwise
+ *                (and on the plan's first call) a new one puts it in
+ *                (2^11, 2^12].
  * Synchronises `stream`. */
 DMU_API dmu_status dmu_debug_gram(dmu_plan plan, int which, int index, float* out, void* stream);
 

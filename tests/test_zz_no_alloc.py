@@ -27,12 +27,12 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else None
 
 
-def _as_plan_image(img, sc):
-    """A bf16 image as the plan path holds it: fp16 at scale sc (fp32 images
-    are kept as they are)."""
-    if img.dtype == torch.float32:
-        return img
-    return (img.float() * sc).half().float() / sc
+def _plan_image(m, sc, dtype):
+    """The image the plan path holds for fp32 values m: fp16 at the power-of
+    -two scale sc, read back in m's units (fp32 plans keep m itself)."""
+    if dtype == "f32":
+        return m
+    return (m * sc).half().float() / sc
 
 
 def _static_call(lib, g, mom, img, inv, dtype_code, beta=BETA):
@@ -66,9 +66,10 @@ def test_static_scratch_matches_plan_path_two_calls(dtype):
         assert st == dmu.OK, lib.dmu_last_error()
         torch.cuda.synchronize()
         assert torch.equal(mom_a, mom_b)
-        # the plan keeps its bf16 image as fp16 scaled by 2^e; the same values
-        # up to fp16's rounding of entries below its normal range
-        assert torch.equal(img_a, _as_plan_image(img_b, sc))
+        # this entry point writes M rounded to the dtype; the plan keeps M in
+        # fp16 at its power-of-two scale 2^e (fp32 plans: M itself)
+        assert torch.equal(img_b, mom_b.to(tdt))
+        assert torch.equal(img_a, _plan_image(mom_a, sc, dtype))
         assert float(inv_b[0]) == pytest.approx(float(inv_a[0]), rel=1e-6)
         x = mom_b.double().cpu().numpy()
         assert float(inv_b[0]) == pytest.approx(1.0 / (np.linalg.norm(x) + EPS), rel=2e-6)
@@ -98,7 +99,8 @@ def test_static_scratch_optional_outputs(drop):
         assert st == dmu.OK, lib.dmu_last_error()
         torch.cuda.synchronize()
         if img_b is not None:
-            assert torch.equal(img_a, _as_plan_image(img_b, sc))
+            assert torch.equal(img_b, g)
+            assert torch.equal(img_a, _plan_image(g.float(), sc, "bf16"))
         else:
             assert torch.equal(mom, g.float())  # beta * 0 + G
         assert float(inv_b[0]) == pytest.approx(float(inv_a[0]), rel=1e-6)
