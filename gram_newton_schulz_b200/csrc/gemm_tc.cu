@@ -180,6 +180,9 @@ __device__ __forceinline__ uint4 ld_row16(const void* p) {
 
 // One CW-column chunk of a Gram-space output tile for the thread's row i.
 // Input and outputs are bf16 hi/lo pairs (FMT_PAIR) or fp32 (FMT_F32).
+// Every rounding step is explicit (__fmul_rn, __fadd_rn, __fmaf_rn), so the
+// on-chip recursion, which repeats this arithmetic, gets the same bits
+// whatever fused multiply-adds the compiler would otherwise form.
 // `tri`: store only i <= j and mirror (symmetric outputs, except the
 // off-diagonal tiles of half-stored outputs, which are written whole).
 __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, int i, int col0,
@@ -195,7 +198,7 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
   }
   float v[CW];
 #pragma unroll
-  for (int c = 0; c < CW; ++c) v[c] = coef * __uint_as_float(r[c]);
+  for (int c = 0; c < CW; ++c) v[c] = __fmul_rn(coef, __uint_as_float(r[c]));
 
   const long long mbase = (long long)mat * pr.mat_stride;
   const long long rowoff = mbase + (long long)i * pr.ld;
@@ -208,15 +211,15 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
 #pragma unroll
       for (int q = 0; q < CW / 4; ++q) {
         const float4 t = pc[q];
-        v[4 * q] += pr.beta * t.x;
-        v[4 * q + 1] += pr.beta * t.y;
-        v[4 * q + 2] += pr.beta * t.z;
-        v[4 * q + 3] += pr.beta * t.w;
+        v[4 * q] = __fmaf_rn(pr.beta, t.x, v[4 * q]);
+        v[4 * q + 1] = __fmaf_rn(pr.beta, t.y, v[4 * q + 1]);
+        v[4 * q + 2] = __fmaf_rn(pr.beta, t.z, v[4 * q + 2]);
+        v[4 * q + 3] = __fmaf_rn(pr.beta, t.w, v[4 * q + 3]);
       }
     } else {
 #pragma unroll
       for (int c = 0; c < CW; ++c)
-        if (col0 + c < N) v[c] += pr.beta * pr.cin_f[rowoff + col0 + c];
+        if (col0 + c < N) v[c] = __fmaf_rn(pr.beta, pr.cin_f[rowoff + col0 + c], v[c]);
     }
   } else if (pr.cin_fmt == FMT_PAIR_H && pr.cin_hi) {
     const __half* ch = reinterpret_cast<const __half*>(pr.cin_hi);
@@ -236,13 +239,14 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
         unpack8_h(uh[q], fh);
         unpack8_h(ul[q], fl);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v[8 * q + e] += pr.beta * (fh[e] + fl[e]);
+        for (int e = 0; e < 8; ++e) v[8 * q + e] = __fmaf_rn(pr.beta, __fadd_rn(fh[e], fl[e]), v[8 * q + e]);
       }
     } else {
 #pragma unroll
       for (int c = 0; c < CW; ++c)
         if (col0 + c < N)
-          v[c] += pr.beta * (__half2float(ch[rowoff + col0 + c]) + __half2float(cl[rowoff + col0 + c]));
+          v[c] = __fmaf_rn(pr.beta, __fadd_rn(__half2float(ch[rowoff + col0 + c]), __half2float(cl[rowoff + col0 + c])),
+                           v[c]);
     }
   } else if (pr.cin_fmt == FMT_PAIR && pr.cin_hi) {
     if (full) {
@@ -259,15 +263,15 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
           for (int e = 0; e < 8; ++e) fl[e] = 0.f;
         }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v[8 * q + e] += pr.beta * (fh[e] + fl[e]);
+        for (int e = 0; e < 8; ++e) v[8 * q + e] = __fmaf_rn(pr.beta, __fadd_rn(fh[e], fl[e]), v[8 * q + e]);
       }
     } else {
 #pragma unroll
       for (int c = 0; c < CW; ++c) {
         if (col0 + c < N) {
           float x = bf2f(pr.cin_hi[rowoff + col0 + c]);
-          if (pr.cin_lo) x += bf2f(pr.cin_lo[rowoff + col0 + c]);
-          v[c] += pr.beta * x;
+          if (pr.cin_lo) x = __fadd_rn(x, bf2f(pr.cin_lo[rowoff + col0 + c]));
+          v[c] = __fmaf_rn(pr.beta, x, v[c]);
         }
       }
     }
@@ -276,7 +280,7 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
   if (dc >= 0 && dc < CW) {
 #pragma unroll
     for (int c = 0; c < CW; ++c)
-      if (c == dc) v[c] += pr.gamma;
+      if (c == dc) v[c] = __fadd_rn(v[c], pr.gamma);
   }
 
   for (int pass = 0; pass < 2; ++pass) {
@@ -284,7 +288,7 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
     if (pass == 1) {
       if (!pr.out2_hi && !pr.out2_f) break;
 #pragma unroll
-      for (int c = 0; c < CW; ++c) v[c] = v[c] * pr.scale2 + (c == dc ? pr.gamma2 : 0.f);
+      for (int c = 0; c < CW; ++c) v[c] = __fmaf_rn(v[c], pr.scale2, c == dc ? pr.gamma2 : 0.f);
     }
     if (fmt == FMT_PAIR_H) {
       __half* oh = reinterpret_cast<__half*>(pass == 0 ? pr.out_hi : pr.out2_hi);

@@ -104,7 +104,10 @@ __device__ __forceinline__ int find_prob(const OnchipParams& p, int t) {
 // One product's epilogue, as in the staged path's Gram epilogue:
 //   v = coef * acc + beta * Cin;  v[i][i] += 0;  out = v;  out2 = v + gamma2 I
 // Cin, out and out2 are shared-memory buffers (byte offsets from the
-// buffer base) or, for the final P, global hi/lo pairs.  Only the upper
+// buffer base) or, for the final P, global hi/lo pairs.  Every rounding
+// step is explicit (__fmul_rn, __fadd_rn, __fmaf_rn), as in the staged
+// epilogue, so the compiler's choice of fused multiply-adds cannot make the
+// two differ.  Only the upper
 // triangle (j >= i) is computed and stored; element (j, i) receives a
 // mirrored copy, so every stored matrix is exactly symmetric.
 struct EpiArgs {
@@ -217,7 +220,7 @@ __device__ __forceinline__ void epilogue(uint8_t* smem, uint32_t tacc, int q, in
     if (i >= m) continue;
     float v[OC_CW];
 #pragma unroll
-    for (int c = 0; c < OC_CW; ++c) v[c] = e.coef * __uint_as_float(r[c]);
+    for (int c = 0; c < OC_CW; ++c) v[c] = __fmul_rn(e.coef, __uint_as_float(r[c]));
     if (e.cin >= 0) {
       const uint8_t* cb = smem + e.cin * OC_BUF;
       if (col0 + OC_CW <= m) {
@@ -232,8 +235,8 @@ __device__ __forceinline__ void epilogue(uint8_t* smem, uint32_t tacc, int q, in
           for (int t = 0; t < 4; ++t) {
             const float2 fh = __bfloat1622float2(h2[t]);
             const float2 fl = __bfloat1622float2(l2[t]);
-            v[8 * qq + 2 * t] += e.beta * (fh.x + fl.x);
-            v[8 * qq + 2 * t + 1] += e.beta * (fh.y + fl.y);
+            v[8 * qq + 2 * t] = __fmaf_rn(e.beta, __fadd_rn(fh.x, fl.x), v[8 * qq + 2 * t]);
+            v[8 * qq + 2 * t + 1] = __fmaf_rn(e.beta, __fadd_rn(fh.y, fl.y), v[8 * qq + 2 * t + 1]);
           }
         }
       } else {
@@ -242,8 +245,8 @@ __device__ __forceinline__ void epilogue(uint8_t* smem, uint32_t tacc, int q, in
           if (col0 + c < m) {
             const uint32_t o = oc_off(i, col0 + c);
             float x = bf(*reinterpret_cast<const __nv_bfloat16*>(cb + o));
-            x += bf(*reinterpret_cast<const __nv_bfloat16*>(cb + OC_PART + o));
-            v[c] += e.beta * x;
+            x = __fadd_rn(x, bf(*reinterpret_cast<const __nv_bfloat16*>(cb + OC_PART + o)));
+            v[c] = __fmaf_rn(e.beta, x, v[c]);
           }
         }
       }
@@ -251,14 +254,14 @@ __device__ __forceinline__ void epilogue(uint8_t* smem, uint32_t tacc, int q, in
     const int dc = i - col0;
 #pragma unroll
     for (int c = 0; c < OC_CW; ++c)
-      if (c == dc) v[c] += 0.f;
+      if (c == dc) v[c] = __fadd_rn(v[c], 0.f);
     if (e.out >= 0)
       store_chunk(smem + e.out * OC_BUF, nullptr, nullptr, 0, m, i, col0, v);
     else
       store_chunk(nullptr, e.g_hi, e.g_lo, e.ld, m, i, col0, v);
     if (e.out2 != -1) {
 #pragma unroll
-      for (int c = 0; c < OC_CW; ++c) v[c] = v[c] * 1.f + (c == dc ? e.gamma2 : 0.f);
+      for (int c = 0; c < OC_CW; ++c) v[c] = __fmaf_rn(v[c], 1.f, c == dc ? e.gamma2 : 0.f);
       if (e.out2 >= 0)
         store_chunk(smem + e.out2 * OC_BUF, nullptr, nullptr, 0, m, i, col0, v);
       else

@@ -146,10 +146,12 @@ __global__ void __launch_bounds__(256, 3) k_momentum(const MomChunk* __restrict_
             float v[8];
             gv[u].get(v);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) v[q] *= gscale;
-            if (mom) {
-              v[0] += beta * ma[u].x; v[1] += beta * ma[u].y; v[2] += beta * ma[u].z; v[3] += beta * ma[u].w;
-              v[4] += beta * mc[u].x; v[5] += beta * mc[u].y; v[6] += beta * mc[u].z; v[7] += beta * mc[u].w;
+            for (int q = 0; q < 8; ++q) v[q] = __fmul_rn(v[q], gscale);
+            if (mom) {  // M = round(beta M + round(s G)), no other contraction
+              v[0] = __fmaf_rn(beta, ma[u].x, v[0]); v[1] = __fmaf_rn(beta, ma[u].y, v[1]);
+              v[2] = __fmaf_rn(beta, ma[u].z, v[2]); v[3] = __fmaf_rn(beta, ma[u].w, v[3]);
+              v[4] = __fmaf_rn(beta, mc[u].x, v[4]); v[5] = __fmaf_rn(beta, mc[u].y, v[5]);
+              v[6] = __fmaf_rn(beta, mc[u].z, v[6]); v[7] = __fmaf_rn(beta, mc[u].w, v[7]);
               float4* q0 = reinterpret_cast<float4*>(mom + i0);
               q0[0] = make_float4(v[0], v[1], v[2], v[3]);
               q0[1] = make_float4(v[4], v[5], v[6], v[7]);
@@ -169,9 +171,9 @@ __global__ void __launch_bounds__(256, 3) k_momentum(const MomChunk* __restrict_
         const long long idx = ch.start + e;
         float v = F32 ? reinterpret_cast<const float*>(g)[idx]
                       : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(g)[idx]);
-        v *= gscale;
+        v = __fmul_rn(v, gscale);
         if (mom) {
-          v += beta * mom[idx];
+          v = __fmaf_rn(beta, mom[idx], v);
           mom[idx] = v;
         }
         ss += v * v;
@@ -264,14 +266,14 @@ __global__ void __launch_bounds__(256) k_image_fix(const MomChunk* __restrict__ 
           gv.load(g, i0);
           gv.get(v);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) v[q] *= gscale;
+          for (int q = 0; q < 8; ++q) v[q] = __fmul_rn(v[q], gscale);
         }
         store8_image_h(mb, mm.mb_off + i0, v, sc);  // ldc == cols on the vector path
       }
     } else {
       for (int e = threadIdx.x; e < ch.len; e += blockDim.x) {
         const long long idx = ch.start + e;
-        const float v = mom ? mom[idx] : __bfloat162float(g[idx]) * gscale;
+        const float v = mom ? mom[idx] : __fmul_rn(__bfloat162float(g[idx]), gscale);
         const long long row = idx / mm.cols, col = idx - row * mm.cols;
         reinterpret_cast<__half*>(mb)[mm.mb_off + row * mm.ldc + col] = __float2half_rn(v * sc);
       }

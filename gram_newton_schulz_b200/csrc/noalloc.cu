@@ -72,8 +72,11 @@ __global__ void __launch_bounds__(256) k_mom_static(const void* __restrict__ gra
         if (mom) {
           float4* pm = reinterpret_cast<float4*>(mom + idx);
           const float4 a = pm[0], b = pm[1];
-          v[0] += beta * a.x; v[1] += beta * a.y; v[2] += beta * a.z; v[3] += beta * a.w;
-          v[4] += beta * b.x; v[5] += beta * b.y; v[6] += beta * b.z; v[7] += beta * b.w;
+          // M = round(beta M + G): one fused multiply-add, as in the plan path
+          v[0] = __fmaf_rn(beta, a.x, v[0]); v[1] = __fmaf_rn(beta, a.y, v[1]);
+          v[2] = __fmaf_rn(beta, a.z, v[2]); v[3] = __fmaf_rn(beta, a.w, v[3]);
+          v[4] = __fmaf_rn(beta, b.x, v[4]); v[5] = __fmaf_rn(beta, b.y, v[5]);
+          v[6] = __fmaf_rn(beta, b.z, v[6]); v[7] = __fmaf_rn(beta, b.w, v[7]);
           pm[0] = make_float4(v[0], v[1], v[2], v[3]);
           pm[1] = make_float4(v[4], v[5], v[6], v[7]);
         }
@@ -99,7 +102,7 @@ __global__ void __launch_bounds__(256) k_mom_static(const void* __restrict__ gra
         float v = grad_f32 ? reinterpret_cast<const float*>(grad)[idx]
                            : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(grad)[idx]);
         if (mom) {
-          v += beta * mom[idx];
+          v = __fmaf_rn(beta, mom[idx], v);
           mom[idx] = v;
         }
         ss += v * v;

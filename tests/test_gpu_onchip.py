@@ -76,7 +76,7 @@ def test_onchip_matches_oracle(dist, monkeypatch):
         p_ref = oracle.gram_trace(x0)[-1]["P"]
         p = plan.debug(7, i).cpu().numpy().astype(np.float64)
         assert np.array_equal(p, p.T)
-        assert rel(p, p_ref) < 2e-3, (r, c, rel(p, p_ref))
+        assert rel(p, p_ref) < 5e-3, (r, c, rel(p, p_ref))
     with pytest.raises(dmu.DmuError, match="on chip"):
         plan.debug(0, 0)
 

@@ -359,6 +359,10 @@ def test_cta_pair_and_single_cta_agree(prec, monkeypatch):
 
 
 def test_autotune_picks_and_caches_schedule(tmp_path):
+    """Per-shape choices: one per Gram class, one per final bucket, each
+    with the times of its candidates in the cache file; a second plan with
+    the same shapes reuses them untimed; the tuned plan then matches the
+    oracle."""
     shapes = [(1024, 4096), (4096, 1024), (512, 2048)]
     w = synth.custom("tune", shapes, seed=33)
     grads = synth.gradients(w, "cuda")
@@ -366,10 +370,13 @@ def test_autotune_picks_and_caches_schedule(tmp_path):
     plan = dmu.Plan(shapes)
     plan.momentum_normalize(grads, None, beta=0.0)
     choice = plan.autotune(cache)
-    assert choice in (0, 1, 2)
+    names = set(dmu.SCHEDULES.values())
+    assert set(choice["gram"]) == {1024, 512} and set(choice["final"]) == set(shapes)
+    assert all(v in names and v != "onchip" for part in choice.values() for v in part.values())
     text = open(cache).read()
-    assert "pair_ms=" in text and "single_ms=" in text and "single128_ms=" in text
-    # a second plan with the same shapes reuses the cached choice
+    assert "s1_ms=" in text and "s0_ms=" in text and "s2_ms=" in text
+    assert "s3_ms=" not in text  # no class here has m <= 128
+    # a second plan with the same shapes reuses the cached choices
     plan2 = dmu.Plan(shapes)
     plan2.momentum_normalize(grads, None, beta=0.0)
     assert plan2.autotune(cache) == choice
