@@ -113,12 +113,33 @@ __global__ void __launch_bounds__(256, 3) k_momentum(const MomChunk* __restrict_
                                                   const float* __restrict__ iscale,
                                                   float* __restrict__ partial, int vec) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // a chunk's descriptor and its matrix's pointers form a chain of dependent
+  // loads: the next chunk's are fetched while this chunk streams
+  struct Meta {
+    MomChunk ch;
+    long long mb_off;
+    float sc;
+    const void* g;
+    float* mom;
+  };
+  auto fetch = [&](int c) {
+    Meta m;
+    m.ch = chunks[c];
+    m.mb_off = mats[m.ch.slot].mb_off;
+    m.sc = F32 ? 1.f : iscale[m.ch.slot];
+    m.g = grads[m.ch.slot];
+    m.mom = momenta ? momenta[m.ch.slot] : nullptr;
+    return m;
+  };
+  Meta next = blockIdx.x < nchunks ? fetch(blockIdx.x) : Meta{};
   for (int c = blockIdx.x; c < nchunks; c += gridDim.x) {
-    const MomChunk ch = chunks[c];
-    const long long mb_off = mats[ch.slot].mb_off;
-    const float sc = F32 ? 1.f : iscale[ch.slot];
-    const void* __restrict__ g = grads[ch.slot];
-    float* __restrict__ mom = momenta ? momenta[ch.slot] : nullptr;
+    const Meta cur = next;
+    if (c + (int)gridDim.x < nchunks) next = fetch(c + gridDim.x);
+    const MomChunk ch = cur.ch;
+    const long long mb_off = cur.mb_off;
+    const float sc = cur.sc;
+    const void* __restrict__ g = cur.g;
+    float* __restrict__ mom = cur.mom;
     const int s0 = warp * MOM_SLICE;
     const int s1 = min(ch.len, s0 + MOM_SLICE);
     float ss = 0.f;
