@@ -752,14 +752,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
 constexpr int BM2 = 256;
 constexpr int HALF_BYTES = 128 * 128;  // 128 rows x 128-byte K row
 
-// K atoms (128-byte rows) per stage.  Measured on the GPU, each stage
-// boundary (commit, barrier wait, fence) costs several hundred cycles of the
-// issuing thread beyond the MMAs, so the one-MMA-per-slice configurations
-// take three atoms (12 MMAs, two 96 KB stages) per stage; the split
-// configurations already issue 8-12 MMAs per atom.
-template <int NA, int NB>
+// K atoms (128-byte rows) per stage.  By default the one-MMA-per-slice
+// configurations take three atoms (12 MMAs, two 96 KB stages) per stage, to
+// amortise the fixed cost of a stage boundary (commit, barrier wait, fence);
+// the split configurations already issue 8-12 MMAs per atom.  KATV > 0
+// overrides the default: fewer atoms per stage mean more stages, so more
+// bytes are in flight while the tensor cores work on one stage (2 atoms:
+// three 64 KB stages; 1 atom: six 32 KB stages).  The schedule cache picks
+// among them per Gram class.
+template <int NA, int NB, int KATV = 0>
 struct Tc2Cfg {
-  static constexpr int KAT = (NA + NB <= 2) ? 3 : 1;
+  static constexpr int KAT = KATV > 0 ? KATV : ((NA + NB <= 2) ? 3 : 1);
   static constexpr int STAGE_BYTES = (NA + NB) * HALF_BYTES * KAT;
   static constexpr int STAGES = (200 * 1024) / STAGE_BYTES;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
@@ -785,10 +788,10 @@ __device__ __forceinline__ bool wait_bar_cluster(uint32_t bar, uint32_t parity, 
   }
 }
 
-template <int NA, int NB, int KIND>
+template <int NA, int NB, int KIND, int KATV>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     k_gemm_tc2(const __grid_constant__ GemmParams p) {
-  using Cfg = Tc2Cfg<NA, NB>;
+  using Cfg = Tc2Cfg<NA, NB, KATV>;
   constexpr int S = Cfg::STAGES;
   constexpr int KATOMS = Cfg::KAT;
   constexpr int ATOM_E = KIND == KIND_TF32 ? 32 : 64;  // elements per 128-byte K row
@@ -1098,10 +1101,10 @@ static cudaError_t configure_one() {
                               TcCfg<NA, NB, TBN>::SMEM_BYTES);
 }
 
-template <int NA, int NB, int KIND>
+template <int NA, int NB, int KIND, int KATV = 0>
 static cudaError_t configure_two() {
-  return cudaFuncSetAttribute(k_gemm_tc2<NA, NB, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              Tc2Cfg<NA, NB>::SMEM_BYTES);
+  return cudaFuncSetAttribute(k_gemm_tc2<NA, NB, KIND, KATV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              Tc2Cfg<NA, NB, KATV>::SMEM_BYTES);
 }
 
 cudaError_t gemm_tc_configure() {
@@ -1123,6 +1126,8 @@ cudaError_t gemm_tc_configure() {
   if ((e = configure_two<2, 2, KIND_BF16>()) != cudaSuccess) return e;
   if ((e = configure_two<1, 1, KIND_TF32>()) != cudaSuccess) return e;
   if ((e = configure_two<1, 1, KIND_F16>()) != cudaSuccess) return e;
+  if ((e = configure_two<1, 1, KIND_F16, 2>()) != cudaSuccess) return e;
+  if ((e = configure_two<1, 1, KIND_F16, 1>()) != cudaSuccess) return e;
   if ((e = configure_two<2, 1, KIND_F16>()) != cudaSuccess) return e;
   return cudaSuccess;
 }
@@ -1145,22 +1150,26 @@ static cudaError_t launch_one(const GemmParams& p, int num_sms, int tbn, cudaStr
   return cudaGetLastError();
 }
 
-template <int NA, int NB, int KIND>
+template <int NA, int NB, int KIND, int KATV = 0>
 static cudaError_t launch_two(const GemmParams& p, int num_sms, cudaStream_t s) {
   int pairs = num_sms / 2;
   if (p.total_tiles < pairs) pairs = p.total_tiles;
   if (pairs <= 0) return cudaSuccess;
-  k_gemm_tc2<NA, NB, KIND><<<2 * pairs, GEMM_THREADS, Tc2Cfg<NA, NB>::SMEM_BYTES, s>>>(p);
+  k_gemm_tc2<NA, NB, KIND, KATV><<<2 * pairs, GEMM_THREADS, Tc2Cfg<NA, NB, KATV>::SMEM_BYTES, s>>>(p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm_tc2(const GemmParams& p, int na, int nb, int kind, int num_sms, cudaStream_t s) {
+cudaError_t launch_gemm_tc2(const GemmParams& p, int na, int nb, int kind, int num_sms, int kat, cudaStream_t s) {
   if (kind == KIND_TF32) {
     if (na == 1 && nb == 1) return launch_two<1, 1, KIND_TF32>(p, num_sms, s);
     return cudaErrorInvalidValue;
   }
   if (kind == KIND_F16) {
-    if (na == 1 && nb == 1) return launch_two<1, 1, KIND_F16>(p, num_sms, s);
+    if (na == 1 && nb == 1) {
+      if (kat == 1) return launch_two<1, 1, KIND_F16, 1>(p, num_sms, s);
+      if (kat == 2) return launch_two<1, 1, KIND_F16, 2>(p, num_sms, s);
+      return launch_two<1, 1, KIND_F16>(p, num_sms, s);
+    }
     if (na == 2 && nb == 1) return launch_two<2, 1, KIND_F16>(p, num_sms, s);
     return cudaErrorInvalidValue;
   }

@@ -120,26 +120,6 @@ struct EpiArgs {
   long long ld;
 };
 
-__device__ __forceinline__ void st_pair_smem(uint8_t* buf, int i, int j, float v) {
-  const __nv_bfloat16 h = __float2bfloat16_rn(v);
-  const __nv_bfloat16 l = __float2bfloat16_rn(v - bf(h));
-  const uint32_t o = oc_off(i, j);
-  *reinterpret_cast<__nv_bfloat16*>(buf + o) = h;
-  *reinterpret_cast<__nv_bfloat16*>(buf + OC_PART + o) = l;
-}
-
-__device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
-  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&hi);
-  __nv_bfloat162* l = reinterpret_cast<__nv_bfloat162*>(&lo);
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const __nv_bfloat16 h0 = __float2bfloat16_rn(v[2 * q]);
-    const __nv_bfloat16 h1 = __float2bfloat16_rn(v[2 * q + 1]);
-    h[q] = __halves2bfloat162(h0, h1);
-    l[q] = __halves2bfloat162(__float2bfloat16_rn(v[2 * q] - bf(h0)), __float2bfloat16_rn(v[2 * q + 1] - bf(h1)));
-  }
-}
-
 __device__ __forceinline__ void split8_h(const float* v, uint4& hi, uint4& lo) {
   __half2* h = reinterpret_cast<__half2*>(&hi);
   __half2* l = reinterpret_cast<__half2*>(&lo);
@@ -159,49 +139,82 @@ __device__ __forceinline__ void st_pair_h(__half* hi, __half* lo, long long o, f
   lo[o] = __float2half_rn(v - __half2float(h));
 }
 
-// Stores of one chunk (row i, columns col0 .. col0 + 15, only j < m) to a
-// shared-memory bf16 pair `buf` or to a global fp16 pair (hi, lo, stride ld).
-__device__ __forceinline__ void store_chunk(uint8_t* buf, __half* ghi, __half* glo, long long ld,
-                                            int m, int i, int col0, const float (&v)[OC_CW]) {
-  const bool full = col0 + OC_CW <= m;
-  const bool all_upper = i <= col0;
-  if (full && all_upper) {
+__device__ __forceinline__ uint32_t bf_bits(__nv_bfloat16 x) { return (uint32_t)__bfloat16_as_ushort(x); }
+
+// Shared-memory stores of one chunk (row i, columns col0 .. col0 + 15, only
+// j < m): row i's upper elements (j >= i) and their mirror images (j, i).
+// Each value is split into its bf16 hi/lo pair once and stored twice; the
+// mirror addresses come from per-thread constants (col0 is a multiple of 16,
+// so j & 7 is known at compile time in the unrolled loop).
+__device__ __forceinline__ void store_chunk_smem(uint8_t* buf, int m, int i, int col0, const float (&v)[OC_CW]) {
+  uint32_t hi[OC_CW], lo[OC_CW];
+#pragma unroll
+  for (int c = 0; c < OC_CW; ++c) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(v[c]);
+    hi[c] = bf_bits(h);
+    lo[c] = bf_bits(__float2bfloat16_rn(__fsub_rn(v[c], bf(h))));
+  }
+  if (col0 + OC_CW <= m && i <= col0) {
 #pragma unroll
     for (int q = 0; q < OC_CW / 8; ++q) {
-      uint4 h, l;
-      if (buf) {
-        split8(v + 8 * q, h, l);
-        const uint32_t o = oc_off(i, col0 + 8 * q);
-        *reinterpret_cast<uint4*>(buf + o) = h;
-        *reinterpret_cast<uint4*>(buf + OC_PART + o) = l;
-      } else {
-        split8_h(v + 8 * q, h, l);
-        *reinterpret_cast<uint4*>(ghi + i * ld + col0 + 8 * q) = h;
-        *reinterpret_cast<uint4*>(glo + i * ld + col0 + 8 * q) = l;
-      }
+      const uint4 h = make_uint4(hi[8 * q] | (hi[8 * q + 1] << 16), hi[8 * q + 2] | (hi[8 * q + 3] << 16),
+                                 hi[8 * q + 4] | (hi[8 * q + 5] << 16), hi[8 * q + 6] | (hi[8 * q + 7] << 16));
+      const uint4 l = make_uint4(lo[8 * q] | (lo[8 * q + 1] << 16), lo[8 * q + 2] | (lo[8 * q + 3] << 16),
+                                 lo[8 * q + 4] | (lo[8 * q + 5] << 16), lo[8 * q + 6] | (lo[8 * q + 7] << 16));
+      const uint32_t o = oc_off(i, col0 + 8 * q);
+      *reinterpret_cast<uint4*>(buf + o) = h;
+      *reinterpret_cast<uint4*>(buf + OC_PART + o) = l;
     }
   } else {
 #pragma unroll
     for (int c = 0; c < OC_CW; ++c) {
       const int j = col0 + c;
       if (j < m && i <= j) {
-        if (buf)
-          st_pair_smem(buf, i, j, v[c]);
-        else
-          st_pair_h(ghi, glo, i * ld + j, v[c]);
+        const uint32_t o = oc_off(i, j);
+        *reinterpret_cast<uint16_t*>(buf + o) = (uint16_t)hi[c];
+        *reinterpret_cast<uint16_t*>(buf + OC_PART + o) = (uint16_t)lo[c];
       }
     }
   }
-  // mirrored stores (j, i) for j > i
+  // mirrored stores (j, i) for j > i: offset (i / 64) ATOM + j 128 +
+  // (((i / 8) % 8) ^ (j % 8)) 16 + (i % 8) 2
+  const uint32_t mbase = (uint32_t)((i >> 6) * OC_ATOM + (i & 7) * 2 + col0 * 128);
+  const uint32_t ci = (uint32_t)((i >> 3) & 7);
 #pragma unroll
   for (int c = 0; c < OC_CW; ++c) {
     const int j = col0 + c;
     if (j < m && i < j) {
-      if (buf)
-        st_pair_smem(buf, j, i, v[c]);
-      else
-        st_pair_h(ghi, glo, j * ld + i, v[c]);
+      const uint32_t o = mbase + c * 128 + ((ci ^ (uint32_t)(c & 7)) << 4);
+      *reinterpret_cast<uint16_t*>(buf + o) = (uint16_t)hi[c];
+      *reinterpret_cast<uint16_t*>(buf + OC_PART + o) = (uint16_t)lo[c];
     }
+  }
+}
+
+// Global stores of one chunk of the final P (row i, columns col0 .. col0 +
+// 15, only j < m) as an fp16 hi/lo pair (row stride ld): the upper elements
+// and their mirror images, as the staged path writes them.
+__device__ __forceinline__ void store_chunk_global(__half* ghi, __half* glo, long long ld, int m, int i, int col0,
+                                                   const float (&v)[OC_CW]) {
+  if (col0 + OC_CW <= m && i <= col0) {
+#pragma unroll
+    for (int q = 0; q < OC_CW / 8; ++q) {
+      uint4 h, l;
+      split8_h(v + 8 * q, h, l);
+      *reinterpret_cast<uint4*>(ghi + i * ld + col0 + 8 * q) = h;
+      *reinterpret_cast<uint4*>(glo + i * ld + col0 + 8 * q) = l;
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < OC_CW; ++c) {
+      const int j = col0 + c;
+      if (j < m && i <= j) st_pair_h(ghi, glo, i * ld + j, v[c]);
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < OC_CW; ++c) {
+    const int j = col0 + c;
+    if (j < m && i < j) st_pair_h(ghi, glo, j * ld + i, v[c]);
   }
 }
 
@@ -256,16 +269,16 @@ __device__ __forceinline__ void epilogue(uint8_t* smem, uint32_t tacc, int q, in
     for (int c = 0; c < OC_CW; ++c)
       if (c == dc) v[c] = __fadd_rn(v[c], 0.f);
     if (e.out >= 0)
-      store_chunk(smem + e.out * OC_BUF, nullptr, nullptr, 0, m, i, col0, v);
+      store_chunk_smem(smem + e.out * OC_BUF, m, i, col0, v);
     else
-      store_chunk(nullptr, e.g_hi, e.g_lo, e.ld, m, i, col0, v);
+      store_chunk_global(e.g_hi, e.g_lo, e.ld, m, i, col0, v);
     if (e.out2 != -1) {
 #pragma unroll
       for (int c = 0; c < OC_CW; ++c) v[c] = __fmaf_rn(v[c], 1.f, c == dc ? e.gamma2 : 0.f);
       if (e.out2 >= 0)
-        store_chunk(smem + e.out2 * OC_BUF, nullptr, nullptr, 0, m, i, col0, v);
+        store_chunk_smem(smem + e.out2 * OC_BUF, m, i, col0, v);
       else
-        store_chunk(nullptr, e.g_hi, e.g_lo, e.ld, m, i, col0, v);
+        store_chunk_global(e.g_hi, e.g_lo, e.ld, m, i, col0, v);
     }
   }
 }

@@ -70,12 +70,21 @@ struct GClass {
   // through MN-major maps (64 x 64 boxes).
   bool half = false;
   int map_t = -1, map_pf_t = -1;
-  // Tile schedule of this class's Gram recursion: -1 the plan's, 0/1/2 the
-  // staged schedules, SCHED_ONCHIP the whole recursion in one CTA per matrix
+  // Tile schedule of this class's Gram recursion: -1 the plan's, a staged
+  // tile schedule (TILE_SCHEDS), or SCHED_ONCHIP: the whole recursion in one
+  // CTA per matrix
   int sched = -1;
 };
 
+// Schedules: 0 single CTAs, 128 x 256 tiles; 1 CTA pairs, 256 x 256 tiles;
+// 2 single CTAs, 128 x 128 tiles; 3 on chip (m <= 128); 4 and 5 CTA pairs
+// whose one-MMA-per-slice fp16 kernels take 2 and 1 K atoms per stage
+// (three and six stages) instead of 3 (two stages).
 constexpr int SCHED_ONCHIP = 3;
+constexpr int TILE_SCHEDS[5] = {0, 1, 2, 4, 5};
+bool is_pair(int sched) { return sched == 1 || sched == 4 || sched == 5; }
+int pair_kat(int sched) { return sched == 4 ? 2 : (sched == 5 ? 1 : 0); }
+bool valid_sched(int v) { return v >= 0 && v <= 5; }
 
 bool onchip_eligible(dmu_dtype dtype, const GClass& g) {
   return dtype == DMU_BF16 && g.prec == DMU_PREC_SPLIT3 && g.m <= ONCHIP_MAX_M;
@@ -271,7 +280,7 @@ dmu_status run_tc(dmu_plan p, std::vector<Prob>& probs, int na, int nb, int kind
       g.b_map = slot(probs[i].bmap);
       g.a_map_t = probs[i].amap_t >= 0 ? slot(probs[i].amap_t) : g.a_map;
       g.b_map_t = probs[i].bmap_t >= 0 ? slot(probs[i].bmap_t) : g.b_map;
-      g.tiles_per_mat = tiles_for(g.M, g.N, g.sym != 0, &g.tiles_m, &g.tiles_n, sched == 1 ? 256 : BM,
+      g.tiles_per_mat = tiles_for(g.M, g.N, g.sym != 0, &g.tiles_m, &g.tiles_n, is_pair(sched) ? 256 : BM,
                                   sched == 2 ? 128 : BN);
       g.tile_begin = tiles;
       tiles += g.count * g.tiles_per_mat;
@@ -283,8 +292,8 @@ dmu_status run_tc(dmu_plan p, std::vector<Prob>& probs, int na, int nb, int kind
     gp.total_tiles = tiles;
     gp.status = p->status_dev();
     gp.timeout_ns = p->timeout_ns;
-    if (sched == 1)
-      CUDA_TRY(launch_gemm_tc2(gp, na, nb, kind, p->num_sms, s));
+    if (is_pair(sched))
+      CUDA_TRY(launch_gemm_tc2(gp, na, nb, kind, p->num_sms, pair_kat(sched), s));
     else
       CUDA_TRY(launch_gemm_tc(gp, na, nb, kind, p->num_sms, sched == 2 ? 128 : 256, s));
     p->launches++;
@@ -529,7 +538,7 @@ dmu_status run_products(dmu_plan p, const std::vector<std::pair<Product, bool>>&
                         const float co[3], int p_in, int p_out, cudaStream_t s) {
   const int precs[5] = {DMU_PREC_F16, DMU_PREC_TF32, DMU_PREC_FAST, DMU_PREC_SPLIT2, DMU_PREC_SPLIT3};
   for (int pr : precs) {
-    for (int sched = 0; sched < SCHED_ONCHIP; ++sched) {
+    for (int sched : TILE_SCHEDS) {
       std::vector<Prob> probs;
       for (size_t c = 0; c < p->classes.size(); ++c) {
         if (p->classes[c].prec != pr || p->class_sched((int)c) != sched) continue;
@@ -648,7 +657,7 @@ dmu_status gram_bf16(dmu_plan p, const float co[3], int steps, cudaStream_t s) {
     syrk_sched.push_back(p->onchip(b.cls) ? p->sched : p->class_sched(b.cls));
   }
   dmu_status st = DMU_OK;
-  for (int sched = 0; sched < SCHED_ONCHIP; ++sched) {
+  for (int sched : TILE_SCHEDS) {
     std::vector<Prob> group;
     for (size_t i = 0; i < syrk.size(); ++i)
       if (syrk_sched[i] == sched) group.push_back(syrk[i]);
@@ -857,7 +866,7 @@ dmu_status final_launch(dmu_plan p, bool with_w, bool with_o, float lr, cudaStre
     probs.push_back(pr);
     scheds.push_back(p->final_sched(b));
   }
-  for (int sched = 0; sched < SCHED_ONCHIP; ++sched) {
+  for (int sched : TILE_SCHEDS) {
     std::vector<Prob> group;
     for (size_t i = 0; i < probs.size(); ++i)
       if (scheds[i] == sched) group.push_back(probs[i]);
@@ -924,7 +933,7 @@ dmu_status dmu_plan_create(const dmu_shape* shapes, int count, dmu_dtype dtype, 
   if (const char* e = std::getenv("DMU_CTA_PAIR")) p->sched = std::atoi(e) != 0 ? 1 : 0;
   if (const char* e = std::getenv("DMU_SCHEDULE")) {
     const int v = std::atoi(e);
-    if (v >= 0 && v <= 2) p->sched = v;
+    if (valid_sched(v) && v != SCHED_ONCHIP) p->sched = v;
   }
   if (const char* e = std::getenv("DMU_HALF")) p->half_store = std::atoi(e) != 0;
 
@@ -1410,7 +1419,7 @@ static std::map<std::string, int> read_cache(const char* path) {
     std::istringstream ls(line);
     std::string k;
     int v = -1;
-    if ((ls >> k >> v) && v >= 0 && v <= SCHED_ONCHIP) out[k] = v;
+    if ((ls >> k >> v) && valid_sched(v)) out[k] = v;
   }
   return out;
 }
@@ -1478,6 +1487,10 @@ dmu_status dmu_autotune(dmu_plan p, const char* cache_path, void* stream) {
       continue;
     }
     std::vector<int> cand = {1, 0, 2};
+    if (g.kind == KIND_F16) {  // stage-depth variants of the CTA-pair fp16 kernel
+      cand.push_back(4);
+      cand.push_back(5);
+    }
     if (onchip_eligible(p->dtype, g)) cand.push_back(SCHED_ONCHIP);
     std::ostringstream times;
     int best = -1;
@@ -1511,7 +1524,7 @@ dmu_status dmu_autotune(dmu_plan p, const char* cache_path, void* stream) {
     const GClass& g = p->classes[b.cls];
     const std::string key = final_key(p, dev, b);
     auto hit = cache.find(key);
-    if (hit != cache.end() && hit->second < SCHED_ONCHIP) {
+    if (hit != cache.end() && hit->second != SCHED_ONCHIP) {
       b.fsched = hit->second;
       continue;
     }

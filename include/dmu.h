@@ -220,8 +220,9 @@ DMU_API dmu_status dmu_debug_gram(dmu_plan plan, int which, int index, float* ou
  * 2.4: per-shape kernel configurations are tuned once and cached).
  *   - Every Gram class (all matrices with one m) is timed alone over the
  *     whole quintic recursion (K = 5) with CTA pairs (256 x 256 tiles),
- *     single CTAs (128 x 256 and 128 x 128 tiles) and, for split-bf16
- *     classes with m <= 128, the on-chip recursion; CTA pairs win ties.
+ *     single CTAs (128 x 256 and 128 x 128 tiles), for scaled-fp16 classes
+ *     CTA pairs with 2 and 1 K atoms per stage, and for split-bf16 classes
+ *     with m <= 128 the on-chip recursion; CTA pairs win ties.
  *   - Every shape bucket's final GEMM + update is then timed alone with the
  *     three tile schedules.  Its weight writes go to the class's free
  *     Gram-space scratch, never to the caller's weights (buckets whose
@@ -243,8 +244,10 @@ DMU_API dmu_status dmu_autotune(dmu_plan plan, const char* cache_path, void* str
 DMU_API int dmu_get_schedule(dmu_plan plan);
 
 /* Schedule of the Gram recursion of matrix `index`'s class (all matrices
- * with its m): 0, 1, 2 as above, or 3 = the whole recursion on chip (one
- * CTA per matrix, m <= 128, split-bf16 precision).  -1 for a bad argument. */
+ * with its m): 0, 1, 2 as above; 3 = the whole recursion on chip (one CTA
+ * per matrix, m <= 128, split-bf16 precision); 4 and 5 = CTA pairs whose
+ * one-MMA-per-slice fp16 kernels stage 2 and 1 K atoms of 64 (three and six
+ * stages) instead of 3 (two stages).  -1 for a bad argument. */
 DMU_API int dmu_get_gram_schedule(dmu_plan plan, int index);
 
 /* Tile schedule (0, 1, 2) of the final GEMM of matrix `index`'s bucket. */

@@ -343,14 +343,16 @@ def test_half_and_full_storage_agree(prec, monkeypatch):
 
 @pytest.mark.parametrize("prec", ["auto", "split3", "tf32"])
 def test_cta_pair_and_single_cta_agree(prec, monkeypatch):
-    """The CTA-pair kernels (256 x 256 tiles, cta_group::2) and the single-CTA
-    kernels (128 x 256 and 128 x 128 tiles) accumulate every element over K
-    in the same order, so they must give bitwise-equal results."""
+    """The CTA-pair kernels (256 x 256 tiles, cta_group::2, with 3, 2 or 1 K
+    atoms per stage) and the single-CTA kernels (128 x 256 and 128 x 128
+    tiles) accumulate every element over K in the same order, so they must
+    give bitwise-equal results."""
     shapes = [(1100, 3000), (3000, 1100), (512, 2048), (520, 200), (384, 384), (128, 512), (100, 300)]
     w = synth.custom("pair", shapes, seed=29)
     monkeypatch.setenv("DMU_SCHEDULE", "1")
     a = run_step(w, prec=prec)
-    for sched in ("0", "2"):
+    # 4 and 5: CTA pairs staging 2 and 1 K atoms per stage (fp16 kernels)
+    for sched in ("0", "2", "4", "5"):
         monkeypatch.setenv("DMU_SCHEDULE", sched)
         b = run_step(w, prec=prec)
         for i in range(w.count):
