@@ -33,8 +33,10 @@
 // formed, buffers R and P are the TMA staging ring (8 stages of 16 KB).
 //
 // TMEM: 4 accumulators of 128 columns (SYRK / G', R, T, P').
-// Warps: 0 TMA producer, 1 MMA issuer (one thread), 2-9 epilogue (two per
-// TMEM lane quarter, each on half of the columns).  Every mbarrier wait is
+// Warps: 0 TMA producer, 1 MMA issuer (one thread), 2-17 epilogue (four per
+// TMEM lane quarter, each on a quarter of the columns, in 8-column chunks:
+// an epilogue is a long dependent chain per warp, so more warps with
+// shorter chains finish it sooner).  Every mbarrier wait is
 // bounded by the plan's time limit; on expiry the CTA sets
 // DMU_FLAG_TIMEOUT and winds down.
 #include "dmu_internal.h"
@@ -43,13 +45,15 @@
 namespace dmu {
 namespace {
 
-constexpr int OC_THREADS = 320;
+constexpr int OC_EPI_WARPS = 16;        // four per TMEM lane quarter
+constexpr int OC_THREADS = 64 + 32 * OC_EPI_WARPS;
 constexpr int OC_ATOM = 16384;            // 128 rows x 128 bytes
 constexpr int OC_PART = 2 * OC_ATOM;      // 128 x 128 bf16
 constexpr int OC_BUF = 2 * OC_PART;       // hi + lo
 constexpr int OC_STAGES = 8;              // SYRK staging in buffers R and P
 constexpr int OC_SMEM = 1024 + 3 * OC_BUF + 512;
-constexpr int OC_CW = 16;                 // epilogue chunk width (columns)
+constexpr int OC_CW = 8;                  // epilogue chunk width (columns): one 16-byte swizzle chunk
+constexpr int OC_SLICE = 128 / (OC_EPI_WARPS / 4);  // columns per epilogue warp
 enum { BUF_G = 0, BUF_R = 1, BUF_P = 2 };
 
 static_assert(OC_STAGES * OC_ATOM == 2 * OC_BUF, "staging ring covers buffers R and P");
@@ -222,13 +226,13 @@ __device__ __forceinline__ void epilogue(uint8_t* smem, uint32_t tacc, int q, in
                                          const EpiArgs& e) {
   const int row_lo = q * 32;
   const int i = row_lo + lane;
-  for (int ch = 0; ch < 64 / OC_CW; ++ch) {
-    const int col0 = half * 64 + ch * OC_CW;
+  for (int ch = 0; ch < OC_SLICE / OC_CW; ++ch) {
+    const int col0 = half * OC_SLICE + ch * OC_CW;
     if (col0 >= m) break;
     if (col0 + OC_CW - 1 < row_lo) continue;  // chunk strictly below the diagonal
     if (row_lo >= m) break;
     uint32_t r[OC_CW];
-    ptx::tmem_ld16(tacc + (uint32_t)col0 + ((uint32_t)(q * 32) << 16), r);
+    ptx::tmem_ld8(tacc + (uint32_t)col0 + ((uint32_t)(q * 32) << 16), r);
     ptx::tmem_wait_ld();
     if (i >= m) continue;
     float v[OC_CW];
@@ -337,10 +341,10 @@ __global__ void __launch_bounds__(OC_THREADS, 1) k_gram_onchip(const __grid_cons
       ptx::mbar_init(bars.empty(s), 1);
     }
     for (int a = 0; a < 4; ++a) ptx::mbar_init(bars.acc(a), 1);
-    ptx::mbar_init(bars.epi_g(), 8);
-    ptx::mbar_init(bars.epi_r(), 8);
-    ptx::mbar_init(bars.epi_p(), 8);
-    ptx::mbar_init(bars.mat_done(), 8);
+    ptx::mbar_init(bars.epi_g(), OC_EPI_WARPS);
+    ptx::mbar_init(bars.epi_r(), OC_EPI_WARPS);
+    ptx::mbar_init(bars.epi_p(), OC_EPI_WARPS);
+    ptx::mbar_init(bars.mat_done(), OC_EPI_WARPS);
     ptx::mbar_init(bars.drain(), 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
@@ -490,10 +494,10 @@ __global__ void __launch_bounds__(OC_THREADS, 1) k_gram_onchip(const __grid_cons
     __syncwarp();
   } else {
     // ------------------------------------------------ epilogue (warps 2..9)
-    const int q = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int q = warp & 3;              // the TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;    // its column slice (OC_SLICE columns)
     uint32_t acc_n[4] = {0, 0, 0, 0};
-    const int ethr = threadIdx.x - 64;  // 0 .. 255
+    const int ethr = threadIdx.x - 64;  // 0 .. 32 * OC_EPI_WARPS - 1
     bool ok = true;
     auto wait_acc = [&](int a) -> bool {
       int w = 1;
@@ -519,7 +523,7 @@ __global__ void __launch_bounds__(OC_THREADS, 1) k_gram_onchip(const __grid_cons
         // never meet the epilogues' stores of elements < m and need no
         // ordering with them; the barrier after this phase orders both
         // before the next MMAs.
-        for (int cidx = ethr; cidx < 6 * 128 * 16; cidx += 256) {
+        for (int cidx = ethr; cidx < 6 * 128 * 16; cidx += 32 * OC_EPI_WARPS) {
           const int part = cidx >> 11, i = (cidx >> 4) & 127, j0 = (cidx & 15) * 8;
           uint8_t* pb = smem + (part >> 1) * OC_BUF + (part & 1) * OC_PART;
           if (i >= m || j0 >= m) {
