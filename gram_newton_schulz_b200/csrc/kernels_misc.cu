@@ -39,7 +39,7 @@ __device__ __forceinline__ void store8_image_h(void* __restrict__ mb, long long 
   __half2* h = reinterpret_cast<__half2*>(&u);
 #pragma unroll
   for (int q = 0; q < 4; ++q) h[q] = __floats2half2_rn(v[2 * q] * sc, v[2 * q + 1] * sc);
-  *reinterpret_cast<uint4*>(reinterpret_cast<__half*>(mb) + o) = u;
+  __stcs(reinterpret_cast<uint4*>(reinterpret_cast<__half*>(mb) + o), u);
 }
 
 __device__ __forceinline__ void store8_image(void* __restrict__ mb, int mb_f32, long long o, const float* v) {
@@ -75,7 +75,8 @@ template <bool F32> struct GradVec;
 template <> struct GradVec<false> {
   uint4 u;
   __device__ __forceinline__ void load(const void* g, long long idx) {
-    u = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(g) + idx));
+    // streamed once: evict-first, so the pass does not churn L2
+    u = __ldcs(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(g) + idx));
   }
   __device__ __forceinline__ void get(float* out) const {
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
@@ -154,8 +155,8 @@ __global__ void __launch_bounds__(256, 3) k_momentum(const MomChunk* __restrict_
             gv[u].load(g, ch.start + eu);
             if (mom) {
               const float4* pm = reinterpret_cast<const float4*>(mom + ch.start + eu);
-              ma[u] = pm[0];
-              mc[u] = pm[1];
+              ma[u] = __ldcs(pm);
+              mc[u] = __ldcs(pm + 1);
             }
           }
         }
@@ -174,8 +175,8 @@ __global__ void __launch_bounds__(256, 3) k_momentum(const MomChunk* __restrict_
               v[4] = __fmaf_rn(beta, mc[u].x, v[4]); v[5] = __fmaf_rn(beta, mc[u].y, v[5]);
               v[6] = __fmaf_rn(beta, mc[u].z, v[6]); v[7] = __fmaf_rn(beta, mc[u].w, v[7]);
               float4* q0 = reinterpret_cast<float4*>(mom + i0);
-              q0[0] = make_float4(v[0], v[1], v[2], v[3]);
-              q0[1] = make_float4(v[4], v[5], v[6], v[7]);
+              __stcs(q0, make_float4(v[0], v[1], v[2], v[3]));
+              __stcs(q0 + 1, make_float4(v[4], v[5], v[6], v[7]));
             }
 #pragma unroll
             for (int q = 0; q < 8; ++q) ss += v[q] * v[q];
