@@ -159,13 +159,13 @@ constexpr int MOM_PARTIALS_PER_CHUNK = 8;
 cudaError_t launch_momentum(const MomChunk* chunks, int nchunks, const MomMat* mats,
                             const void* const* grads, float* const* momenta, int grad_f32,
                             void* mb, int mb_f32, float beta, float gscale, const float* iscale,
-                            float* partial, int vec_ok, int num_sms, cudaStream_t s);
+                            int* fix_count, float* partial, int vec_ok, int num_sms, cudaStream_t s);
 cudaError_t launch_norm_finalize(const MomMat* mats, int nmats, const float* partial,
                                  float eps, float* inv, float* iscale, float* inv_img, int* fix,
-                                 unsigned int* status, cudaStream_t s);
+                                 int* fix_count, unsigned int* status, cudaStream_t s);
 cudaError_t launch_image_fix(const MomChunk* chunks, int nchunks, const MomMat* mats, const void* const* grads,
                              float* const* momenta, float gscale, void* mb, const float* iscale, const int* fix,
-                             int vec_ok, int num_sms, cudaStream_t s);
+                             const int* fix_count, int vec_ok, int num_sms, cudaStream_t s);
 cudaError_t launch_simt_gemm(const SimtProblem& p, cudaStream_t s);
 cudaError_t launch_identity16(void* hi, void* lo, int count, int m, long long ld, long long mat_stride, int f16,
                               cudaStream_t s);

@@ -111,9 +111,12 @@ __global__ void __launch_bounds__(256, 3) k_momentum(const MomChunk* __restrict_
                                                   const void* const* __restrict__ grads,
                                                   float* const* __restrict__ momenta,
                                                   void* __restrict__ mb, float beta, float gscale,
-                                                  const float* __restrict__ iscale,
+                                                  const float* __restrict__ iscale, int* __restrict__ fix_count,
                                                   float* __restrict__ partial, int vec) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // k_norm_finalize counts the matrices whose image needs rewriting; the
+  // previous call's fix-up pass has finished reading the count (stream order)
+  if (fix_count && blockIdx.x == 0 && threadIdx.x == 0) *fix_count = 0;
   // a chunk's descriptor and its matrix's pointers form a chain of dependent
   // loads: the next chunk's are fetched while this chunk streams
   struct Meta {
@@ -224,7 +227,7 @@ __global__ void __launch_bounds__(256, 3) k_momentum(const MomChunk* __restrict_
 __global__ void k_norm_finalize(const MomMat* __restrict__ mats, int nmats,
                                 const float* __restrict__ partial, float eps, float* __restrict__ inv,
                                 float* __restrict__ iscale, float* __restrict__ inv_img, int* __restrict__ fix,
-                                unsigned int* status) {
+                                int* __restrict__ fix_count, unsigned int* status) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= nmats) return;
@@ -252,6 +255,7 @@ __global__ void k_norm_finalize(const MomMat* __restrict__ mats, int nmats,
         iscale[warp] = sc;
       }
       fix[warp] = keep ? 0 : 1;
+      if (!keep) atomicAdd(fix_count, 1);
       inv_img[warp] = iv / sc;  // exact: sc is a power of two
     }
   }
@@ -259,14 +263,17 @@ __global__ void k_norm_finalize(const MomMat* __restrict__ mats, int nmats,
 
 // The fp16 image 2^e M of the matrices k_norm_finalize flagged, recomputed
 // from their source: M as the momentum pass left it, or, without momentum
-// state, gscale * G exactly as the momentum pass formed it.  Chunks of
-// matrices that keep their scale return at once.
+// state, gscale * G exactly as the momentum pass formed it.  When no matrix
+// is flagged (a steady run) every CTA returns after one load; otherwise
+// chunks of matrices that keep their scale are skipped.
 __global__ void __launch_bounds__(256) k_image_fix(const MomChunk* __restrict__ chunks, int nchunks,
                                                    const MomMat* __restrict__ mats,
                                                    const void* const* __restrict__ grads,
                                                    float* const* __restrict__ momenta, float gscale,
                                                    void* __restrict__ mb, const float* __restrict__ iscale,
-                                                   const int* __restrict__ fix, int vec) {
+                                                   const int* __restrict__ fix, const int* __restrict__ fix_count,
+                                                   int vec) {
+  if (*fix_count == 0) return;
   for (int c = blockIdx.x; c < nchunks; c += gridDim.x) {
     const MomChunk ch = chunks[c];
     if (!fix[ch.slot]) continue;
@@ -305,18 +312,19 @@ __global__ void __launch_bounds__(256) k_image_fix(const MomChunk* __restrict__ 
 
 cudaError_t launch_image_fix(const MomChunk* chunks, int nchunks, const MomMat* mats, const void* const* grads,
                              float* const* momenta, float gscale, void* mb, const float* iscale, const int* fix,
-                             int vec_ok, int num_sms, cudaStream_t s) {
+                             const int* fix_count, int vec_ok, int num_sms, cudaStream_t s) {
   if (nchunks <= 0) return cudaSuccess;
   int grid = num_sms * 8;
   if (grid > nchunks) grid = nchunks;
-  k_image_fix<<<grid, 256, 0, s>>>(chunks, nchunks, mats, grads, momenta, gscale, mb, iscale, fix, vec_ok);
+  k_image_fix<<<grid, 256, 0, s>>>(chunks, nchunks, mats, grads, momenta, gscale, mb, iscale, fix, fix_count,
+                                   vec_ok);
   return cudaGetLastError();
 }
 
 cudaError_t launch_momentum(const MomChunk* chunks, int nchunks, const MomMat* mats,
                             const void* const* grads, float* const* momenta, int grad_f32, void* mb,
-                            int mb_f32, float beta, float gscale, const float* iscale, float* partial, int vec_ok,
-                            int num_sms, cudaStream_t s) {
+                            int mb_f32, float beta, float gscale, const float* iscale, int* fix_count,
+                            float* partial, int vec_ok, int num_sms, cudaStream_t s) {
   if (nchunks <= 0) return cudaSuccess;
   int grid = num_sms * 3;  // the resident CTAs per SM of the launch bounds
   if (grid > nchunks) grid = nchunks;
@@ -324,21 +332,21 @@ cudaError_t launch_momentum(const MomChunk* chunks, int nchunks, const MomMat* m
   // bf16 plans write fp16 at the kept scale
   if (grad_f32 != mb_f32) return cudaErrorInvalidValue;
   if (grad_f32)
-    k_momentum<true><<<grid, 256, 0, s>>>(chunks, nchunks, mats, grads, momenta, mb, beta, gscale, nullptr, partial,
-                                          vec_ok);
+    k_momentum<true><<<grid, 256, 0, s>>>(chunks, nchunks, mats, grads, momenta, mb, beta, gscale, nullptr, nullptr,
+                                          partial, vec_ok);
   else
-    k_momentum<false><<<grid, 256, 0, s>>>(chunks, nchunks, mats, grads, momenta, mb, beta, gscale, iscale, partial,
-                                           vec_ok);
+    k_momentum<false><<<grid, 256, 0, s>>>(chunks, nchunks, mats, grads, momenta, mb, beta, gscale, iscale,
+                                           fix_count, partial, vec_ok);
   return cudaGetLastError();
 }
 
 cudaError_t launch_norm_finalize(const MomMat* mats, int nmats, const float* partial, float eps,
-                                 float* inv, float* iscale, float* inv_img, int* fix, unsigned int* status,
-                                 cudaStream_t s) {
+                                 float* inv, float* iscale, float* inv_img, int* fix, int* fix_count,
+                                 unsigned int* status, cudaStream_t s) {
   if (nmats <= 0) return cudaSuccess;
   const int threads = 256, per = threads / 32;
   k_norm_finalize<<<(nmats + per - 1) / per, threads, 0, s>>>(mats, nmats, partial, eps, inv, iscale, inv_img,
-                                                             fix, status);
+                                                             fix, fix_count, status);
   return cudaGetLastError();
 }
 

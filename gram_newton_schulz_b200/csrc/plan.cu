@@ -167,6 +167,7 @@ struct dmu_plan_s {
   float* iscale_dev() const { return reinterpret_cast<float*>(ws + off_iscale); }
   float* invimg_dev() const { return reinterpret_cast<float*>(ws + off_invimg); }
   int* fix_dev() const { return reinterpret_cast<int*>(ws + off_fix); }  // image needs rewriting
+  int* fix_count_dev() const { return fix_dev() + count; }              // how many are flagged
   // the scale the tensor-core kernels apply to image products
   const float* inv_kernel() const { return dtype == DMU_BF16 ? invimg_dev() : inv_dev(); }
   float* partial_dev() const { return reinterpret_cast<float*>(ws + off_partial); }
@@ -800,14 +801,15 @@ dmu_status run_normalize(dmu_plan p, int tbl, bool with_mom, float beta, float g
   // yet) are rewritten by the fix-up pass, which reads M (or the gradient)
   CUDA_TRY(launch_momentum(p->chunks_dev(), (int)p->chunks.size(), p->mats_dev(), src, moms, f32 ? 1 : 0,
                            p->mb_dev(), f32 ? 1 : 0, beta, gscale, f32 ? nullptr : p->iscale_dev(),
-                           p->partial_dev(), vec ? 1 : 0, p->num_sms, s));
+                           f32 ? nullptr : p->fix_count_dev(), p->partial_dev(), vec ? 1 : 0, p->num_sms, s));
   CUDA_TRY(launch_norm_finalize(p->mats_dev(), p->count, p->partial_dev(), eps, p->inv_dev(),
                                 f32 ? nullptr : p->iscale_dev(), f32 ? nullptr : p->invimg_dev(),
-                                f32 ? nullptr : p->fix_dev(), p->status_dev(), s));
+                                f32 ? nullptr : p->fix_dev(), f32 ? nullptr : p->fix_count_dev(), p->status_dev(),
+                                s));
   p->launches += 2;
   if (!f32) {
     CUDA_TRY(launch_image_fix(p->chunks_dev(), (int)p->chunks.size(), p->mats_dev(), src, moms, gscale, p->mb_dev(),
-                              p->iscale_dev(), p->fix_dev(), vec ? 1 : 0, p->num_sms, s));
+                              p->iscale_dev(), p->fix_dev(), p->fix_count_dev(), vec ? 1 : 0, p->num_sms, s));
     p->launches++;
   }
   p->eps = eps;
@@ -1049,7 +1051,7 @@ dmu_status dmu_plan_create(const dmu_shape* shapes, int count, dmu_dtype dtype, 
   p->off_invimg = off;
   off = align_up(off + sizeof(float) * count, 256);
   p->off_fix = off;
-  off = align_up(off + sizeof(int) * count, 256);
+  off = align_up(off + sizeof(int) * (count + 1), 256);
   p->off_partial = off;
   off = align_up(off + sizeof(float) * MOM_PARTIALS_PER_CHUNK * p->chunks.size(), 256);
   p->off_chunks = off;
