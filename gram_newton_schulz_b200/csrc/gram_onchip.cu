@@ -145,58 +145,102 @@ __device__ __forceinline__ void st_pair_h(__half* hi, __half* lo, long long o, f
 
 __device__ __forceinline__ uint32_t bf_bits(__nv_bfloat16 x) { return (uint32_t)__bfloat16_as_ushort(x); }
 
-// Shared-memory stores of one chunk (row i, columns col0 .. col0 + 15, only
-// j < m): row i's upper elements (j >= i) and their mirror images (j, i).
-// Each value is split into its bf16 hi/lo pair once and stored twice; the
-// mirror addresses come from per-thread constants (col0 is a multiple of 16,
-// so j & 7 is known at compile time in the unrolled loop).
-__device__ __forceinline__ void store_chunk_smem(uint8_t* buf, int m, int i, int col0, const float (&v)[OC_CW]) {
-  uint32_t hi[OC_CW], lo[OC_CW];
+// Row stores of one chunk (row i, columns col0 .. col0 + 7, only i, j < m)
+// as a bf16 hi/lo pair: rows above the chunk's diagonal 8 x 8 block and rows
+// inside it store all eight values (inside the block, the values left of
+// the diagonal are then replaced by mirror_chunk); rows below store nothing.
+__device__ __forceinline__ void store_chunk_rows(uint8_t* buf, int m, int i, int col0, const float (&v)[OC_CW]) {
+  if (i >= m || i >= col0 + OC_CW) return;
+  uint32_t hi[OC_CW / 2], lo[OC_CW / 2];  // packed pairs of columns
 #pragma unroll
-  for (int c = 0; c < OC_CW; ++c) {
-    const __nv_bfloat16 h = __float2bfloat16_rn(v[c]);
-    hi[c] = bf_bits(h);
-    lo[c] = bf_bits(__float2bfloat16_rn(__fsub_rn(v[c], bf(h))));
+  for (int c = 0; c < OC_CW; c += 2) {
+    const __nv_bfloat16 h0 = __float2bfloat16_rn(v[c]), h1 = __float2bfloat16_rn(v[c + 1]);
+    hi[c / 2] = bf_bits(h0) | (bf_bits(h1) << 16);
+    lo[c / 2] = bf_bits(__float2bfloat16_rn(__fsub_rn(v[c], bf(h0)))) |
+                (bf_bits(__float2bfloat16_rn(__fsub_rn(v[c + 1], bf(h1)))) << 16);
   }
-  if (col0 + OC_CW <= m && i <= col0) {
-#pragma unroll
-    for (int q = 0; q < OC_CW / 8; ++q) {
-      const uint4 h = make_uint4(hi[8 * q] | (hi[8 * q + 1] << 16), hi[8 * q + 2] | (hi[8 * q + 3] << 16),
-                                 hi[8 * q + 4] | (hi[8 * q + 5] << 16), hi[8 * q + 6] | (hi[8 * q + 7] << 16));
-      const uint4 l = make_uint4(lo[8 * q] | (lo[8 * q + 1] << 16), lo[8 * q + 2] | (lo[8 * q + 3] << 16),
-                                 lo[8 * q + 4] | (lo[8 * q + 5] << 16), lo[8 * q + 6] | (lo[8 * q + 7] << 16));
-      const uint32_t o = oc_off(i, col0 + 8 * q);
-      *reinterpret_cast<uint4*>(buf + o) = h;
-      *reinterpret_cast<uint4*>(buf + OC_PART + o) = l;
-    }
+  if (col0 + OC_CW <= m) {
+    const uint32_t o = oc_off(i, col0);
+    *reinterpret_cast<uint4*>(buf + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(buf + OC_PART + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
   } else {
 #pragma unroll
     for (int c = 0; c < OC_CW; ++c) {
-      const int j = col0 + c;
-      if (j < m && i <= j) {
-        const uint32_t o = oc_off(i, j);
-        *reinterpret_cast<uint16_t*>(buf + o) = (uint16_t)hi[c];
-        *reinterpret_cast<uint16_t*>(buf + OC_PART + o) = (uint16_t)lo[c];
+      if (col0 + c < m) {
+        const uint32_t o = oc_off(i, col0 + c);
+        *reinterpret_cast<uint16_t*>(buf + o) = (uint16_t)(hi[c / 2] >> (16 * (c & 1)));
+        *reinterpret_cast<uint16_t*>(buf + OC_PART + o) = (uint16_t)(lo[c / 2] >> (16 * (c & 1)));
       }
-    }
-  }
-  // mirrored stores (j, i) for j > i: offset (i / 64) ATOM + j 128 +
-  // (((i / 8) % 8) ^ (j % 8)) 16 + (i % 8) 2
-  const uint32_t mbase = (uint32_t)((i >> 6) * OC_ATOM + (i & 7) * 2 + col0 * 128);
-  const uint32_t ci = (uint32_t)((i >> 3) & 7);
-#pragma unroll
-  for (int c = 0; c < OC_CW; ++c) {
-    const int j = col0 + c;
-    if (j < m && i < j) {
-      const uint32_t o = mbase + c * 128 + ((ci ^ (uint32_t)(c & 7)) << 4);
-      *reinterpret_cast<uint16_t*>(buf + o) = (uint16_t)hi[c];
-      *reinterpret_cast<uint16_t*>(buf + OC_PART + o) = (uint16_t)lo[c];
     }
   }
 }
 
+// A fragment register holding destination elements (row, col) (low half)
+// and (row, col + 1) (high half), with the halves in the padding (row or
+// column >= m) cleared.
+__device__ __forceinline__ uint32_t pad_clear(uint32_t x, int row, int col, int m) {
+  if (row >= m || col >= m) return 0u;
+  return col + 1 < m ? x : (x & 0x0000FFFFu);
+}
+
+// The mirror images (j, i), i < j, of one chunk's upper elements (rows of
+// lane quarter q, columns col0 .. col0 + 7, as store_chunk_rows left them),
+// moved as 8 x 8 blocks: each block of 8 rows above the chunk's diagonal
+// block is loaded transposed and stored into rows col0 .. col0 + 7; the
+// diagonal block keeps its upper half and takes the transpose of that as its
+// lower half.  Destination elements in the padding are written as zero, so
+// this never meets the padding clear with a different value.  Warp-collective;
+// the warp's row stores must be ordered before it (__syncwarp).
+__device__ __forceinline__ void mirror_chunk(uint32_t buf, int m, int q, int lane, int col0) {
+  const int rq = q * 32;
+  const bool ragged = col0 + OC_CW > m || rq + 32 > m;
+  const int fr = lane >> 2, fc = 2 * (lane & 3);  // fragment elements (fr, fc) and (fr, fc + 1)
+  if (col0 >= rq + 32) {
+    // all four blocks lie above the chunk's columns
+    uint32_t h[4], l[4];
+    const uint32_t src = buf + oc_off(rq + lane, col0);
+    ptx::ldsm_x4_trans(src, h);
+    ptx::ldsm_x4_trans(src + OC_PART, l);
+    if (ragged) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        h[k] = pad_clear(h[k], col0 + fr, rq + 8 * k + fc, m);
+        l[k] = pad_clear(l[k], col0 + fr, rq + 8 * k + fc, m);
+      }
+    }
+    const uint32_t dst = buf + oc_off(col0 + (lane & 7), rq + 8 * (lane >> 3));
+    ptx::stsm_x4(dst, h);
+    ptx::stsm_x4(dst + OC_PART, l);
+    return;
+  }
+  // the chunk holds the diagonal of this quarter: blocks 0 .. kd - 1 lie above
+  const int kd = (col0 - rq) >> 3;
+  const uint32_t part = (lane & 8) ? (uint32_t)OC_PART : 0u;  // matrix 0: hi, matrix 1: lo
+  for (int k = 0; k < kd; ++k) {
+    uint32_t a, b;
+    ptx::ldsm_x2_trans(buf + oc_off(rq + 8 * k + (lane & 7), col0) + part, a, b);
+    if (ragged) {
+      a = pad_clear(a, col0 + fr, rq + 8 * k + fc, m);
+      b = pad_clear(b, col0 + fr, rq + 8 * k + fc, m);
+    }
+    ptx::stsm_x2(buf + oc_off(col0 + (lane & 7), rq + 8 * k) + part, a, b);
+  }
+  const uint32_t d = buf + oc_off(col0 + (lane & 7), col0) + part;
+  uint32_t a, b, at, bt;
+  ptx::ldsm_x2(d, a, b);
+  ptx::ldsm_x2_trans(d, at, bt);
+  const uint32_t sel = (fr > fc ? 0x0000FFFFu : 0u) | (fr > fc + 1 ? 0xFFFF0000u : 0u);
+  a = (a & ~sel) | (at & sel);
+  b = (b & ~sel) | (bt & sel);
+  if (ragged) {
+    a = pad_clear(a, col0 + fr, col0 + fc, m);
+    b = pad_clear(b, col0 + fr, col0 + fc, m);
+  }
+  ptx::stsm_x2(d, a, b);
+}
+
 // Global stores of one chunk of the final P (row i, columns col0 .. col0 +
-// 15, only j < m) as an fp16 hi/lo pair (row stride ld): the upper elements
+// 7, only j < m) as an fp16 hi/lo pair (row stride ld): the upper elements
 // and their mirror images, as the staged path writes them.
 __device__ __forceinline__ void store_chunk_global(__half* ghi, __half* glo, long long ld, int m, int i, int col0,
                                                    const float (&v)[OC_CW]) {
@@ -222,8 +266,8 @@ __device__ __forceinline__ void store_chunk_global(__half* ghi, __half* glo, lon
   }
 }
 
-__device__ __forceinline__ void epilogue(uint8_t* smem, uint32_t tacc, int q, int half, int lane, int m,
-                                         const EpiArgs& e) {
+__device__ __forceinline__ void epilogue(uint8_t* smem, uint32_t sbase, uint32_t tacc, int q, int half, int lane,
+                                         int m, const EpiArgs& e) {
   const int row_lo = q * 32;
   const int i = row_lo + lane;
   for (int ch = 0; ch < OC_SLICE / OC_CW; ++ch) {
@@ -234,7 +278,8 @@ __device__ __forceinline__ void epilogue(uint8_t* smem, uint32_t tacc, int q, in
     uint32_t r[OC_CW];
     ptx::tmem_ld8(tacc + (uint32_t)col0 + ((uint32_t)(q * 32) << 16), r);
     ptx::tmem_wait_ld();
-    if (i >= m) continue;
+    // rows >= m go through the arithmetic too (their values are never
+    // stored): the block moves below are warp-collective
     float v[OC_CW];
 #pragma unroll
     for (int c = 0; c < OC_CW; ++c) v[c] = __fmul_rn(e.coef, __uint_as_float(r[c]));
@@ -273,16 +318,21 @@ __device__ __forceinline__ void epilogue(uint8_t* smem, uint32_t tacc, int q, in
     for (int c = 0; c < OC_CW; ++c)
       if (c == dc) v[c] = __fadd_rn(v[c], 0.f);
     if (e.out >= 0)
-      store_chunk_smem(smem + e.out * OC_BUF, m, i, col0, v);
-    else
+      store_chunk_rows(smem + e.out * OC_BUF, m, i, col0, v);
+    else if (i < m)
       store_chunk_global(e.g_hi, e.g_lo, e.ld, m, i, col0, v);
     if (e.out2 != -1) {
 #pragma unroll
       for (int c = 0; c < OC_CW; ++c) v[c] = __fmaf_rn(v[c], 1.f, c == dc ? e.gamma2 : 0.f);
       if (e.out2 >= 0)
-        store_chunk_smem(smem + e.out2 * OC_BUF, m, i, col0, v);
-      else
+        store_chunk_rows(smem + e.out2 * OC_BUF, m, i, col0, v);
+      else if (i < m)
         store_chunk_global(e.g_hi, e.g_lo, e.ld, m, i, col0, v);
+    }
+    if (e.out >= 0 || e.out2 >= 0) {
+      __syncwarp();
+      if (e.out >= 0) mirror_chunk(sbase + e.out * OC_BUF, m, q, lane, col0);
+      if (e.out2 >= 0) mirror_chunk(sbase + e.out2 * OC_BUF, m, q, lane, col0);
     }
   }
 }
@@ -537,7 +587,7 @@ __global__ void __launch_bounds__(OC_THREADS, 1) k_gram_onchip(const __grid_cons
         float coef = 1.f;
         coef *= s * s;
         EpiArgs e{coef, 0.f, 0.f, -1, BUF_G, -1, nullptr, nullptr, 0};
-        epilogue(smem, tmem_base, q, half, lane, m, e);
+        epilogue(smem, base, tmem_base, q, half, lane, m, e);
       }
       epi_done(bars.epi_g(), lane);
       for (int k = 0; k < K; ++k) {
@@ -546,28 +596,28 @@ __global__ void __launch_bounds__(OC_THREADS, 1) k_gram_onchip(const __grid_cons
         if (!wait_acc(1)) { ok = false; break; }
         {
           EpiArgs e{p.c, p.b, p.a, BUF_G, BUF_R, k == 0 ? (last ? -2 : BUF_P) : -1, g_hi, g_lo, pr.ld};
-          epilogue(smem, tmem_base + 128, q, half, lane, m, e);
+          epilogue(smem, base, tmem_base + 128, q, half, lane, m, e);
         }
         epi_done(bars.epi_r(), lane);
         if (!last) {
           // ---- T = a G + R G, into buffer G
           if (!wait_acc(2)) { ok = false; break; }
           EpiArgs e{1.f, p.a, 0.f, BUF_G, BUF_G, -1, nullptr, nullptr, 0};
-          epilogue(smem, tmem_base + 256, q, half, lane, m, e);
+          epilogue(smem, base, tmem_base + 256, q, half, lane, m, e);
           epi_done(bars.epi_g(), lane);
         }
         if (k >= 1) {
           // ---- P' = a P + R P, in place (the last one to global)
           if (!wait_acc(3)) { ok = false; break; }
           EpiArgs e{1.f, p.a, 0.f, BUF_P, last ? -1 : BUF_P, -1, g_hi, g_lo, pr.ld};
-          epilogue(smem, tmem_base + 384, q, half, lane, m, e);
+          epilogue(smem, base, tmem_base + 384, q, half, lane, m, e);
           epi_done(bars.epi_p(), lane);
         }
         if (!last) {
           // ---- G' = a T + T R, in place
           if (!wait_acc(0)) { ok = false; break; }
           EpiArgs e{1.f, p.a, 0.f, BUF_G, BUF_G, -1, nullptr, nullptr, 0};
-          epilogue(smem, tmem_base, q, half, lane, m, e);
+          epilogue(smem, base, tmem_base, q, half, lane, m, e);
           epi_done(bars.epi_g(), lane);
         }
       }
