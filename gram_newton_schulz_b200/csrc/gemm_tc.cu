@@ -32,13 +32,17 @@
 
 namespace dmu {
 
+// Per-warp shared scratch of the symmetric diagonal-tile epilogue (block
+// transposes of the mirror images), after the barrier area.
+constexpr int EPI_SCRATCH_BYTES = EPI_WARPS * 2048;
+
 template <int NA, int NB, int TBN = BN>
 struct TcCfg {  // stage geometry is the same for both operand kinds
   static constexpr int B_PART = TBN * BK * 2;  // TBN rows of one 128-byte K row
   static constexpr int STAGE_BYTES = NA * A_PART_BYTES + NB * B_PART;
   static constexpr int STAGES = (200 * 1024) / STAGE_BYTES;
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + EPI_SCRATCH_BYTES;
   static_assert(STAGES >= 2 && STAGES <= 13, "stage count (barrier area holds 13)");
   static_assert(TBN == 128 || TBN == 256, "tile width");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
@@ -178,6 +182,67 @@ __device__ __forceinline__ uint4 ld_row16(const void* p) {
   return r;
 }
 
+// Symmetric diagonal tiles: the mirror images (j, i), i < j, of a chunk's
+// upper elements are moved as 8 x 8 blocks through a per-warp shared-memory
+// scratch (ldmatrix .trans / stmatrix) and written as 16-byte rows, instead
+// of one 2-byte store per element.  Scratch per epilogue warp: 32 source rows
+// x 32 bytes (the chunk as the lanes computed it) and 16 destination rows x
+// 64 bytes (its transpose); 16-byte segments are XOR-swizzled so that the
+// 8-row accesses of ldmatrix / stmatrix fall on distinct banks.
+constexpr int TRI_SCRATCH = 2048;
+static_assert(EPI_SCRATCH_BYTES == EPI_WARPS * TRI_SCRATCH, "scratch per epilogue warp");
+static_assert(CW == 16, "the block-transpose mirror moves 32 x 16 chunks");
+__device__ __forceinline__ uint32_t tri_src(uint32_t scr, int r, int seg) {
+  return scr + r * 32 + ((seg ^ ((r >> 2) & 1)) << 4);
+}
+__device__ __forceinline__ uint32_t tri_dst(uint32_t scr, int r, int seg) {
+  return scr + 1024 + r * 64 + ((seg ^ ((r >> 1) & 3)) << 4);
+}
+
+// One 16-bit part (hi or lo) of the mirror images of a 32 x CW chunk (rows
+// row_lo .. row_lo + 31, one per lane, x0 / x1 = this lane's 16 packed
+// values; columns col0 .. col0 + 15; the whole chunk inside the matrix).
+// Destination rows R = col0 .. col0 + 15, 8-column segments C0 = row_lo +
+// 8 s: segments left of the diagonal are written from the transpose, the
+// segment holding (R, R) merges the transpose (C < R) with row R's own
+// values (C >= R, from the source rows), segments right of it are skipped.
+// Warp-collective; the lanes' direct stores precede it.
+__device__ __forceinline__ void tri_mirror_part(uint16_t* o, long long mbase, long long ld, int row_lo, int col0,
+                                                int lane, uint4 x0, uint4 x1, uint32_t scr) {
+  ptx::sts128(tri_src(scr, lane, 0), x0);
+  ptx::sts128(tri_src(scr, lane, 1), x1);
+  __syncwarp();
+#pragma unroll
+  for (int cb = 0; cb < 2; ++cb) {
+    // matrix rb = lanes 8 rb .. 8 rb + 7, columns 8 cb .. 8 cb + 7; its
+    // transpose is destination rows 8 cb .. 8 cb + 7, segment rb
+    uint32_t t[4];
+    ptx::ldsm_x4_trans(tri_src(scr, lane, cb), t);
+    ptx::stsm_x4(tri_dst(scr, 8 * cb + (lane & 7), lane >> 3), t);
+  }
+  __syncwarp();
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int s = lane + 32 * h, dr = s >> 2, sg = s & 3;
+    const int R = col0 + dr, C0 = row_lo + 8 * sg;
+    if (C0 > R) continue;
+    uint4 val = ptx::lds128(tri_dst(scr, dr, sg));
+    if (C0 + 7 >= R) {
+      const uint4 d = ptx::lds128(tri_src(scr, R - row_lo, (C0 - col0) >> 3));
+      const int e0 = R - C0;  // elements e >= e0 lie on or right of the diagonal
+      uint32_t* pv = reinterpret_cast<uint32_t*>(&val);
+      const uint32_t* pd = reinterpret_cast<const uint32_t*>(&d);
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const uint32_t keep = (2 * w < e0 ? 0x0000FFFFu : 0u) | (2 * w + 1 < e0 ? 0xFFFF0000u : 0u);
+        pv[w] = (pv[w] & keep) | (pd[w] & ~keep);
+      }
+    }
+    *reinterpret_cast<uint4*>(o + mbase + (long long)R * ld + C0) = val;
+  }
+  __syncwarp();
+}
+
 // One CW-column chunk of a Gram-space output tile for the thread's row i.
 // Input and outputs are bf16 hi/lo pairs (FMT_PAIR) or fp32 (FMT_F32).
 // Every rounding step is explicit (__fmul_rn, __fadd_rn, __fmaf_rn), so the
@@ -186,8 +251,13 @@ __device__ __forceinline__ uint4 ld_row16(const void* p) {
 // `tri`: store only i <= j and mirror (symmetric outputs, except the
 // off-diagonal tiles of half-stored outputs, which are written whole).
 __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, int i, int col0,
-                                               const uint32_t (&r)[CW], bool tri) {
+                                               const uint32_t (&r)[CW], bool tri, uint32_t scr) {
   const int M = pr.M, N = pr.N;
+  const int lane = (int)(threadIdx.x & 31u);
+  const int row_lo = i - lane;
+  // whole-chunk symmetric diagonal tiles take the block-transpose mirror
+  // (warp-uniform: every lane of the chunk lies inside the matrix)
+  const bool fast = tri && scr != 0u && col0 + CW <= N && row_lo + 32 <= M;
   if (i >= M) return;
   float coef = pr.alpha;
   if (pr.alpha_mode == ALPHA_INV2) {
@@ -294,6 +364,26 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
       __half* oh = reinterpret_cast<__half*>(pass == 0 ? pr.out_hi : pr.out2_hi);
       __half* ol = reinterpret_cast<__half*>(pass == 0 ? pr.out_lo : pr.out2_lo);
       if (!oh) continue;
+      if (fast) {
+        uint4 h0, l0, h1, l1;
+        split8_h(v, h0, l0);
+        split8_h(v + 8, h1, l1);
+        // rows above the chunk's diagonal 16 x 16 block and inside it store
+        // all 16 values (the block's lower half is rewritten by the mirror)
+        if (i < col0 + CW) {
+          uint4* dh = reinterpret_cast<uint4*>(oh + rowoff + col0);
+          dh[0] = h0;
+          dh[1] = h1;
+          if (ol) {
+            uint4* dl = reinterpret_cast<uint4*>(ol + rowoff + col0);
+            dl[0] = l0;
+            dl[1] = l1;
+          }
+        }
+        tri_mirror_part(reinterpret_cast<uint16_t*>(oh), mbase, pr.ld, row_lo, col0, lane, h0, h1, scr);
+        if (ol) tri_mirror_part(reinterpret_cast<uint16_t*>(ol), mbase, pr.ld, row_lo, col0, lane, l0, l1, scr);
+        continue;
+      }
       if (full && all_upper) {
         uint4* dh = reinterpret_cast<uint4*>(oh + rowoff + col0);
         uint4* dl = ol ? reinterpret_cast<uint4*>(ol + rowoff + col0) : nullptr;
@@ -346,6 +436,24 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
     __nv_bfloat16* oh = pass == 0 ? pr.out_hi : pr.out2_hi;
     __nv_bfloat16* ol = pass == 0 ? pr.out_lo : pr.out2_lo;
     if (!oh) continue;
+    if (fast) {
+      uint4 h0, l0, h1, l1;
+      split8(v, h0, l0);
+      split8(v + 8, h1, l1);
+      if (i < col0 + CW) {
+        uint4* dh = reinterpret_cast<uint4*>(oh + rowoff + col0);
+        dh[0] = h0;
+        dh[1] = h1;
+        if (ol) {
+          uint4* dl = reinterpret_cast<uint4*>(ol + rowoff + col0);
+          dl[0] = l0;
+          dl[1] = l1;
+        }
+      }
+      tri_mirror_part(reinterpret_cast<uint16_t*>(oh), mbase, pr.ld, row_lo, col0, lane, h0, h1, scr);
+      if (ol) tri_mirror_part(reinterpret_cast<uint16_t*>(ol), mbase, pr.ld, row_lo, col0, lane, l0, l1, scr);
+      continue;
+    }
     // direct stores (i, j), j >= i when symmetric
     if (full && all_upper) {
       uint4* dh = reinterpret_cast<uint4*>(oh + rowoff + col0);
@@ -692,6 +800,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
   } else {
     // ------------------------------------------------ epilogue (warps 2..9)
     const int q = warp & 3;                        // TMEM lane quarter this warp may access
+    const uint32_t scr = bars + Cfg::BAR_BYTES + (uint32_t)(warp - 2) * TRI_SCRATCH;
     const int ch_begin = ((warp - 2) >> 2) * (TBN / 2 / CW);  // column half of the tile
     const int ch_end = ch_begin + TBN / 2 / CW;
     int acc = 0;
@@ -716,7 +825,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
         ptx::tmem_ld16(tmem_base + (uint32_t)(acc * TBN + ch * CW) + ((uint32_t)(q * 32) << 16), r);
         ptx::tmem_wait_ld();
         if (pr.epi == EPI_GRAM)
-          epi_gram_chunk(pr, tc.mat, i, col0, r, tri);
+          epi_gram_chunk(pr, tc.mat, i, col0, r, tri, scr);
         else
           epi_update_chunk(pr, tc.mat, i, col0, r);
       }
@@ -765,7 +874,7 @@ struct Tc2Cfg {
   static constexpr int KAT = KATV > 0 ? KATV : ((NA + NB <= 2) ? 3 : 1);
   static constexpr int STAGE_BYTES = (NA + NB) * HALF_BYTES * KAT;
   static constexpr int STAGES = (200 * 1024) / STAGE_BYTES;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256 + EPI_SCRATCH_BYTES;
   static_assert(STAGES >= 2 && STAGES <= 8, "stage count");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
@@ -1022,6 +1131,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   } else {
     // ------------------------------------------------ epilogue (both CTAs, warps 2..9)
     const int q = warp & 3;
+    const uint32_t scr = bars + 256u + (uint32_t)(warp - 2) * TRI_SCRATCH;
     const int ch_begin = ((warp - 2) >> 2) * (BN / 2 / CW);
     const int ch_end = ch_begin + BN / 2 / CW;
     int acc = 0;
@@ -1046,7 +1156,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         ptx::tmem_ld16(tmem_base + (uint32_t)(acc * BN + ch * CW) + ((uint32_t)(q * 32) << 16), r);
         ptx::tmem_wait_ld();
         if (pr.epi == EPI_GRAM)
-          epi_gram_chunk(pr, tc.mat, i, col0, r, tri);
+          epi_gram_chunk(pr, tc.mat, i, col0, r, tri, scr);
         else
           epi_update_chunk(pr, tc.mat, i, col0, r);
       }
