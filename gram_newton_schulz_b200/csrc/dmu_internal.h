@@ -159,7 +159,9 @@ constexpr int MOM_PARTIALS_PER_CHUNK = 8;
 cudaError_t launch_momentum(const MomChunk* chunks, int nchunks, const MomMat* mats,
                             const void* const* grads, float* const* momenta, int grad_f32,
                             void* mb, int mb_f32, float beta, float gscale, const float* iscale,
-                            int* fix_count, float* partial, int vec_ok, int num_sms, cudaStream_t s);
+                            int* fix_count, float* partial, int vec_ok, int num_sms, long long timeout_ns,
+                            unsigned int* status, cudaStream_t s);
+cudaError_t momentum_configure();
 cudaError_t launch_norm_finalize(const MomMat* mats, int nmats, const float* partial,
                                  float eps, float* inv, float* iscale, float* inv_img, int* fix,
                                  int* fix_count, unsigned int* status, cudaStream_t s);

@@ -11,6 +11,7 @@
 #include <cuda_fp16.h>
 
 #include "dmu_internal.h"
+#include "ptx.cuh"
 
 namespace dmu {
 
@@ -61,8 +62,10 @@ __device__ __forceinline__ void store8_image(void* __restrict__ mb, int mb_f32, 
 // partial sum of M^2 (partial[chunk * 8 + warp]), so no block-wide barrier
 // stalls the stream at chunk ends, and the partials -- hence the norm --
 // do not depend on the grid size.  Vector path: every thread issues the
-// loads of four 8-element vectors (G, M) before any arithmetic or store.
-// G, M and the image are distinct buffers (restrict).
+// loads of four 8-element vectors (G, M; two for fp32 gradients) before any
+// arithmetic or store.  G, M and the image are distinct buffers (restrict).
+// bf16 plans on the vector path use k_momentum_bulk below, which computes
+// the same values from shared memory.
 constexpr int MOM_WARPS = 8;
 constexpr int MOM_SLICE = MOM_CHUNK / MOM_WARPS;  // 2048 elements per warp
 constexpr int MOM_VEC = 4;                        // vectors in flight per thread
@@ -147,12 +150,14 @@ __global__ void __launch_bounds__(256, 3) k_momentum(const MomChunk* __restrict_
     const int s0 = warp * MOM_SLICE;
     const int s1 = min(ch.len, s0 + MOM_SLICE);
     float ss = 0.f;
+    // fp32 gradients hold twice the registers per vector in flight
+    constexpr int VEC = F32 ? MOM_VEC / 2 : MOM_VEC;
     if (vec) {
-      for (int e = s0 + lane * 8; e < s1; e += 32 * 8 * MOM_VEC) {
-        GradVec<F32> gv[MOM_VEC];
-        float4 ma[MOM_VEC], mc[MOM_VEC];
+      for (int e = s0 + lane * 8; e < s1; e += 32 * 8 * VEC) {
+        GradVec<F32> gv[VEC];
+        float4 ma[VEC], mc[VEC];
 #pragma unroll
-        for (int u = 0; u < MOM_VEC; ++u) {
+        for (int u = 0; u < VEC; ++u) {
           const int eu = e + u * 256;
           if (eu < s1) {
             gv[u].load(g, ch.start + eu);
@@ -164,7 +169,7 @@ __global__ void __launch_bounds__(256, 3) k_momentum(const MomChunk* __restrict_
           }
         }
 #pragma unroll
-        for (int u = 0; u < MOM_VEC; ++u) {
+        for (int u = 0; u < VEC; ++u) {
           const int eu = e + u * 256;
           if (eu < s1) {
             const long long i0 = ch.start + eu;
@@ -182,7 +187,7 @@ __global__ void __launch_bounds__(256, 3) k_momentum(const MomChunk* __restrict_
               __stcs(q0 + 1, make_float4(v[4], v[5], v[6], v[7]));
             }
 #pragma unroll
-            for (int q = 0; q < 8; ++q) ss += v[q] * v[q];
+            for (int q = 0; q < 8; ++q) ss = __fmaf_rn(v[q], v[q], ss);
             if (F32)
               store8_image(mb, 1, mb_off + i0, v);  // ldc == cols on the vector path
             else if (sc > 0.f)
@@ -201,7 +206,7 @@ __global__ void __launch_bounds__(256, 3) k_momentum(const MomChunk* __restrict_
           v = __fmaf_rn(beta, mom[idx], v);
           mom[idx] = v;
         }
-        ss += v * v;
+        ss = __fmaf_rn(v, v, ss);
         const long long row = idx / mm.cols, col = idx - row * mm.cols;
         const long long o = mm.mb_off + row * mm.ldc + col;
         if (F32)
@@ -213,6 +218,142 @@ __global__ void __launch_bounds__(256, 3) k_momentum(const MomChunk* __restrict_
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
     if (lane == 0) partial[(long long)c * MOM_WARPS + warp] = ss;
+  }
+}
+
+// Momentum pass of bf16 plans on the vector path, fed by bulk copies
+// (cp.async.bulk): one producer thread streams each chunk's G and M into
+// shared memory MB_STAGES chunks ahead, so the bytes in flight are bounded
+// by shared memory (192 KB per SM) rather than by registers.  The eight
+// consumer warps take the same elements, arithmetic and partial sums as
+// k_momentum (bitwise-equal M, image and partials) from shared memory and
+// write M and the fp16 image with 16-byte streaming stores.  Every wait is
+// bounded; on expiry the CTA sets DMU_FLAG_TIMEOUT and winds down.
+constexpr int MB_STAGES = 2;
+constexpr int MB_G = MOM_CHUNK * 2;  // bf16 G of one chunk
+constexpr int MB_M = MOM_CHUNK * 4;  // fp32 M of one chunk
+constexpr int MB_STAGE = MB_G + MB_M;
+constexpr int MB_THREADS = 32 * (MOM_WARPS + 1);
+constexpr int MB_SMEM = MB_STAGES * MB_STAGE + 16 * MB_STAGES;
+static_assert(MB_SMEM <= 232448, "shared memory per CTA");
+
+__device__ __forceinline__ bool mb_wait(uint32_t bar, uint32_t parity, long long timeout_ns, unsigned int* status) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  while (!ptx::mbar_try_wait(bar, parity)) {
+    if ((long long)(ptx::globaltimer() - t0) > timeout_ns) {
+      atomicOr(status, DMU_FLAG_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+__global__ void __launch_bounds__(MB_THREADS, 1)
+    k_momentum_bulk(const MomChunk* __restrict__ chunks, int nchunks, const MomMat* __restrict__ mats,
+                    const void* const* __restrict__ grads, float* const* __restrict__ momenta, void* __restrict__ mb,
+                    float beta, float gscale, const float* __restrict__ iscale, int* __restrict__ fix_count,
+                    float* __restrict__ partial, long long timeout_ns, unsigned int* status) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const uint32_t sbase = ptx::smem_u32(smem);
+  const uint32_t bars = sbase + MB_STAGES * MB_STAGE;
+  auto full = [&](int s) { return bars + 8u * s; };
+  auto empty = [&](int s) { return bars + 8u * (MB_STAGES + s); };
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // k_norm_finalize counts the matrices whose image needs rewriting; the
+  // previous call's fix-up pass has finished reading the count (stream order)
+  if (fix_count && blockIdx.x == 0 && threadIdx.x == 0) *fix_count = 0;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < MB_STAGES; ++s) {
+      ptx::mbar_init(full(s), 1);
+      ptx::mbar_init(empty(s), MOM_WARPS);
+    }
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == MOM_WARPS) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, par = 0;
+      for (int c = blockIdx.x; c < nchunks; c += gridDim.x) {
+        if (!mb_wait(empty(stage), phase ^ 1u, timeout_ns, status)) break;
+        const MomChunk ch = chunks[c];
+        const float* mom = momenta ? momenta[ch.slot] : nullptr;
+        const uint32_t gbytes = (uint32_t)ch.len * 2u, mbytes = mom ? (uint32_t)ch.len * 4u : 0u;
+        ptx::mbar_arrive_expect_tx(full(stage), gbytes + mbytes);
+        ptx::bulk_g2s(sbase + stage * MB_STAGE,
+                      reinterpret_cast<const __nv_bfloat16*>(grads[ch.slot]) + ch.start, gbytes, full(stage));
+        if (mom) ptx::bulk_g2s(sbase + stage * MB_STAGE + MB_G, mom + ch.start, mbytes, full(stage));
+        issued |= 1u << stage;
+        par = (par & ~(1u << stage)) | (phase << stage);
+        if (++stage == MB_STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      // every issued copy has landed before the CTA exits
+      for (int s = 0; s < MB_STAGES; ++s)
+        if (issued & (1u << s)) mb_wait(full(s), (par >> s) & 1u, timeout_ns, status);
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------ consumers
+  int stage = 0;
+  uint32_t phase = 0;
+  for (int c = blockIdx.x; c < nchunks; c += gridDim.x) {
+    const MomChunk ch = chunks[c];
+    const long long mb_off = mats[ch.slot].mb_off;
+    const float sc = iscale[ch.slot];
+    float* __restrict__ mom = momenta ? momenta[ch.slot] : nullptr;
+    int ok = 1;
+    if (lane == 0) ok = mb_wait(full(stage), phase, timeout_ns, status) ? 1 : 0;
+    if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+    const uint8_t* sg = smem + stage * MB_STAGE;
+    const float* sm = reinterpret_cast<const float*>(smem + stage * MB_STAGE + MB_G);
+    const int s0 = warp * MOM_SLICE;
+    const int s1 = min(ch.len, s0 + MOM_SLICE);
+    float ss = 0.f;
+    for (int e = s0 + lane * 8; e < s1; e += 256) {
+      const uint4 u = *reinterpret_cast<const uint4*>(sg + 2 * e);
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+      float v[8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 t = __bfloat1622float2(h[q]);
+        v[2 * q] = t.x;
+        v[2 * q + 1] = t.y;
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = __fmul_rn(v[q], gscale);
+      const long long i0 = ch.start + e;
+      if (mom) {  // M = round(beta M + round(s G)), no other contraction
+        const float4 a = *reinterpret_cast<const float4*>(sm + e);
+        const float4 b = *reinterpret_cast<const float4*>(sm + e + 4);
+        v[0] = __fmaf_rn(beta, a.x, v[0]); v[1] = __fmaf_rn(beta, a.y, v[1]);
+        v[2] = __fmaf_rn(beta, a.z, v[2]); v[3] = __fmaf_rn(beta, a.w, v[3]);
+        v[4] = __fmaf_rn(beta, b.x, v[4]); v[5] = __fmaf_rn(beta, b.y, v[5]);
+        v[6] = __fmaf_rn(beta, b.z, v[6]); v[7] = __fmaf_rn(beta, b.w, v[7]);
+        float4* q0 = reinterpret_cast<float4*>(mom + i0);
+        __stcs(q0, make_float4(v[0], v[1], v[2], v[3]));
+        __stcs(q0 + 1, make_float4(v[4], v[5], v[6], v[7]));
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) ss = __fmaf_rn(v[q], v[q], ss);
+      if (sc > 0.f) store8_image_h(mb, mb_off + i0, v, sc);  // ldc == cols on the vector path
+    }
+    // this warp is done with the stage: the producer may refill it
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(empty(stage));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    if (lane == 0) partial[(long long)c * MOM_WARPS + warp] = ss;
+    if (++stage == MB_STAGES) {
+      stage = 0;
+      phase ^= 1u;
+    }
   }
 }
 
@@ -321,11 +462,22 @@ cudaError_t launch_image_fix(const MomChunk* chunks, int nchunks, const MomMat* 
   return cudaGetLastError();
 }
 
+cudaError_t momentum_configure() {
+  return cudaFuncSetAttribute(k_momentum_bulk, cudaFuncAttributeMaxDynamicSharedMemorySize, MB_SMEM);
+}
+
 cudaError_t launch_momentum(const MomChunk* chunks, int nchunks, const MomMat* mats,
                             const void* const* grads, float* const* momenta, int grad_f32, void* mb,
                             int mb_f32, float beta, float gscale, const float* iscale, int* fix_count,
-                            float* partial, int vec_ok, int num_sms, cudaStream_t s) {
+                            float* partial, int vec_ok, int num_sms, long long timeout_ns, unsigned int* status,
+                            cudaStream_t s) {
   if (nchunks <= 0) return cudaSuccess;
+  if (!grad_f32 && !mb_f32 && vec_ok) {
+    const int grid = nchunks < num_sms ? nchunks : num_sms;
+    k_momentum_bulk<<<grid, MB_THREADS, MB_SMEM, s>>>(chunks, nchunks, mats, grads, momenta, mb, beta, gscale,
+                                                       iscale, fix_count, partial, timeout_ns, status);
+    return cudaGetLastError();
+  }
   int grid = num_sms * 3;  // the resident CTAs per SM of the launch bounds
   if (grid > nchunks) grid = nchunks;
   // the image has the gradients' element type for fp32 plans (fp32 -> fp32);

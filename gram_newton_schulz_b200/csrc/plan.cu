@@ -801,7 +801,8 @@ dmu_status run_normalize(dmu_plan p, int tbl, bool with_mom, float beta, float g
   // yet) are rewritten by the fix-up pass, which reads M (or the gradient)
   CUDA_TRY(launch_momentum(p->chunks_dev(), (int)p->chunks.size(), p->mats_dev(), src, moms, f32 ? 1 : 0,
                            p->mb_dev(), f32 ? 1 : 0, beta, gscale, f32 ? nullptr : p->iscale_dev(),
-                           f32 ? nullptr : p->fix_count_dev(), p->partial_dev(), vec ? 1 : 0, p->num_sms, s));
+                           f32 ? nullptr : p->fix_count_dev(), p->partial_dev(), vec ? 1 : 0, p->num_sms,
+                           p->timeout_ns, p->status_dev(), s));
   CUDA_TRY(launch_norm_finalize(p->mats_dev(), p->count, p->partial_dev(), eps, p->inv_dev(),
                                 f32 ? nullptr : p->iscale_dev(), f32 ? nullptr : p->invimg_dev(),
                                 f32 ? nullptr : p->fix_dev(), f32 ? nullptr : p->fix_count_dev(), p->status_dev(),
@@ -1112,6 +1113,7 @@ dmu_status dmu_set_workspace(dmu_plan p, void* dev_ptr, size_t bytes) {
   if (p->dtype == DMU_BF16) {
     CUDA_TRY(gemm_tc_configure());
     CUDA_TRY(onchip_configure());
+    CUDA_TRY(momentum_configure());
     for (Bucket& b : p->buckets) {
       CUtensorMap mk, mn;
       void* base = p->mb_dev() + 2 * (size_t)b.mb_off;
