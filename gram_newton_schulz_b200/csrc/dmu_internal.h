@@ -149,7 +149,8 @@ cudaError_t launch_gemm_tc(const GemmParams& p, int na, int nb, int kind, int nu
 // a 256-row block), clusters of 2 CTAs, tcgen05.mma.cta_group::2.  `kat`:
 // K atoms per stage of the one-MMA-per-slice fp16 kernels (1, 2, or 0 for
 // the default of 3); other configurations ignore it.
-cudaError_t launch_gemm_tc2(const GemmParams& p, int na, int nb, int kind, int num_sms, int kat, cudaStream_t s);
+cudaError_t launch_gemm_tc2(const GemmParams& p, int na, int nb, int kind, int num_sms, int kat, int tn,
+                            cudaStream_t s);
 cudaError_t gemm_tc_configure();
 cudaError_t launch_wait_selftest(unsigned int* status, long long timeout_ns, cudaStream_t s);
 int gemm_tc_stages(int na, int nb);

@@ -869,14 +869,20 @@ constexpr int HALF_BYTES = 128 * 128;  // 128 rows x 128-byte K row
 // bytes are in flight while the tensor cores work on one stage (2 atoms:
 // three 64 KB stages; 1 atom: six 32 KB stages).  The schedule cache picks
 // among them per Gram class.
-template <int NA, int NB, int KATV = 0>
+template <int NA, int NB, int KATV = 0, int TN = 256>
 struct Tc2Cfg {
-  static constexpr int KAT = KATV > 0 ? KATV : ((NA + NB <= 2) ? 3 : 1);
-  static constexpr int STAGE_BYTES = (NA + NB) * HALF_BYTES * KAT;
+  // TN = 512: the pair's tile is 256 x 512 (two N = 256 MMAs per K slice
+  // share the A operand), one 512-column accumulator per CTA
+  static constexpr int NH = TN == 512 ? 2 : 1;  // B halves per part
+  static constexpr int NACC = TN == 512 ? 1 : 2;  // TMEM accumulators
+  static constexpr int KAT = KATV > 0 ? KATV : (TN == 512 ? 1 : ((NA + NB <= 2) ? 3 : 1));
+  static constexpr int STAGE_BYTES = (NA + NB * NH) * HALF_BYTES * KAT;
   static constexpr int STAGES = (200 * 1024) / STAGE_BYTES;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256 + EPI_SCRATCH_BYTES;
   static_assert(STAGES >= 2 && STAGES <= 8, "stage count");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+  static_assert(TN == 256 || TN == 512, "pair tile width");
+  static_assert(NACC * TN == TMEM_COLS, "accumulators fill TMEM");
 };
 
 __device__ __forceinline__ bool wait_bar_cluster(uint32_t bar, uint32_t parity, volatile int* abort_flag,
@@ -897,10 +903,12 @@ __device__ __forceinline__ bool wait_bar_cluster(uint32_t bar, uint32_t parity, 
   }
 }
 
-template <int NA, int NB, int KIND, int KATV>
+template <int NA, int NB, int KIND, int KATV, int TN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     k_gemm_tc2(const __grid_constant__ GemmParams p) {
-  using Cfg = Tc2Cfg<NA, NB, KATV>;
+  using Cfg = Tc2Cfg<NA, NB, KATV, TN>;
+  constexpr int NH = Cfg::NH;
+  constexpr int NACC = Cfg::NACC;
   constexpr int S = Cfg::STAGES;
   constexpr int KATOMS = Cfg::KAT;
   constexpr int ATOM_E = KIND == KIND_TF32 ? 32 : 64;  // elements per 128-byte K row
@@ -965,7 +973,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       bool ok = true;
       uint32_t issued_mask = 0, issued_par = 0;
       for (int t = pair; ok && t < p.total_tiles; t += npairs) {
-        const TileCoord tc = decode_tile<BM2>(p, t);
+        const TileCoord tc = decode_tile<BM2, TN>(p, t);
         const GemmProblem& pr = p.prob[tc.pi];
         // Per-tile operand parameters, read from the parameter space once:
         // the K loop below issues only TMA copies and barrier operations.
@@ -973,15 +981,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         const CUtensorMap* bm = &p.maps[pr.b_map];
         const CUtensorMap* am_t = pr.half_a ? &p.maps[pr.a_map_t] : am;
         const CUtensorMap* bm_t = pr.half_b ? &p.maps[pr.b_map_t] : bm;
-        const int thr_a = pr.half_a ? tc.bi : 0, thr_b = pr.half_b ? tc.bj : 0;
+        // half-stored operands: row block r, K block c < r reads the stored
+        // transpose (thresholds in HALF_BLOCK units; B half h is block NH bj + h)
+        const int thr_a = pr.half_a ? tc.bi : 0;
+        const int thr_b0 = pr.half_b ? NH * tc.bj : 0, thr_b1 = pr.half_b ? NH * tc.bj + 1 : 0;
         const bool a_mn = pr.a_mn != 0, b_mn = pr.b_mn != 0;
         const int za0 = pr.a_z[0] + tc.mat, za1 = pr.a_z[1] + tc.mat;
         const int zb0 = pr.b_z[0] + tc.mat, zb1 = pr.b_z[1] + tc.mat;
         const int na = (NA > 1 && (pr.terms & TERM_LH)) ? 2 : 1;
         const int nb = (NB > 1 && (pr.terms & TERM_HL)) ? 2 : 1;
-        const uint32_t bytes_pair = 2u * (uint32_t)(na + nb) * HALF_BYTES * KATOMS;
+        const uint32_t bytes_pair = 2u * (uint32_t)(na + nb * NH) * HALF_BYTES * KATOMS;
         const int nk = (pr.K + BKE - 1) / BKE;
-        const int arow = tc.bi * BM2 + (int)rank * 128, brow = tc.bj * BN + (int)rank * 128;
+        const int arow = tc.bi * BM2 + (int)rank * 128, brow0 = tc.bj * TN + (int)rank * 128;
         for (int kb = 0; kb < nk; ++kb) {
           if (!wait_bar(empty_bar(stage), phase ^ 1u, abort_flag, p)) {
             ok = false;
@@ -1001,9 +1012,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
             const int k0 = kb * BKE + at * ATOM_E;
             const int ktile = k0 / HALF_BLOCK;
             const bool a_t = ktile < thr_a;  // rows of block bi, K in an earlier block
-            const bool b_t = ktile < thr_b;
             const CUtensorMap* am_k = a_t ? am_t : am;
-            const CUtensorMap* bm_k = b_t ? bm_t : bm;
             for (int part = 0; part < na; ++part) {
               const uint32_t dst = sa + (part * KATOMS + at) * HALF_BYTES;
               const int z = part ? za1 : za0;
@@ -1014,14 +1023,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
                 ptx::tma_load_3d_pair(dst + 8192, am_k, fb_leader, arow + 64, k0, z);
               }
             }
-            for (int part = 0; part < nb; ++part) {
-              const uint32_t dst = sb + (part * KATOMS + at) * HALF_BYTES;
-              const int z = part ? zb1 : zb0;
-              if (!b_mn && !b_t) {
-                ptx::tma_load_3d_pair(dst, bm_k, fb_leader, k0, brow, z);
-              } else {
-                ptx::tma_load_3d_pair(dst, bm_k, fb_leader, brow, k0, z);
-                ptx::tma_load_3d_pair(dst + 8192, bm_k, fb_leader, brow + 64, k0, z);
+            // B layout: [part][half][atom], 16 KB each
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+              const bool b_t = ktile < (h ? thr_b1 : thr_b0);
+              const CUtensorMap* bm_k = b_t ? bm_t : bm;
+              const int brow = brow0 + h * 256;
+              for (int part = 0; part < nb; ++part) {
+                const uint32_t dst = sb + ((part * NH + h) * KATOMS + at) * HALF_BYTES;
+                const int z = part ? zb1 : zb0;
+                if (!b_mn && !b_t) {
+                  ptx::tma_load_3d_pair(dst, bm_k, fb_leader, k0, brow, z);
+                } else {
+                  ptx::tma_load_3d_pair(dst, bm_k, fb_leader, brow, k0, z);
+                  ptx::tma_load_3d_pair(dst + 8192, bm_k, fb_leader, brow + 64, k0, z);
+                }
               }
             }
           }
@@ -1056,7 +1072,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       bool ok = true;
       bool issued = false;
       for (int t = pair; ok && t < p.total_tiles; t += npairs) {
-        const TileCoord tc = decode_tile<BM2>(p, t);
+        const TileCoord tc = decode_tile<BM2, TN>(p, t);
         const GemmProblem& pr = p.prob[tc.pi];
         const int nk = (pr.K + BKE - 1) / BKE;
         if (!wait_bar_cluster(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p)) {
@@ -1064,10 +1080,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
           break;
         }
         ptx::tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        uint32_t accumulate = 0;
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * TN);
+        uint32_t accumulate[2] = {0u, 0u};  // per N = 256 half of the accumulator
         const int terms = pr.terms, pr_a_mn = pr.a_mn, pr_b_mn = pr.b_mn;
-        const int thr_a = pr.half_a ? tc.bi : 0, thr_b = pr.half_b ? tc.bj : 0;
+        const int thr_a = pr.half_a ? tc.bi : 0;
+        const int thr_b0 = pr.half_b ? NH * tc.bj : 0, thr_b1 = pr.half_b ? NH * tc.bj + 1 : 0;
         const uint32_t idesc0 = ptx::make_idesc(BM2, BN, 0, 0, OPFMT);
         const uint64_t hi_k = ptx::make_sw128_desc(0u, 16u, 1024u), hi_mn = ptx::make_sw128_desc(0u, 8192u, 1024u);
         for (int kb = 0; kb < nk; ++kb) {
@@ -1082,26 +1099,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
           for (int at = 0; at < KATOMS; ++at) {
             const int ktile = (kb * BKE + at * ATOM_E) / HALF_BLOCK;
             const uint32_t a_mn = (uint32_t)(pr_a_mn | (ktile < thr_a ? 1 : 0));
-            const uint32_t b_mn = (uint32_t)(pr_b_mn | (ktile < thr_b ? 1 : 0));
-            const uint32_t idesc = idesc0 | (a_mn << 15) | (b_mn << 16);
-            const uint64_t a_hi = a_mn ? hi_mn : hi_k, b_hi = b_mn ? hi_mn : hi_k;
-            const uint32_t a_ks = a_mn ? 2048u : 32u, b_ks = b_mn ? 2048u : 32u;
+            const uint64_t a_hi = a_mn ? hi_mn : hi_k;
+            const uint32_t a_ks = a_mn ? 2048u : 32u;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
+              // the NH halves of the tile share this K slice's A operand
 #pragma unroll
-              for (int term = 0; term < 3; ++term) {
-                if (term == 1 && NB < 2) continue;
-                if (term == 2 && NA < 2) continue;
-                if (!(terms & (1 << term))) continue;
-                const uint32_t pa = sa + ((term == 2 ? KATOMS : 0) + at) * HALF_BYTES + kk * a_ks;
-                const uint32_t pb = sb + ((term == 1 ? KATOMS : 0) + at) * HALF_BYTES + kk * b_ks;
-                const uint64_t ad = a_hi | (uint64_t)((pa >> 4) & 0x3FFFu);
-                const uint64_t bd = b_hi | (uint64_t)((pb >> 4) & 0x3FFFu);
-                if (KIND == KIND_TF32)
-                  ptx::mma2_tf32(d_tmem, ad, bd, idesc, accumulate);
-                else
-                  ptx::mma2_f16(d_tmem, ad, bd, idesc, accumulate);
-                accumulate = 1;
+              for (int h = 0; h < NH; ++h) {
+                const uint32_t b_mn = (uint32_t)(pr_b_mn | (ktile < (h ? thr_b1 : thr_b0) ? 1 : 0));
+                const uint32_t idesc = idesc0 | (a_mn << 15) | (b_mn << 16);
+                const uint64_t b_hi = b_mn ? hi_mn : hi_k;
+                const uint32_t b_ks = b_mn ? 2048u : 32u;
+#pragma unroll
+                for (int term = 0; term < 3; ++term) {
+                  if (term == 1 && NB < 2) continue;
+                  if (term == 2 && NA < 2) continue;
+                  if (!(terms & (1 << term))) continue;
+                  const uint32_t pa = sa + ((term == 2 ? KATOMS : 0) + at) * HALF_BYTES + kk * a_ks;
+                  const uint32_t pb = sb + (((term == 1 ? NH : 0) + h) * KATOMS + at) * HALF_BYTES + kk * b_ks;
+                  const uint64_t ad = a_hi | (uint64_t)((pa >> 4) & 0x3FFFu);
+                  const uint64_t bd = b_hi | (uint64_t)((pb >> 4) & 0x3FFFu);
+                  if (KIND == KIND_TF32)
+                    ptx::mma2_tf32(d_tmem + (uint32_t)(h * 256), ad, bd, idesc, accumulate[h]);
+                  else
+                    ptx::mma2_f16(d_tmem + (uint32_t)(h * 256), ad, bd, idesc, accumulate[h]);
+                  accumulate[h] = 1;
+                }
               }
             }
           }
@@ -1114,7 +1137,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         }
         if (!ok) break;
         ptx::mma2_commit_both(tfull_bar(acc));
-        if (++acc == 2) {
+        if (++acc == NACC) {
           acc = 0;
           acc_phase ^= 1u;
         }
@@ -1132,12 +1155,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     // ------------------------------------------------ epilogue (both CTAs, warps 2..9)
     const int q = warp & 3;
     const uint32_t scr = bars + 256u + (uint32_t)(warp - 2) * TRI_SCRATCH;
-    const int ch_begin = ((warp - 2) >> 2) * (BN / 2 / CW);
-    const int ch_end = ch_begin + BN / 2 / CW;
+    const int ch_begin = ((warp - 2) >> 2) * (TN / 2 / CW);
+    const int ch_end = ch_begin + TN / 2 / CW;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = pair; t < p.total_tiles; t += npairs) {
-      const TileCoord tc = decode_tile<BM2>(p, t);
+      const TileCoord tc = decode_tile<BM2, TN>(p, t);
       const GemmProblem& pr = p.prob[tc.pi];
       int ok = 1;
       if (lane == 0) ok = wait_bar_cluster(tfull_bar(acc), acc_phase, abort_flag, p) ? 1 : 0;
@@ -1145,15 +1168,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       if (!ok) break;
       ptx::tc_fence_after();
       const int row_lo = tc.bi * BM2 + (int)rank * 128 + q * 32;
-      const bool tri = pr.sym && (!pr.half_out || tc.bi == tc.bj);
       const int i = row_lo + lane;
       for (int ch = ch_begin; ch < ch_end; ++ch) {
-        const int col0 = tc.bj * BN + ch * CW;
+        const int col0 = tc.bj * TN + ch * CW;
         if (col0 >= pr.N) break;
+        // half-stored outputs: lower blocks are never written, the diagonal
+        // block is mirrored, upper blocks are written whole
+        const int cblk = col0 / HALF_BLOCK;
+        if (pr.sym && pr.half_out && cblk < tc.bi) continue;
+        const bool tri = pr.sym && (!pr.half_out || cblk == tc.bi);
         if (tri && col0 + CW - 1 < row_lo) continue;
         if (row_lo >= pr.M) break;
         uint32_t r[CW];
-        ptx::tmem_ld16(tmem_base + (uint32_t)(acc * BN + ch * CW) + ((uint32_t)(q * 32) << 16), r);
+        ptx::tmem_ld16(tmem_base + (uint32_t)(acc * TN + ch * CW) + ((uint32_t)(q * 32) << 16), r);
         ptx::tmem_wait_ld();
         if (pr.epi == EPI_GRAM)
           epi_gram_chunk(pr, tc.mat, i, col0, r, tri, scr);
@@ -1163,7 +1190,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive_cluster(ptx::mapa_shared(tempty_bar(acc), 0));
-      if (++acc == 2) {
+      if (++acc == NACC) {
         acc = 0;
         acc_phase ^= 1u;
       }
@@ -1211,10 +1238,10 @@ static cudaError_t configure_one() {
                               TcCfg<NA, NB, TBN>::SMEM_BYTES);
 }
 
-template <int NA, int NB, int KIND, int KATV = 0>
+template <int NA, int NB, int KIND, int KATV = 0, int TN = 256>
 static cudaError_t configure_two() {
-  return cudaFuncSetAttribute(k_gemm_tc2<NA, NB, KIND, KATV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              Tc2Cfg<NA, NB, KATV>::SMEM_BYTES);
+  return cudaFuncSetAttribute(k_gemm_tc2<NA, NB, KIND, KATV, TN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              Tc2Cfg<NA, NB, KATV, TN>::SMEM_BYTES);
 }
 
 cudaError_t gemm_tc_configure() {
@@ -1239,6 +1266,8 @@ cudaError_t gemm_tc_configure() {
   if ((e = configure_two<1, 1, KIND_F16, 2>()) != cudaSuccess) return e;
   if ((e = configure_two<1, 1, KIND_F16, 1>()) != cudaSuccess) return e;
   if ((e = configure_two<2, 1, KIND_F16>()) != cudaSuccess) return e;
+  if ((e = configure_two<1, 1, KIND_F16, 0, 512>()) != cudaSuccess) return e;
+  if ((e = configure_two<2, 1, KIND_F16, 0, 512>()) != cudaSuccess) return e;
   return cudaSuccess;
 }
 
@@ -1260,16 +1289,24 @@ static cudaError_t launch_one(const GemmParams& p, int num_sms, int tbn, cudaStr
   return cudaGetLastError();
 }
 
-template <int NA, int NB, int KIND, int KATV = 0>
+template <int NA, int NB, int KIND, int KATV = 0, int TN = 256>
 static cudaError_t launch_two(const GemmParams& p, int num_sms, cudaStream_t s) {
   int pairs = num_sms / 2;
   if (p.total_tiles < pairs) pairs = p.total_tiles;
   if (pairs <= 0) return cudaSuccess;
-  k_gemm_tc2<NA, NB, KIND, KATV><<<2 * pairs, GEMM_THREADS, Tc2Cfg<NA, NB, KATV>::SMEM_BYTES, s>>>(p);
+  k_gemm_tc2<NA, NB, KIND, KATV, TN><<<2 * pairs, GEMM_THREADS, Tc2Cfg<NA, NB, KATV, TN>::SMEM_BYTES, s>>>(p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm_tc2(const GemmParams& p, int na, int nb, int kind, int num_sms, int kat, cudaStream_t s) {
+cudaError_t launch_gemm_tc2(const GemmParams& p, int na, int nb, int kind, int num_sms, int kat, int tn,
+                            cudaStream_t s) {
+  if (tn == 512) {  // 256 x 512 pair tiles: scaled-fp16 operands only
+    if (kind != KIND_F16) return cudaErrorInvalidValue;
+    if (na == 1 && nb == 1) return launch_two<1, 1, KIND_F16, 0, 512>(p, num_sms, s);
+    if (na == 2 && nb == 1) return launch_two<2, 1, KIND_F16, 0, 512>(p, num_sms, s);
+    return cudaErrorInvalidValue;
+  }
+  if (tn != 256) return cudaErrorInvalidValue;
   if (kind == KIND_TF32) {
     if (na == 1 && nb == 1) return launch_two<1, 1, KIND_TF32>(p, num_sms, s);
     return cudaErrorInvalidValue;

@@ -79,12 +79,17 @@ struct GClass {
 // Schedules: 0 single CTAs, 128 x 256 tiles; 1 CTA pairs, 256 x 256 tiles;
 // 2 single CTAs, 128 x 128 tiles; 3 on chip (m <= 128); 4 and 5 CTA pairs
 // whose one-MMA-per-slice fp16 kernels take 2 and 1 K atoms per stage
-// (three and six stages) instead of 3 (two stages).
+// (three and six stages) instead of 3 (two stages); 6 CTA pairs with
+// 256 x 512 tiles (two N = 256 MMAs per K slice share A: a quarter fewer
+// operand bytes per MMA, one 512-column accumulator, so the epilogue does
+// not overlap the next tile), scaled-fp16 launches only (others run 1).
 constexpr int SCHED_ONCHIP = 3;
-constexpr int TILE_SCHEDS[5] = {0, 1, 2, 4, 5};
-bool is_pair(int sched) { return sched == 1 || sched == 4 || sched == 5; }
+constexpr int SCHED_WIDE = 6;
+constexpr int TILE_SCHEDS[6] = {0, 1, 2, 4, 5, 6};
+bool is_pair(int sched) { return sched == 1 || sched == 4 || sched == 5 || sched == SCHED_WIDE; }
 int pair_kat(int sched) { return sched == 4 ? 2 : (sched == 5 ? 1 : 0); }
-bool valid_sched(int v) { return v >= 0 && v <= 5; }
+bool valid_sched(int v) { return v >= 0 && v <= 6; }
+int tile_n(int sched) { return sched == 2 ? 128 : (sched == SCHED_WIDE ? 512 : BN); }
 
 bool onchip_eligible(dmu_dtype dtype, const GClass& g) {
   return dtype == DMU_BF16 && g.prec == DMU_PREC_SPLIT3 && g.m <= ONCHIP_MAX_M;
@@ -252,6 +257,7 @@ struct Prob {
 };
 
 dmu_status run_tc(dmu_plan p, std::vector<Prob>& probs, int na, int nb, int kind, int sched, cudaStream_t s) {
+  if (sched == SCHED_WIDE && kind != KIND_F16) sched = 1;  // the wide pair tile is built for fp16 operands
   size_t i = 0;
   while (i < probs.size()) {
     GemmParams gp;
@@ -282,7 +288,7 @@ dmu_status run_tc(dmu_plan p, std::vector<Prob>& probs, int na, int nb, int kind
       g.a_map_t = probs[i].amap_t >= 0 ? slot(probs[i].amap_t) : g.a_map;
       g.b_map_t = probs[i].bmap_t >= 0 ? slot(probs[i].bmap_t) : g.b_map;
       g.tiles_per_mat = tiles_for(g.M, g.N, g.sym != 0, &g.tiles_m, &g.tiles_n, is_pair(sched) ? 256 : BM,
-                                  sched == 2 ? 128 : BN);
+                                  tile_n(sched));
       g.tile_begin = tiles;
       tiles += g.count * g.tiles_per_mat;
       gp.prob[nprob++] = g;
@@ -294,7 +300,7 @@ dmu_status run_tc(dmu_plan p, std::vector<Prob>& probs, int na, int nb, int kind
     gp.status = p->status_dev();
     gp.timeout_ns = p->timeout_ns;
     if (is_pair(sched))
-      CUDA_TRY(launch_gemm_tc2(gp, na, nb, kind, p->num_sms, pair_kat(sched), s));
+      CUDA_TRY(launch_gemm_tc2(gp, na, nb, kind, p->num_sms, pair_kat(sched), tile_n(sched), s));
     else
       CUDA_TRY(launch_gemm_tc(gp, na, nb, kind, p->num_sms, sched == 2 ? 128 : 256, s));
     p->launches++;
@@ -1491,9 +1497,10 @@ dmu_status dmu_autotune(dmu_plan p, const char* cache_path, void* stream) {
       continue;
     }
     std::vector<int> cand = {1, 0, 2};
-    if (g.kind == KIND_F16) {  // stage-depth variants of the CTA-pair fp16 kernel
+    if (g.kind == KIND_F16) {  // stage-depth and tile-width variants of the CTA-pair fp16 kernel
       cand.push_back(4);
       cand.push_back(5);
+      cand.push_back(SCHED_WIDE);
     }
     if (onchip_eligible(p->dtype, g)) cand.push_back(SCHED_ONCHIP);
     std::ostringstream times;
@@ -1546,7 +1553,7 @@ dmu_status dmu_autotune(dmu_plan p, const char* cache_path, void* stream) {
     std::ostringstream times;
     int best = -1;
     float best_ms = 0.f;
-    for (int sc : {1, 0, 2}) {
+    for (int sc : {1, 0, 2, SCHED_WIDE}) {
       b.fsched = sc;
       const float ms = time_min([&] { return final_launch(p, true, false, 0.f, s); });
       if (st != DMU_OK) break;

@@ -29,7 +29,7 @@ DTYPES = {"bf16": 0, "f32": 1}
 PRECS = {"auto": 0, "fast": 1, "split2": 2, "split3": 3, "tf32": 4, "f16": 5}
 FLAG_NONFINITE, FLAG_TIMEOUT = 1, 2
 SCHEDULES = {0: "single_cta", 1: "cta_pair", 2: "single_cta_n128", 3: "onchip", 4: "cta_pair_k2",
-             5: "cta_pair_k1"}
+             5: "cta_pair_k1", 6: "cta_pair_n512"}
 
 # name -> (restype, argtypes); every symbol of include/dmu.h
 _VP = ctypes.c_void_p

@@ -52,10 +52,11 @@
  *     tcgen05.mma.cta_group::2) by default.  Two single-CTA schedules
  *     exist: 128 x 256 tiles, and 128 x 128 tiles for many small matrices.
  *     dmu_autotune picks one by measurement.  At plan creation the
- *     environment variable DMU_SCHEDULE=0|1|2 (0 = 128 x 256 single CTAs,
- *     1 = CTA pairs, 2 = 128 x 128 single CTAs) overrides the default, and
- *     so does DMU_CTA_PAIR=0|1.  Every schedule accumulates each element
- *     over K in the same order, so all give bitwise-equal results.
+ *     environment variable DMU_SCHEDULE=0|1|2|4|5|6 (0 = 128 x 256 single
+ *     CTAs, 1 = CTA pairs, 2 = 128 x 128 single CTAs, 4-6 as in
+ *     dmu_get_gram_schedule) overrides the default, and so does
+ *     DMU_CTA_PAIR=0|1.  Every schedule accumulates each element over K in
+ *     the same order, so all give bitwise-equal results.
  */
 #ifndef DMU_H
 #define DMU_H
@@ -247,10 +248,14 @@ DMU_API int dmu_get_schedule(dmu_plan plan);
  * with its m): 0, 1, 2 as above; 3 = the whole recursion on chip (one CTA
  * per matrix, m <= 128, split-bf16 precision); 4 and 5 = CTA pairs whose
  * one-MMA-per-slice fp16 kernels stage 2 and 1 K atoms of 64 (three and six
- * stages) instead of 3 (two stages).  -1 for a bad argument. */
+ * stages) instead of 3 (two stages); 6 = CTA pairs with 256 x 512 tiles
+ * (two N = 256 MMAs per K slice share the A operand; scaled-fp16 launches
+ * only, the others of a class on schedule 6 run as schedule 1).  -1 for a
+ * bad argument. */
 DMU_API int dmu_get_gram_schedule(dmu_plan plan, int index);
 
-/* Tile schedule (0, 1, 2) of the final GEMM of matrix `index`'s bucket. */
+/* Tile schedule (0, 1, 2 or 6) of the final GEMM of matrix `index`'s
+ * bucket. */
 DMU_API int dmu_get_final_schedule(dmu_plan plan, int index);
 
 /* Number of kernel launches the last compute call enqueued. */

@@ -232,3 +232,12 @@ def test_per_class_schedule_queries(monkeypatch):
     st, h, keep = _create(pairs)
     assert st == dmu.OK and lib.dmu_get_gram_schedule(h, 0) == 1
     lib.dmu_plan_destroy(h)
+    # DMU_SCHEDULE takes the tile schedules (6: 256 x 512 CTA-pair tiles);
+    # 3 (on chip) and values outside 0..6 leave the default
+    for env, want in (("6", 6), ("4", 4), ("3", 1), ("7", 1), ("-1", 1)):
+        monkeypatch.setenv("DMU_SCHEDULE", env)
+        st, h, keep = _create(pairs)
+        assert st == dmu.OK
+        assert lib.dmu_get_schedule(h) == want, env
+        assert lib.dmu_get_final_schedule(h, 4) == want, env
+        lib.dmu_plan_destroy(h)

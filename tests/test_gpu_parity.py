@@ -344,15 +344,16 @@ def test_half_and_full_storage_agree(prec, monkeypatch):
 @pytest.mark.parametrize("prec", ["auto", "split3", "tf32"])
 def test_cta_pair_and_single_cta_agree(prec, monkeypatch):
     """The CTA-pair kernels (256 x 256 tiles, cta_group::2, with 3, 2 or 1 K
-    atoms per stage) and the single-CTA kernels (128 x 256 and 128 x 128
-    tiles) accumulate every element over K in the same order, so they must
-    give bitwise-equal results."""
+    atoms per stage; 256 x 512 tiles), and the single-CTA kernels (128 x 256
+    and 128 x 128 tiles) accumulate every element over K in the same order,
+    so they must give bitwise-equal results."""
     shapes = [(1100, 3000), (3000, 1100), (512, 2048), (520, 200), (384, 384), (128, 512), (100, 300)]
     w = synth.custom("pair", shapes, seed=29)
     monkeypatch.setenv("DMU_SCHEDULE", "1")
     a = run_step(w, prec=prec)
-    # 4 and 5: CTA pairs staging 2 and 1 K atoms per stage (fp16 kernels)
-    for sched in ("0", "2", "4", "5"):
+    # 4 and 5: CTA pairs staging 2 and 1 K atoms per stage (fp16 kernels);
+    # 6: 256 x 512 CTA-pair tiles (fp16 launches; the others run as 1)
+    for sched in ("0", "2", "4", "5", "6"):
         monkeypatch.setenv("DMU_SCHEDULE", sched)
         b = run_step(w, prec=prec)
         for i in range(w.count):
@@ -378,6 +379,7 @@ def test_autotune_picks_and_caches_schedule(tmp_path):
     text = open(cache).read()
     assert "s1_ms=" in text and "s0_ms=" in text and "s2_ms=" in text
     assert "s3_ms=" not in text  # no class here has m <= 128
+    assert "s6_ms=" in text  # 256 x 512 CTA-pair tiles: the fp16 class and the finals
     # a second plan with the same shapes reuses the cached choices
     plan2 = dmu.Plan(shapes)
     plan2.momentum_normalize(grads, None, beta=0.0)
