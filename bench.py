@@ -142,8 +142,9 @@ def momentum_bytes(shapes, grad_bytes=2, image16=False):
 
 def schedule_summary(sch):
     """Plan.schedules() as JSON-friendly text: one entry per Gram class (by
-    m) and per final-GEMM bucket (by rows x cols)."""
+    m) and per SYRK and final-GEMM bucket (by rows x cols)."""
     return {"gram": {f"m{m}": v for m, v in sorted(sch["gram"].items())},
+            "syrk": {f"{r}x{c}": v for (r, c), v in sorted(sch["syrk"].items())},
             "final": {f"{r}x{c}": v for (r, c), v in sorted(sch["final"].items())}}
 
 

@@ -54,6 +54,7 @@ struct Bucket {
   int64_t mb_off = 0;  // element offset of the bucket's first image
   int map_k = -1, map_mn = -1;
   int fsched = -1;     // tile schedule of this bucket's final GEMM (-1: the plan's)
+  int ssched = -1;     // tile schedule of this bucket's SYRK (-1: its class's)
 };
 
 struct GClass {
@@ -83,6 +84,9 @@ struct GClass {
 // 256 x 512 tiles (two N = 256 MMAs per K slice share A: a quarter fewer
 // operand bytes per MMA, one 512-column accumulator, so the epilogue does
 // not overlap the next tile), scaled-fp16 launches only (others run 1).
+// The Gram products and the final lose more to the exposed epilogue than
+// they gain (measured), so schedule 6 is an autotune candidate only for the
+// SYRK, whose K is the long side n.
 constexpr int SCHED_ONCHIP = 3;
 constexpr int SCHED_WIDE = 6;
 constexpr int TILE_SCHEDS[6] = {0, 1, 2, 4, 5, 6};
@@ -160,6 +164,7 @@ struct dmu_plan_s {
   int sched = 1;
   bool half_store = true;  // half-stored symmetric Gram-space matrices
   int tune_class = -1, tune_bucket = -1;  // autotune: run one class / one bucket only
+  int tune_syrk = -1;                      // autotune: the SYRK of one bucket only
   int tune_count = 0;                      // autotune: matrices of the tuned bucket's final (0: all)
 
   int class_sched(int c) const { return classes[c].sched >= 0 ? classes[c].sched : sched; }
@@ -627,6 +632,7 @@ dmu_status gram_bf16(dmu_plan p, const float co[3], int steps, cudaStream_t s) {
   for (const Bucket& b : p->buckets) {
     const GClass& gc = p->classes[b.cls];
     if (p->tune_class >= 0 && b.cls != p->tune_class) continue;
+    if (p->tune_syrk >= 0 && &b != &p->buckets[p->tune_syrk]) continue;
     if (steps >= 1 && p->onchip(b.cls)) continue;
     Prob pr;
     std::memset(&pr, 0, sizeof(pr));
@@ -661,7 +667,7 @@ dmu_status gram_bf16(dmu_plan p, const float co[3], int steps, cudaStream_t s) {
     pr.amap = pr.bmap = b.tall ? b.map_mn : b.map_k;
     g.half_out = gc.half ? 1 : 0;
     syrk.push_back(pr);
-    syrk_sched.push_back(p->onchip(b.cls) ? p->sched : p->class_sched(b.cls));
+    syrk_sched.push_back(p->onchip(b.cls) ? p->sched : (b.ssched >= 0 ? b.ssched : p->class_sched(b.cls)));
   }
   dmu_status st = DMU_OK;
   for (int sched : TILE_SCHEDS) {
@@ -1420,6 +1426,12 @@ static std::string final_key(dmu_plan p, const std::string& dev, const Bucket& b
   return k.str();
 }
 
+static std::string syrk_key(dmu_plan p, const std::string& dev, const Bucket& b) {
+  std::ostringstream k;
+  k << dev << "/syrk/" << b.rows << "x" << b.cols << "/n" << b.count << "/p" << p->classes[b.cls].prec;
+  return k.str();
+}
+
 static std::map<std::string, int> read_cache(const char* path) {
   std::map<std::string, int> out;
   if (!path) return out;
@@ -1449,6 +1461,14 @@ int dmu_get_final_schedule(dmu_plan p, int index) {
   for (const Bucket& b : p->buckets)
     for (int i : b.mats)
       if (i == index) return p->final_sched(b);
+  return -1;
+}
+
+int dmu_get_syrk_schedule(dmu_plan p, int index) {
+  if (!p || index < 0 || index >= p->count) return -1;
+  for (const Bucket& b : p->buckets)
+    for (int i : b.mats)
+      if (i == index) return p->onchip(b.cls) ? SCHED_ONCHIP : (b.ssched >= 0 ? b.ssched : p->class_sched(b.cls));
   return -1;
 }
 
@@ -1497,10 +1517,9 @@ dmu_status dmu_autotune(dmu_plan p, const char* cache_path, void* stream) {
       continue;
     }
     std::vector<int> cand = {1, 0, 2};
-    if (g.kind == KIND_F16) {  // stage-depth and tile-width variants of the CTA-pair fp16 kernel
+    if (g.kind == KIND_F16) {  // stage-depth variants of the CTA-pair fp16 kernel
       cand.push_back(4);
       cand.push_back(5);
-      cand.push_back(SCHED_WIDE);
     }
     if (onchip_eligible(p->dtype, g)) cand.push_back(SCHED_ONCHIP);
     std::ostringstream times;
@@ -1520,6 +1539,45 @@ dmu_status dmu_autotune(dmu_plan p, const char* cache_path, void* stream) {
     p->tune_class = -1;
     if (st != DMU_OK) break;
     g.sched = best;
+    cache[key] = best;
+    lines.push_back(key + " " + std::to_string(best) + times.str());
+  }
+  // ---- SYRK of every bucket off the on-chip schedule: its class's tile
+  // schedule, or the 256 x 512 CTA-pair tile, whose epilogue does not
+  // overlap the next tile but whose operands cost a quarter less per MMA
+  // (the long K of a wide or tall bucket amortises the epilogue)
+  for (size_t bi = 0; st == DMU_OK && bi < p->buckets.size(); ++bi) {
+    Bucket& b = p->buckets[bi];
+    const GClass& g = p->classes[b.cls];
+    if (p->onchip(b.cls)) continue;
+    const std::string key = syrk_key(p, dev, b);
+    auto hit = cache.find(key);
+    if (hit != cache.end() && hit->second != SCHED_ONCHIP) {
+      b.ssched = hit->second;
+      continue;
+    }
+    std::ostringstream times;
+    int best = -1;
+    float best_ms = 0.f;
+    p->tune_class = b.cls;
+    p->tune_syrk = (int)bi;
+    const int own = p->class_sched(b.cls);
+    for (int sc : {own, SCHED_WIDE}) {
+      if (sc == SCHED_WIDE && own == SCHED_WIDE) break;
+      b.ssched = sc;
+      const float ms = time_min([&] { return gram_bf16(p, co, 0, s); });
+      if (st != DMU_OK) break;
+      times << " s" << sc << "_ms=" << ms;
+      if (best < 0 || ms < best_ms) {
+        best = sc;
+        best_ms = ms;
+      }
+    }
+    p->tune_class = -1;
+    p->tune_syrk = -1;
+    if (st != DMU_OK) break;
+    (void)g;
+    b.ssched = best;
     cache[key] = best;
     lines.push_back(key + " " + std::to_string(best) + times.str());
   }
@@ -1553,7 +1611,7 @@ dmu_status dmu_autotune(dmu_plan p, const char* cache_path, void* stream) {
     std::ostringstream times;
     int best = -1;
     float best_ms = 0.f;
-    for (int sc : {1, 0, 2, SCHED_WIDE}) {
+    for (int sc : {1, 0, 2}) {
       b.fsched = sc;
       const float ms = time_min([&] { return final_launch(p, true, false, 0.f, s); });
       if (st != DMU_OK) break;

@@ -50,6 +50,7 @@ SIGNATURES = {
     "dmu_get_schedule": (ctypes.c_int, [_VP]),
     "dmu_get_gram_schedule": (ctypes.c_int, [_VP, ctypes.c_int]),
     "dmu_get_final_schedule": (ctypes.c_int, [_VP, ctypes.c_int]),
+    "dmu_get_syrk_schedule": (ctypes.c_int, [_VP, ctypes.c_int]),
     "dmu_momentum_norm_static": (ctypes.c_int, [_VP, _VP, _VP, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
                                                 ctypes.c_float, ctypes.c_float, _VP, _VP]),
     "dmu_demuon_track": (ctypes.c_int, [ctypes.c_int, ctypes.c_int64, _VP, ctypes.c_float, _VP, _VP, _VP, _VP,
@@ -218,13 +219,14 @@ class Plan:
         return self.schedules()
 
     def schedules(self) -> dict:
-        """{"gram": {m: name}, "final": {(rows, cols): name}} with the
-        schedule names of SCHEDULES."""
-        gram, final = {}, {}
+        """{"gram": {m: name}, "syrk": {(rows, cols): name}, "final":
+        {(rows, cols): name}} with the schedule names of SCHEDULES."""
+        gram, syrk, final = {}, {}, {}
         for i, (r, c) in enumerate(self.shapes):
             gram[min(r, c)] = SCHEDULES.get(int(self.lib.dmu_get_gram_schedule(self.handle, i)), "?")
+            syrk[(r, c)] = SCHEDULES.get(int(self.lib.dmu_get_syrk_schedule(self.handle, i)), "?")
             final[(r, c)] = SCHEDULES.get(int(self.lib.dmu_get_final_schedule(self.handle, i)), "?")
-        return {"gram": gram, "final": final}
+        return {"gram": gram, "syrk": syrk, "final": final}
 
     def read_status(self) -> int:
         flags = ctypes.c_uint32(0)

@@ -254,9 +254,15 @@ DMU_API int dmu_get_schedule(dmu_plan plan);
  * bad argument. */
 DMU_API int dmu_get_gram_schedule(dmu_plan plan, int index);
 
-/* Tile schedule (0, 1, 2 or 6) of the final GEMM of matrix `index`'s
- * bucket. */
+/* Tile schedule (0, 1 or 2) of the final GEMM of matrix `index`'s bucket.
+ * -1 for a bad argument. */
 DMU_API int dmu_get_final_schedule(dmu_plan plan, int index);
+
+/* Schedule of the SYRK (G0 = s^2 X X^T) of matrix `index`'s bucket: its
+ * class's tile schedule, or 6 when dmu_autotune measured the 256 x 512
+ * CTA-pair tile faster for that bucket (its K is the long side n); 3 when
+ * the class runs on chip.  -1 for a bad argument. */
+DMU_API int dmu_get_syrk_schedule(dmu_plan plan, int index);
 
 /* Number of kernel launches the last compute call enqueued. */
 DMU_API int dmu_last_launch_count(dmu_plan plan);

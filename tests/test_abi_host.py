@@ -222,6 +222,8 @@ def test_per_class_schedule_queries(monkeypatch):
     assert st == dmu.OK
     assert [lib.dmu_get_gram_schedule(h, i) for i in range(5)] == [3, 3, 1, 3, 1]
     assert [lib.dmu_get_final_schedule(h, i) for i in range(5)] == [1] * 5
+    assert [lib.dmu_get_syrk_schedule(h, i) for i in range(5)] == [3, 3, 1, 3, 1]
+    assert lib.dmu_get_syrk_schedule(h, 5) == -1 and lib.dmu_get_syrk_schedule(None, 0) == -1
     assert lib.dmu_get_gram_schedule(h, 5) == -1 and lib.dmu_get_final_schedule(h, -1) == -1
     assert lib.dmu_get_gram_schedule(None, 0) == -1
     lib.dmu_plan_destroy(h)

@@ -375,11 +375,13 @@ def test_autotune_picks_and_caches_schedule(tmp_path):
     choice = plan.autotune(cache)
     names = set(dmu.SCHEDULES.values())
     assert set(choice["gram"]) == {1024, 512} and set(choice["final"]) == set(shapes)
+    assert set(choice["syrk"]) == set(shapes)
     assert all(v in names and v != "onchip" for part in choice.values() for v in part.values())
     text = open(cache).read()
     assert "s1_ms=" in text and "s0_ms=" in text and "s2_ms=" in text
     assert "s3_ms=" not in text  # no class here has m <= 128
-    assert "s6_ms=" in text  # 256 x 512 CTA-pair tiles: the fp16 class and the finals
+    assert "s6_ms=" in text  # 256 x 512 CTA-pair tiles: a candidate for every bucket's SYRK
+    assert sum("/syrk/" in line for line in text.splitlines()) == len(shapes)
     # a second plan with the same shapes reuses the cached choices
     plan2 = dmu.Plan(shapes)
     plan2.momentum_normalize(grads, None, beta=0.0)
