@@ -99,10 +99,7 @@ def _check(st: int):
 
 
 def _ptr_array(ptrs):
-    arr = (ctypes.c_void_p * len(ptrs))()
-    for i, p in enumerate(ptrs):
-        arr[i] = p
-    return arr
+    return (ctypes.c_void_p * len(ptrs))(*ptrs)
 
 
 def _stream_handle(stream, device):
@@ -120,6 +117,7 @@ class Plan:
         self.lib = load()
         self.shapes = [(int(r), int(c)) for r, c in shapes]
         self.count = len(self.shapes)
+        self._sizes = [torch.Size(sh) for sh in self.shapes]
         self._shape_arr = (Shape * self.count)(*[Shape(r, c) for r, c in self.shapes])
         self.device = torch.device("cuda", torch.cuda.current_device() if device is None else
                                    torch.device(device).index or 0)
@@ -148,10 +146,18 @@ class Plan:
             pass
 
     def _check_tensors(self, ts, what, dtype):
+        # one pass of cheap comparisons (torch.Size equality, dtype identity,
+        # integer device index): thousands of matrices per call
         if len(ts) != self.count:
             raise ValueError(f"{what}: expected {self.count} tensors, got {len(ts)}")
-        for t, (r, c) in zip(ts, self.shapes):
-            if tuple(t.shape) != (r, c) or not t.is_contiguous() or t.dtype != dtype or t.device != self.device:
+        sizes = getattr(self, "_sizes", None)
+        if sizes is None:
+            import torch
+            sizes = self._sizes = [torch.Size(sh) for sh in self.shapes]
+        dev = self.device.index
+        for k, t in enumerate(ts):
+            if t.shape != sizes[k] or t.dtype is not dtype or not t.is_contiguous() or t.get_device() != dev:
+                r, c = self.shapes[k]
                 raise ValueError(f"{what}: tensor {tuple(t.shape)} {t.dtype} {t.device} does not match "
                                  f"({r}, {c}) {dtype} contiguous on {self.device}")
 
