@@ -96,12 +96,13 @@ def gemm_alg_bytes(shapes, k=K_STEPS):
     return tot
 
 
-# DRAM traffic of the tensor-core kernel measured by ncu (one pass:
+# DRAM traffic of the tensor-core launches measured by ncu (one pass:
 # gpu__time_duration.sum, dram__bytes_read.sum, dram__bytes_write.sum) on a
 # two-layer slice of the 28-layer set (1/14 of its matrices, small enough
-# for counter captures), scaled by the units processed (x 14) to the whole
-# step.  The figure applies only while gemm_tc.cu + plan.cu hash to the
-# captured build: a changed kernel reports null.
+# for counter captures) run with the 28-layer set's schedule choices, scaled
+# by the units processed (x 14) to the whole step.  The figure applies only
+# while gemm_tc.cu + plan.cu hash to the captured build and the run uses
+# the captured schedules: otherwise the line reports null.
 TRAFFIC_CAPTURE = {
     "sources": ["gram_newton_schulz_b200/csrc/gemm_tc.cu", "gram_newton_schulz_b200/csrc/plan.cu"],
     "sha256": "1deff850c10b9549df8d57593dd6bc0146f39527674e3a33e83aa64c8953d8eb",
@@ -109,16 +110,19 @@ TRAFFIC_CAPTURE = {
     "captured_on": "3584x3584*4,512x3584*4,18944x3584*4,3584x18944*2 (2 of 28 layers)",
     "scale": 14,
     "dram_bytes_per_step": 15.321e9 * 14,
-    "launches_per_step": 30,
+    "schedule": None,  # the schedule summary the capture ran with (None: any)
 }
 
 
-def captured_traffic(workload_name):
-    """Measured DRAM bytes per tensor-core launch, or None when the capture
-    does not apply (other workload, or kernel sources changed since)."""
+def captured_traffic(workload_name, schedule=None):
+    """Measured DRAM bytes of the tensor-core launches of one step, or None
+    when the capture does not apply (other workload or schedules, or kernel
+    sources changed since)."""
     import hashlib
     cap = TRAFFIC_CAPTURE
     if workload_name != cap["workload"]:
+        return None
+    if cap.get("schedule") is not None and schedule != cap["schedule"]:
         return None
     h = hashlib.sha256()
     for rel in cap["sources"]:
@@ -129,7 +133,7 @@ def captured_traffic(workload_name):
             h.update(fh.read())
     if h.hexdigest() != cap["sha256"]:
         return None
-    return cap["dram_bytes_per_step"] / cap["launches_per_step"]
+    return cap["dram_bytes_per_step"]
 
 
 def momentum_bytes(shapes, grad_bytes=2, image16=False):
@@ -730,10 +734,8 @@ def main():
     clk = clocks.stop()
     total_ms *= K
     # per-rank launches are those of the captured run only for the whole
-    # layer set at the default precision
-    all_pairs = all(v == "cta_pair" for part in schedule.values() for v in part.values()) \
-        if isinstance(schedule, dict) else False
-    traffic = captured_traffic(w_full.name) if args.prec == "auto" and all_pairs else None
+    # layer set at the default precision, under the captured schedules
+    traffic = captured_traffic(w_full.name, schedule) if args.prec == "auto" else None
     step_ms = owners.max_over_ranks(total_ms / K, device=dev)
     eager_max = owners.max_over_ranks(eager_ms, device=dev)
     status = plan.read_status()
@@ -854,7 +856,7 @@ def main():
             "eager_ms_per_step": round(eager_max, 3),
             "roofline": {"bound": "tensor", "achieved": round(achieved_tf, 1), "peak": peak_tf,
                          "unit": "TFLOP/s", "frac": round(achieved_tf / peak_tf, 4),
-                         "traffic": traffic,
+                         "traffic": round(traffic / max(tc_launches, 1)) if traffic else None,
                          "alg_bytes_per_launch": round(gemm_alg_bytes(w.shapes) / max(tc_launches, 1)),
                          "kernel": "k_gemm_tc2 (all Gram-space and final launches)",
                          "peak_kind": f"{peak_kind} cuBLAS bf16 GEMM, sustained (achievable)",

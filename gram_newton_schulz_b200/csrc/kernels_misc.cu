@@ -505,16 +505,19 @@ cudaError_t launch_norm_finalize(const MomMat* mats, int nmats, const float* par
 // ------------------------------------------------------------- helpers
 // Identity as a 16-bit hi/lo pair; `one` is the bit pattern of 1.0 in the
 // pair's format (0x3F80 bf16, 0x3C00 fp16).
+// One block per row (grid-stride over the count * m rows), so a thread's
+// index arithmetic is a 32-bit division per row rather than 64-bit
+// divisions per element.
 __global__ void k_identity16(uint16_t* hi, uint16_t* lo, int count, int m, long long ld, long long mat_stride,
                              uint16_t one) {
-  const long long total = (long long)count * m * m;
-  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
-       e += (long long)gridDim.x * blockDim.x) {
-    const long long mat = e / ((long long)m * m);
-    const long long r = (e / m) % m, c = e % m;
-    const long long o = mat * mat_stride + r * ld + c;
-    hi[o] = r == c ? one : (uint16_t)0;
-    lo[o] = 0;
+  const int rows = count * m;
+  for (int row = blockIdx.x; row < rows; row += gridDim.x) {
+    const int mat = row / m, r = row - mat * m;
+    const long long o = (long long)mat * mat_stride + (long long)r * ld;
+    for (int c = threadIdx.x; c < m; c += blockDim.x) {
+      hi[o + c] = c == r ? one : (uint16_t)0;
+      lo[o + c] = 0;
+    }
   }
 }
 
@@ -575,7 +578,10 @@ static int grid_for(long long total) {
 
 cudaError_t launch_identity16(void* hi, void* lo, int count, int m, long long ld, long long mat_stride, int f16,
                               cudaStream_t s) {
-  k_identity16<<<grid_for((long long)count * m * m), 256, 0, s>>>(
+  if ((long long)count * m > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const int rows = count * m;
+  if (rows <= 0) return cudaSuccess;
+  k_identity16<<<rows < 8192 ? rows : 8192, 256, 0, s>>>(
       reinterpret_cast<uint16_t*>(hi), reinterpret_cast<uint16_t*>(lo), count, m, ld, mat_stride,
       f16 ? (uint16_t)0x3C00 : (uint16_t)0x3F80);
   return cudaGetLastError();

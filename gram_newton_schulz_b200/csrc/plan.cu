@@ -683,6 +683,7 @@ dmu_status gram_bf16(dmu_plan p, const float co[3], int steps, cudaStream_t s) {
     for (size_t c = 0; c < p->classes.size(); ++c) {
       const GClass& gc = p->classes[c];
       if (p->tune_class >= 0 && (int)c != p->tune_class) continue;
+      if (p->tune_syrk >= 0) continue;  // timing one bucket's SYRK alone
       // P_0 = I as an fp16 pair: in P buffer A for F16 classes, in the
       // final-P area for the others
       const bool f16 = gc.kind == KIND_F16;
