@@ -565,7 +565,8 @@ def run_demuon(args, w_full, dev, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: 20; 5 for --impl reference, whose steps are oracle samples)")
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="dmu", choices=["dmu", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
@@ -597,6 +598,8 @@ def main():
                     help="schedule cache file for dmu_autotune (read and appended)")
     ap.add_argument("--ref-budget", type=float, default=10.0)
     args = ap.parse_args()
+    if args.steps is None:
+        args.steps = 5 if args.impl == "reference" else 20
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
