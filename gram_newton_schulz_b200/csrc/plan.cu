@@ -86,7 +86,8 @@ struct GClass {
 // not overlap the next tile), scaled-fp16 launches only (others run 1).
 // The Gram products and the final lose more to the exposed epilogue than
 // they gain (measured), so schedule 6 is an autotune candidate only for the
-// SYRK, whose K is the long side n.
+// SYRK, whose K is the long side n (with schedules 0 and 4 beside the
+// class's own).
 constexpr int SCHED_ONCHIP = 3;
 constexpr int SCHED_WIDE = 6;
 constexpr int TILE_SCHEDS[6] = {0, 1, 2, 4, 5, 6};
@@ -1562,9 +1563,15 @@ dmu_status dmu_autotune(dmu_plan p, const char* cache_path, void* stream) {
     float best_ms = 0.f;
     p->tune_class = b.cls;
     p->tune_syrk = (int)bi;
+    // candidates: the class's own schedule first (it wins ties), then the
+    // single-CTA tiles, the three-stage CTA pairs and the 256 x 512 pairs
+    // (measured alone on long-K SYRKs: 2 K atoms x 3 stages and single CTAs
+    // can beat the class's choice, which is tuned for the products' epilogue)
     const int own = p->class_sched(b.cls);
-    for (int sc : {own, SCHED_WIDE}) {
-      if (sc == SCHED_WIDE && own == SCHED_WIDE) break;
+    std::vector<int> cand = {own};
+    for (int sc : {0, 4, SCHED_WIDE})
+      if (sc != own) cand.push_back(sc);
+    for (int sc : cand) {
       b.ssched = sc;
       const float ms = time_min([&] { return gram_bf16(p, co, 0, s); });
       if (st != DMU_OK) break;

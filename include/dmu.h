@@ -259,9 +259,10 @@ DMU_API int dmu_get_gram_schedule(dmu_plan plan, int index);
 DMU_API int dmu_get_final_schedule(dmu_plan plan, int index);
 
 /* Schedule of the SYRK (G0 = s^2 X X^T) of matrix `index`'s bucket: its
- * class's tile schedule, or 6 when dmu_autotune measured the 256 x 512
- * CTA-pair tile faster for that bucket (its K is the long side n); 3 when
- * the class runs on chip.  -1 for a bad argument. */
+ * class's tile schedule unless dmu_autotune measured another one faster
+ * for that bucket's SYRK alone (candidates 0, 4 and 6 besides the class's;
+ * its K is the long side n); 3 when the class runs on chip.  -1 for a bad
+ * argument. */
 DMU_API int dmu_get_syrk_schedule(dmu_plan plan, int index);
 
 /* Number of kernel launches the last compute call enqueued. */
