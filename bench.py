@@ -781,7 +781,9 @@ def main():
     if not args.no_e2e and e2e is None:
         E = args.e2e_steps
         g_buf = [grads, [torch.empty_like(g) for g in grads]]
-        w_stage = [torch.empty_like(x) for x in weights]  # device copy of W that the download reads
+        # two device copies of W that the downloads read, alternating, so the
+        # staging of step k waits only for the download of step k - 2
+        w_stage = [[torch.empty_like(x) for x in weights] for _ in range(2)]
         h2d = sum(t.numel() * t.element_size() for t in h_grads)
         d2h = sum(t.numel() * t.element_size() for t in h_w)
         s_in = torch.cuda.Stream(dev)
@@ -812,15 +814,16 @@ def main():
             plan.apply_update(weights, lr=w.lr, stream=stream)
             # stage W in device memory (one fast device copy), so the next
             # update need not wait for this step's download
-            if k >= 1:
-                stream.wait_event(out_done[k - 1])  # the stage's previous download is done
-            for st_, x in zip(w_stage, weights):
+            stage = w_stage[k % 2]
+            if k >= 2:
+                stream.wait_event(out_done[k - 2])  # this stage's previous download is done
+            for st_, x in zip(stage, weights):
                 st_.copy_(x, non_blocking=True)
             upd = torch.cuda.Event()
             upd.record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(upd)
-                for hw, x in zip(h_w, w_stage):
+                for hw, x in zip(h_w, stage):
                     hw.copy_(x, non_blocking=True)
                 out_done[k].record(s_out)
         stream.wait_event(out_done[E - 1])
@@ -830,8 +833,8 @@ def main():
         e2e_ms = owners.max_over_ranks(e0.elapsed_time(e1) / E, device=dev)
         e2e = {"value": round(e2e_ms, 3), "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "overlap": "H2D of step k+1 and D2H of step k overlap compute on separate copy streams; "
-                          "W is staged by a device copy after each update, so the next update does not "
-                          "wait for the download",
+                          "W is staged by a device copy after each update into one of two stage buffers, "
+                          "so neither the next update nor the next staging waits for this download",
                "host_link": host_link_rates(h_grads, grads, h_w, weights, s_in, s_out, dev)}
 
     cpu = None
