@@ -106,16 +106,16 @@ def gemm_alg_bytes(shapes, k=K_STEPS):
 # captured ones (close calls of the autotuner can differ from box to box).
 TRAFFIC_CAPTURE = {
     "sources": ["gram_newton_schulz_b200/csrc/gemm_tc.cu", "gram_newton_schulz_b200/csrc/plan.cu"],
-    "sha256": "1bd9ba78a6728b2984652452f8423b7e09bfdecb26f5feab6b25a1b96600599d",
+    "sha256": "199c54b8168a091124b98048e0114aaf5a1a349b208109fcac0de92ad319b7ff",
     "workload": "qwen2.5-7b-layer-set-x28",
     "captured_on": "3584x3584*4,512x3584*4,18944x3584*4,3584x18944*2 (2 of 28 layers)",
     "scale": 14,
-    "dram_bytes_per_step": 14.715e9 * 14,
+    "dram_bytes_per_step": 15.423e9 * 14,
     "schedule": {
         "gram": {"m512": "single_cta_n128", "m3584": "cta_pair"},
-        "syrk": {"512x3584": "single_cta_n128", "3584x3584": "cta_pair", "3584x18944": "cta_pair_n512",
-                 "18944x3584": "cta_pair_n512"},
-        "final": {"512x3584": "single_cta", "3584x3584": "single_cta", "3584x18944": "cta_pair",
+        "syrk": {"512x3584": "cta_pair_k2", "3584x3584": "single_cta", "3584x18944": "single_cta",
+                 "18944x3584": "single_cta"},
+        "final": {"512x3584": "single_cta", "3584x3584": "single_cta", "3584x18944": "single_cta",
                   "18944x3584": "single_cta"},
     },
 }
