@@ -403,8 +403,13 @@ def run_owner(args, w_full, dev, world, rank, local, barrier):
     owned = osd.owned_shapes()
     moms = [torch.zeros(s, dtype=torch.float32, device=dev) for s in owned]
     kw = dict(beta=w_full.beta, lr=w_full.lr, eps=1e-7, coeffs=dmu.QUINTIC, steps=K_STEPS)
-    for _ in range(args.warmup):
+    for k in range(args.warmup):
         osd.step(gflat, wflat, moms, **kw)
+        if k == 0 and not args.no_autotune:  # schedules per shape, on this rank's data
+            cache = args.schedule_cache
+            if cache and world > 1:
+                cache = f"{cache}.rank{rank}"  # one file per rank: no interleaved appends
+            osd.autotune(cache)
     torch.cuda.synchronize(dev)
     if osd.read_status() != 0:
         raise SystemExit("device status word set during warm-up")

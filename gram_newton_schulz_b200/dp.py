@@ -152,6 +152,11 @@ class PlanCompute:
         n2 = self.plan.last_launch_count()
         self.launches, self.tc_launches = n0 + n1 + n2, n1 + n2
 
+    def autotune(self, cache_path=None):
+        """Per-shape schedule choice for this group's plan (needs the data
+        of a prior call); see `dmu.Plan.autotune`."""
+        return self.plan.autotune(cache_path) if self.plan is not None else {}
+
     def close(self):
         if self.plan is not None:
             self.plan.close()
@@ -204,6 +209,12 @@ class OwnerShardedStep:
     @property
     def tc_launches(self) -> int:
         return sum(getattr(c, "tc_launches", 0) for c in set(self.computes))
+
+    def autotune(self, cache_path=None):
+        """Per-shape schedule choice for each publish group's plan, after a
+        step has given the plans data.  Local to this rank: schedules change
+        no collective, so the ranks need not agree on them."""
+        return [c.autotune(cache_path) for c in self.computes if hasattr(c, "autotune")]
 
     def read_status(self) -> int:
         """OR of the device status words of the groups' plans."""
