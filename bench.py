@@ -106,7 +106,7 @@ def gemm_alg_bytes(shapes, k=K_STEPS):
 # captured ones (close calls of the autotuner can differ from box to box).
 TRAFFIC_CAPTURE = {
     "sources": ["gram_newton_schulz_b200/csrc/gemm_tc.cu", "gram_newton_schulz_b200/csrc/plan.cu"],
-    "sha256": "199c54b8168a091124b98048e0114aaf5a1a349b208109fcac0de92ad319b7ff",
+    "sha256": "8884bb97dc0fa6147c07bb61e3ff32889137c9c1f58e58ce921b3f7aaa5950ef",
     "workload": "qwen2.5-7b-layer-set-x28",
     "captured_on": "3584x3584*4,512x3584*4,18944x3584*4,3584x18944*2 (2 of 28 layers)",
     "scale": 14,

@@ -19,8 +19,10 @@
 //              K=16) into one of two TMEM accumulators (2 x 256 columns);
 //   warps 2-9  epilogue: tcgen05.ld of their 32-lane quarter (two warps per
 //              quarter, each on half of the tile's columns), fp32 affine
-//              epilogue, hi/lo split, direct + mirrored stores; the
-//              epilogue of tile t overlaps the main loop of tile t+1.
+//              epilogue, hi/lo split, direct stores; in diagonal tiles the
+//              mirror images move as 8 x 8 block transposes through a
+//              per-warp shared scratch; the epilogue of tile t overlaps
+//              the main loop of tile t+1.
 // Operand precision: each stage holds up to two bf16 parts of A (hi, lo)
 // and of B; the problem's term bits choose hi*hi, hi*lo, lo*hi.
 // Every mbarrier wait is bounded by a wall-clock limit; on expiry the CTA
@@ -858,6 +860,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
 // bytes and issues the MMAs; its commits arrive on both CTAs' barriers;
 // both epilogues arrive on the leader's TMEM-empty barrier.  No load uses
 // cluster multicast: every byte a CTA reads comes from its own TMA loads.
+// With TN = 512 the pair's tile is 256 x 512: two N = 256 MMAs per K slice
+// share the A operand (a quarter fewer operand bytes per MMA), and the
+// 512-column accumulator fills TMEM, so the epilogue of a tile does not
+// overlap the next tile's main loop.
 constexpr int BM2 = 256;
 constexpr int HALF_BYTES = 128 * 128;  // 128 rows x 128-byte K row
 
