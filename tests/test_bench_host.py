@@ -82,6 +82,16 @@ def test_captured_traffic_applies_only_to_its_sources(monkeypatch):
     assert bench.captured_traffic(cap["workload"]) == cap["dram_bytes_per_step"]
 
 
+def test_schedule_summary_has_gram_syrk_and_final_entries():
+    sch = {"gram": {3584: "cta_pair", 512: "single_cta_n128"},
+           "syrk": {(3584, 18944): "cta_pair_n512", (512, 3584): "cta_pair_k2"},
+           "final": {(3584, 18944): "single_cta"}}
+    out = bench.schedule_summary(sch)
+    assert out == {"gram": {"m3584": "cta_pair", "m512": "single_cta_n128"},
+                   "syrk": {"3584x18944": "cta_pair_n512", "512x3584": "cta_pair_k2"},
+                   "final": {"3584x18944": "single_cta"}}
+
+
 def test_captured_traffic_names_its_schedules():
     # the capture records the schedule choices it ran under, in the bench
     # line's own form, so a run can say whether its choices were the same

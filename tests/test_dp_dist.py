@@ -166,6 +166,8 @@ def test_single_process_step_matches_oracle():
     moms = [torch.from_numpy(_momentum0(i)).clone() for i in step.mine]
     step.step(gf, wf, moms, beta=BETA, lr=LR, eps=EPS)
     assert compute.calls == [len(g) for g in step.publish]  # one call per publish group
+    # a stand-in compute has no schedules to tune: autotune is a no-op
+    assert step.autotune() == []
     ew, em = _expected(1)
     for i in range(len(SHAPES)):
         assert np.array_equal(b.view(wf, i).numpy(), ew[i])
