@@ -91,16 +91,13 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
                                          const GemmParams& p) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer();
-  uint32_t n = 0;
   for (;;) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
-    if ((++n & 63u) == 0) {
-      if (*abort_flag) return false;
-      if ((long long)(ptx::globaltimer() - t0) > p.timeout_ns) {
-        *abort_flag = 1;
-        atomicOr(p.status, DMU_FLAG_TIMEOUT);
-        return false;
-      }
+    if (*abort_flag) return false;
+    if ((long long)(ptx::globaltimer() - t0) > p.timeout_ns) {
+      *abort_flag = 1;
+      atomicOr(p.status, DMU_FLAG_TIMEOUT);
+      return false;
     }
   }
 }
@@ -895,16 +892,13 @@ __device__ __forceinline__ bool wait_bar_cluster(uint32_t bar, uint32_t parity, 
                                                  const GemmParams& p) {
   if (ptx::mbar_try_wait_cluster(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer();
-  uint32_t n = 0;
   for (;;) {
     if (ptx::mbar_try_wait_cluster(bar, parity)) return true;
-    if ((++n & 63u) == 0) {
-      if (*abort_flag) return false;
-      if ((long long)(ptx::globaltimer() - t0) > p.timeout_ns) {
-        *abort_flag = 1;
-        atomicOr(p.status, DMU_FLAG_TIMEOUT);
-        return false;
-      }
+    if (*abort_flag) return false;
+    if ((long long)(ptx::globaltimer() - t0) > p.timeout_ns) {
+      *abort_flag = 1;
+      atomicOr(p.status, DMU_FLAG_TIMEOUT);
+      return false;
     }
   }
 }
@@ -1222,10 +1216,9 @@ __global__ void k_wait_selftest(unsigned int* status, long long timeout_ns) {
   __syncthreads();
   if (threadIdx.x == 0) {
     const uint64_t t0 = ptx::globaltimer();
-    uint32_t n = 0;
     for (;;) {
       if (ptx::mbar_try_wait(ptx::smem_u32(&bar), 0)) break;
-      if ((++n & 63u) == 0 && (long long)(ptx::globaltimer() - t0) > timeout_ns) {
+      if ((long long)(ptx::globaltimer() - t0) > timeout_ns) {
         atomicOr(status, DMU_FLAG_TIMEOUT);
         break;
       }

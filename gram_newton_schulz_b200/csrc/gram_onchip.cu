@@ -84,16 +84,13 @@ __device__ __forceinline__ bool oc_wait(uint32_t bar, uint32_t parity, volatile 
                                         const OnchipParams& p) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer();
-  uint32_t n = 0;
   for (;;) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
-    if ((++n & 63u) == 0) {
-      if (*abort_flag) return false;
-      if ((long long)(ptx::globaltimer() - t0) > p.timeout_ns) {
-        *abort_flag = 1;
-        atomicOr(p.status, DMU_FLAG_TIMEOUT);
-        return false;
-      }
+    if (*abort_flag) return false;
+    if ((long long)(ptx::globaltimer() - t0) > p.timeout_ns) {
+      *abort_flag = 1;
+      atomicOr(p.status, DMU_FLAG_TIMEOUT);
+      return false;
     }
   }
 }
