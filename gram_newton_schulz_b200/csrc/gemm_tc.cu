@@ -115,16 +115,17 @@ __device__ __forceinline__ void unpack8(const uint4& u, float* f) {
   }
 }
 
+// hi = RN(v), lo = RN(v - hi), two values per packed conversion (v - hi is
+// exact in fp32, so the pair carries v to 16 + 8 bits).
 __device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
   __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&hi);
   __nv_bfloat162* l = reinterpret_cast<__nv_bfloat162*>(&lo);
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    __nv_bfloat16 h0 = __float2bfloat16_rn(v[2 * q]);
-    __nv_bfloat16 h1 = __float2bfloat16_rn(v[2 * q + 1]);
-    h[q] = __halves2bfloat162(h0, h1);
-    l[q] = __halves2bfloat162(__float2bfloat16_rn(v[2 * q] - bf2f(h0)),
-                              __float2bfloat16_rn(v[2 * q + 1] - bf2f(h1)));
+    const __nv_bfloat162 hq = __floats2bfloat162_rn(v[2 * q], v[2 * q + 1]);
+    const float2 f = __bfloat1622float2(hq);
+    h[q] = hq;
+    l[q] = __floats2bfloat162_rn(__fsub_rn(v[2 * q], f.x), __fsub_rn(v[2 * q + 1], f.y));
   }
 }
 
@@ -143,11 +144,10 @@ __device__ __forceinline__ void split8_h(const float* v, uint4& hi, uint4& lo) {
   __half2* l = reinterpret_cast<__half2*>(&lo);
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    __half h0 = __float2half_rn(v[2 * q]);
-    __half h1 = __float2half_rn(v[2 * q + 1]);
-    h[q] = __halves2half2(h0, h1);
-    l[q] = __halves2half2(__float2half_rn(v[2 * q] - __half2float(h0)),
-                          __float2half_rn(v[2 * q + 1] - __half2float(h1)));
+    const __half2 hq = __floats2half2_rn(v[2 * q], v[2 * q + 1]);
+    const float2 f = __half22float2(hq);
+    h[q] = hq;
+    l[q] = __floats2half2_rn(__fsub_rn(v[2 * q], f.x), __fsub_rn(v[2 * q + 1], f.y));
   }
 }
 

@@ -121,16 +121,17 @@ struct EpiArgs {
   long long ld;
 };
 
+// hi = RN(v), lo = RN(v - hi) (v - hi is exact), two values per packed
+// conversion.
 __device__ __forceinline__ void split8_h(const float* v, uint4& hi, uint4& lo) {
   __half2* h = reinterpret_cast<__half2*>(&hi);
   __half2* l = reinterpret_cast<__half2*>(&lo);
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    const __half h0 = __float2half_rn(v[2 * q]);
-    const __half h1 = __float2half_rn(v[2 * q + 1]);
-    h[q] = __halves2half2(h0, h1);
-    l[q] = __halves2half2(__float2half_rn(v[2 * q] - __half2float(h0)),
-                          __float2half_rn(v[2 * q + 1] - __half2float(h1)));
+    const __half2 hq = __floats2half2_rn(v[2 * q], v[2 * q + 1]);
+    const float2 f = __half22float2(hq);
+    h[q] = hq;
+    l[q] = __floats2half2_rn(__fsub_rn(v[2 * q], f.x), __fsub_rn(v[2 * q + 1], f.y));
   }
 }
 
@@ -140,7 +141,6 @@ __device__ __forceinline__ void st_pair_h(__half* hi, __half* lo, long long o, f
   lo[o] = __float2half_rn(v - __half2float(h));
 }
 
-__device__ __forceinline__ uint32_t bf_bits(__nv_bfloat16 x) { return (uint32_t)__bfloat16_as_ushort(x); }
 
 // Row stores of one chunk (row i, columns col0 .. col0 + 7, only i, j < m)
 // as a bf16 hi/lo pair: rows above the chunk's diagonal 8 x 8 block and rows
@@ -151,10 +151,12 @@ __device__ __forceinline__ void store_chunk_rows(uint8_t* buf, int m, int i, int
   uint32_t hi[OC_CW / 2], lo[OC_CW / 2];  // packed pairs of columns
 #pragma unroll
   for (int c = 0; c < OC_CW; c += 2) {
-    const __nv_bfloat16 h0 = __float2bfloat16_rn(v[c]), h1 = __float2bfloat16_rn(v[c + 1]);
-    hi[c / 2] = bf_bits(h0) | (bf_bits(h1) << 16);
-    lo[c / 2] = bf_bits(__float2bfloat16_rn(__fsub_rn(v[c], bf(h0)))) |
-                (bf_bits(__float2bfloat16_rn(__fsub_rn(v[c + 1], bf(h1)))) << 16);
+    // hi = RN(v), lo = RN(v - hi) (exact difference), two per conversion
+    const __nv_bfloat162 hq = __floats2bfloat162_rn(v[c], v[c + 1]);
+    const float2 f = __bfloat1622float2(hq);
+    const __nv_bfloat162 lq = __floats2bfloat162_rn(__fsub_rn(v[c], f.x), __fsub_rn(v[c + 1], f.y));
+    hi[c / 2] = *reinterpret_cast<const uint32_t*>(&hq);
+    lo[c / 2] = *reinterpret_cast<const uint32_t*>(&lq);
   }
   if (col0 + OC_CW <= m) {
     const uint32_t o = oc_off(i, col0);
