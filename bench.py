@@ -583,7 +583,7 @@ def main():
     ap.add_argument("--shapes", default=None,
                     help="custom spiked bf16 workload for profiling, e.g. 3584x3584*8,512x3584*4")
     ap.add_argument("--prec", default="auto")
-    ap.add_argument("--e2e-steps", type=int, default=12,
+    ap.add_argument("--e2e-steps", type=int, default=20,
                     help="steps of the e2e leg; its first upload and last download overlap no compute, "
                          "so longer runs approach the steady state")
     ap.add_argument("--no-e2e", action="store_true")
