@@ -242,6 +242,43 @@ __device__ __forceinline__ void tri_mirror_part(uint16_t* o, long long mbase, lo
   __syncwarp();
 }
 
+// The Cin row segment of one chunk (16 values of row i), loaded ahead of its
+// use so that its latency overlaps the previous chunk's epilogue (or, for a
+// tile's first chunk, the main loop): a 16-bit pair as raw[0..1] (hi) and
+// raw[2..3] (lo), or fp32 as raw[0..3].  `ok` is set only for a whole chunk
+// inside the matrix with an input to read; other chunks load per element.
+// Cin is never written by the launch that reads it, so loading early is safe.
+struct CinRow {
+  uint4 raw[4];
+  bool ok;
+};
+
+__device__ __forceinline__ void cin_fetch(const GemmProblem& pr, int mat, int i, int col0, CinRow& c) {
+  c.ok = false;
+  if (i >= pr.M || col0 + CW > pr.N) return;
+  const long long off = (long long)mat * pr.mat_stride + (long long)i * pr.ld + col0;
+  if (pr.cin_fmt == FMT_F32 && pr.cin_f) {
+    const uint4* pf = reinterpret_cast<const uint4*>(pr.cin_f + off);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) c.raw[q] = ld_row16(pf + q);
+    c.ok = true;
+  } else if ((pr.cin_fmt == FMT_PAIR_H || pr.cin_fmt == FMT_PAIR) && pr.cin_hi) {
+    // both 16-bit formats are addressed as 2-byte elements
+    const uint4* ph = reinterpret_cast<const uint4*>(pr.cin_hi + off);
+    c.raw[0] = ld_row16(ph);
+    c.raw[1] = ld_row16(ph + 1);
+    if (pr.cin_lo) {
+      const uint4* pl = reinterpret_cast<const uint4*>(pr.cin_lo + off);
+      c.raw[2] = ld_row16(pl);
+      c.raw[3] = ld_row16(pl + 1);
+    } else {
+      c.raw[2] = make_uint4(0u, 0u, 0u, 0u);  // +0 in both formats: hi + 0 = hi exactly
+      c.raw[3] = c.raw[2];
+    }
+    c.ok = true;
+  }
+}
+
 // One CW-column chunk of a Gram-space output tile for the thread's row i.
 // Input and outputs are bf16 hi/lo pairs (FMT_PAIR) or fp32 (FMT_F32).
 // Every rounding step is explicit (__fmul_rn, __fadd_rn, __fmaf_rn), so the
@@ -250,7 +287,8 @@ __device__ __forceinline__ void tri_mirror_part(uint16_t* o, long long mbase, lo
 // `tri`: store only i <= j and mirror (symmetric outputs, except the
 // off-diagonal tiles of half-stored outputs, which are written whole).
 __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, int i, int col0,
-                                               const uint32_t (&r)[CW], bool tri, uint32_t scr) {
+                                               const uint32_t (&r)[CW], bool tri, uint32_t scr,
+                                               const CinRow& cin) {
   const int M = pr.M, N = pr.N;
   const int lane = (int)(threadIdx.x & 31u);
   const int row_lo = i - lane;
@@ -274,67 +312,48 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
   const bool full = (col0 + CW <= N);
   const bool all_upper = !tri || (i <= col0);
 
-  if (pr.cin_fmt == FMT_F32 && pr.cin_f) {
-    if (full) {
-      const float4* pc = reinterpret_cast<const float4*>(pr.cin_f + rowoff + col0);
+  if (cin.ok) {
+    // the whole chunk's row segment, loaded by cin_fetch
+    if (pr.cin_fmt == FMT_F32) {
 #pragma unroll
-      for (int q = 0; q < CW / 4; ++q) {
-        const float4 t = pc[q];
-        v[4 * q] = __fmaf_rn(pr.beta, t.x, v[4 * q]);
-        v[4 * q + 1] = __fmaf_rn(pr.beta, t.y, v[4 * q + 1]);
-        v[4 * q + 2] = __fmaf_rn(pr.beta, t.z, v[4 * q + 2]);
-        v[4 * q + 3] = __fmaf_rn(pr.beta, t.w, v[4 * q + 3]);
+      for (int q = 0; q < 4; ++q) {
+        v[4 * q] = __fmaf_rn(pr.beta, __uint_as_float(cin.raw[q].x), v[4 * q]);
+        v[4 * q + 1] = __fmaf_rn(pr.beta, __uint_as_float(cin.raw[q].y), v[4 * q + 1]);
+        v[4 * q + 2] = __fmaf_rn(pr.beta, __uint_as_float(cin.raw[q].z), v[4 * q + 2]);
+        v[4 * q + 3] = __fmaf_rn(pr.beta, __uint_as_float(cin.raw[q].w), v[4 * q + 3]);
       }
     } else {
 #pragma unroll
-      for (int c = 0; c < CW; ++c)
-        if (col0 + c < N) v[c] = __fmaf_rn(pr.beta, pr.cin_f[rowoff + col0 + c], v[c]);
-    }
-  } else if (pr.cin_fmt == FMT_PAIR_H && pr.cin_hi) {
-    const __half* ch = reinterpret_cast<const __half*>(pr.cin_hi);
-    const __half* cl = reinterpret_cast<const __half*>(pr.cin_lo);
-    if (full) {
-      const uint4* ph = reinterpret_cast<const uint4*>(ch + rowoff + col0);
-      const uint4* pl = reinterpret_cast<const uint4*>(cl + rowoff + col0);
-      uint4 uh[CW / 8], ul[CW / 8];
-#pragma unroll
-      for (int q = 0; q < CW / 8; ++q) {
-        uh[q] = ld_row16(ph + q);
-        ul[q] = ld_row16(pl + q);
-      }
-#pragma unroll
       for (int q = 0; q < CW / 8; ++q) {
         float fh[8], fl[8];
-        unpack8_h(uh[q], fh);
-        unpack8_h(ul[q], fl);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v[8 * q + e] = __fmaf_rn(pr.beta, __fadd_rn(fh[e], fl[e]), v[8 * q + e]);
-      }
-    } else {
-#pragma unroll
-      for (int c = 0; c < CW; ++c)
-        if (col0 + c < N)
-          v[c] = __fmaf_rn(pr.beta, __fadd_rn(__half2float(ch[rowoff + col0 + c]), __half2float(cl[rowoff + col0 + c])),
-                           v[c]);
-    }
-  } else if (pr.cin_fmt == FMT_PAIR && pr.cin_hi) {
-    if (full) {
-      const uint4* ph = reinterpret_cast<const uint4*>(pr.cin_hi + rowoff + col0);
-      const uint4* pl = pr.cin_lo ? reinterpret_cast<const uint4*>(pr.cin_lo + rowoff + col0) : nullptr;
-#pragma unroll
-      for (int q = 0; q < CW / 8; ++q) {
-        float fh[8], fl[8];
-        unpack8(ld_row16(ph + q), fh);
-        if (pl) {
-          unpack8(ld_row16(pl + q), fl);
+        if (pr.cin_fmt == FMT_PAIR_H) {
+          unpack8_h(cin.raw[q], fh);
+          unpack8_h(cin.raw[2 + q], fl);
         } else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) fl[e] = 0.f;
+          unpack8(cin.raw[q], fh);
+          unpack8(cin.raw[2 + q], fl);
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) v[8 * q + e] = __fmaf_rn(pr.beta, __fadd_rn(fh[e], fl[e]), v[8 * q + e]);
       }
-    } else {
+    }
+  } else if (!full) {
+    // ragged chunk: per-element loads of the columns inside the matrix
+    if (pr.cin_fmt == FMT_F32 && pr.cin_f) {
+#pragma unroll
+      for (int c = 0; c < CW; ++c)
+        if (col0 + c < N) v[c] = __fmaf_rn(pr.beta, pr.cin_f[rowoff + col0 + c], v[c]);
+    } else if (pr.cin_fmt == FMT_PAIR_H && pr.cin_hi) {
+      const __half* ch = reinterpret_cast<const __half*>(pr.cin_hi);
+      const __half* cl = reinterpret_cast<const __half*>(pr.cin_lo);
+#pragma unroll
+      for (int c = 0; c < CW; ++c)
+        if (col0 + c < N) {
+          float x = __half2float(ch[rowoff + col0 + c]);
+          if (cl) x = __fadd_rn(x, __half2float(cl[rowoff + col0 + c]));
+          v[c] = __fmaf_rn(pr.beta, x, v[c]);
+        }
+    } else if (pr.cin_fmt == FMT_PAIR && pr.cin_hi) {
 #pragma unroll
       for (int c = 0; c < CW; ++c) {
         if (col0 + c < N) {
@@ -807,26 +826,39 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
     for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
       const TileCoord tc = decode_tile<BM, TBN>(p, t);
       const GemmProblem& pr = p.prob[tc.pi];
+      const int row_lo = tc.bi * BM + q * 32;
+      const bool tri = pr.sym && (!pr.half_out || (tc.bi * BM) / HALF_BLOCK == (tc.bj * TBN) / HALF_BLOCK);
+      const int i = row_lo + lane;
+      // this warp's chunks of the tile, [c_lo, c_hi): inside the matrix and,
+      // in symmetric diagonal tiles, not strictly below the diagonal
+      int c_lo = ch_begin, c_hi = ch_end;
+      const int c_in = (pr.N - tc.bj * TBN + CW - 1) / CW;
+      if (c_hi > c_in) c_hi = c_in;
+      if (row_lo >= pr.M) c_hi = c_lo;
+      while (tri && c_lo < c_hi && tc.bj * TBN + c_lo * CW + CW - 1 < row_lo) ++c_lo;
+      const bool gram = pr.epi == EPI_GRAM;
+      CinRow cin;
+      cin.ok = false;
+      if (gram && c_lo < c_hi) cin_fetch(pr, tc.mat, i, tc.bj * TBN + c_lo * CW, cin);  // overlaps the main loop
       int ok = 1;
       if (lane == 0) ok = wait_bar(tfull_bar(acc), acc_phase, abort_flag, p) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       ptx::tc_fence_after();
-      const int row_lo = tc.bi * BM + q * 32;
-      const bool tri = pr.sym && (!pr.half_out || (tc.bi * BM) / HALF_BLOCK == (tc.bj * TBN) / HALF_BLOCK);
-      const int i = row_lo + lane;
-      for (int ch = ch_begin; ch < ch_end; ++ch) {
+      for (int ch = c_lo; ch < c_hi; ++ch) {
         const int col0 = tc.bj * TBN + ch * CW;
-        if (col0 >= pr.N) break;
-        if (tri && col0 + CW - 1 < row_lo) continue;  // chunk strictly below the diagonal
-        if (row_lo >= pr.M) break;
         uint32_t r[CW];
         ptx::tmem_ld16(tmem_base + (uint32_t)(acc * TBN + ch * CW) + ((uint32_t)(q * 32) << 16), r);
         ptx::tmem_wait_ld();
-        if (pr.epi == EPI_GRAM)
-          epi_gram_chunk(pr, tc.mat, i, col0, r, tri, scr);
-        else
+        if (gram) {
+          CinRow nxt;
+          nxt.ok = false;
+          if (ch + 1 < c_hi) cin_fetch(pr, tc.mat, i, col0 + CW, nxt);
+          epi_gram_chunk(pr, tc.mat, i, col0, r, tri, scr, cin);
+          cin = nxt;
+        } else {
           epi_update_chunk(pr, tc.mat, i, col0, r);
+        }
       }
       ptx::tc_fence_before();
       __syncwarp();
@@ -1162,30 +1194,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     for (int t = pair; t < p.total_tiles; t += npairs) {
       const TileCoord tc = decode_tile<BM2, TN>(p, t);
       const GemmProblem& pr = p.prob[tc.pi];
+      const int row_lo = tc.bi * BM2 + (int)rank * 128 + q * 32;
+      const int i = row_lo + lane;
+      // half-stored outputs: lower blocks are never written, the diagonal
+      // block is mirrored, upper blocks are written whole
+      auto chunk_tri = [&](int col0) { return pr.sym && (!pr.half_out || col0 / HALF_BLOCK == tc.bi); };
+      // this warp's chunks of the tile, [c_lo, c_hi): inside the matrix, not
+      // in a lower block, not strictly below the diagonal (the skipped
+      // chunks of a tile are always its leftmost ones)
+      int c_lo = ch_begin, c_hi = ch_end;
+      const int c_in = (pr.N - tc.bj * TN + CW - 1) / CW;
+      if (c_hi > c_in) c_hi = c_in;
+      if (row_lo >= pr.M) c_hi = c_lo;
+      while (c_lo < c_hi) {
+        const int col0 = tc.bj * TN + c_lo * CW;
+        if (pr.sym && pr.half_out && col0 / HALF_BLOCK < tc.bi) { ++c_lo; continue; }
+        if (chunk_tri(col0) && col0 + CW - 1 < row_lo) { ++c_lo; continue; }
+        break;
+      }
+      const bool gram = pr.epi == EPI_GRAM;
+      CinRow cin;
+      cin.ok = false;
+      if (gram && c_lo < c_hi) cin_fetch(pr, tc.mat, i, tc.bj * TN + c_lo * CW, cin);  // overlaps the main loop
       int ok = 1;
       if (lane == 0) ok = wait_bar_cluster(tfull_bar(acc), acc_phase, abort_flag, p) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       ptx::tc_fence_after();
-      const int row_lo = tc.bi * BM2 + (int)rank * 128 + q * 32;
-      const int i = row_lo + lane;
-      for (int ch = ch_begin; ch < ch_end; ++ch) {
+      for (int ch = c_lo; ch < c_hi; ++ch) {
         const int col0 = tc.bj * TN + ch * CW;
-        if (col0 >= pr.N) break;
-        // half-stored outputs: lower blocks are never written, the diagonal
-        // block is mirrored, upper blocks are written whole
-        const int cblk = col0 / HALF_BLOCK;
-        if (pr.sym && pr.half_out && cblk < tc.bi) continue;
-        const bool tri = pr.sym && (!pr.half_out || cblk == tc.bi);
-        if (tri && col0 + CW - 1 < row_lo) continue;
-        if (row_lo >= pr.M) break;
         uint32_t r[CW];
         ptx::tmem_ld16(tmem_base + (uint32_t)(acc * TN + ch * CW) + ((uint32_t)(q * 32) << 16), r);
         ptx::tmem_wait_ld();
-        if (pr.epi == EPI_GRAM)
-          epi_gram_chunk(pr, tc.mat, i, col0, r, tri, scr);
-        else
+        if (gram) {
+          CinRow nxt;
+          nxt.ok = false;
+          if (ch + 1 < c_hi) cin_fetch(pr, tc.mat, i, col0 + CW, nxt);
+          epi_gram_chunk(pr, tc.mat, i, col0, r, chunk_tri(col0), scr, cin);
+          cin = nxt;
+        } else {
           epi_update_chunk(pr, tc.mat, i, col0, r);
+        }
       }
       ptx::tc_fence_before();
       __syncwarp();
