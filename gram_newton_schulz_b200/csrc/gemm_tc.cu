@@ -205,9 +205,11 @@ __device__ __forceinline__ uint32_t tri_dst(uint32_t scr, int r, int seg) {
 // 8 s: segments left of the diagonal are written from the transpose, the
 // segment holding (R, R) merges the transpose (C < R) with row R's own
 // values (C >= R, from the source rows), segments right of it are skipped.
-// Warp-collective; the lanes' direct stores precede it.
-__device__ __forceinline__ void tri_mirror_part(uint16_t* o, long long mbase, long long ld, int row_lo, int col0,
-                                                int lane, uint4 x0, uint4 x1, uint32_t scr) {
+// om is the matrix's base; in-matrix offsets fit 32 bits (m <= 65536, so
+// row * ld + column < 2^32).  Warp-collective; the lanes' direct stores
+// precede it.
+__device__ __forceinline__ void tri_mirror_part(uint16_t* om, uint32_t ld, int row_lo, int col0, int lane, uint4 x0,
+                                                uint4 x1, uint32_t scr) {
   ptx::sts128(tri_src(scr, lane, 0), x0);
   ptx::sts128(tri_src(scr, lane, 1), x1);
   __syncwarp();
@@ -237,7 +239,7 @@ __device__ __forceinline__ void tri_mirror_part(uint16_t* o, long long mbase, lo
         pv[w] = (pv[w] & keep) | (pd[w] & ~keep);
       }
     }
-    *reinterpret_cast<uint4*>(o + mbase + (long long)R * ld + C0) = val;
+    *reinterpret_cast<uint4*>(om + ((uint32_t)R * ld + (uint32_t)C0)) = val;
   }
   __syncwarp();
 }
@@ -398,8 +400,8 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
             dl[1] = l1;
           }
         }
-        tri_mirror_part(reinterpret_cast<uint16_t*>(oh), mbase, pr.ld, row_lo, col0, lane, h0, h1, scr);
-        if (ol) tri_mirror_part(reinterpret_cast<uint16_t*>(ol), mbase, pr.ld, row_lo, col0, lane, l0, l1, scr);
+        tri_mirror_part(reinterpret_cast<uint16_t*>(oh) + mbase, (uint32_t)pr.ld, row_lo, col0, lane, h0, h1, scr);
+        if (ol) tri_mirror_part(reinterpret_cast<uint16_t*>(ol) + mbase, (uint32_t)pr.ld, row_lo, col0, lane, l0, l1, scr);
         continue;
       }
       if (full && all_upper) {
@@ -468,8 +470,8 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
           dl[1] = l1;
         }
       }
-      tri_mirror_part(reinterpret_cast<uint16_t*>(oh), mbase, pr.ld, row_lo, col0, lane, h0, h1, scr);
-      if (ol) tri_mirror_part(reinterpret_cast<uint16_t*>(ol), mbase, pr.ld, row_lo, col0, lane, l0, l1, scr);
+      tri_mirror_part(reinterpret_cast<uint16_t*>(oh) + mbase, (uint32_t)pr.ld, row_lo, col0, lane, h0, h1, scr);
+      if (ol) tri_mirror_part(reinterpret_cast<uint16_t*>(ol) + mbase, (uint32_t)pr.ld, row_lo, col0, lane, l0, l1, scr);
       continue;
     }
     // direct stores (i, j), j >= i when symmetric
@@ -500,6 +502,156 @@ __device__ __forceinline__ void epi_gram_chunk(const GemmProblem& pr, int mat, i
       }
     }
   }
+}
+
+// Gram products whose input (if any) and output are 16-bit hi/lo pairs and
+// that have no second output -- every product of the split-bf16 and
+// scaled-fp16 classes, and the SYRK -- take a specialised chunk epilogue:
+// the formats are template parameters, the tile-uniform fields are read
+// once per tile into GramTile, and in-matrix offsets are 32-bit.  The
+// arithmetic is epi_gram_chunk's, operation for operation, so the bits are
+// the same; other problems, and chunks at a ragged matrix edge, keep
+// epi_gram_chunk.
+struct GramTile {
+  const uint16_t* cin_hi;  // this matrix's input pair (null: no input; lo may be null)
+  const uint16_t* cin_lo;
+  uint16_t* out_hi;        // this matrix's output pair (lo may be null)
+  uint16_t* out_lo;
+  float coef, beta, gamma;
+  uint32_t ld;
+  int kind;                // GRAM_GENERAL: epi_gram_chunk; else the formats
+};
+enum GramKind : int { GRAM_GENERAL = 0, GRAM_BB = 1, GRAM_HH = 2, GRAM_BH = 3 };  // Cin (or none) -> out formats
+
+__device__ __forceinline__ GramTile gram_tile(const GemmProblem& pr, int mat) {
+  GramTile g;
+  g.kind = GRAM_GENERAL;
+  g.cin_hi = g.cin_lo = nullptr;
+  g.out_hi = g.out_lo = nullptr;
+  g.coef = g.beta = g.gamma = 0.f;
+  g.ld = 0;
+  if (pr.epi != EPI_GRAM || !pr.out_hi || pr.out_fmt == FMT_F32 || pr.out2_hi || pr.out2_f) return g;
+  if (pr.cin_fmt == FMT_F32) return g;
+  const bool cin_h = pr.cin_hi && pr.cin_fmt == FMT_PAIR_H, out_h = pr.out_fmt == FMT_PAIR_H;
+  if (cin_h && !out_h) return g;
+  g.kind = out_h ? (pr.cin_hi && !cin_h ? GRAM_BH : GRAM_HH) : GRAM_BB;
+  const long long mbase = (long long)mat * pr.mat_stride;
+  g.out_hi = reinterpret_cast<uint16_t*>(pr.out_hi) + mbase;
+  g.out_lo = pr.out_lo ? reinterpret_cast<uint16_t*>(pr.out_lo) + mbase : nullptr;
+  if (pr.cin_hi) {
+    g.cin_hi = reinterpret_cast<const uint16_t*>(pr.cin_hi) + mbase;
+    g.cin_lo = pr.cin_lo ? reinterpret_cast<const uint16_t*>(pr.cin_lo) + mbase : nullptr;
+  }
+  float coef = pr.alpha;
+  if (pr.alpha_mode == ALPHA_INV2) {
+    float sv = pr.inv[pr.inv_base + mat];
+    coef *= sv * sv;
+  } else if (pr.alpha_mode == ALPHA_INV) {
+    coef *= pr.inv[pr.inv_base + mat];
+  }
+  g.coef = coef;
+  g.beta = pr.beta;
+  g.gamma = pr.gamma;
+  g.ld = (uint32_t)pr.ld;
+  return g;
+}
+
+// The row segment of a chunk's input pair (see CinRow), for gram_tile16.
+__device__ __forceinline__ void cin16_fetch(const GramTile& g, int i, int col0, CinRow& c) {
+  c.ok = g.cin_hi != nullptr;
+  if (!c.ok) return;
+  const uint32_t off = (uint32_t)i * g.ld + (uint32_t)col0;
+  const uint4* ph = reinterpret_cast<const uint4*>(g.cin_hi + off);
+  c.raw[0] = ld_row16(ph);
+  c.raw[1] = ld_row16(ph + 1);
+  if (g.cin_lo) {
+    const uint4* pl = reinterpret_cast<const uint4*>(g.cin_lo + off);
+    c.raw[2] = ld_row16(pl);
+    c.raw[3] = ld_row16(pl + 1);
+  } else {
+    c.raw[2] = make_uint4(0u, 0u, 0u, 0u);
+    c.raw[3] = c.raw[2];
+  }
+}
+
+// A warp's chunks [c_lo, c_hi) of one tile of a GramTile product, every
+// chunk whole (all 32 rows and 16 columns inside the matrix).  tmem: the
+// accumulator's column 0 in this warp's lane quarter; col_base: the tile's
+// first column; chunks with col0 < tri_end are symmetric diagonal chunks
+// (mirrored); cin: the first chunk's input, already loaded.  The next
+// chunk's input is loaded as soon as this chunk's has been consumed, so
+// one CinRow is live at a time.
+template <bool CIN_H, bool OUT_H>
+__device__ __forceinline__ void gram_tile16(const GramTile& g, uint32_t tmem, int col_base, int c_lo, int c_hi,
+                                            int row_lo, int lane, int tri_end, uint32_t scr, CinRow cin) {
+  const int i = row_lo + lane;
+  const bool has_cin = g.cin_hi != nullptr;
+  for (int ch = c_lo; ch < c_hi; ++ch) {
+    const int col0 = col_base + ch * CW;
+    uint32_t r[CW];
+    ptx::tmem_ld16(tmem + (uint32_t)(ch * CW), r);
+    ptx::tmem_wait_ld();
+    float v[CW];
+#pragma unroll
+    for (int c = 0; c < CW; ++c) v[c] = __fmul_rn(g.coef, __uint_as_float(r[c]));
+    if (has_cin) {
+#pragma unroll
+      for (int q = 0; q < CW / 8; ++q) {
+        float fh[8], fl[8];
+        if (CIN_H) {
+          unpack8_h(cin.raw[q], fh);
+          unpack8_h(cin.raw[2 + q], fl);
+        } else {
+          unpack8(cin.raw[q], fh);
+          unpack8(cin.raw[2 + q], fl);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[8 * q + e] = __fmaf_rn(g.beta, __fadd_rn(fh[e], fl[e]), v[8 * q + e]);
+      }
+      if (ch + 1 < c_hi) cin16_fetch(g, i, col0 + CW, cin);
+    }
+    const int dc = i - col0;  // diagonal column within the chunk
+    if (dc >= 0 && dc < CW) {
+#pragma unroll
+      for (int c = 0; c < CW; ++c)
+        if (c == dc) v[c] = __fadd_rn(v[c], g.gamma);
+    }
+    uint4 h0, l0, h1, l1;
+    if (OUT_H) {
+      split8_h(v, h0, l0);
+      split8_h(v + 8, h1, l1);
+    } else {
+      split8(v, h0, l0);
+      split8(v + 8, h1, l1);
+    }
+    // direct row stores: every row of an upper chunk; in a diagonal chunk
+    // the rows above its diagonal 16 x 16 block and inside it (the block's
+    // lower half is rewritten by the mirror)
+    const bool tri = col0 < tri_end;
+    const uint32_t off = (uint32_t)i * g.ld + (uint32_t)col0;
+    if (!tri || i < col0 + CW) {
+      uint4* dh = reinterpret_cast<uint4*>(g.out_hi + off);
+      dh[0] = h0;
+      dh[1] = h1;
+      if (g.out_lo) {
+        uint4* dl = reinterpret_cast<uint4*>(g.out_lo + off);
+        dl[0] = l0;
+        dl[1] = l1;
+      }
+    }
+    if (tri) {
+      tri_mirror_part(g.out_hi, g.ld, row_lo, col0, lane, h0, h1, scr);
+      if (g.out_lo) tri_mirror_part(g.out_lo, g.ld, row_lo, col0, lane, l0, l1, scr);
+    }
+  }
+}
+
+// GramTile of a warp's part of a tile: the specialised epilogue only when
+// all of the warp's chunks are whole.
+__device__ __forceinline__ GramTile gram_tile_for(const GemmProblem& pr, int mat, int row_lo, int col_end) {
+  GramTile g = gram_tile(pr, mat);
+  if (col_end > pr.N || row_lo + 32 > pr.M) g.kind = GRAM_GENERAL;
+  return g;
 }
 
 // One CW-column chunk of the final O = P X0 tile, fused with the update.
@@ -837,27 +989,43 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_gemm_tc(const __grid_consta
       if (row_lo >= pr.M) c_hi = c_lo;
       while (tri && c_lo < c_hi && tc.bj * TBN + c_lo * CW + CW - 1 < row_lo) ++c_lo;
       const bool gram = pr.epi == EPI_GRAM;
+      const int col_base = tc.bj * TBN;
+      GramTile gt;
+      gt.kind = GRAM_GENERAL;
+      if (gram) gt = gram_tile_for(pr, tc.mat, row_lo, col_base + c_hi * CW);
       CinRow cin;
       cin.ok = false;
-      if (gram && c_lo < c_hi) cin_fetch(pr, tc.mat, i, tc.bj * TBN + c_lo * CW, cin);  // overlaps the main loop
+      if (gram && c_lo < c_hi) {  // the first chunk's input: overlaps the main loop
+        if (gt.kind != GRAM_GENERAL)
+          cin16_fetch(gt, i, col_base + c_lo * CW, cin);
+        else
+          cin_fetch(pr, tc.mat, i, col_base + c_lo * CW, cin);
+      }
       int ok = 1;
       if (lane == 0) ok = wait_bar(tfull_bar(acc), acc_phase, abort_flag, p) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       ptx::tc_fence_after();
-      for (int ch = c_lo; ch < c_hi; ++ch) {
-        const int col0 = tc.bj * TBN + ch * CW;
-        uint32_t r[CW];
-        ptx::tmem_ld16(tmem_base + (uint32_t)(acc * TBN + ch * CW) + ((uint32_t)(q * 32) << 16), r);
-        ptx::tmem_wait_ld();
-        if (gram) {
-          CinRow nxt;
-          nxt.ok = false;
-          if (ch + 1 < c_hi) cin_fetch(pr, tc.mat, i, col0 + CW, nxt);
-          epi_gram_chunk(pr, tc.mat, i, col0, r, tri, scr, cin);
-          cin = nxt;
-        } else {
-          epi_update_chunk(pr, tc.mat, i, col0, r);
+      const uint32_t tacc = tmem_base + (uint32_t)(acc * TBN) + ((uint32_t)(q * 32) << 16);
+      const int tri_end = tri ? INT_MAX : INT_MIN;
+      if (gt.kind == GRAM_BB) {
+        gram_tile16<false, false>(gt, tacc, col_base, c_lo, c_hi, row_lo, lane, tri_end, scr, cin);
+      } else if (gt.kind == GRAM_HH) {
+        gram_tile16<true, true>(gt, tacc, col_base, c_lo, c_hi, row_lo, lane, tri_end, scr, cin);
+      } else if (gt.kind == GRAM_BH) {
+        gram_tile16<false, true>(gt, tacc, col_base, c_lo, c_hi, row_lo, lane, tri_end, scr, cin);
+      } else {
+        for (int ch = c_lo; ch < c_hi; ++ch) {
+          const int col0 = col_base + ch * CW;
+          uint32_t r[CW];
+          ptx::tmem_ld16(tacc + (uint32_t)(ch * CW), r);
+          ptx::tmem_wait_ld();
+          if (gram) {
+            epi_gram_chunk(pr, tc.mat, i, col0, r, tri, scr, cin);
+            if (ch + 1 < c_hi) cin_fetch(pr, tc.mat, i, col0 + CW, cin);  // overlaps the next accumulator load
+          } else {
+            epi_update_chunk(pr, tc.mat, i, col0, r);
+          }
         }
       }
       ptx::tc_fence_before();
@@ -1213,27 +1381,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         break;
       }
       const bool gram = pr.epi == EPI_GRAM;
+      const int col_base = tc.bj * TN;
+      GramTile gt;
+      gt.kind = GRAM_GENERAL;
+      if (gram) gt = gram_tile_for(pr, tc.mat, row_lo, col_base + c_hi * CW);
       CinRow cin;
       cin.ok = false;
-      if (gram && c_lo < c_hi) cin_fetch(pr, tc.mat, i, tc.bj * TN + c_lo * CW, cin);  // overlaps the main loop
+      if (gram && c_lo < c_hi) {  // the first chunk's input: overlaps the main loop
+        if (gt.kind != GRAM_GENERAL)
+          cin16_fetch(gt, i, col_base + c_lo * CW, cin);
+        else
+          cin_fetch(pr, tc.mat, i, col_base + c_lo * CW, cin);
+      }
       int ok = 1;
       if (lane == 0) ok = wait_bar_cluster(tfull_bar(acc), acc_phase, abort_flag, p) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       ptx::tc_fence_after();
-      for (int ch = c_lo; ch < c_hi; ++ch) {
-        const int col0 = tc.bj * TN + ch * CW;
-        uint32_t r[CW];
-        ptx::tmem_ld16(tmem_base + (uint32_t)(acc * TN + ch * CW) + ((uint32_t)(q * 32) << 16), r);
-        ptx::tmem_wait_ld();
-        if (gram) {
-          CinRow nxt;
-          nxt.ok = false;
-          if (ch + 1 < c_hi) cin_fetch(pr, tc.mat, i, col0 + CW, nxt);
-          epi_gram_chunk(pr, tc.mat, i, col0, r, chunk_tri(col0), scr, cin);
-          cin = nxt;
-        } else {
-          epi_update_chunk(pr, tc.mat, i, col0, r);
+      const uint32_t tacc = tmem_base + (uint32_t)(acc * TN) + ((uint32_t)(q * 32) << 16);
+      // symmetric chunks: all (not half-stored) or those of the diagonal block
+      const int tri_end = !pr.sym ? INT_MIN : (!pr.half_out ? INT_MAX : (tc.bi + 1) * HALF_BLOCK);
+      if (gt.kind == GRAM_BB) {
+        gram_tile16<false, false>(gt, tacc, col_base, c_lo, c_hi, row_lo, lane, tri_end, scr, cin);
+      } else if (gt.kind == GRAM_HH) {
+        gram_tile16<true, true>(gt, tacc, col_base, c_lo, c_hi, row_lo, lane, tri_end, scr, cin);
+      } else if (gt.kind == GRAM_BH) {
+        gram_tile16<false, true>(gt, tacc, col_base, c_lo, c_hi, row_lo, lane, tri_end, scr, cin);
+      } else {
+        for (int ch = c_lo; ch < c_hi; ++ch) {
+          const int col0 = col_base + ch * CW;
+          uint32_t r[CW];
+          ptx::tmem_ld16(tacc + (uint32_t)(ch * CW), r);
+          ptx::tmem_wait_ld();
+          if (gram) {
+            epi_gram_chunk(pr, tc.mat, i, col0, r, chunk_tri(col0), scr, cin);
+            if (ch + 1 < c_hi) cin_fetch(pr, tc.mat, i, col0 + CW, cin);  // overlaps the next accumulator load
+          } else {
+            epi_update_chunk(pr, tc.mat, i, col0, r);
+          }
         }
       }
       ptx::tc_fence_before();
