@@ -106,16 +106,16 @@ def gemm_alg_bytes(shapes, k=K_STEPS):
 # captured ones (close calls of the autotuner can differ from box to box).
 TRAFFIC_CAPTURE = {
     "sources": ["gram_newton_schulz_b200/csrc/gemm_tc.cu", "gram_newton_schulz_b200/csrc/plan.cu"],
-    "sha256": "5dd5a4cd019c3d3e75d74d8e8c67355972b70b41255ddaa3fa25a5d1cd69f7f3",
+    "sha256": "127ceaff98071631ed3ebe3828de6403486087cfb5f444ce7cb11094b50aa156",
     "workload": "qwen2.5-7b-layer-set-x28",
     "captured_on": "3584x3584*4,512x3584*4,18944x3584*4,3584x18944*2 (2 of 28 layers)",
     "scale": 14,
-    "dram_bytes_per_step": 15.203e9 * 14,
+    "dram_bytes_per_step": 15.137e9 * 14,
     "schedule": {
         "gram": {"m512": "single_cta_n128", "m3584": "cta_pair"},
-        "syrk": {"512x3584": "single_cta_n128", "3584x3584": "cta_pair_k2", "3584x18944": "cta_pair_k2",
+        "syrk": {"512x3584": "cta_pair_k2", "3584x3584": "cta_pair_k2", "3584x18944": "cta_pair_k2",
                  "18944x3584": "single_cta"},
-        "final": {"512x3584": "single_cta", "3584x3584": "single_cta", "3584x18944": "single_cta",
+        "final": {"512x3584": "single_cta", "3584x3584": "single_cta", "3584x18944": "cta_pair",
                   "18944x3584": "single_cta"},
     },
 }
