@@ -1293,6 +1293,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
             break;
           }
           ptx::tc_fence_after();
+          // Descriptors: the start address (bits 0-13, bytes / 16) sits in
+          // the low word and never carries out of its field (shared
+          // addresses are below 256 KB), so each MMA's descriptor is an atom
+          // base plus a constant, one 32-bit add.
           const uint32_t sa = ring + stage * Cfg::STAGE_BYTES;
           const uint32_t sb = sa + NA * KATOMS * HALF_BYTES;
 #pragma unroll
@@ -1300,7 +1304,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
             const int ktile = (kb * BKE + at * ATOM_E) / HALF_BLOCK;
             const uint32_t a_mn = (uint32_t)(pr_a_mn | (ktile < thr_a ? 1 : 0));
             const uint64_t a_hi = a_mn ? hi_mn : hi_k;
-            const uint32_t a_ks = a_mn ? 2048u : 32u;
+            const uint32_t a_up = (uint32_t)(a_hi >> 32), a_dk = a_mn ? 2048u / 16u : 32u / 16u;
+            const uint32_t a_lo0 = (uint32_t)a_hi | ((sa + at * HALF_BYTES) >> 4);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               // the NH halves of the tile share this K slice's A operand
@@ -1309,16 +1314,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
                 const uint32_t b_mn = (uint32_t)(pr_b_mn | (ktile < (h ? thr_b1 : thr_b0) ? 1 : 0));
                 const uint32_t idesc = idesc0 | (a_mn << 15) | (b_mn << 16);
                 const uint64_t b_hi = b_mn ? hi_mn : hi_k;
-                const uint32_t b_ks = b_mn ? 2048u : 32u;
+                const uint32_t b_up = (uint32_t)(b_hi >> 32), b_dk = b_mn ? 2048u / 16u : 32u / 16u;
+                const uint32_t b_lo0 = (uint32_t)b_hi | ((sb + (h * KATOMS + at) * HALF_BYTES) >> 4);
 #pragma unroll
                 for (int term = 0; term < 3; ++term) {
                   if (term == 1 && NB < 2) continue;
                   if (term == 2 && NA < 2) continue;
                   if (!(terms & (1 << term))) continue;
-                  const uint32_t pa = sa + ((term == 2 ? KATOMS : 0) + at) * HALF_BYTES + kk * a_ks;
-                  const uint32_t pb = sb + (((term == 1 ? NH : 0) + h) * KATOMS + at) * HALF_BYTES + kk * b_ks;
-                  const uint64_t ad = a_hi | (uint64_t)((pa >> 4) & 0x3FFFu);
-                  const uint64_t bd = b_hi | (uint64_t)((pb >> 4) & 0x3FFFu);
+                  const uint32_t a_lo = a_lo0 + kk * a_dk + (term == 2 ? KATOMS * HALF_BYTES / 16 : 0);
+                  const uint32_t b_lo = b_lo0 + kk * b_dk + (term == 1 ? NH * KATOMS * HALF_BYTES / 16 : 0);
+                  const uint64_t ad = ((uint64_t)a_up << 32) | a_lo;
+                  const uint64_t bd = ((uint64_t)b_up << 32) | b_lo;
                   if (KIND == KIND_TF32)
                     ptx::mma2_tf32(d_tmem + (uint32_t)(h * 256), ad, bd, idesc, accumulate[h]);
                   else
