@@ -141,6 +141,40 @@ def captured_traffic(workload_name):
     return cap["dram_bytes_per_step"]
 
 
+def graph_phase_split(plan, grads, moms, weights, w, K, stream, dev):
+    """Device time of the momentum, Gram and update phases over K steps,
+    each phase captured as its own CUDA graph and the three replayed in
+    turn with events between them.  Returns (times, None), or (None, why)
+    if a capture fails."""
+    import torch
+
+    from gram_newton_schulz_b200 import dmu
+    try:
+        gp = [torch.cuda.CUDAGraph() for _ in range(3)]
+        calls = (lambda: plan.momentum_normalize(grads, moms, beta=w.beta, eps=1e-7),
+                 lambda: plan.gram_ns_batched(None, dmu.QUINTIC, K_STEPS),
+                 lambda: plan.apply_update(weights, lr=w.lr))
+        torch.cuda.synchronize(dev)
+        for g, call in zip(gp, calls):
+            with torch.cuda.graph(g, capture_error_mode="thread_local"):
+                call()
+        for g in gp:
+            g.replay()
+        torch.cuda.synchronize(dev)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+        for k in range(K):
+            for i, g in enumerate(gp):
+                ev[k][i].record(stream)
+                g.replay()
+            ev[k][3].record(stream)
+        torch.cuda.synchronize(dev)
+        out = tuple(sum(e[i].elapsed_time(e[i + 1]) for e in ev) for i in range(3))
+        del gp
+        return out, None
+    except Exception as e:  # keep the eager split, say why
+        return None, f"{type(e).__name__}: {str(e)[:120]}"
+
+
 def momentum_bytes(shapes, grad_bytes=2, image16=False):
     """HBM bytes of the momentum phase: read G and M, write M and the bf16
     image; with ``image16`` also the in-place conversion of the image to
@@ -714,6 +748,7 @@ def main():
     # comes from the eager steps; the headline value is the graph replay
     # when capture succeeded.
     graph_note = "off (--no-graph)"
+    split_note = "eager steps"
     total_ms = eager_ms
     if not args.no_graph:
         g = None
@@ -745,6 +780,17 @@ def main():
             torch.cuda.synchronize(dev)
             barrier()
             total_ms = gev[0].elapsed_time(gev[1]) / K
+            # The phase split (roofline and HBM fractions below) from the
+            # device alone: the step's three phases captured as three graphs
+            # and replayed in turn, events between them, so the eager
+            # split's host time (marshalling thousands of tensors per call
+            # while the GPU idles) stays out of the kernels' durations.
+            split, why = graph_phase_split(plan, grads, moms, weights, w, K, stream, dev)
+            if all_ranks_ok(split is not None, dev, world):
+                t_mom, t_gram, t_upd = split
+                split_note = "graph replay of each phase"
+            else:
+                split_note = f"eager steps (phase capture failed: {why})" if why else "eager steps"
         del g
     clk = clocks.stop()
     total_ms *= K
@@ -872,6 +918,7 @@ def main():
                                                        if clk and clk.get("sm_mhz") else None)},
             "split_ms": {"momentum": round(t_mom / K, 3), "gram": round(t_gram / K, 3),
                          "update": round(t_upd / K, 3)},
+            "split_source": split_note,
             "eager_ms_per_step": round(eager_max, 3),
             "roofline": {"bound": "tensor", "achieved": round(achieved_tf, 1), "peak": peak_tf,
                          "unit": "TFLOP/s", "frac": round(achieved_tf / peak_tf, 4),
