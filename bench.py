@@ -744,9 +744,9 @@ def main():
     # The same step captured once into a CUDA graph and replayed: the
     # launches of a step (tens of them) cost no host time.  Steady-state
     # calls of the library only enqueue kernels (pointer tables are uploaded
-    # only when they change), so a step is capturable.  The phase split above
-    # comes from the eager steps; the headline value is the graph replay
-    # when capture succeeded.
+    # only when they change), so a step is capturable.  The headline value is
+    # the graph replay when capture succeeded, and the eager phase split above
+    # is then replaced by the per-phase replay below.
     graph_note = "off (--no-graph)"
     split_note = "eager steps"
     total_ms = eager_ms
